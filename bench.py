@@ -1,0 +1,346 @@
+#!/usr/bin/env python3
+"""Throughput of the Gated DeltaNet-2 chunkwise forward (gdn2_chunk_fwd) on B200.
+
+Workload: the long-context 16K x 1 token budget of the pages' throughput
+figure -- B=1, T=16384, H=16, dk=dv=128, bf16 q/k/v/out, fp32 gates with
+strong per-channel decay variety, seeded synthetic inputs (workloads.py,
+workload 2).  A step is one gdn2_chunk_fwd call over the whole batch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun (one process per GPU, NCCL for the barrier and the
+max-over-ranks reduction only): every rank runs an independent replica of the
+workload ("replicas only": the operator needs no exchange between sequences).
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN2 chunk-fwd tokens/s (B·T) at H=16,dk=dv=128,bf16 on 1 B200; % of roofline"
+UNIT = "tokens/s"
+WORKLOAD_ID = 2
+B, T, H, DK, DV = 1, 16384, 16, 128, 128
+TH = B * T * H
+# Algorithmic work of the method per token-head (bf16 I/O, d = 128, chunk 64):
+# q, k, v in bf16 (768 B) + log_alpha, b, w in fp32 (1536 B) + O in bf16 (256 B);
+# per (sequence, head) the fp32 final state (64 KiB); h0 is zero and not read.
+ALG_BYTES_PER_TH = 2560
+ALG_BYTES = TH * ALG_BYTES_PER_TH + B * H * DK * DV * 4
+# Chunk-form FLOPs per token-head: 6*dk*dv + 5*C*d + C^2/3 with C = 64.
+ALG_FLOPS = TH * (6 * DK * DV + 5 * 64 * 128 + 64 * 64 / 3)
+# Compulsory bytes of the two kernels given the stored chunk factors (bf16
+# W, U~, Kbar, Q_eff, O_part = 1280 B per token-head, exp(g_n) fp32 8 B).
+PREP_BYTES = TH * (2304 + 1280 + 8)
+WALK_BYTES = TH * (1280 + 8 + 256) + B * H * DK * DV * 4
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "200"]
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(self.cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        except OSError:
+            return None
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        torch.cuda.set_device(0)
+        return 0, 1, 0
+    import datetime
+
+    import torch.distributed as dist
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return dist.get_rank(), dist.get_world_size(), local
+
+
+def barrier_sync(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(x, target_s, max_tokens=T):
+    """Time the fp64 oracle (as it stands) on the first `t` tokens of every
+    head, with `t` chosen so that one run takes about `target_s` seconds."""
+    import oracle
+    cores = min(oracle.default_threads(), H * B)
+    t_tok = 256
+    while True:
+        s = slice(0, t_tok)
+        args = [a[:, s] for a in (x.q, x.k, x.v, x.log_alpha, x.b, x.w)]
+        t0 = time.perf_counter()
+        oracle.recurrent(*args, x.scale, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or t_tok >= max_tokens:
+            return B * t_tok / dt, cores, t_tok, dt
+        t_tok = int(min(max_tokens, max(t_tok * 2, t_tok * target_s / max(dt, 1e-3))))
+
+
+def run_reference(args, rank):
+    """The oracle as the reference arm: each step is a bounded sample of the
+    workload (all 16 heads, the first t tokens), timed on the host cores."""
+    if rank != 0:
+        return
+    from workloads import config
+    x = config(WORKLOAD_ID)
+    per_step = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    _, cores, t_tok, _ = cpu_oracle_sample(x, per_step)
+    import oracle
+    s = slice(0, t_tok)
+    sample = [a[:, s] for a in (x.q, x.k, x.v, x.log_alpha, x.b, x.w)]
+    for _ in range(args.warmup):
+        oracle.recurrent(*sample, x.scale, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrent(*sample, x.scale, nthreads=cores)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = B * t_tok / dt
+    desc = f"fp64 C oracle on tokens [0,{t_tok}) of every head of the 16Kx1 workload"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "16Kx1 B=1 T=16384 H=16 dk=dv=128 (sampled)", "sample_tokens": t_tok},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    from workloads import config
+    gdn2.load_library()
+    x = config(WORKLOAD_ID)
+    dev = torch.device("cuda", local)
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
+    bf, f32 = torch.bfloat16, torch.float32
+    q, k, v = t(x.q, bf), t(x.k, bf), t(x.v, bf)
+    la, b, w = t(x.log_alpha, f32), t(x.b, f32), t(x.w, f32)
+    out = torch.empty_like(v)
+    hT = torch.empty((B, H, DK, DV), dtype=f32, device=dev)
+    ws = torch.empty(gdn2.workspace_size(B, T, H, DK, DV, gdn2.GDN2_IO_BF16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn2.chunk_fwd(q, k, v, la, b, w, x.scale, out=out, hT=hT, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier_sync(world)
+    if sampler:
+        sampler.__enter__()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    barrier_sync(world)
+    if sampler:
+        sampler.__exit__(None, None, None)
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(ms, world)
+    launches_per_step = 3  # plan, prep, walk
+
+    # per-kernel durations of the same work through the stage entry points
+    kt = {"prep": [], "walk": []}
+    nk = max(3, min(args.steps, 50))
+    for i in range(nk):
+        flush.zero_()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        gdn2.chunk_prep(q, k, v, la, b, w, workspace=ws, stream=stream)
+        e1.record(stream)
+        gdn2.chunk_walk(ws, (B, T, H, DK, DV), bf, x.scale, out=out, hT=hT, stream=stream)
+        e2.record(stream)
+        kt["prep"].append((e0, e1))
+        kt["walk"].append((e1, e2))
+    torch.cuda.synchronize()
+    kern_ms = {kname: sum(a.elapsed_time(bb) for a, bb in ev) / len(ev) for kname, ev in kt.items()}
+
+    # end to end: pinned host inputs -> device -> chunk_fwd -> O, hT back to pinned host
+    host = {n: getattr(x, n) for n in ("q", "k", "v", "log_alpha", "b", "w")}
+    pin = {}
+    for n, a in host.items():
+        dt = bf if n in ("q", "k", "v") else f32
+        pin[n] = torch.from_numpy(np.ascontiguousarray(a)).to(dt).pin_memory()
+    dev_in = {"q": q, "k": k, "v": v, "log_alpha": la, "b": b, "w": w}
+    out_h = torch.empty(out.shape, dtype=bf).pin_memory()
+    hT_h = torch.empty(hT.shape, dtype=f32).pin_memory()
+    h2d = sum(p.numel() * p.element_size() for p in pin.values())
+    d2h = out_h.numel() * out_h.element_size() + hT_h.numel() * hT_h.element_size()
+    ne = max(2, min(args.steps, 10))
+    barrier_sync(world)
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_s.record(stream)
+    for _ in range(ne):
+        for n in dev_in:
+            dev_in[n].copy_(pin[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        hT_h.copy_(hT, non_blocking=True)
+    e_e.record(stream)
+    barrier_sync(world)
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / ne, world)
+
+    if rank != 0:
+        return
+    hbm, tflops, src = peaks()
+    tokens = B * T
+    value = world * tokens / (ms / 1e3)
+    t_roof = max(ALG_BYTES / (hbm * 1e9), ALG_FLOPS / (tflops * 1e12))
+    dom = max(kern_ms, key=kern_ms.get)
+    dom_bytes = PREP_BYTES if dom == "prep" else WALK_BYTES
+    dom_gbs = dom_bytes / (kern_ms[dom] / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "16Kx1 B=1 T=16384 H=16 dk=dv=128 bf16 I/O, fp32 gates (strong decay)",
+                   "global_batch": world * B, "seq_len": T, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MiB write)"},
+        "roofline": {"bound": "hbm", "achieved": dom_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": dom_gbs / hbm, "traffic": None, "kernel": dom,
+                     "kernel_ms": kern_ms[dom], "alg_bytes_per_launch": dom_bytes,
+                     "peak_source": f"{src} (MEASURED_PEAKS hbm_gbs)" if src == "measured" else src},
+        "roofline_step": {"alg_bytes": ALG_BYTES, "alg_flops": ALG_FLOPS, "t_roof_us": t_roof * 1e6,
+                          "t_meas_us": ms * 1e3, "frac": t_roof / (ms / 1e3),
+                          "achieved_gbs": ALG_BYTES / (ms / 1e3) / 1e9},
+        "kernels_ms": kern_ms,
+        "e2e": {"value": world * tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ne},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    clk = sampler.summary() if sampler else None
+    line["clocks"] = clk
+    if world == 1 and not args.no_cpu_baseline:
+        tps, cores, t_tok, dt = cpu_oracle_sample(x, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"fp64 C oracle, tokens [0,{t_tok}) of all 16 heads "
+                                          f"({dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", 0))
+        run_reference(args, rank)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

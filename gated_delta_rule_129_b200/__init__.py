@@ -1,0 +1,264 @@
+"""B200 (sm_100a) Gated DeltaNet-2 forward operator -- Python binding.
+
+A thin ctypes layer over ``libgdn2.so`` (declared in ``include/gdn2.h``).  It
+only marshals arguments: every step of the computation runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There
+is no CPU fallback: if the library is missing, every call raises.
+
+Public functions mirror the C entry points:
+
+* :func:`chunk_fwd`        -- ``gdn2_chunk_fwd``
+* :func:`chunk_prep`       -- ``gdn2_chunk_prep`` (gate prep + intra-chunk WY)
+* :func:`chunk_walk`       -- ``gdn2_chunk_walk`` (state walk + output)
+* :func:`recurrent_step`   -- ``gdn2_recurrent_step`` (one decode token)
+* :func:`workspace_size`, :func:`workspace_layout`, :func:`status_string`
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = ["chunk_fwd", "chunk_prep", "chunk_walk", "recurrent_step", "workspace_size",
+           "workspace_layout", "status_string", "GDN2Error", "lib_path", "load_library"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgdn2.so")
+_lock = threading.Lock()
+_lib = None
+
+GDN2_IO_F32 = 0
+GDN2_IO_BF16 = 1
+
+STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_NULL", 2: "GDN2_ERR_SHAPE", 3: "GDN2_ERR_DTYPE",
+          4: "GDN2_ERR_ALIGN", 5: "GDN2_ERR_SEQLENS", 6: "GDN2_ERR_WORKSPACE",
+          7: "GDN2_ERR_CUDA", 8: "GDN2_ERR_DEVICE_TIMEOUT", 9: "GDN2_ERR_UNSUPPORTED"}
+
+EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_prep",
+            "gdn2_chunk_walk", "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version")
+
+
+class GDN2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("num_seqs", ctypes.c_int),
+                ("io", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("max_chunks", ctypes.c_int),
+                ("factor_elem_bytes", ctypes.c_int), ("off_W", ctypes.c_size_t),
+                ("off_Ut", ctypes.c_size_t), ("off_Kbar", ctypes.c_size_t),
+                ("off_Qeff", ctypes.c_size_t), ("off_Opart", ctypes.c_size_t),
+                ("off_gamma_last", ctypes.c_size_t), ("off_chunk_offsets", ctypes.c_size_t),
+                ("off_status", ctypes.c_size_t)]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load ``libgdn2.so``; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m gated_delta_rule_129_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        dp = ctypes.POINTER(Desc)
+        lib.gdn2_workspace_size.argtypes = [dp]
+        lib.gdn2_workspace_size.restype = sz
+        lib.gdn2_workspace_layout.argtypes = [dp, ctypes.POINTER(WsLayout)]
+        lib.gdn2_workspace_layout.restype = i
+        lib.gdn2_chunk_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
+        lib.gdn2_chunk_fwd.restype = i
+        lib.gdn2_chunk_prep.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.gdn2_chunk_prep.restype = i
+        lib.gdn2_chunk_walk.argtypes = [dp, f, vp, vp, vp, vp, vp, vp]
+        lib.gdn2_chunk_walk.restype = i
+        lib.gdn2_recurrent_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp]
+        lib.gdn2_recurrent_step.restype = i
+        lib.gdn2_status_string.argtypes = [i]
+        lib.gdn2_status_string.restype = ctypes.c_char_p
+        lib.gdn2_version.argtypes = []
+        lib.gdn2_version.restype = i
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().gdn2_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise GDN2Error(status, where)
+
+
+# ------------------------------------------------------------------ helpers --
+
+def _torch():
+    import torch
+    return torch
+
+
+def _io_of(dtype) -> int:
+    torch = _torch()
+    if dtype == torch.float32:
+        return GDN2_IO_F32
+    if dtype == torch.bfloat16:
+        return GDN2_IO_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_desc(B, T, H, dk, dv, io, num_seqs=0, workspace=None, workspace_bytes=0) -> Desc:
+    return Desc(int(B), int(T), int(H), int(dk), int(dv), int(num_seqs), int(io),
+                None if workspace is None else ctypes.c_void_p(workspace),
+                int(workspace_bytes))
+
+
+def workspace_size(B, T, H, dk, dv, io=GDN2_IO_BF16, num_seqs=0) -> int:
+    d = make_desc(B, T, H, dk, dv, io, num_seqs)
+    return int(load_library().gdn2_workspace_size(ctypes.byref(d)))
+
+
+def workspace_layout(B, T, H, dk, dv, io=GDN2_IO_BF16, num_seqs=0) -> dict:
+    d = make_desc(B, T, H, dk, dv, io, num_seqs)
+    lay = WsLayout()
+    _check(load_library().gdn2_workspace_layout(ctypes.byref(d), ctypes.byref(lay)),
+           "gdn2_workspace_layout")
+    return lay.as_dict()
+
+
+def _shapes(q, v, cu_seqlens):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+    return B, T, H, dk, dv, num_seqs
+
+
+def _alloc_workspace(desc_args, device):
+    torch = _torch()
+    nbytes = workspace_size(*desc_args)
+    if nbytes == 0:
+        raise GDN2Error(2, "gdn2_workspace_size")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _need_contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+# -------------------------------------------------------------- entry points --
+
+def chunk_fwd(q, k, v, log_alpha, b, w, scale=None, h0=None, cu_seqlens=None, *,
+              out=None, hT=None, workspace=None, output_final_state=True, stream=None):
+    """Gated DeltaNet-2 chunkwise forward.  Returns ``(out, hT)``.
+
+    ``q, k, v`` are float32 or bfloat16 ``[B, T, H, d]`` CUDA tensors;
+    ``log_alpha, b, w`` float32 of the same leading shape; ``h0`` float32
+    ``[N, H, dk, dv]`` or None; ``cu_seqlens`` int32 ``[N + 1]`` CUDA tensor
+    or None.  ``scale`` defaults to ``dk ** -0.5``.
+    """
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    io = _io_of(q.dtype)
+    N = ns if cu_seqlens is not None else B
+    if scale is None:
+        scale = dk ** -0.5
+    _need_contig(q, k, v, log_alpha, b, w, h0, cu_seqlens)
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _alloc_workspace((B, T, H, dk, dv, io, ns), q.device)
+    d = make_desc(B, T, H, dk, dv, io, ns, workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                       _ptr(b), _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens),
+                                       _ptr(out), _ptr(hT), _stream(stream))
+    _check(st, "gdn2_chunk_fwd")
+    return out, hT
+
+
+def chunk_prep(q, k, v, log_alpha, b, w, cu_seqlens=None, *, workspace=None, stream=None):
+    """Stage 1 only.  Returns the workspace tensor holding the chunk factors."""
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    io = _io_of(q.dtype)
+    _need_contig(q, k, v, log_alpha, b, w, cu_seqlens)
+    if workspace is None:
+        workspace = _alloc_workspace((B, T, H, dk, dv, io, ns), q.device)
+    d = make_desc(B, T, H, dk, dv, io, ns, workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_prep(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                        _ptr(b), _ptr(w), _ptr(cu_seqlens), _stream(stream))
+    _check(st, "gdn2_chunk_prep")
+    return workspace
+
+
+def chunk_walk(workspace, shape, io_dtype, scale, h0=None, cu_seqlens=None, *, out=None, hT=None,
+               chunk_states=None, stream=None):
+    """Stage 2 only, from a workspace filled by :func:`chunk_prep`.
+
+    ``shape`` is ``(B, T, H, dk, dv)``; ``io_dtype`` the torch dtype of q/k/v.
+    Returns ``(out, hT)``.
+    """
+    torch = _torch()
+    B, T, H, dk, dv = shape
+    ns = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+    N = ns if cu_seqlens is not None else B
+    io = _io_of(io_dtype)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=io_dtype, device=workspace.device)
+    if hT is None:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=workspace.device)
+    d = make_desc(B, T, H, dk, dv, io, ns, workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_walk(ctypes.byref(d), float(scale), _ptr(h0), _ptr(cu_seqlens),
+                                        _ptr(out), _ptr(hT), _ptr(chunk_states), _stream(stream))
+    _check(st, "gdn2_chunk_walk")
+    return out, hT
+
+
+def recurrent_step(q, k, v, log_alpha, b, w, scale, state, *, out=None, stream=None):
+    """One decode token; ``state`` ``[B, H, dk, dv]`` fp32 is updated in place.
+
+    ``q, k, log_alpha, b`` are ``[B, H, dk]``; ``v, w`` ``[B, H, dv]``.
+    Returns ``out`` ``[B, H, dv]``.
+    """
+    torch = _torch()
+    Bn, H, dk = q.shape
+    dv = v.shape[-1]
+    io = _io_of(q.dtype)
+    _need_contig(q, k, v, log_alpha, b, w, state)
+    if out is None:
+        out = torch.empty((Bn, H, dv), dtype=q.dtype, device=q.device)
+    d = make_desc(Bn, 1, H, dk, dv, io)
+    st = load_library().gdn2_recurrent_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                            _ptr(b), _ptr(w), float(scale), _ptr(state), _ptr(out),
+                                            _stream(stream))
+    _check(st, "gdn2_recurrent_step")
+    return out

@@ -1,0 +1,71 @@
+// common.cuh -- small device helpers shared by the Gated DeltaNet-2 kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn2 {
+
+// Chunk length of the WY form (page "Gated DeltaNet-2：将擦除与写入分开",
+// section "词元路径与并行训练": training uses 64-token chunks).
+constexpr int kChunk = 64;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Sequence bookkeeping shared by every chunked kernel.  Sequence n covers
+// tokens [seq_begin(n), seq_end(n)); its chunks are global indices
+// [chunk_off[n], chunk_off[n+1]) and chunk j of it starts at token
+// seq_begin(n) + 64 j.
+struct SeqMap {
+  const int32_t* cu;        // packed boundaries or nullptr (dense)
+  const int32_t* chunk_off; // [N + 1], written by the plan kernel
+  int N;                    // sequences
+  int T;                    // dense tokens per sequence (unused when packed)
+
+  __device__ __forceinline__ int seq_begin(int n) const { return cu ? cu[n] : n * T; }
+  __device__ __forceinline__ int seq_end(int n) const { return cu ? cu[n + 1] : (n + 1) * T; }
+
+  // The sequence owning global chunk c (c < chunk_off[N]): the largest n with
+  // chunk_off[n] <= c; empty sequences (equal offsets) are skipped over.
+  __device__ __forceinline__ int seq_of_chunk(int c) const {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (chunk_off[mid] <= c) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+};
+
+// Where one chunk sits in the token stream.
+struct ChunkPos {
+  int seq, t0, len;
+};
+
+__device__ __forceinline__ ChunkPos chunk_pos(const SeqMap& m, int c) {
+  ChunkPos p;
+  p.seq = m.seq_of_chunk(c);
+  const int j = c - m.chunk_off[p.seq];
+  p.t0 = m.seq_begin(p.seq) + j * kChunk;
+  p.len = min(kChunk, m.seq_end(p.seq) - p.t0);
+  return p;
+}
+
+}  // namespace gdn2

@@ -1,0 +1,345 @@
+// gdn2_api.cu -- the C ABI declared in include/gdn2.h.
+//
+// Host side only: argument checks (no CUDA call happens before they pass),
+// workspace carving, and dispatch of the kernels for (dk, dv, io dtype).
+// Nothing here allocates device memory or synchronises a stream.
+#include "gdn2.h"
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "plan.cuh"
+#include "prep_simt.cuh"
+#include "walk_simt.cuh"
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+using gdn2::kChunk;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn2_status check_dims(const gdn2_desc* d, bool packed) {
+  if (!d) return GDN2_ERR_NULL;
+  if (d->io != GDN2_IO_F32 && d->io != GDN2_IO_BF16) return GDN2_ERR_DTYPE;
+  if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128)) return GDN2_ERR_SHAPE;
+  if (d->H < 1 || d->B < 1 || d->T < 0) return GDN2_ERR_SHAPE;
+  // packed calls describe num_seqs >= 1 sequences in one row; dense calls
+  // leave num_seqs at 0 (this keeps gdn2_workspace_size consistent)
+  if (packed && (d->B != 1 || d->num_seqs < 1)) return GDN2_ERR_SHAPE;
+  if (!packed && d->num_seqs != 0) return GDN2_ERR_SHAPE;
+  // all token-level indices are computed in 64-bit, but token and chunk
+  // counts themselves must fit in int32
+  const long long tokens = (long long)d->B * d->T;
+  if (tokens > INT32_MAX / 2) return GDN2_ERR_SHAPE;
+  return GDN2_OK;
+}
+
+struct Layout {
+  gdn2_ws_layout l;
+  int N;
+};
+
+gdn2_status make_layout(const gdn2_desc* d, bool packed, Layout* out) {
+  gdn2_status st = check_dims(d, packed);
+  if (st != GDN2_OK) return st;
+  const int N = packed ? d->num_seqs : d->B;
+  const long long tokens = (long long)d->B * d->T;
+  const long long max_chunks =
+      packed ? tokens / kChunk + N : (long long)d->B * ((d->T + kChunk - 1) / kChunk);
+  if (max_chunks > INT32_MAX / 2) return GDN2_ERR_SHAPE;
+  gdn2_ws_layout& L = out->l;
+  std::memset(&L, 0, sizeof(L));
+  L.max_chunks = (int)max_chunks;
+  L.factor_elem_bytes = d->io == GDN2_IO_F32 ? 4 : 2;
+  const size_t tiles = (size_t)max_chunks * d->H * kChunk;
+  const size_t eb = (size_t)L.factor_elem_bytes;
+  size_t off = 0;
+  L.off_W = off;          off = align_up(off + tiles * d->dk * eb);
+  L.off_Ut = off;         off = align_up(off + tiles * d->dv * eb);
+  L.off_Kbar = off;       off = align_up(off + tiles * d->dk * eb);
+  L.off_Qeff = off;       off = align_up(off + tiles * d->dk * eb);
+  L.off_Opart = off;      off = align_up(off + tiles * d->dv * eb);
+  L.off_gamma_last = off; off = align_up(off + (size_t)max_chunks * d->H * d->dk * sizeof(float));
+  L.off_chunk_offsets = off; off = align_up(off + (size_t)(N + 1) * sizeof(int32_t));
+  L.off_status = off;     off = align_up(off + sizeof(int32_t));
+  L.total_bytes = off;
+  out->N = N;
+  return GDN2_OK;
+}
+
+gdn2_status check_workspace(const gdn2_desc* d, const Layout& L) {
+  if (!d->workspace) return GDN2_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(d->workspace) & (kAlign - 1)) != 0) return GDN2_ERR_ALIGN;
+  if (d->workspace_bytes < L.l.total_bytes) return GDN2_ERR_WORKSPACE;
+  return GDN2_OK;
+}
+
+gdn2_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+gdn2::SeqMap seq_map(const gdn2_desc* d, const Layout& L, const int32_t* cu) {
+  gdn2::SeqMap m;
+  m.cu = cu;
+  m.chunk_off = at<const int32_t>(d->workspace, L.l.off_chunk_offsets);
+  m.N = L.N;
+  m.T = d->T;
+  return m;
+}
+
+gdn2_status launch_plan(const gdn2_desc* d, const Layout& L, const int32_t* cu, cudaStream_t s) {
+  gdn2::plan_kernel<<<1, gdn2::kPlanThreads, 0, s>>>(
+      cu, L.N, d->T, d->B * d->T, at<int32_t>(d->workspace, L.l.off_chunk_offsets),
+      at<int32_t>(d->workspace, L.l.off_status), (int)GDN2_ERR_SEQLENS);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- prep ----
+template <int DK, int DV, typename IO, typename FT>
+gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, const void* k,
+                          const void* v, const float* la, const float* b, const float* w,
+                          const int32_t* cu, cudaStream_t s) {
+  gdn2::PrepArgs<IO, FT> a;
+  a.q = static_cast<const IO*>(q);
+  a.k = static_cast<const IO*>(k);
+  a.v = static_cast<const IO*>(v);
+  a.la = la;
+  a.b = b;
+  a.w = w;
+  a.map = seq_map(d, L, cu);
+  a.H = d->H;
+  a.W = at<FT>(d->workspace, L.l.off_W);
+  a.Ut = at<FT>(d->workspace, L.l.off_Ut);
+  a.Kbar = at<FT>(d->workspace, L.l.off_Kbar);
+  a.Qeff = at<FT>(d->workspace, L.l.off_Qeff);
+  a.Opart = at<FT>(d->workspace, L.l.off_Opart);
+  a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
+  if (L.l.max_chunks == 0) return GDN2_OK;
+  constexpr size_t smem = gdn2::prep_simt_smem_bytes<DK, DV>();
+  auto kern = gdn2::prep_simt_kernel<DK, DV, IO, FT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  dim3 grid(L.l.max_chunks, d->H);
+  kern<<<grid, gdn2::kPrepSimtThreads, smem, s>>>(a);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- walk ----
+template <int DK, int DV, typename IO, typename FT>
+gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, const float* h0,
+                          const int32_t* cu, void* out, float* hT, float* chunk_states,
+                          cudaStream_t s) {
+  gdn2::WalkArgs<IO, FT> a;
+  a.W = at<const FT>(d->workspace, L.l.off_W);
+  a.Ut = at<const FT>(d->workspace, L.l.off_Ut);
+  a.Kbar = at<const FT>(d->workspace, L.l.off_Kbar);
+  a.Qeff = at<const FT>(d->workspace, L.l.off_Qeff);
+  a.Opart = at<const FT>(d->workspace, L.l.off_Opart);
+  a.gamma_last = at<const float>(d->workspace, L.l.off_gamma_last);
+  a.map = seq_map(d, L, cu);
+  a.H = d->H;
+  a.scale = scale;
+  a.h0 = h0;
+  a.out = static_cast<IO*>(out);
+  a.hT = hT;
+  a.chunk_states = chunk_states;
+  if (L.N == 0) return GDN2_OK;
+  constexpr size_t smem = gdn2::walk_simt_smem_bytes<DK, DV>();
+  auto kern = gdn2::walk_simt_kernel<DK, DV, IO, FT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  const long long blocks = (long long)L.N * d->H * (DV / gdn2::kWalkSimtDVS);
+  if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+  kern<<<(unsigned)blocks, gdn2::kWalkSimtThreads, smem, s>>>(a);
+  return launch_status();
+}
+
+// ----------------------------------------------------------- dispatch ----
+template <template <int, int, typename, typename> class F, typename... Args>
+gdn2_status dispatch(const gdn2_desc* d, Args... args) {
+  const bool f32 = d->io == GDN2_IO_F32;
+#define GDN2_CASE(DK_, DV_)                                                        \
+  if (d->dk == DK_ && d->dv == DV_)                                                \
+    return f32 ? F<DK_, DV_, float, float>::run(d, args...)                        \
+               : F<DK_, DV_, bf16, bf16>::run(d, args...);
+  GDN2_CASE(64, 64)
+  GDN2_CASE(64, 128)
+  GDN2_CASE(128, 64)
+  GDN2_CASE(128, 128)
+#undef GDN2_CASE
+  return GDN2_ERR_SHAPE;
+}
+
+template <int DK, int DV, typename IO, typename FT>
+struct PrepOp {
+  template <typename... A>
+  static gdn2_status run(const gdn2_desc* d, A... a) { return launch_prep_t<DK, DV, IO, FT>(d, a...); }
+};
+template <int DK, int DV, typename IO, typename FT>
+struct WalkOp {
+  template <typename... A>
+  static gdn2_status run(const gdn2_desc* d, A... a) { return launch_walk_t<DK, DV, IO, FT>(d, a...); }
+};
+
+template <int DK, int DV, typename IO, typename FT>
+struct DecodeOp {
+  static gdn2_status run(const gdn2_desc* d, const void* q, const void* k, const void* v,
+                         const float* la, const float* b, const float* w, float scale,
+                         float* state, void* out, cudaStream_t s) {
+    gdn2::DecodeArgs<IO> a;
+    a.q = static_cast<const IO*>(q);
+    a.k = static_cast<const IO*>(k);
+    a.v = static_cast<const IO*>(v);
+    a.la = la;
+    a.b = b;
+    a.w = w;
+    a.state = state;
+    a.out = static_cast<IO*>(out);
+    a.H = d->H;
+    a.scale = scale;
+    constexpr int cols = DV < 32 ? DV : 32;
+    const long long blocks = (long long)d->B * d->H * (DV / cols);
+    if (blocks == 0) return GDN2_OK;
+    if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+    gdn2::decode_kernel<DK, DV, IO><<<(unsigned)blocks, gdn2::kDecodeThreads, 0, s>>>(a);
+    return launch_status();
+  }
+};
+
+bool device_ok() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+// Token arrays may be NULL only when there are no tokens (an empty tensor has
+// no storage); non-NULL pointers must always be 16-byte aligned.
+gdn2_status check_inputs(const void* q, const void* k, const void* v, const float* la,
+                         const float* b, const float* w, long long tokens = 1) {
+  if (tokens > 0 && (!q || !k || !v || !la || !b || !w)) return GDN2_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(la) || !aligned16(b) ||
+      !aligned16(w))
+    return GDN2_ERR_ALIGN;
+  return GDN2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn2_workspace_size(const gdn2_desc* desc) {
+  if (!desc) return 0;
+  Layout L;
+  const bool packed = desc->num_seqs > 0;
+  if (make_layout(desc, packed, &L) != GDN2_OK) return 0;
+  return L.l.total_bytes;
+}
+
+gdn2_status gdn2_workspace_layout(const gdn2_desc* desc, gdn2_ws_layout* layout) {
+  if (!desc || !layout) return GDN2_ERR_NULL;
+  Layout L;
+  const bool packed = desc->num_seqs > 0;
+  const gdn2_status st = make_layout(desc, packed, &L);
+  if (st != GDN2_OK) return st;
+  *layout = L.l;
+  return GDN2_OK;
+}
+
+gdn2_status gdn2_chunk_prep(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                            const float* log_alpha, const float* b, const float* w,
+                            const int32_t* cu_seqlens, cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, (long long)desc->B * desc->T)) != GDN2_OK) return st;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if ((st = launch_plan(desc, L, cu_seqlens, stream)) != GDN2_OK) return st;
+  return dispatch<PrepOp>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, stream);
+}
+
+gdn2_status gdn2_chunk_walk(const gdn2_desc* desc, float scale, const float* h0,
+                            const int32_t* cu_seqlens, void* out, float* hT, float* chunk_states,
+                            cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  if (!out && (long long)desc->B * desc->T > 0) return GDN2_ERR_NULL;
+  if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT)) ||
+      (chunk_states && !aligned16(chunk_states)))
+    return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  return dispatch<WalkOp>(desc, L, scale, h0, cu_seqlens, out, hT, chunk_states, stream);
+}
+
+gdn2_status gdn2_chunk_fwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* b, const float* w, float scale,
+                           const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                           cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  const long long tokens = (long long)desc->B * desc->T;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, tokens)) != GDN2_OK) return st;
+  if (!out && tokens > 0) return GDN2_ERR_NULL;
+  if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if ((st = launch_plan(desc, L, cu_seqlens, stream)) != GDN2_OK) return st;
+  if ((st = dispatch<PrepOp>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, stream)) != GDN2_OK)
+    return st;
+  return dispatch<WalkOp>(desc, L, scale, h0, cu_seqlens, out, hT, (float*)nullptr, stream);
+}
+
+gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* b, const float* w, float scale,
+                                float* state, void* out, cudaStream_t stream) {
+  if (!desc) return GDN2_ERR_NULL;
+  if (desc->io != GDN2_IO_F32 && desc->io != GDN2_IO_BF16) return GDN2_ERR_DTYPE;
+  if ((desc->dk != 64 && desc->dk != 128) || (desc->dv != 64 && desc->dv != 128)) return GDN2_ERR_SHAPE;
+  if (desc->B < 0 || desc->H < 1) return GDN2_ERR_SHAPE;
+  gdn2_status st = check_inputs(q, k, v, log_alpha, b, w, desc->B);
+  if (st != GDN2_OK) return st;
+  if (desc->B > 0 && (!state || !out)) return GDN2_ERR_NULL;
+  if (!aligned16(state) || !aligned16(out)) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  return dispatch<DecodeOp>(desc, q, k, v, log_alpha, b, w, scale, state, out, stream);
+}
+
+const char* gdn2_status_string(gdn2_status s) {
+  switch (s) {
+    case GDN2_OK: return "ok";
+    case GDN2_ERR_NULL: return "a required pointer is NULL";
+    case GDN2_ERR_SHAPE: return "unsupported or inconsistent sizes";
+    case GDN2_ERR_DTYPE: return "unknown io dtype";
+    case GDN2_ERR_ALIGN: return "a pointer is not 16-byte aligned (workspace: 256-byte)";
+    case GDN2_ERR_SEQLENS: return "cu_seqlens is malformed";
+    case GDN2_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDN2_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case GDN2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    case GDN2_ERR_UNSUPPORTED: return "the current device is not sm_100 (B200 class)";
+  }
+  return "unknown status";
+}
+
+int gdn2_version(void) { return 100; }
+
+}  // extern "C"

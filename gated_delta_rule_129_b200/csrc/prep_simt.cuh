@@ -1,0 +1,176 @@
+// prep_simt.cuh -- gate preparation + intra-chunk WY factors, fp32 on CUDA cores.
+//
+// One CTA per (chunk, head).  This is the fp32-I/O path (the 1e-4 accuracy
+// mode) and the portable baseline of the bf16 path; the tensor-core kernel in
+// prep_tc.cuh computes the same factors.
+//
+// Per chunk of n <= 64 tokens (page "Gated DeltaNet-2：将擦除与写入分开",
+// sections "在两个维度上独立控制" and "词元路径与并行训练"; the algebra below is the
+// recurrence unrolled over one chunk):
+//   g_i    = cumulative sum of log_alpha over the chunk          (fp32)
+//   e_i    = b_i * k_i,  z_i = w_i * v_i
+//   A_ij   = sum_c e_ic k_jc exp(g_ic - g_jc),   j < i
+//   P_ij   = sum_c q_ic k_jc exp(g_ic - g_jc),   j <= i
+//   (I + A) W  = E~ = e * exp(g)       forward substitution, fp32
+//   (I + A) U~ = Z                     same solve
+//   Kbar_i = k_i * exp(g_n - g_i)
+//   Q_eff  = q * exp(g) - P W,   O_part = P U~
+// Every decay factor has a non-positive exponent, so none can overflow.
+// Rows past the chunk's last token are written as zeros.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn2 {
+
+template <typename IO, typename FT>
+struct PrepArgs {
+  const IO* q;
+  const IO* k;
+  const IO* v;
+  const float* la;
+  const float* b;
+  const float* w;
+  SeqMap map;
+  int H;
+  FT* W;
+  FT* Ut;
+  FT* Kbar;
+  FT* Qeff;
+  FT* Opart;
+  float* gamma_last;
+};
+
+constexpr int kPrepSimtThreads = 256;
+
+template <int DK, int DV>
+constexpr size_t prep_simt_smem_bytes() {
+  return sizeof(float) * (size_t)(4 * kChunk * (DK + 1) + kChunk * (DV + 1) + 2 * kChunk * (kChunk + 1));
+}
+
+template <int DK, int DV, typename IO, typename FT>
+__global__ void __launch_bounds__(kPrepSimtThreads)
+prep_simt_kernel(const PrepArgs<IO, FT> a) {
+  static_assert(DK + DV <= kPrepSimtThreads, "one thread per solve column");
+  constexpr int LK = DK + 1, LV = DV + 1, LA = kChunk + 1;
+  const int c = blockIdx.x, h = blockIdx.y, H = a.H;
+  if (c >= a.map.chunk_off[a.map.N]) return;
+  const ChunkPos pos = chunk_pos(a.map, c);
+  const int len = pos.len;
+
+  extern __shared__ float smem[];
+  float* sg = smem;                 // [64][LK]  cumulative log-decay
+  float* sk = sg + kChunk * LK;     // [64][LK]  k
+  float* se = sk + kChunk * LK;     // [64][LK]  e, then E~, then W
+  float* sq = se + kChunk * LK;     // [64][LK]  q, then Q~
+  float* sz = sq + kChunk * LK;     // [64][LV]  z, then U~
+  float* sA = sz + kChunk * LV;     // [64][LA]  A (strictly lower)
+  float* sP = sA + kChunk * LA;     // [64][LA]  P (lower, diagonal included)
+  const int tid = threadIdx.x;
+
+  for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
+    const int i = idx / DK, cc = idx % DK;
+    float kv = 0.f, bv = 0.f, qv = 0.f, lv = 0.f;
+    if (i < len) {
+      const size_t off = ((size_t)(pos.t0 + i) * H + h) * DK + cc;
+      kv = to_f32(a.k[off]);
+      qv = to_f32(a.q[off]);
+      bv = a.b[off];
+      lv = a.la[off];
+    }
+    sk[i * LK + cc] = kv;
+    se[i * LK + cc] = bv * kv;
+    sq[i * LK + cc] = qv;
+    sg[i * LK + cc] = lv;
+  }
+  for (int idx = tid; idx < kChunk * DV; idx += kPrepSimtThreads) {
+    const int i = idx / DV, cc = idx % DV;
+    float z = 0.f;
+    if (i < len) {
+      const size_t off = ((size_t)(pos.t0 + i) * H + h) * DV + cc;
+      z = a.w[off] * to_f32(a.v[off]);
+    }
+    sz[i * LV + cc] = z;
+  }
+  for (int idx = tid; idx < kChunk * LA; idx += kPrepSimtThreads) {
+    sA[idx] = 0.f;
+    sP[idx] = 0.f;
+  }
+  __syncthreads();
+  // In-chunk cumulative sum, one thread per key channel.  Padded rows carry
+  // log_alpha = 0, so g stays at g_{n-1} past the last token.
+  if (tid < DK) {
+    float acc = 0.f;
+    for (int i = 0; i < kChunk; ++i) {
+      acc += sg[i * LK + tid];
+      sg[i * LK + tid] = acc;
+    }
+  }
+  __syncthreads();
+  // A and P: one warp per (i, j) pair, lanes over key channels.
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int i = warp; i < len; i += kPrepSimtThreads / 32) {
+    for (int j = 0; j <= i; ++j) {
+      float acc_a = 0.f, acc_p = 0.f;
+#pragma unroll
+      for (int cc = lane; cc < DK; cc += 32) {
+        const float kd = sk[j * LK + cc] * expf(sg[i * LK + cc] - sg[j * LK + cc]);
+        acc_a = fmaf(se[i * LK + cc], kd, acc_a);
+        acc_p = fmaf(sq[i * LK + cc], kd, acc_p);
+      }
+      acc_a = warp_sum(acc_a);
+      acc_p = warp_sum(acc_p);
+      if (lane == 0) {
+        if (j < i) sA[i * LA + j] = acc_a;
+        sP[i * LA + j] = acc_p;
+      }
+    }
+  }
+  __syncthreads();
+  // Kbar and gamma_last go straight out; E~ and Q~ are formed in place.
+  const size_t tile_k = ((size_t)c * H + h) * kChunk * DK;
+  const size_t tile_v = ((size_t)c * H + h) * kChunk * DV;
+  for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
+    const int i = idx / DK, cc = idx % DK;
+    const float gi = sg[i * LK + cc];
+    const float kb = i < len ? sk[i * LK + cc] * expf(sg[(kChunk - 1) * LK + cc] - gi) : 0.f;
+    a.Kbar[tile_k + idx] = from_f32<FT>(kb);
+    const float gam = expf(gi);
+    se[i * LK + cc] *= gam;
+    sq[i * LK + cc] *= gam;
+  }
+  if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
+  __syncthreads();
+  // Forward substitution, row by row: W_i = E~_i - sum_{j<i} A_ij W_j, and the
+  // same for U~ with Z.  One thread per column of [W | U~].
+  for (int i = 1; i < len; ++i) {
+    if (tid < DK) {
+      float acc = se[i * LK + tid];
+      for (int j = 0; j < i; ++j) acc = fmaf(-sA[i * LA + j], se[j * LK + tid], acc);
+      se[i * LK + tid] = acc;
+    } else if (tid < DK + DV) {
+      const int col = tid - DK;
+      float acc = sz[i * LV + col];
+      for (int j = 0; j < i; ++j) acc = fmaf(-sA[i * LA + j], sz[j * LV + col], acc);
+      sz[i * LV + col] = acc;
+    }
+    __syncthreads();
+  }
+  // Q_eff = Q~ - P W and O_part = P U~ (P is lower triangular with diagonal).
+  for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
+    const int i = idx / DK, cc = idx % DK;
+    float acc = sq[i * LK + cc];
+    for (int j = 0; j <= i && j < len; ++j) acc = fmaf(-sP[i * LA + j], se[j * LK + cc], acc);
+    a.Qeff[tile_k + idx] = from_f32<FT>(acc);
+    a.W[tile_k + idx] = from_f32<FT>(se[i * LK + cc]);
+  }
+  for (int idx = tid; idx < kChunk * DV; idx += kPrepSimtThreads) {
+    const int i = idx / DV, cc = idx % DV;
+    float acc = 0.f;
+    for (int j = 0; j <= i && j < len; ++j) acc = fmaf(sP[i * LA + j], sz[j * LV + cc], acc);
+    a.Opart[tile_v + idx] = from_f32<FT>(acc);
+    a.Ut[tile_v + idx] = from_f32<FT>(sz[i * LV + cc]);
+  }
+}
+
+}  // namespace gdn2

@@ -1,0 +1,184 @@
+/*
+ * gdn2.h -- C ABI of the B200 (sm_100a) Gated DeltaNet-2 forward operator.
+ *
+ * The operator is the Gated Delta Rule-2 recurrence.  Per (sequence, head),
+ * for t = 1..T (page "Gated DeltaNet-2：将擦除与写入分开", iplexlaw blog,
+ * section "在两个维度上独立控制"):
+ *
+ *     e_t = b_t * k_t                   erase vector, key channels
+ *     z_t = w_t * v_t                   write vector, value channels
+ *     Sbar = diag(alpha_t) S_{t-1}      channel-wise decay on the key axis
+ *     r_t = Sbar^T e_t                  read along the erase vector
+ *     S_t = Sbar + k_t (z_t - r_t)^T
+ *     o_t = scale * S_t^T q_t           the query reads the updated state
+ *
+ * with alpha_t = exp(log_alpha_t).  The state S is dk x dv (row = key channel,
+ * column = value channel).  gdn2_chunk_fwd evaluates the recurrence in the
+ * 64-token chunkwise WY form (same page, section "词元路径与并行训练": 64-token
+ * chunks, cumulative channel-wise decay folded into the erase factors, an
+ * in-chunk triangular solve plus dense products, fp32 for the decay, the state
+ * and the solve).  Results equal the token recurrence up to rounding.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.   Every tensor argument is a DEVICE pointer owned by the caller,
+ *             16-byte aligned and densely packed in the layout given below.
+ *             The library allocates no memory and never synchronises a
+ *             stream; all work is enqueued on `stream` (0 = legacy default).
+ * Layouts.    Token-major.  q, k, log_alpha, b : [B, T, H, dk];
+ *             v, w, out : [B, T, H, dv]; states h0, hT : [N, H, dk, dv] fp32
+ *             with N = B (dense) or N = num_seqs (packed).
+ * Precision.  q, k, v and out are fp32 (GDN2_IO_F32) or bf16 (GDN2_IO_BF16);
+ *             log_alpha, b, w, h0, hT and state are always fp32.  The decay,
+ *             the state and the triangular solve are computed in fp32.
+ * Packing.    With cu_seqlens != NULL the batch is one packed row (B must be
+ *             1, T = total tokens) holding num_seqs sequences; sequence n
+ *             covers tokens [cu_seqlens[n], cu_seqlens[n+1]).  cu_seqlens is
+ *             an int32 device array of num_seqs + 1 entries, starting at 0,
+ *             non-decreasing and ending at T.  Chunks start at each sequence's
+ *             first token, so a sequence's result does not depend on what it
+ *             is packed with (bitwise).
+ * Shapes.     dk and dv are each 64 or 128; H >= 1; B >= 1; T >= 0.
+ * Errors.     Returned as gdn2_status, never thrown; the library never exits,
+ *             aborts or traps.  A returned GDN2_OK means the host-side checks
+ *             passed and the launches were accepted.  cu_seqlens lives on the
+ *             device, so its contents are checked on the device: a bad array
+ *             leaves the outputs unspecified and stores GDN2_ERR_SEQLENS in the
+ *             workspace status word (see gdn2_workspace_layout).
+ */
+#ifndef GDN2_H_
+#define GDN2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn2_status {
+  GDN2_OK = 0,
+  GDN2_ERR_NULL = 1,          /* a required pointer is NULL                       */
+  GDN2_ERR_SHAPE = 2,         /* unsupported or inconsistent sizes                */
+  GDN2_ERR_DTYPE = 3,         /* unknown gdn2_io_dtype                            */
+  GDN2_ERR_ALIGN = 4,         /* a pointer is not 16-byte aligned                 */
+  GDN2_ERR_SEQLENS = 5,       /* cu_seqlens is malformed (device status word)     */
+  GDN2_ERR_WORKSPACE = 6,     /* workspace missing or smaller than required       */
+  GDN2_ERR_CUDA = 7,          /* a CUDA runtime call or launch failed             */
+  GDN2_ERR_DEVICE_TIMEOUT = 8,/* a bounded device-side wait gave up               */
+  GDN2_ERR_UNSUPPORTED = 9    /* the current device is not sm_100 (B200 class)    */
+} gdn2_status;
+
+typedef enum gdn2_io_dtype {
+  GDN2_IO_F32 = 0,   /* q, k, v, out in fp32 (correctness mode)                  */
+  GDN2_IO_BF16 = 1   /* q, k, v, out in bf16 (the fast path)                    */
+} gdn2_io_dtype;
+
+/* Problem description.  `workspace` is a caller-owned device buffer of at
+ * least gdn2_workspace_size(desc) bytes, 256-byte aligned; its contents on
+ * entry do not matter and are overwritten. */
+typedef struct gdn2_desc {
+  int B;                   /* batch size (1 when packed)                         */
+  int T;                   /* tokens per sequence, or total tokens when packed   */
+  int H;                   /* heads                                              */
+  int dk;                  /* key dimension, 64 or 128                           */
+  int dv;                  /* value dimension, 64 or 128                         */
+  int num_seqs;            /* packed: sequences in the row (>= 1, with         */
+                           /* cu_seqlens); dense: must be 0                     */
+  gdn2_io_dtype io;        /* dtype of q, k, v, out                              */
+  void* workspace;         /* device scratch, caller-owned                       */
+  size_t workspace_bytes;  /* its size in bytes                                  */
+} gdn2_desc;
+
+/* Where the per-chunk WY factors live inside the workspace, so that callers
+ * (and tests) can inspect what gdn2_chunk_prep produced.  All offsets are in
+ * bytes from `workspace`.  Factor tensors are [max_chunks, H, 64, d] in the
+ * element size `factor_elem_bytes` (4 = fp32 for GDN2_IO_F32, 2 = bf16 for
+ * GDN2_IO_BF16); rows past a chunk's last token are zero.  Chunk c of
+ * sequence n has global index chunk_offsets[n] + c (int32 array of N + 1
+ * entries); gamma_last is [max_chunks, H, dk] fp32. */
+typedef struct gdn2_ws_layout {
+  size_t total_bytes;
+  int max_chunks;            /* upper bound on chunks: T_total/64 + N            */
+  int factor_elem_bytes;
+  size_t off_W;              /* W     = T E~           [., H, 64, dk]            */
+  size_t off_Ut;             /* U~    = T Z            [., H, 64, dv]            */
+  size_t off_Kbar;           /* Kbar  = k exp(g_n - g) [., H, 64, dk]            */
+  size_t off_Qeff;           /* Q_eff = Q~ - P W       [., H, 64, dk]            */
+  size_t off_Opart;          /* O_part= P U~           [., H, 64, dv]            */
+  size_t off_gamma_last;     /* exp(g_n)               [., H, dk] fp32           */
+  size_t off_chunk_offsets;  /* int32 [N + 1]                                    */
+  size_t off_status;         /* int32 status word (a gdn2_status value)          */
+} gdn2_ws_layout;
+
+/* Bytes of workspace gdn2_chunk_fwd needs for `desc` (0 if desc is invalid).
+ * num_seqs > 0 describes a packed call (cu_seqlens given), 0 a dense one. */
+GDN2_API size_t gdn2_workspace_size(const gdn2_desc* desc);
+
+/* Fill *layout for `desc`.  Host-only, no CUDA call. */
+GDN2_API gdn2_status gdn2_workspace_layout(const gdn2_desc* desc, gdn2_ws_layout* layout);
+
+/* Chunkwise forward pass: O and the final state.
+ *   q, k       : [B, T, H, dk]  io dtype
+ *   v          : [B, T, H, dv]  io dtype
+ *   log_alpha  : [B, T, H, dk]  fp32, log of the channel-wise decay (<= 0)
+ *   b          : [B, T, H, dk]  fp32 erase gate (key channels)
+ *   w          : [B, T, H, dv]  fp32 write gate (value channels)
+ *   scale      : output scale (the usual choice dk^-1/2 is the caller's)
+ *   h0         : [N, H, dk, dv] fp32 initial state, or NULL for zeros
+ *   cu_seqlens : int32 [num_seqs + 1] (device) or NULL for B dense sequences
+ *   out        : [B, T, H, dv]  io dtype
+ *   hT         : [N, H, dk, dv] fp32 final state, or NULL to skip; may alias h0
+ * Asynchronous on `stream`.  Runs gdn2_chunk_prep then gdn2_chunk_walk. */
+GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* b, const float* w, float scale,
+                           const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                           cudaStream_t stream);
+
+/* Stage 1 of gdn2_chunk_fwd: gate preparation and the intra-chunk WY factors
+ * of every (chunk, head), written to the workspace (layout above).  Depends
+ * only on the inputs of each chunk, not on any state. */
+GDN2_API gdn2_status gdn2_chunk_prep(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                            const float* log_alpha, const float* b, const float* w,
+                            const int32_t* cu_seqlens, cudaStream_t stream);
+
+/* Stage 2 of gdn2_chunk_fwd: the inter-chunk state walk and the outputs,
+ * reading the factors gdn2_chunk_prep left in the workspace.  If
+ * chunk_states is not NULL it receives the state at the START of every chunk,
+ * [max_chunks, H, dk, dv] fp32 indexed by global chunk index (diagnostics). */
+GDN2_API gdn2_status gdn2_chunk_walk(const gdn2_desc* desc, float scale, const float* h0,
+                            const int32_t* cu_seqlens, void* out, float* hT,
+                            float* chunk_states, cudaStream_t stream);
+
+/* One decode token for a batch of states, updated in place.
+ * desc: B = batch, H, dk, dv, io (T, num_seqs and the workspace are ignored).
+ *   q, k, log_alpha, b : [B, H, dk]   (q, k in io dtype; the rest fp32)
+ *   v, w               : [B, H, dv]   (v in io dtype; w fp32)
+ *   state              : [B, H, dk, dv] fp32, read and overwritten
+ *   out                : [B, H, dv]   io dtype
+ * Same recurrence as gdn2_chunk_fwd with T = 1 (constant-memory decoding,
+ * page "Gated DeltaNet-2: Decoupling Erase and Write in Linear Attention",
+ * cere-bro blog, section "TL;DR"). */
+GDN2_API gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* b, const float* w, float scale,
+                                float* state, void* out, cudaStream_t stream);
+
+/* Static description of a status code. */
+GDN2_API const char* gdn2_status_string(gdn2_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDN2_API int gdn2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H_ */

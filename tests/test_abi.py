@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+that include/gdn2.h declares, and rejects bad arguments with the documented
+status codes before it makes any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_129_b200 as gdn2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn2.h")
+
+OK, NULL, SHAPE, DTYPE, ALIGN, SEQLENS, WORKSPACE, CUDA, TIMEOUT, UNSUPPORTED = range(10)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN2_API\s+[\w\s\*]*?\b(gdn2_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_129_b200 import build
+    build.build()
+    return gdn2.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 8
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) <= set(gdn2.EXPORTED) | set(syms)
+
+
+def test_status_strings(lib):
+    for code in range(10):
+        assert gdn2.status_string(code)
+    assert gdn2.status_string(0) == "ok"
+    assert lib.gdn2_version() >= 100
+
+
+def test_workspace_layout_sizes(lib):
+    lay = gdn2.workspace_layout(1, 16384, 16, 128, 128, gdn2.GDN2_IO_BF16)
+    assert lay["max_chunks"] == 256 and lay["factor_elem_bytes"] == 2
+    tile = 256 * 16 * 64 * 128 * 2
+    assert lay["off_Ut"] - lay["off_W"] >= tile
+    offs = sorted(v for k, v in lay.items() if k.startswith("off_"))
+    assert all(o % 256 == 0 for o in offs)
+    assert lay["total_bytes"] >= offs[-1] + 4
+    # packed: the bound is T_total/64 + N chunks
+    lay2 = gdn2.workspace_layout(1, 1000, 2, 64, 128, gdn2.GDN2_IO_F32, num_seqs=7)
+    assert lay2["max_chunks"] == 1000 // 64 + 7 and lay2["factor_elem_bytes"] == 4
+    assert gdn2.workspace_size(1, 1000, 2, 64, 128, gdn2.GDN2_IO_F32, num_seqs=7) == lay2["total_bytes"]
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=96), SHAPE), (dict(dv=32), SHAPE), (dict(H=0), SHAPE), (dict(T=-1), SHAPE),
+    (dict(io=7), DTYPE), (dict(B=2, num_seqs=3), SHAPE),
+])
+def test_layout_rejects_bad_desc(lib, kw, code):
+    args = dict(B=1, T=128, H=2, dk=64, dv=64, io=0, num_seqs=0)
+    args.update(kw)
+    d = gdn2.make_desc(**args)
+    lay = gdn2.WsLayout()
+    assert lib.gdn2_workspace_layout(ctypes.byref(d), ctypes.byref(lay)) == code
+    assert lib.gdn2_workspace_size(ctypes.byref(d)) == 0
+
+
+def _fwd(lib, d, ptrs, out=0x20000, h0=None, cu=None, hT=None):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn2_chunk_fwd(ctypes.byref(d), *(P(p) for p in ptrs), 0.125, P(h0), P(cu), P(out),
+                              P(hT), None)
+
+
+def test_chunk_fwd_host_checks(lib):
+    """Fake, never-dereferenced device addresses: every call below must return
+    before any CUDA call (or with UNSUPPORTED where no B200 is present)."""
+    size = gdn2.workspace_size(1, 128, 2, 64, 64, 0)
+    good = [0x10000 + 0x100 * i for i in range(6)]
+    d = gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, 0x100000, size)
+    assert lib.gdn2_chunk_fwd(None, *(ctypes.c_void_p(p) for p in good), 0.1, None, None,
+                              ctypes.c_void_p(0x20000), None, None) == NULL
+    bad_null = list(good)
+    bad_null[3] = None
+    assert _fwd(lib, d, bad_null) == NULL
+    assert _fwd(lib, d, good, out=None) == NULL
+    bad_align = list(good)
+    bad_align[1] += 4
+    assert _fwd(lib, d, bad_align) == ALIGN
+    assert _fwd(lib, d, good, h0=0x30004) == ALIGN
+    small = gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, 0x100000, size - 1)
+    assert _fwd(lib, small, good) == WORKSPACE
+    nows = gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, None, size)
+    assert _fwd(lib, nows, good) == WORKSPACE
+    misws = gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, 0x100010, size)
+    assert _fwd(lib, misws, good) == ALIGN
+    # packed call without cu_seqlens / dense call with num_seqs set
+    pk = gdn2.make_desc(1, 128, 2, 64, 64, 0, 3, 0x100000, 1 << 30)
+    assert _fwd(lib, pk, good) == SHAPE
+    assert _fwd(lib, d, good, cu=0x40000) == SHAPE
+    # with valid arguments the only remaining check is the device itself
+    rc = _fwd(lib, d, good)
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:  # pragma: no cover
+        has_gpu = False
+    if not has_gpu:
+        assert rc == UNSUPPORTED
+
+
+def test_recurrent_step_host_checks(lib):
+    good = [ctypes.c_void_p(0x10000 + 0x100 * i) for i in range(6)]
+    d = gdn2.make_desc(4, 1, 2, 128, 128, 1)
+    st, out = ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000)
+    assert lib.gdn2_recurrent_step(ctypes.byref(d), *good, 0.1, None, out, None) == NULL
+    assert lib.gdn2_recurrent_step(ctypes.byref(d), *good, 0.1, ctypes.c_void_p(0x50008), out, None) == ALIGN
+    bad = gdn2.make_desc(4, 1, 2, 128, 80, 1)
+    assert lib.gdn2_recurrent_step(ctypes.byref(bad), *good, 0.1, st, out, None) == SHAPE
+    bad = gdn2.make_desc(4, 1, 2, 128, 128, 5)
+    assert lib.gdn2_recurrent_step(ctypes.byref(bad), *good, 0.1, st, out, None) == DTYPE
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    """The product path has no fallback: a missing library is an error."""
+    monkeypatch.setattr(gdn2, "_lib", None)
+    monkeypatch.setattr(gdn2, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        gdn2.load_library()

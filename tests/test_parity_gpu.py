@@ -1,0 +1,238 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (rel-L2 over the whole tensor, fp64): 1e-4 with fp32 I/O and
+2e-2 with bf16 I/O, for O and for hT; bitwise equality between a packed
+(varlen) call and per-sequence calls."""
+import numpy as np
+import pytest
+
+from tests.helpers import TOL, compare, rel_l2, run_gpu, to_device
+from workloads import config, decode_inputs, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_device):
+    import gated_delta_rule_129_b200 as gdn2
+    gdn2.load_library()
+
+
+# --- end-to-end, small sizes spanning several chunks and a ragged tail ----------
+
+def test_tiny_fp32_workload():
+    x = config(0)
+    o, hT = run_gpu(x)
+    ro, rh = compare(x, o, hT)
+    assert ro <= TOL["f32"] and rh <= TOL["f32"], (ro, rh)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_shapes(io, dk, dv, T):
+    x = make_inputs(2, T, 3, dk, dv, io=io, seed=100 + T + dk + dv, h0_std=0.05)
+    o, hT = run_gpu(x)
+    ro, rh = compare(x, o, hT)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(hT))
+    assert ro <= TOL[io] and rh <= TOL[io], (ro, rh)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_strong_decay(io):
+    x = make_inputs(1, 640, 4, 128, 128, io=io, seed=7, decay="strong", h0_std=0.05)
+    o, hT = run_gpu(x)
+    ro, rh = compare(x, o, hT)
+    assert ro <= TOL[io] and rh <= TOL[io], (ro, rh)
+
+
+# --- the stages, one at a time ------------------------------------------------
+
+def _factors(ws, lay, H, dk, dv, io):
+    import torch
+    dt = torch.float32 if io == "f32" else torch.bfloat16
+    mc = lay["max_chunks"]
+
+    def view(off, d):
+        n = mc * H * 64 * d
+        eb = lay["factor_elem_bytes"]
+        return ws[off: off + n * eb].view(dt).view(mc, H, 64, d).float().cpu().numpy()
+    f = dict(W=view(lay["off_W"], dk), Ut=view(lay["off_Ut"], dv), Kbar=view(lay["off_Kbar"], dk),
+             Q_eff=view(lay["off_Qeff"], dk), O_part=view(lay["off_Opart"], dv))
+    g = ws[lay["off_gamma_last"]: lay["off_gamma_last"] + mc * H * dk * 4].view(torch.float32)
+    f["gamma_last"] = g.view(mc, H, dk).cpu().numpy()
+    return f
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_prep_factors_match_oracle(io):
+    """Gate prep + intra-chunk WY (W, U~, Kbar, Q_eff, O_part, exp(g_n)) per
+    chunk against the fp64 chunkwise restatement."""
+    import gated_delta_rule_129_b200 as gdn2
+    from oracle.chunk_wy import chunk_wy
+    lens = [130, 64, 5]
+    H, dk, dv = 2, 128, 64
+    x = make_inputs(1, sum(lens), H, dk, dv, io=io, seed=31, decay="strong", lengths=lens)
+    d = to_device(x)
+    ws = gdn2.chunk_prep(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["cu_seqlens"])
+    import torch
+    torch.cuda.synchronize()
+    lay = gdn2.workspace_layout(1, sum(lens), H, dk, dv, 0 if io == "f32" else 1, num_seqs=len(lens))
+    got = _factors(ws, lay, H, dk, dv, io)
+    _, _, inter = chunk_wy(x.q, x.k, x.v, x.log_alpha, x.b, x.w, x.scale, cu_seqlens=x.cu_seqlens,
+                           return_intermediates=True)
+    assert len(inter) == 5
+    for c, r in enumerate(inter):
+        n = r["len"]
+        for key in ("W", "Ut", "Kbar", "Q_eff", "O_part"):
+            ref = r[key]
+            g = got[key][c]
+            assert rel_l2(g[:, :n], ref) <= TOL[io], (c, key, rel_l2(g[:, :n], ref))
+            assert np.all(g[:, n:] == 0), (c, key)   # padded rows are exact zeros
+        assert rel_l2(got["gamma_last"][c], r["gamma_last"]) <= 1e-6
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_walk_states_match_oracle(io):
+    """The state walk: the state at the start of every chunk, and hT."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    from oracle.chunk_wy import chunk_wy
+    x = make_inputs(2, 200, 2, 64, 128, io=io, seed=32, h0_std=0.1)
+    d = to_device(x)
+    ws = gdn2.chunk_prep(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"])
+    lay = gdn2.workspace_layout(2, 200, 2, 64, 128, 0 if io == "f32" else 1)
+    cs = torch.zeros((lay["max_chunks"], 2, 64, 128), dtype=torch.float32, device="cuda")
+    io_dt = torch.float32 if io == "f32" else torch.bfloat16
+    o, hT = gdn2.chunk_walk(ws, (2, 200, 2, 64, 128), io_dt, x.scale, h0=d["h0"], chunk_states=cs)
+    _, hT_ref, inter = chunk_wy(x.q, x.k, x.v, x.log_alpha, x.b, x.w, x.scale, h0=x.h0,
+                                return_intermediates=True)
+    cs = cs.cpu().numpy()
+    assert len(inter) == 8
+    for c, r in enumerate(inter):
+        assert rel_l2(cs[c], r["S0"]) <= TOL[io], c
+    assert rel_l2(hT.cpu().numpy(), hT_ref) <= TOL[io]
+
+
+# --- varlen, state chaining, in place ------------------------------------------------
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_varlen_bitwise_equals_per_sequence(io):
+    import gated_delta_rule_129_b200 as gdn2
+    lens = [65, 0, 1, 64, 130, 63, 200]
+    x = make_inputs(1, sum(lens), 3, 128, 128, io=io, seed=33, h0_std=0.05, lengths=lens)
+    o, hT = run_gpu(x)
+    d = to_device(x)
+    cu = x.cu_seqlens
+    for n, L in enumerate(lens):
+        s = slice(int(cu[n]), int(cu[n + 1]))
+        sub = lambda t: t[:, s].contiguous()  # noqa: E731
+        on, hn = gdn2.chunk_fwd(sub(d["q"]), sub(d["k"]), sub(d["v"]), sub(d["log_alpha"]),
+                                sub(d["b"]), sub(d["w"]), x.scale, h0=d["h0"][n:n + 1].contiguous())
+        assert np.array_equal(on.float().cpu().numpy(), o[:, s]), n
+        assert np.array_equal(hn[0].cpu().numpy(), hT[n]), n
+    ro, rh = compare(x, o, hT)
+    assert ro <= TOL[io] and rh <= TOL[io], (ro, rh)
+
+
+def test_state_chaining_equals_one_call():
+    """Checkpoint/resume through h0/hT: [0,T1) then [T1,T) from hT."""
+    import gated_delta_rule_129_b200 as gdn2
+    x = make_inputs(1, 300, 2, 128, 128, io="f32", seed=34, h0_std=0.05)
+    o, hT = run_gpu(x)
+    d = to_device(x)
+    a = lambda t, s: t[:, s].contiguous()  # noqa: E731
+    s1, s2 = slice(0, 100), slice(100, 300)
+    o1, h1 = gdn2.chunk_fwd(*(a(d[k], s1) for k in ("q", "k", "v", "log_alpha", "b", "w")), x.scale, h0=d["h0"])
+    o2, h2 = gdn2.chunk_fwd(*(a(d[k], s2) for k in ("q", "k", "v", "log_alpha", "b", "w")), x.scale, h0=h1)
+    oc = np.concatenate([o1.cpu().numpy(), o2.cpu().numpy()], axis=1)
+    assert rel_l2(oc, o) <= 1e-5 and rel_l2(h2.cpu().numpy(), hT) <= 1e-5
+
+
+def test_final_state_may_alias_initial_state():
+    import gated_delta_rule_129_b200 as gdn2
+    x = make_inputs(2, 150, 2, 128, 128, io="bf16", seed=35, h0_std=0.05)
+    o_ref, hT_ref = run_gpu(x)
+    d = to_device(x)
+    state = d["h0"].clone()
+    o, h = gdn2.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], x.scale,
+                          h0=state, hT=state)
+    assert np.array_equal(state.cpu().numpy(), hT_ref)
+    assert np.array_equal(o.float().cpu().numpy(), o_ref)
+
+
+def test_empty_inputs():
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    x = make_inputs(2, 0, 2, 64, 64, io="bf16", seed=36, h0_std=0.1)
+    o, hT = run_gpu(x)
+    assert o.shape == (2, 0, 2, 64)
+    assert np.array_equal(hT, x.h0)
+    # packed row where every sequence is empty
+    x = make_inputs(1, 0, 2, 64, 64, io="bf16", seed=37, h0_std=0.1, lengths=[0, 0, 0])
+    o, hT = run_gpu(x)
+    assert np.array_equal(hT, x.h0)
+    # no h0 and no hT requested
+    d = to_device(make_inputs(1, 70, 2, 64, 64, io="bf16", seed=38))
+    o, hT = gdn2.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], 0.125,
+                           output_final_state=False)
+    torch.cuda.synchronize()
+    assert hT is None and torch.isfinite(o.float()).all()
+
+
+def test_malformed_seqlens_sets_status_word():
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    x = make_inputs(1, 200, 2, 64, 64, io="bf16", seed=39, lengths=[100, 100])
+    d = to_device(x)
+    lay = gdn2.workspace_layout(1, 200, 2, 64, 64, 1, num_seqs=2)
+    for bad in ([0, 120, 100], [5, 100, 200], [0, 100, 199]):
+        cu = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        ws = torch.zeros(lay["total_bytes"], dtype=torch.uint8, device="cuda")
+        gdn2.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], 0.125,
+                       cu_seqlens=cu, workspace=ws)
+        st = ws[lay["off_status"]: lay["off_status"] + 4].view(torch.int32).item()
+        assert st == 5, bad
+    cu = torch.tensor([0, 100, 200], dtype=torch.int32, device="cuda")
+    ws = torch.full((lay["total_bytes"],), 0xFF, dtype=torch.uint8, device="cuda")
+    gdn2.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], 0.125, cu_seqlens=cu, workspace=ws)
+    assert ws[lay["off_status"]: lay["off_status"] + 4].view(torch.int32).item() == 0
+
+
+# --- decode step -----------------------------------------------------------------
+
+@pytest.mark.parametrize("io,dk,dv,B", [("bf16", 128, 128, 256), ("f32", 64, 128, 5), ("bf16", 128, 64, 3)])
+def test_recurrent_step_matches_oracle(io, dk, dv, B):
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    import oracle
+    di = decode_inputs(B=B, H=16 if B == 256 else 2, dk=dk, dv=dv, io=io, seed=41 + B)
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    t = lambda a, ty: torch.from_numpy(a).to("cuda", ty)  # noqa: E731
+    state = t(di.state, torch.float32)
+    out = gdn2.recurrent_step(t(di.q, dt), t(di.k, dt), t(di.v, dt), t(di.log_alpha, torch.float32),
+                              t(di.b, torch.float32), t(di.w, torch.float32), di.scale, state)
+    o_ref, s_ref = oracle.recurrent_step(di.q, di.k, di.v, di.log_alpha, di.b, di.w, di.scale, di.state)
+    assert rel_l2(out.float().cpu().numpy(), o_ref) <= TOL[io]
+    assert rel_l2(state.cpu().numpy(), s_ref) <= 1e-5
+
+
+def test_decode_steps_equal_chunk_forward():
+    """Decoding token by token from h0 reproduces the chunked forward."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    x = make_inputs(2, 70, 2, 128, 128, io="f32", seed=42, h0_std=0.05)
+    o, hT = run_gpu(x)
+    d = to_device(x)
+    state = d["h0"].clone()
+    outs = []
+    for t in range(70):
+        s = lambda k: d[k][:, t].contiguous()  # noqa: E731
+        outs.append(gdn2.recurrent_step(s("q"), s("k"), s("v"), s("log_alpha"), s("b"), s("w"), x.scale, state))
+    od = torch.stack(outs, dim=1).cpu().numpy()
+    assert rel_l2(od, o) <= 1e-5 and rel_l2(state.cpu().numpy(), hT) <= 1e-5
