@@ -89,7 +89,8 @@ def test_prep_factors_match_oracle(io):
             g = got[key][c]
             assert rel_l2(g[:, :n], ref) <= TOL[io], (c, key, rel_l2(g[:, :n], ref))
             assert np.all(g[:, n:] == 0), (c, key)   # padded rows are exact zeros
-        assert rel_l2(got["gamma_last"][c], r["gamma_last"]) <= 1e-6
+        # fp32 cumulative sum of up to 64 log-decays: relative error ~1e-6
+        assert rel_l2(got["gamma_last"][c], r["gamma_last"]) <= 1e-4
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
