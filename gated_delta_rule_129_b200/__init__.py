@@ -53,10 +53,12 @@ class Desc(ctypes.Structure):
 
 class WsLayout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t), ("max_chunks", ctypes.c_int),
-                ("factor_elem_bytes", ctypes.c_int), ("off_W", ctypes.c_size_t),
+                ("factor_elem_bytes", ctypes.c_int), ("factor_set", ctypes.c_int),
+                ("reserved", ctypes.c_int), ("off_W", ctypes.c_size_t),
                 ("off_Ut", ctypes.c_size_t), ("off_Kbar", ctypes.c_size_t),
                 ("off_Qeff", ctypes.c_size_t), ("off_Opart", ctypes.c_size_t),
-                ("off_gamma_last", ctypes.c_size_t), ("off_chunk_offsets", ctypes.c_size_t),
+                ("off_gamma_last", ctypes.c_size_t), ("off_Mp", ctypes.c_size_t),
+                ("off_Nc", ctypes.c_size_t), ("off_chunk_offsets", ctypes.c_size_t),
                 ("off_status", ctypes.c_size_t)]
 
     def as_dict(self):

@@ -8,14 +8,18 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "decode.cuh"
 #include "plan.cuh"
 #include "prep_simt.cuh"
+#include "tmap.cuh"
 #include "walk_simt.cuh"
+#include "walk_tc.cuh"
 
 namespace {
 
@@ -48,6 +52,11 @@ struct Layout {
   int N;
 };
 
+// The bf16 path with dk = 128 stores each chunk's affine state map and walks
+// with one tensor-core product per chunk; every other case stores the WY
+// factors and walks on CUDA cores.
+bool uses_affine(const gdn2_desc* d) { return d->io == GDN2_IO_BF16 && d->dk == 128; }
+
 gdn2_status make_layout(const gdn2_desc* d, bool packed, Layout* out) {
   gdn2_status st = check_dims(d, packed);
   if (st != GDN2_OK) return st;
@@ -60,15 +69,20 @@ gdn2_status make_layout(const gdn2_desc* d, bool packed, Layout* out) {
   std::memset(&L, 0, sizeof(L));
   L.max_chunks = (int)max_chunks;
   L.factor_elem_bytes = d->io == GDN2_IO_F32 ? 4 : 2;
+  L.factor_set = uses_affine(d) ? 1 : 0;
+  const bool wy = L.factor_set == 0;
   const size_t tiles = (size_t)max_chunks * d->H * kChunk;
+  const size_t mats = (size_t)max_chunks * d->H * d->dk;
   const size_t eb = (size_t)L.factor_elem_bytes;
   size_t off = 0;
-  L.off_W = off;          off = align_up(off + tiles * d->dk * eb);
-  L.off_Ut = off;         off = align_up(off + tiles * d->dv * eb);
-  L.off_Kbar = off;       off = align_up(off + tiles * d->dk * eb);
+  L.off_W = off;          off = align_up(off + (wy ? tiles * d->dk * eb : 0));
+  L.off_Ut = off;         off = align_up(off + (wy ? tiles * d->dv * eb : 0));
+  L.off_Kbar = off;       off = align_up(off + (wy ? tiles * d->dk * eb : 0));
   L.off_Qeff = off;       off = align_up(off + tiles * d->dk * eb);
   L.off_Opart = off;      off = align_up(off + tiles * d->dv * eb);
   L.off_gamma_last = off; off = align_up(off + (size_t)max_chunks * d->H * d->dk * sizeof(float));
+  L.off_Mp = off;         off = align_up(off + (wy ? 0 : mats * d->dk * eb));
+  L.off_Nc = off;         off = align_up(off + (wy ? 0 : mats * d->dv * eb));
   L.off_chunk_offsets = off; off = align_up(off + (size_t)(N + 1) * sizeof(int32_t));
   L.off_status = off;     off = align_up(off + sizeof(int32_t));
   L.total_bytes = off;
@@ -129,13 +143,56 @@ gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, co
   a.Qeff = at<FT>(d->workspace, L.l.off_Qeff);
   a.Opart = at<FT>(d->workspace, L.l.off_Opart);
   a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
+  a.Mp = at<FT>(d->workspace, L.l.off_Mp);
+  a.Nc = at<FT>(d->workspace, L.l.off_Nc);
   if (L.l.max_chunks == 0) return GDN2_OK;
   constexpr size_t smem = gdn2::prep_simt_smem_bytes<DK, DV>();
-  auto kern = gdn2::prep_simt_kernel<DK, DV, IO, FT>;
+  auto kern = L.l.factor_set == 1 ? gdn2::prep_simt_kernel<DK, DV, IO, FT, true>
+                                  : gdn2::prep_simt_kernel<DK, DV, IO, FT, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return GDN2_ERR_CUDA;
   dim3 grid(L.l.max_chunks, d->H);
   kern<<<grid, gdn2::kPrepSimtThreads, smem, s>>>(a);
+  return launch_status();
+}
+
+// ------------------------------------------------------- walk (tensor) ----
+// bf16 I/O with dk = 128: the affine walk on the tensor cores.
+template <int DV>
+gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const float* h0,
+                           const int32_t* cu, void* out, float* hT, float* chunk_states, cudaStream_t s) {
+  using C = gdn2::WalkTcCfg<DV>;
+  gdn2::WalkTcArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const long long rows_mp = (long long)std::max(L.l.max_chunks, 1) * d->H * 128;
+  if (rows_mp >= (1ll << 31)) return GDN2_ERR_SHAPE;  // TMA coordinates are int32
+  const uint64_t dims_mp[2] = {128, (uint64_t)rows_mp};
+  const uint64_t dims_qe[2] = {128, (uint64_t)rows_mp / 2};
+  const uint64_t strides[1] = {256};
+  const uint32_t box_mp[2] = {64, 128}, box_qe[2] = {64, 64};
+  if (!gdn2::make_tmap(&a.tm_Mp, at<void>(d->workspace, L.l.off_Mp), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims_mp,
+                       strides, box_mp, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !gdn2::make_tmap(&a.tm_Qe, at<void>(d->workspace, L.l.off_Qeff), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims_qe,
+                       strides, box_qe, CU_TENSOR_MAP_SWIZZLE_128B))
+    return GDN2_ERR_CUDA;
+  a.Nc = at<const bf16>(d->workspace, L.l.off_Nc);
+  a.Opart = at<const bf16>(d->workspace, L.l.off_Opart);
+  a.gamma_last = at<const float>(d->workspace, L.l.off_gamma_last);
+  a.map = seq_map(d, L, cu);
+  a.H = d->H;
+  a.scale = scale;
+  a.h0 = h0;
+  a.out = static_cast<bf16*>(out);
+  a.hT = hT;
+  a.chunk_states = chunk_states;
+  a.status = at<int32_t>(d->workspace, L.l.off_status);
+  if (L.N == 0) return GDN2_OK;
+  auto kern = gdn2::walk_tc_kernel<DV>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  const long long blocks = (long long)L.N * d->H;
+  if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+  kern<<<(unsigned)blocks, C::THREADS, C::SMEM, s>>>(a);
   return launch_status();
 }
 
@@ -158,6 +215,9 @@ gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, cons
   a.out = static_cast<IO*>(out);
   a.hT = hT;
   a.chunk_states = chunk_states;
+  if constexpr (DK == 128 && std::is_same<IO, bf16>::value) {
+    if (L.l.factor_set == 1) return launch_walk_tc<DV>(d, L, scale, h0, cu, out, hT, chunk_states, s);
+  }
   if (L.N == 0) return GDN2_OK;
   constexpr size_t smem = gdn2::walk_simt_smem_bytes<DK, DV>();
   auto kern = gdn2::walk_simt_kernel<DK, DV, IO, FT>;

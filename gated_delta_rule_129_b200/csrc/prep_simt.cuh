@@ -39,6 +39,8 @@ struct PrepArgs {
   FT* Qeff;
   FT* Opart;
   float* gamma_last;
+  FT* Mp;  // affine factor set only: Kbar^T W   [., H, DK, DK]
+  FT* Nc;  // affine factor set only: Kbar^T U~  [., H, DK, DV]
 };
 
 constexpr int kPrepSimtThreads = 256;
@@ -48,7 +50,9 @@ constexpr size_t prep_simt_smem_bytes() {
   return sizeof(float) * (size_t)(4 * kChunk * (DK + 1) + kChunk * (DV + 1) + 2 * kChunk * (kChunk + 1));
 }
 
-template <int DK, int DV, typename IO, typename FT>
+// AFFINE selects the factor set: false stores W, U~, Kbar (WY set); true
+// stores Mp = Kbar^T W and Nc = Kbar^T U~ (the chunk's affine state map).
+template <int DK, int DV, typename IO, typename FT, bool AFFINE>
 __global__ void __launch_bounds__(kPrepSimtThreads)
 prep_simt_kernel(const PrepArgs<IO, FT> a) {
   static_assert(DK + DV <= kPrepSimtThreads, "one thread per solve column");
@@ -127,17 +131,24 @@ prep_simt_kernel(const PrepArgs<IO, FT> a) {
     }
   }
   __syncthreads();
-  // Kbar and gamma_last go straight out; E~ and Q~ are formed in place.
+  // Kbar (kept in sk, rows past the last token zero) and gamma_last; E~ and
+  // Q~ are formed in place.
   const size_t tile_k = ((size_t)c * H + h) * kChunk * DK;
   const size_t tile_v = ((size_t)c * H + h) * kChunk * DV;
   for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
     const int i = idx / DK, cc = idx % DK;
     const float gi = sg[i * LK + cc];
     const float kb = i < len ? sk[i * LK + cc] * expf(sg[(kChunk - 1) * LK + cc] - gi) : 0.f;
-    a.Kbar[tile_k + idx] = from_f32<FT>(kb);
+    if constexpr (!AFFINE) a.Kbar[tile_k + idx] = from_f32<FT>(kb);
     const float gam = expf(gi);
     se[i * LK + cc] *= gam;
     sq[i * LK + cc] *= gam;
+  }
+  // (sg is still read above by other threads; Kbar replaces k only after a barrier)
+  __syncthreads();
+  for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
+    const int i = idx / DK, cc = idx % DK;
+    sk[i * LK + cc] = i < len ? sk[i * LK + cc] * expf(sg[(kChunk - 1) * LK + cc] - sg[i * LK + cc]) : 0.f;
   }
   if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
   __syncthreads();
@@ -162,14 +173,32 @@ prep_simt_kernel(const PrepArgs<IO, FT> a) {
     float acc = sq[i * LK + cc];
     for (int j = 0; j <= i && j < len; ++j) acc = fmaf(-sP[i * LA + j], se[j * LK + cc], acc);
     a.Qeff[tile_k + idx] = from_f32<FT>(acc);
-    a.W[tile_k + idx] = from_f32<FT>(se[i * LK + cc]);
+    if constexpr (!AFFINE) a.W[tile_k + idx] = from_f32<FT>(se[i * LK + cc]);
   }
   for (int idx = tid; idx < kChunk * DV; idx += kPrepSimtThreads) {
     const int i = idx / DV, cc = idx % DV;
     float acc = 0.f;
     for (int j = 0; j <= i && j < len; ++j) acc = fmaf(sP[i * LA + j], sz[j * LV + cc], acc);
     a.Opart[tile_v + idx] = from_f32<FT>(acc);
-    a.Ut[tile_v + idx] = from_f32<FT>(sz[i * LV + cc]);
+    if constexpr (!AFFINE) a.Ut[tile_v + idx] = from_f32<FT>(sz[i * LV + cc]);
+  }
+  if constexpr (AFFINE) {
+    // The chunk's affine state map: S' = diag(gamma) S - Mp S + Nc with
+    // Mp = Kbar^T W and Nc = Kbar^T U~ (sums over the chunk's tokens).
+    const size_t mat_k = ((size_t)c * H + h) * DK * DK;
+    const size_t mat_v = ((size_t)c * H + h) * DK * DV;
+    for (int idx = tid; idx < DK * DK; idx += kPrepSimtThreads) {
+      const int m = idx / DK, kk = idx % DK;
+      float acc = 0.f;
+      for (int i = 0; i < len; ++i) acc = fmaf(sk[i * LK + m], se[i * LK + kk], acc);
+      a.Mp[mat_k + idx] = from_f32<FT>(acc);
+    }
+    for (int idx = tid; idx < DK * DV; idx += kPrepSimtThreads) {
+      const int m = idx / DV, j = idx % DV;
+      float acc = 0.f;
+      for (int i = 0; i < len; ++i) acc = fmaf(sk[i * LK + m], sz[i * LV + j], acc);
+      a.Nc[mat_v + idx] = from_f32<FT>(acc);
+    }
   }
 }
 

@@ -51,13 +51,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: spins at most `limit` polls (each try_wait itself blocks for
-// a hardware-defined short interval).  Returns false if the phase never
-// completed; the caller records the timeout and winds down.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 24)) {
-  for (uint32_t i = 0; i < limit; ++i)
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: polls until the phase with `parity` has completed or
+// `budget_ns` of wall time (default 2 s) has passed.  Returns false on a
+// timeout; the caller records it and winds down instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t budget_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-  return false;
+    if (global_ns() - t0 > budget_ns) return false;
+  }
 }
 
 // ------------------------------------------------------------------ TMA ----

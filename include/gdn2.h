@@ -98,23 +98,35 @@ typedef struct gdn2_desc {
   size_t workspace_bytes;  /* its size in bytes                                  */
 } gdn2_desc;
 
-/* Where the per-chunk WY factors live inside the workspace, so that callers
+/* Where the per-chunk factors live inside the workspace, so that callers
  * (and tests) can inspect what gdn2_chunk_prep produced.  All offsets are in
- * bytes from `workspace`.  Factor tensors are [max_chunks, H, 64, d] in the
- * element size `factor_elem_bytes` (4 = fp32 for GDN2_IO_F32, 2 = bf16 for
+ * bytes from `workspace`.  Factor tensors are indexed [max_chunks, H, ...] in
+ * the element size `factor_elem_bytes` (4 = fp32 for GDN2_IO_F32, 2 = bf16 for
  * GDN2_IO_BF16); rows past a chunk's last token are zero.  Chunk c of
  * sequence n has global index chunk_offsets[n] + c (int32 array of N + 1
- * entries); gamma_last is [max_chunks, H, dk] fp32. */
+ * entries); gamma_last is [max_chunks, H, dk] fp32.
+ *
+ * Two factor sets exist.  Both hold Q_eff, O_part and gamma_last.
+ *  factor_set 0 ("WY", fp32 I/O and dk = 64): W, U~ and Kbar, with which the
+ *    walk computes U = U~ - W S and S' = diag(gamma) S + Kbar^T U.
+ *  factor_set 1 ("affine", bf16 I/O with dk = 128): the chunk's affine state
+ *    map, Mp = Kbar^T W [dk, dk] and Nc = Kbar^T U~ [dk, dv], so that
+ *    S' = diag(gamma) S - Mp S + Nc (one matrix product per chunk).
+ * Tensors of the other set have zero size. */
 typedef struct gdn2_ws_layout {
   size_t total_bytes;
   int max_chunks;            /* upper bound on chunks: T_total/64 + N            */
   int factor_elem_bytes;
-  size_t off_W;              /* W     = T E~           [., H, 64, dk]            */
-  size_t off_Ut;             /* U~    = T Z            [., H, 64, dv]            */
-  size_t off_Kbar;           /* Kbar  = k exp(g_n - g) [., H, 64, dk]            */
+  int factor_set;            /* 0 = WY, 1 = affine (see above)                   */
+  int reserved;
+  size_t off_W;              /* W     = T E~           [., H, 64, dk]   set 0    */
+  size_t off_Ut;             /* U~    = T Z            [., H, 64, dv]   set 0    */
+  size_t off_Kbar;           /* Kbar  = k exp(g_n - g) [., H, 64, dk]   set 0    */
   size_t off_Qeff;           /* Q_eff = Q~ - P W       [., H, 64, dk]            */
   size_t off_Opart;          /* O_part= P U~           [., H, 64, dv]            */
   size_t off_gamma_last;     /* exp(g_n)               [., H, dk] fp32           */
+  size_t off_Mp;             /* Mp    = Kbar^T W       [., H, dk, dk]   set 1    */
+  size_t off_Nc;             /* Nc    = Kbar^T U~      [., H, dk, dv]   set 1    */
   size_t off_chunk_offsets;  /* int32 [N + 1]                                    */
   size_t off_status;         /* int32 status word (a gdn2_status value)          */
 } gdn2_ws_layout;

@@ -44,9 +44,14 @@ def test_status_strings(lib):
 
 def test_workspace_layout_sizes(lib):
     lay = gdn2.workspace_layout(1, 16384, 16, 128, 128, gdn2.GDN2_IO_BF16)
-    assert lay["max_chunks"] == 256 and lay["factor_elem_bytes"] == 2
+    assert lay["max_chunks"] == 256 and lay["factor_elem_bytes"] == 2 and lay["factor_set"] == 1
     tile = 256 * 16 * 64 * 128 * 2
-    assert lay["off_Ut"] - lay["off_W"] >= tile
+    assert lay["off_W"] == lay["off_Ut"] == lay["off_Kbar"] == lay["off_Qeff"]   # WY set absent
+    assert lay["off_Opart"] - lay["off_Qeff"] >= tile
+    assert lay["off_Nc"] - lay["off_Mp"] >= 256 * 16 * 128 * 128 * 2
+    wy = gdn2.workspace_layout(1, 16384, 16, 128, 128, gdn2.GDN2_IO_F32)
+    assert wy["factor_set"] == 0 and wy["off_Ut"] - wy["off_W"] >= 2 * tile
+    assert wy["off_Nc"] == wy["off_Mp"] == wy["off_chunk_offsets"]              # affine set absent
     offs = sorted(v for k, v in lay.items() if k.startswith("off_"))
     assert all(o % 256 == 0 for o in offs)
     assert lay["total_bytes"] >= offs[-1] + 4

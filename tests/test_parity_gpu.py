@@ -52,68 +52,88 @@ def _factors(ws, lay, H, dk, dv, io):
     import torch
     dt = torch.float32 if io == "f32" else torch.bfloat16
     mc = lay["max_chunks"]
+    eb = lay["factor_elem_bytes"]
 
-    def view(off, d):
-        n = mc * H * 64 * d
-        eb = lay["factor_elem_bytes"]
-        return ws[off: off + n * eb].view(dt).view(mc, H, 64, d).float().cpu().numpy()
-    f = dict(W=view(lay["off_W"], dk), Ut=view(lay["off_Ut"], dv), Kbar=view(lay["off_Kbar"], dk),
-             Q_eff=view(lay["off_Qeff"], dk), O_part=view(lay["off_Opart"], dv))
+    def view(off, *shape):
+        n = int(np.prod(shape))
+        return ws[off: off + n * eb].view(dt).view(*shape).float().cpu().numpy()
+    f = dict(Q_eff=view(lay["off_Qeff"], mc, H, 64, dk), O_part=view(lay["off_Opart"], mc, H, 64, dv))
+    if lay["factor_set"] == 0:
+        f.update(W=view(lay["off_W"], mc, H, 64, dk), Ut=view(lay["off_Ut"], mc, H, 64, dv),
+                 Kbar=view(lay["off_Kbar"], mc, H, 64, dk))
+    else:
+        f.update(Mp=view(lay["off_Mp"], mc, H, dk, dk), Nc=view(lay["off_Nc"], mc, H, dk, dv))
     g = ws[lay["off_gamma_last"]: lay["off_gamma_last"] + mc * H * dk * 4].view(torch.float32)
     f["gamma_last"] = g.view(mc, H, dk).cpu().numpy()
     return f
 
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
-def test_prep_factors_match_oracle(io):
-    """Gate prep + intra-chunk WY (W, U~, Kbar, Q_eff, O_part, exp(g_n)) per
-    chunk against the fp64 chunkwise restatement."""
+@pytest.mark.parametrize("io,dk,dv", [("f32", 128, 64), ("bf16", 128, 64), ("bf16", 64, 128),
+                                      ("bf16", 128, 128)])
+def test_prep_factors_match_oracle(io, dk, dv):
+    """Gate prep + intra-chunk WY per chunk against the fp64 chunkwise
+    restatement: W, U~, Kbar (WY factor set) or the affine state map
+    Mp = Kbar^T W, Nc = Kbar^T U~ (affine set), plus Q_eff, O_part, exp(g_n)."""
+    import torch
+
     import gated_delta_rule_129_b200 as gdn2
     from oracle.chunk_wy import chunk_wy
     lens = [130, 64, 5]
-    H, dk, dv = 2, 128, 64
+    H = 2
     x = make_inputs(1, sum(lens), H, dk, dv, io=io, seed=31, decay="strong", lengths=lens)
     d = to_device(x)
     ws = gdn2.chunk_prep(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["cu_seqlens"])
-    import torch
     torch.cuda.synchronize()
     lay = gdn2.workspace_layout(1, sum(lens), H, dk, dv, 0 if io == "f32" else 1, num_seqs=len(lens))
+    assert lay["factor_set"] == (1 if (io == "bf16" and dk == 128) else 0)
     got = _factors(ws, lay, H, dk, dv, io)
     _, _, inter = chunk_wy(x.q, x.k, x.v, x.log_alpha, x.b, x.w, x.scale, cu_seqlens=x.cu_seqlens,
                            return_intermediates=True)
     assert len(inter) == 5
     for c, r in enumerate(inter):
         n = r["len"]
-        for key in ("W", "Ut", "Kbar", "Q_eff", "O_part"):
-            ref = r[key]
+        ref = {"Q_eff": r["Q_eff"], "O_part": r["O_part"]}
+        if lay["factor_set"] == 0:
+            ref.update(W=r["W"], Ut=r["Ut"], Kbar=r["Kbar"])
+        else:
+            ref.update(Mp=np.einsum("hic,hik->hck", r["Kbar"], r["W"]),
+                       Nc=np.einsum("hic,hij->hcj", r["Kbar"], r["Ut"]))
+        for key, rv in ref.items():
             g = got[key][c]
-            assert rel_l2(g[:, :n], ref) <= TOL[io], (c, key, rel_l2(g[:, :n], ref))
-            assert np.all(g[:, n:] == 0), (c, key)   # padded rows are exact zeros
+            if key in ("Mp", "Nc"):
+                assert rel_l2(g, rv) <= TOL[io], (c, key, rel_l2(g, rv))
+            else:
+                assert rel_l2(g[:, :n], rv) <= TOL[io], (c, key, rel_l2(g[:, :n], rv))
+                assert np.all(g[:, n:] == 0), (c, key)   # padded rows are exact zeros
         # fp32 cumulative sum of up to 64 log-decays: relative error ~1e-6
         assert rel_l2(got["gamma_last"][c], r["gamma_last"]) <= 1e-4
 
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
-def test_walk_states_match_oracle(io):
+@pytest.mark.parametrize("io,dk,dv", [("f32", 64, 128), ("bf16", 64, 128), ("bf16", 128, 128),
+                                      ("bf16", 128, 64)])
+def test_walk_states_match_oracle(io, dk, dv):
     """The state walk: the state at the start of every chunk, and hT."""
     import torch
 
     import gated_delta_rule_129_b200 as gdn2
     from oracle.chunk_wy import chunk_wy
-    x = make_inputs(2, 200, 2, 64, 128, io=io, seed=32, h0_std=0.1)
+    x = make_inputs(2, 200, 2, dk, dv, io=io, seed=32, h0_std=0.1)
     d = to_device(x)
     ws = gdn2.chunk_prep(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"])
-    lay = gdn2.workspace_layout(2, 200, 2, 64, 128, 0 if io == "f32" else 1)
-    cs = torch.zeros((lay["max_chunks"], 2, 64, 128), dtype=torch.float32, device="cuda")
+    lay = gdn2.workspace_layout(2, 200, 2, dk, dv, 0 if io == "f32" else 1)
+    cs = torch.zeros((lay["max_chunks"], 2, dk, dv), dtype=torch.float32, device="cuda")
     io_dt = torch.float32 if io == "f32" else torch.bfloat16
-    o, hT = gdn2.chunk_walk(ws, (2, 200, 2, 64, 128), io_dt, x.scale, h0=d["h0"], chunk_states=cs)
-    _, hT_ref, inter = chunk_wy(x.q, x.k, x.v, x.log_alpha, x.b, x.w, x.scale, h0=x.h0,
-                                return_intermediates=True)
+    o, hT = gdn2.chunk_walk(ws, (2, 200, 2, dk, dv), io_dt, x.scale, h0=d["h0"], chunk_states=cs)
+    o_ref, hT_ref, inter = chunk_wy(x.q, x.k, x.v, x.log_alpha, x.b, x.w, x.scale, h0=x.h0,
+                                    return_intermediates=True)
     cs = cs.cpu().numpy()
     assert len(inter) == 8
     for c, r in enumerate(inter):
         assert rel_l2(cs[c], r["S0"]) <= TOL[io], c
     assert rel_l2(hT.cpu().numpy(), hT_ref) <= TOL[io]
+    assert rel_l2(o.float().cpu().numpy(), o_ref) <= TOL[io]
+    st = ws[lay["off_status"]: lay["off_status"] + 4].view(torch.int32).item()
+    assert st == 0
 
 
 # --- varlen, state chaining, in place ------------------------------------------------
