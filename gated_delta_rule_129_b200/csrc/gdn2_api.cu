@@ -166,18 +166,19 @@ gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, con
   std::memset(&a, 0, sizeof(a));
   const long long rows_mp = (long long)std::max(L.l.max_chunks, 1) * d->H * 128;
   if (rows_mp >= (1ll << 31)) return GDN2_ERR_SHAPE;  // TMA coordinates are int32
-  const uint64_t dims_mp[2] = {128, (uint64_t)rows_mp};
-  const uint64_t dims_qe[2] = {128, (uint64_t)rows_mp / 2};
-  const uint64_t strides[1] = {256};
-  const uint32_t box_mp[2] = {64, 128}, box_qe[2] = {64, 64};
-  if (!gdn2::make_tmap(&a.tm_Mp, at<void>(d->workspace, L.l.off_Mp), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims_mp,
-                       strides, box_mp, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !gdn2::make_tmap(&a.tm_Qe, at<void>(d->workspace, L.l.off_Qeff), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims_qe,
-                       strides, box_qe, CU_TENSOR_MAP_SWIZZLE_128B))
+  const uint64_t rows_k = (uint64_t)rows_mp, rows_t = rows_k / 2, rows_g = rows_k / 128;
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t d_mp[2] = {128, rows_k}, d_qe[2] = {128, rows_t};
+  const uint64_t d_nc[2] = {(uint64_t)DV, rows_k}, d_op[2] = {(uint64_t)DV, rows_t}, d_g[2] = {128, rows_g};
+  const uint64_t st_k[1] = {256}, st_v[1] = {(uint64_t)DV * 2}, st_g[1] = {512};
+  const uint32_t b_mp[2] = {64, 128}, b_qe[2] = {64, 64}, b_nc[2] = {32, 128}, b_op[2] = {32, 64}, b_g[2] = {128, 1};
+  if (!gdn2::make_tmap(&a.tm_Mp, at<void>(d->workspace, L.l.off_Mp), BF, 2, d_mp, st_k, b_mp, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !gdn2::make_tmap(&a.tm_Qe, at<void>(d->workspace, L.l.off_Qeff), BF, 2, d_qe, st_k, b_qe, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !gdn2::make_tmap(&a.tm_Nc, at<void>(d->workspace, L.l.off_Nc), BF, 2, d_nc, st_v, b_nc, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !gdn2::make_tmap(&a.tm_Op, at<void>(d->workspace, L.l.off_Opart), BF, 2, d_op, st_v, b_op, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !gdn2::make_tmap(&a.tm_g, at<void>(d->workspace, L.l.off_gamma_last), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d_g, st_g,
+                       b_g, CU_TENSOR_MAP_SWIZZLE_NONE))
     return GDN2_ERR_CUDA;
-  a.Nc = at<const bf16>(d->workspace, L.l.off_Nc);
-  a.Opart = at<const bf16>(d->workspace, L.l.off_Opart);
-  a.gamma_last = at<const float>(d->workspace, L.l.off_gamma_last);
   a.map = seq_map(d, L, cu);
   a.H = d->H;
   a.scale = scale;
@@ -190,7 +191,7 @@ gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, con
   auto kern = gdn2::walk_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;
-  const long long blocks = (long long)L.N * d->H;
+  const long long blocks = (long long)L.N * d->H * C::SLICES;
   if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM, s>>>(a);
   return launch_status();

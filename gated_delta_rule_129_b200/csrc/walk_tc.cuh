@@ -1,29 +1,33 @@
 // walk_tc.cuh -- inter-chunk state walk + chunk output on the tensor cores
 // (bf16 I/O, dk = 128, dv in {64, 128}).
 //
-// One CTA per (sequence, head).  The head's dk x dv state stays in fp32
-// registers for the whole walk (16 epilogue warps; warp w owns key rows
-// 32*(w%4) .. +31 and value columns (w/4)*dv/4 .. +dv/4, matching the TMEM
-// lane quarter the warp may read).  A bf16 copy of the state in shared memory
-// is the B operand of two UMMAs per chunk:
+// One CTA per (sequence, head, 32-column value slice).  The columns of the
+// state evolve independently (every update is a left product), so a head's
+// dv columns are split over dv/32 CTAs; each CTA keeps its 128 x 32 slice of
+// the state in fp32 registers for the whole walk (4 epilogue warps: warp w
+// owns key rows 32w .. 32w+31, the TMEM lane quarter it may read; each thread
+// one key row x 32 columns).  A bf16 copy of the slice in shared memory is the
+// B operand of two UMMAs per chunk:
 //
-//   D_S = Mp . S        (M = 128 key rows,  K = 128, N = dv)
-//   D_O = Q_eff . S     (M = 64 tokens,     K = 128, N = dv)
+//   D_S = Mp . S        (M = 128 key rows,  K = 128, N = 32)
+//   D_O = Q_eff . S     (M = 64 tokens,     K = 128, N = 32)
 //
 // and then   S <- diag(gamma) S - D_S + Nc      (fp32, in registers)
 //            O  = scale * (D_O + O_part)        (query reads the updated state)
 //
 // which is the recurrence over one 64-token chunk in its affine form (the
 // factors Mp = Kbar^T W, Nc = Kbar^T U~, Q_eff = Q~ - P W, O_part = P U~ come
-// from the prep kernel).  The serial dependency per chunk is one UMMA plus
-// one register epilogue.  Mp and Q_eff tiles are streamed by TMA through a
-// 3-stage ring; Nc, O_part and gamma rows are prefetched into registers one
-// chunk ahead.  D_O is double-buffered in TMEM so the output epilogue of
-// chunk j overlaps the UMMA of chunk j+1.
+// from the prep kernel).  The serial dependency per chunk is one UMMA (D_S)
+// plus one register epilogue; D_O is issued after D_S, double-buffered in
+// TMEM, and the bf16 state operand is double-buffered in shared memory, so
+// the output epilogue of chunk j overlaps the critical path of chunk j+1.
 //
-// Warp 16 is the producer: one lane issues the TMA loads and the UMMAs.
-// Every wait is bounded; on a timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT
-// in the status word, drains what it issued and exits.
+// Two TMA rings feed it: ring A (Mp, Q_eff; read only by the UMMAs, released
+// by tcgen05.commit) and ring B (the CTA's Nc and O_part columns and gamma;
+// read by the epilogue warps, released by them).  Warp 4 is the producer: one
+// lane issues the TMA loads and the UMMAs.  Every wait is bounded; on a
+// timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT in the status word, drains
+// what it issued and exits.
 #pragma once
 
 #include <cuda.h>
@@ -34,11 +38,11 @@
 namespace gdn2 {
 
 struct WalkTcArgs {
-  CUtensorMap tm_Mp;   // [max_chunks*H*128 rows, 128] bf16, box {64, 128}, SW128
-  CUtensorMap tm_Qe;   // [max_chunks*H*64 rows, 128]  bf16, box {64, 64},  SW128
-  const __nv_bfloat16* Nc;     // [max_chunks, H, 128, DV]
-  const __nv_bfloat16* Opart;  // [max_chunks, H, 64, DV]
-  const float* gamma_last;     // [max_chunks, H, 128]
+  CUtensorMap tm_Mp;   // Mp    [rows = max_chunks*H*128, 128] bf16, box {64, 128}, SW128
+  CUtensorMap tm_Qe;   // Q_eff [rows = max_chunks*H*64,  128] bf16, box {64, 64},  SW128
+  CUtensorMap tm_Nc;   // Nc    [rows = max_chunks*H*128, dv]  bf16, box {32, 128}
+  CUtensorMap tm_Op;   // O_part[rows = max_chunks*H*64,  dv]  bf16, box {32, 64}
+  CUtensorMap tm_g;    // gamma [rows = max_chunks*H,     128] fp32, box {128, 1}
   SeqMap map;
   int H;
   float scale;
@@ -52,18 +56,27 @@ struct WalkTcArgs {
 template <int DV>
 struct WalkTcCfg {
   static constexpr int DK = 128;
-  static constexpr int EPI_WARPS = 16;
+  static constexpr int NSL = 32;                 // value columns per CTA
+  static constexpr int SLICES = DV / NSL;
+  static constexpr int EPI_WARPS = 4;
   static constexpr int THREADS = EPI_WARPS * 32 + 32;
-  static constexpr int CPT = DV / 4;  // state columns per epilogue thread
-  static constexpr int STAGES = 3;
-  static constexpr int MP_BYTES = DK * DK * 2;
-  static constexpr int QE_BYTES = kChunk * DK * 2;
-  static constexpr int STAGE_BYTES = MP_BYTES + QE_BYTES;
-  static constexpr int S_BYTES = DK * DV * 2;
+  static constexpr int STAGES_A = 3;
+  static constexpr int STAGES_B = 4;
+  static constexpr int MP_BYTES = DK * DK * 2;             // 32 KiB
+  static constexpr int QE_BYTES = kChunk * DK * 2;         // 16 KiB
+  static constexpr int A_BYTES = MP_BYTES + QE_BYTES;
+  static constexpr int NC_BYTES = DK * NSL * 2;            // 8 KiB
+  static constexpr int OP_BYTES = kChunk * NSL * 2;        // 4 KiB
+  static constexpr int G_BYTES = DK * 4;                   // 512 B
+  static constexpr int B_BYTES = NC_BYTES + OP_BYTES + G_BYTES;
+  static constexpr int B_STRIDE = (B_BYTES + 1023) / 1024 * 1024;
+  // bf16 state operand, MN-major interleaved core matrices (8 key rows x 8
+  // columns, 128 B): offset(kg, ng) = kg * S_LBO + ng * 128
+  static constexpr int S_LBO = (NSL / 8) * 128;
+  static constexpr int S_BYTES = DK * NSL * 2;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + S_BYTES + BAR_BYTES;
-  static constexpr int TMEM_COLS = DV == 128 ? 512 : 256;  // D_S, D_O[0], D_O[1]
-  static_assert(CPT % 16 == 0, "whole 16-column TMEM loads per thread");
+  static constexpr int SMEM = 1024 + STAGES_A * A_BYTES + STAGES_B * B_STRIDE + 2 * S_BYTES + BAR_BYTES;
+  static constexpr int TMEM_COLS = 128;  // D_S [0,32), D_O[0] [32,64), D_O[1] [64,96)
 };
 
 __device__ __forceinline__ void set_timeout(int* status, int* s_abort) {
@@ -71,35 +84,51 @@ __device__ __forceinline__ void set_timeout(int* status, int* s_abort) {
   *reinterpret_cast<volatile int*>(s_abort) = 1;
 }
 
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
 template <int DV>
 __global__ void __launch_bounds__(WalkTcCfg<DV>::THREADS, 1)
 walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
   using C = WalkTcCfg<DV>;
-  constexpr int DK = C::DK, CPT = C::CPT;
+  constexpr int DK = C::DK, NSL = C::NSL;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sS = sm + C::STAGES * C::STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sS + C::S_BYTES);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* mma_done = empty + C::STAGES;
-  uint64_t* s_ready = mma_done + 1;
+  uint8_t* ringA = sm;
+  uint8_t* ringB = ringA + C::STAGES_A * C::A_BYTES;
+  uint8_t* sS = ringB + C::STAGES_B * C::B_STRIDE;          // [2][S_BYTES]
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(sS + 2 * C::S_BYTES);
+  uint64_t* emptyA = fullA + C::STAGES_A;
+  uint64_t* fullB = emptyA + C::STAGES_A;
+  uint64_t* emptyB = fullB + C::STAGES_B;
+  uint64_t* s_done = emptyB + C::STAGES_B;   // D_S of the current chunk is ready
+  uint64_t* o_done = s_done + 1;             // D_O of the current chunk is ready
+  uint64_t* s_ready = o_done + 1;            // bf16 state operand written
   uint32_t* tslot = reinterpret_cast<uint32_t*>(s_ready + 1);
   int* s_abort = reinterpret_cast<int*>(tslot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  const int sl = blockIdx.x % C::SLICES;
+  const int h = (blockIdx.x / C::SLICES) % H;
+  const int n = blockIdx.x / (C::SLICES * H);
+  const int col0 = sl * NSL;
   const int c_begin = a.map.chunk_off[n];
   const int nch = a.map.chunk_off[n + 1] - c_begin;
   const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
 
   if (tid == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], 1);
+    for (int s = 0; s < C::STAGES_A; ++s) {
+      tc::mbar_init(&fullA[s], 1);
+      tc::mbar_init(&emptyA[s], 1);
     }
-    tc::mbar_init(mma_done, 1);
+    for (int s = 0; s < C::STAGES_B; ++s) {
+      tc::mbar_init(&fullB[s], 1);
+      tc::mbar_init(&emptyB[s], C::EPI_WARPS);
+    }
+    tc::mbar_init(s_done, 1);
+    tc::mbar_init(o_done, 1);
     tc::mbar_init(s_ready, C::EPI_WARPS);
     *s_abort = 0;
     tc::fence_mbar_init();
@@ -115,189 +144,197 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
 
   if (warp < C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue --
-    const int q = warp & 3, cg = warp >> 2;
-    const int row = 32 * q + lane;  // key channel (TMEM lane)
-    const int c0 = cg * CPT;        // first value column
-    const size_t sbase = ((size_t)n * H + h) * DK * DV + (size_t)row * DV + c0;
-    float S[CPT];
+    const int row = 32 * warp + lane;  // key channel = TMEM lane
+    const size_t sbase = ((size_t)n * H + h) * DK * DV + (size_t)row * DV + col0;
+    float S[NSL];
 #pragma unroll
-    for (int i = 0; i < CPT; i += 4) {
-      float4 v = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + sbase + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < NSL; i += 4) {
+      const float4 v = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + sbase + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
     }
-    // bf16 state operand, MN-major SW128: element (k = row, n = col) of panel
-    // col / 64 at sw128_off(row, col % 64); this thread's columns are
-    // CPT / 8 whole 16-byte units of one panel.
-    uint8_t* srow = sS + (c0 / 64) * (DK * 128) + row * 128;
-    const int u0 = (c0 % 64) / 8;
-    auto store_state = [&]() {
+    // this thread's row in the interleaved operand: core matrix (row/8, g),
+    // 16-byte line row%8
+    const uint32_t srow = (row >> 3) * C::S_LBO + (row & 7) * 16;
+    auto store_state = [&](int buf) {
+      uint8_t* base = sS + buf * C::S_BYTES + srow;
 #pragma unroll
-      for (int u = 0; u < CPT / 8; ++u) {
+      for (int g = 0; g < NSL / 8; ++g) {
         uint4 pk;
-        pk.x = tc::pack_bf16(S[8 * u + 0], S[8 * u + 1]);
-        pk.y = tc::pack_bf16(S[8 * u + 2], S[8 * u + 3]);
-        pk.z = tc::pack_bf16(S[8 * u + 4], S[8 * u + 5]);
-        pk.w = tc::pack_bf16(S[8 * u + 6], S[8 * u + 7]);
-        *reinterpret_cast<uint4*>(srow + ((((u0 + u) ^ (row & 7)) << 4))) = pk;
+        pk.x = tc::pack_bf16(S[8 * g + 0], S[8 * g + 1]);
+        pk.y = tc::pack_bf16(S[8 * g + 2], S[8 * g + 3]);
+        pk.z = tc::pack_bf16(S[8 * g + 4], S[8 * g + 5]);
+        pk.w = tc::pack_bf16(S[8 * g + 6], S[8 * g + 7]);
+        *reinterpret_cast<uint4*>(base + g * 128) = pk;
       }
       tc::fence_async_smem();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_ready);
     };
-    store_state();
-
-    // per-chunk row data, prefetched one chunk ahead
-    uint32_t nc_r[CPT / 2], op_r[CPT / 2];  // bf16 pairs
-    float gam = 0.f;
-    auto prefetch = [&](int j) {
-      const int c = c_begin + j;
-      const size_t mat = ((size_t)c * H + h) * DK;
-      const uint4* np = reinterpret_cast<const uint4*>(a.Nc + (mat + row) * DV + c0);
-#pragma unroll
-      for (int u = 0; u < CPT / 8; ++u) {
-        const uint4 t = __ldg(np + u);
-        nc_r[4 * u] = t.x; nc_r[4 * u + 1] = t.y; nc_r[4 * u + 2] = t.z; nc_r[4 * u + 3] = t.w;
-      }
-      gam = __ldg(a.gamma_last + mat + row);
-      if (lane < 16) {
-        const size_t orow = ((size_t)c * H + h) * kChunk + 16 * q + lane;
-        const uint4* op = reinterpret_cast<const uint4*>(a.Opart + orow * DV + c0);
-#pragma unroll
-        for (int u = 0; u < CPT / 8; ++u) {
-          const uint4 t = __ldg(op + u);
-          op_r[4 * u] = t.x; op_r[4 * u + 1] = t.y; op_r[4 * u + 2] = t.z; op_r[4 * u + 3] = t.w;
-        }
-      }
-    };
-    if (nch > 0) prefetch(0);
+    store_state(0);
 
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int c = c_begin + j;
+      const int sb = j % C::STAGES_B;
+      const uint8_t* stB = ringB + sb * C::B_STRIDE;
       if (a.chunk_states) {
-        float* cs = a.chunk_states + ((size_t)c * H + h) * DK * DV + (size_t)row * DV + c0;
+        float* cs = a.chunk_states + ((size_t)c * H + h) * DK * DV + (size_t)row * DV + col0;
 #pragma unroll
-        for (int i = 0; i < CPT; i += 4) *reinterpret_cast<float4*>(cs + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
+        for (int i = 0; i < NSL; i += 4) *reinterpret_cast<float4*>(cs + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
       }
-      if (!tc::mbar_wait(mma_done, j & 1)) {
+      if (!tc::mbar_wait(&fullB[sb], (j / C::STAGES_B) & 1) || !tc::mbar_wait(s_done, j & 1)) {
         set_timeout(a.status, s_abort);
         break;
       }
       tc::tc_fence_after();
-      // state: S <- gamma * S - Mp S + Nc
+      // state: S <- gamma * S - Mp S + Nc   (Nc row: 32 bf16 = 64 B)
+      const float gam = reinterpret_cast<const float*>(stB + C::NC_BYTES + C::OP_BYTES)[row];
+      uint32_t ncw[NSL / 2];
 #pragma unroll
-      for (int m = 0; m < CPT / 16; ++m) {
+      for (int u = 0; u < NSL / 8; ++u) {
+        const uint4 t = reinterpret_cast<const uint4*>(stB + row * NSL * 2)[u];
+        ncw[4 * u] = t.x; ncw[4 * u + 1] = t.y; ncw[4 * u + 2] = t.z; ncw[4 * u + 3] = t.w;
+      }
+#pragma unroll
+      for (int m = 0; m < NSL / 16; ++m) {
         float d[16];
-        tc::tmem_ld16(tc::tmem_addr(tbase, 32 * q, c0 + 16 * m), d);
+        tc::tmem_ld16(tc::tmem_addr(tbase, 32 * warp, 16 * m), d);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 16; i += 2) {
           const int e = 16 * m + i;
-          const uint32_t w2 = nc_r[e / 2];
-          const float nv = __uint_as_float((e & 1) ? (w2 & 0xFFFF0000u) : (w2 << 16));
-          S[e] = fmaf(gam, S[e], nv - d[i]);
+          const uint32_t w2 = ncw[e / 2];
+          S[e] = fmaf(gam, S[e], bf16_lo(w2) - d[i]);
+          S[e + 1] = fmaf(gam, S[e + 1], bf16_hi(w2) - d[i + 1]);
         }
       }
-      store_state();
-      // output of chunk j from D_O[j & 1]: token rows 16 q + lane (lane < 16)
+      store_state((j + 1) & 1);
+      // output of chunk j: token rows 16 warp + lane (lane < 16) of D_O[j & 1]
+      if (!tc::mbar_wait(o_done, j & 1)) {
+        set_timeout(a.status, s_abort);
+        break;
+      }
+      tc::tc_fence_after();
       const int t0 = s_begin + j * kChunk;
       const int len = min(kChunk, s_end - t0);
-      const uint32_t ocol = (uint32_t)DV * (1u + (j & 1));
+      const int i_tok = 16 * warp + lane;
+      const uint32_t ocol = (uint32_t)NSL * (1u + (j & 1));
 #pragma unroll
-      for (int m = 0; m < CPT / 16; ++m) {
+      for (int m = 0; m < NSL / 16; ++m) {
         float d[16];
-        tc::tmem_ld16(tc::tmem_addr(tbase, 32 * q, ocol + c0 + 16 * m), d);
+        tc::tmem_ld16(tc::tmem_addr(tbase, 32 * warp, ocol + 16 * m), d);
         tc::tmem_wait_ld();
-        const int i_tok = 16 * q + lane;
         if (lane < 16 && i_tok < len) {
+          const uint4* op = reinterpret_cast<const uint4*>(stB + C::NC_BYTES + i_tok * NSL * 2 + 32 * m);
+          const uint4 o0 = op[0], o1 = op[1];
+          const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
           uint32_t pw[8];
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const int e = 16 * m + i;
-            const uint32_t w2 = op_r[e / 2];
-            const float o0 = a.scale * (d[i] + __uint_as_float(w2 << 16));
-            const float o1 = a.scale * (d[i + 1] + __uint_as_float(w2 & 0xFFFF0000u));
-            pw[i / 2] = tc::pack_bf16(o0, o1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)(t0 + i_tok) * H + h) * DV + c0 + 16 * m);
+          for (int i = 0; i < 8; ++i)
+            pw[i] = tc::pack_bf16(a.scale * (d[2 * i] + bf16_lo(ow[i])), a.scale * (d[2 * i + 1] + bf16_hi(ow[i])));
+          uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)(t0 + i_tok) * H + h) * DV + col0 + 16 * m);
           dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
           dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
         }
       }
       tc::tc_fence_before();
-      if (j + 1 < nch) prefetch(j + 1);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
     }
     if (a.hT && !*reinterpret_cast<volatile int*>(s_abort)) {
 #pragma unroll
-      for (int i = 0; i < CPT; i += 4)
+      for (int i = 0; i < NSL; i += 4)
         *reinterpret_cast<float4*>(a.hT + sbase + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
     }
   } else if (lane == 0) {
     // ------------------------------------------------- producer + UMMA issue --
     tc::prefetch_tmap(&a.tm_Mp);
     tc::prefetch_tmap(&a.tm_Qe);
-    auto load = [&](int j) {
-      const int st = j % C::STAGES;
+    tc::prefetch_tmap(&a.tm_Nc);
+    tc::prefetch_tmap(&a.tm_Op);
+    tc::prefetch_tmap(&a.tm_g);
+    auto loadA = [&](int j) {
+      const int st = j % C::STAGES_A;
       const int c = c_begin + j;
-      uint8_t* dst = sm + st * C::STAGE_BYTES;
-      tc::mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+      uint8_t* dst = ringA + st * C::A_BYTES;
+      tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
       const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
-      tc::tma_load_2d(dst, &a.tm_Mp, &full[st], 0, rm);
-      tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &full[st], 64, rm);
-      tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &full[st], 0, rq);
-      tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &full[st], 64, rq);
+      tc::tma_load_2d(dst, &a.tm_Mp, &fullA[st], 0, rm);
+      tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &fullA[st], 64, rm);
+      tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
+      tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
     };
-    const int pre = nch < C::STAGES ? nch : C::STAGES;
-    for (int j = 0; j < pre; ++j) load(j);
-    int loaded = pre, committed = 0;
-    constexpr uint32_t idS = tc::idesc_bf16(128, DV, false, true);
-    constexpr uint32_t idO = tc::idesc_bf16(64, DV, false, true);
-    const uint32_t sS_addr = tc::smem_u32(sS);
-    bool ok = true;
-    for (int j = 0; j < nch && ok; ++j) {
-      const int st = j % C::STAGES;
-      ok = tc::mbar_wait(&full[st], (j / C::STAGES) & 1) && tc::mbar_wait(s_ready, j & 1);
-      if (!ok || *reinterpret_cast<volatile int*>(s_abort)) {
-        if (!ok) set_timeout(a.status, s_abort);
-        ok = false;
+    auto loadB = [&](int j) {
+      const int st = j % C::STAGES_B;
+      const int c = c_begin + j;
+      uint8_t* dst = ringB + st * C::B_STRIDE;
+      tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
+      tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
+      tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
+      tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
+    };
+    int loadedA = nch < C::STAGES_A ? nch : C::STAGES_A;
+    int loadedB = nch < C::STAGES_B ? nch : C::STAGES_B;
+    for (int j = 0; j < loadedA; ++j) loadA(j);
+    for (int j = 0; j < loadedB; ++j) loadB(j);
+    constexpr uint32_t idS = tc::idesc_bf16(128, NSL, false, true);
+    constexpr uint32_t idO = tc::idesc_bf16(64, NSL, false, true);
+    int committed = 0;
+    for (int j = 0; j < nch; ++j) {
+      const int st = j % C::STAGES_A;
+      if (!tc::mbar_wait(&fullA[st], (j / C::STAGES_A) & 1) || !tc::mbar_wait(s_ready, j & 1)) {
+        set_timeout(a.status, s_abort);
         break;
       }
+      if (*reinterpret_cast<volatile int*>(s_abort)) break;
       tc::tc_fence_after();
-      const uint32_t mp = tc::smem_u32(sm + st * C::STAGE_BYTES);
+      const uint32_t mp = tc::smem_u32(ringA + st * C::A_BYTES);
       const uint32_t qe = mp + C::MP_BYTES;
+      const uint32_t sb = tc::smem_u32(sS + (j & 1) * C::S_BYTES);
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s) {
-        const uint32_t koff = (s % 4) * 32;
-        const uint64_t bd = tc::sdesc(sS_addr + s * 16 * 128, DK * 128, 1024, tc::kLayoutSW128);
-        const uint64_t ad = tc::sdesc(mp + (s / 4) * (DK * 128) + koff, 16, 1024, tc::kLayoutSW128);
+        const uint64_t bd = tc::sdesc(sb + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
+        const uint64_t ad = tc::sdesc(mp + (s / 4) * (DK * 128) + (s % 4) * 32, 16, 1024, tc::kLayoutSW128);
         tc::umma_f16(tbase, ad, bd, idS, s > 0);
       }
+      tc::umma_commit(s_done);
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s) {
-        const uint32_t koff = (s % 4) * 32;
-        const uint64_t bd = tc::sdesc(sS_addr + s * 16 * 128, DK * 128, 1024, tc::kLayoutSW128);
-        const uint64_t ad = tc::sdesc(qe + (s / 4) * (kChunk * 128) + koff, 16, 1024, tc::kLayoutSW128);
-        tc::umma_f16(tbase + (uint32_t)DV * (1u + (j & 1)), ad, bd, idO, s > 0);
+        const uint64_t bd = tc::sdesc(sb + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
+        const uint64_t ad = tc::sdesc(qe + (s / 4) * (kChunk * 128) + (s % 4) * 32, 16, 1024, tc::kLayoutSW128);
+        tc::umma_f16(tbase + (uint32_t)NSL * (1u + (j & 1)), ad, bd, idO, s > 0);
       }
-      tc::umma_commit(mma_done);
-      tc::umma_commit(&empty[st]);
+      tc::umma_commit(o_done);
+      tc::umma_commit(&emptyA[st]);
       committed = j + 1;
-      if (loaded < nch) {
-        // stage st is reused for chunk `loaded` once these UMMAs have read it
-        if (!tc::mbar_wait(&empty[st], (j / C::STAGES) & 1)) {
+      // refill ring A with chunk j + STAGES_A once this chunk's UMMAs are done
+      if (loadedA < nch) {
+        if (!tc::mbar_wait(&emptyA[st], (j / C::STAGES_A) & 1)) {
           set_timeout(a.status, s_abort);
-          ok = false;
           break;
         }
-        load(loaded);
-        ++loaded;
+        loadA(loadedA++);
+      }
+      // refill ring B with chunk (j - 1) + STAGES_B once the epilogue is done with j - 1
+      if (j >= 1 && loadedB < nch) {
+        const int jb = j - 1;
+        if (!tc::mbar_wait(&emptyB[jb % C::STAGES_B], (jb / C::STAGES_B) & 1)) {
+          set_timeout(a.status, s_abort);
+          break;
+        }
+        loadB(loadedB++);
       }
     }
-    // drain: every issued load has landed and every issued UMMA has finished
-    // before the CTA releases its shared and tensor memory
-    for (int j = committed; j < loaded; ++j) tc::mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
-    if (committed > 0) tc::mbar_wait(mma_done, (committed - 1) & 1);
+    // drain: issued loads have landed and issued UMMAs have finished before
+    // the CTA releases its shared and tensor memory
+    // (each stage holds at most one outstanding load, so waiting on the last
+    // load of every stage covers all of them, including ones already consumed)
+    for (int j = loadedA > C::STAGES_A ? loadedA - C::STAGES_A : 0; j < loadedA; ++j)
+      tc::mbar_wait(&fullA[j % C::STAGES_A], (j / C::STAGES_A) & 1);
+    for (int j = loadedB > C::STAGES_B ? loadedB - C::STAGES_B : 0; j < loadedB; ++j)
+      tc::mbar_wait(&fullB[j % C::STAGES_B], (j / C::STAGES_B) & 1);
+    if (committed > 0) tc::mbar_wait(&emptyA[(committed - 1) % C::STAGES_A], ((committed - 1) / C::STAGES_A) & 1);
   }
   tc::tc_fence_before();
   __syncthreads();
