@@ -59,7 +59,7 @@ class WsLayout(ctypes.Structure):
                 ("off_Qeff", ctypes.c_size_t), ("off_Opart", ctypes.c_size_t),
                 ("off_gamma_last", ctypes.c_size_t), ("off_Mp", ctypes.c_size_t),
                 ("off_Nc", ctypes.c_size_t), ("off_chunk_offsets", ctypes.c_size_t),
-                ("off_status", ctypes.c_size_t)]
+                ("off_status", ctypes.c_size_t), ("off_fix", ctypes.c_size_t)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}

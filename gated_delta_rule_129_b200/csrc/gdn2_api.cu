@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "plan.cuh"
 #include "prep_simt.cuh"
+#include "prep_tc.cuh"
 #include "tmap.cuh"
 #include "walk_simt.cuh"
 #include "walk_tc.cuh"
@@ -85,6 +86,7 @@ gdn2_status make_layout(const gdn2_desc* d, bool packed, Layout* out) {
   L.off_Nc = off;         off = align_up(off + (wy ? 0 : mats * d->dv * eb));
   L.off_chunk_offsets = off; off = align_up(off + (size_t)(N + 1) * sizeof(int32_t));
   L.off_status = off;     off = align_up(off + sizeof(int32_t));
+  L.off_fix = off;        off = align_up(off + (wy ? 0 : (size_t)(1 + (size_t)max_chunks * d->H) * sizeof(int32_t)));
   L.total_bytes = off;
   out->N = N;
   return GDN2_OK;
@@ -119,7 +121,46 @@ gdn2::SeqMap seq_map(const gdn2_desc* d, const Layout& L, const int32_t* cu) {
 gdn2_status launch_plan(const gdn2_desc* d, const Layout& L, const int32_t* cu, cudaStream_t s) {
   gdn2::plan_kernel<<<1, gdn2::kPlanThreads, 0, s>>>(
       cu, L.N, d->T, d->B * d->T, at<int32_t>(d->workspace, L.l.off_chunk_offsets),
-      at<int32_t>(d->workspace, L.l.off_status), (int)GDN2_ERR_SEQLENS);
+      at<int32_t>(d->workspace, L.l.off_status), (int)GDN2_ERR_SEQLENS,
+      L.l.factor_set == 1 ? at<int32_t>(d->workspace, L.l.off_fix) : nullptr);
+  return launch_status();
+}
+
+// ------------------------------------------------------- prep (tensor) ----
+// bf16 I/O with dk = 128: gate prep, intra-chunk WY and the affine state map
+// on the tensor cores.
+template <int DV>
+gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
+                           const float* la, const float* b, const float* w, const int32_t* cu, cudaStream_t s) {
+  using C = gdn2::PrepTcCfg<DV>;
+  gdn2::PrepTcArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const uint64_t T_total = (uint64_t)d->B * d->T;
+  if (T_total == 0) return GDN2_OK;
+  const uint64_t dk[3] = {128, (uint64_t)d->H, T_total}, dv[3] = {(uint64_t)DV, (uint64_t)d->H, T_total};
+  const uint64_t sk2[2] = {128 * 2, (uint64_t)d->H * 128 * 2}, sk4[2] = {128 * 4, (uint64_t)d->H * 128 * 4};
+  const uint64_t sv2[2] = {(uint64_t)DV * 2, (uint64_t)d->H * DV * 2}, sv4[2] = {(uint64_t)DV * 4, (uint64_t)d->H * DV * 4};
+  const uint32_t bk[3] = {32, 1, 64}, bv[3] = {(uint32_t)C::VS, 1, 64};
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUtensorMapSwizzle NS = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!gdn2::make_tmap(&a.tm_q, q, BF, 3, dk, sk2, bk, NS) || !gdn2::make_tmap(&a.tm_k, k, BF, 3, dk, sk2, bk, NS) ||
+      !gdn2::make_tmap(&a.tm_v, v, BF, 3, dv, sv2, bv, NS) || !gdn2::make_tmap(&a.tm_la, la, F32, 3, dk, sk4, bk, NS) ||
+      !gdn2::make_tmap(&a.tm_b, b, F32, 3, dk, sk4, bk, NS) || !gdn2::make_tmap(&a.tm_w, w, F32, 3, dv, sv4, bv, NS))
+    return GDN2_ERR_CUDA;
+  a.map = seq_map(d, L, cu);
+  a.H = d->H;
+  a.Qeff = at<bf16>(d->workspace, L.l.off_Qeff);
+  a.Opart = at<bf16>(d->workspace, L.l.off_Opart);
+  a.Mp = at<bf16>(d->workspace, L.l.off_Mp);
+  a.Nc = at<bf16>(d->workspace, L.l.off_Nc);
+  a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
+  a.fix_list = at<int32_t>(d->workspace, L.l.off_fix);
+  a.status = at<int32_t>(d->workspace, L.l.off_status);
+  auto kern = gdn2::prep_tc_kernel<DV>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  dim3 grid(L.l.max_chunks, d->H);
+  kern<<<grid, C::THREADS, C::SMEM, s>>>(a);
   return launch_status();
 }
 
@@ -147,6 +188,19 @@ gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, co
   a.Nc = at<FT>(d->workspace, L.l.off_Nc);
   if (L.l.max_chunks == 0) return GDN2_OK;
   constexpr size_t smem = gdn2::prep_simt_smem_bytes<DK, DV>();
+  if constexpr (DK == 128 && std::is_same<IO, bf16>::value) {
+    if (L.l.factor_set == 1) {
+      const gdn2_status st = launch_prep_tc<DV>(d, L, q, k, v, la, b, w, cu, s);
+      if (st != GDN2_OK) return st;
+      // exact redo of the chunks the tensor-core prep handed back
+      auto fix = gdn2::prep_fixup_kernel<DK, DV, IO, FT>;
+      if (cudaFuncSetAttribute(fix, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+      const int grid = std::min(L.l.max_chunks * d->H, 148);
+      fix<<<grid, gdn2::kPrepSimtThreads, smem, s>>>(a, at<const int32_t>(d->workspace, L.l.off_fix));
+      return launch_status();
+    }
+  }
   auto kern = L.l.factor_set == 1 ? gdn2::prep_simt_kernel<DK, DV, IO, FT, true>
                                   : gdn2::prep_simt_kernel<DK, DV, IO, FT, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)

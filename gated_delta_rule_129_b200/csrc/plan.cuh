@@ -18,7 +18,8 @@ constexpr int kPlanThreads = 1024;
 
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int32_t* __restrict__ cu, int N, int T_dense, int T_total,
-            int32_t* __restrict__ chunk_off, int32_t* __restrict__ status, int err_code) {
+            int32_t* __restrict__ chunk_off, int32_t* __restrict__ status, int err_code,
+            int32_t* __restrict__ fix_count) {
   __shared__ int s_scan[kPlanThreads];
   __shared__ int s_bad;
   const int tid = threadIdx.x;
@@ -56,7 +57,10 @@ plan_kernel(const int32_t* __restrict__ cu, int N, int T_dense, int T_total,
     }
   }
   if (tid == kPlanThreads - 1) chunk_off[N] = any_bad ? 0 : s_scan[tid];
-  if (tid == 0) *status = any_bad ? err_code : 0;
+  if (tid == 0) {
+    *status = any_bad ? err_code : 0;
+    if (fix_count) *fix_count = 0;
+  }
 }
 
 }  // namespace gdn2

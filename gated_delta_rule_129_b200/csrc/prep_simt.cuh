@@ -52,17 +52,15 @@ constexpr size_t prep_simt_smem_bytes() {
 
 // AFFINE selects the factor set: false stores W, U~, Kbar (WY set); true
 // stores Mp = Kbar^T W and Nc = Kbar^T U~ (the chunk's affine state map).
+// One (chunk c, head h) per call; all kPrepSimtThreads threads take part.
 template <int DK, int DV, typename IO, typename FT, bool AFFINE>
-__global__ void __launch_bounds__(kPrepSimtThreads)
-prep_simt_kernel(const PrepArgs<IO, FT> a) {
+__device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c, int h, float* smem) {
   static_assert(DK + DV <= kPrepSimtThreads, "one thread per solve column");
   constexpr int LK = DK + 1, LV = DV + 1, LA = kChunk + 1;
-  const int c = blockIdx.x, h = blockIdx.y, H = a.H;
-  if (c >= a.map.chunk_off[a.map.N]) return;
+  const int H = a.H;
   const ChunkPos pos = chunk_pos(a.map, c);
   const int len = pos.len;
 
-  extern __shared__ float smem[];
   float* sg = smem;                 // [64][LK]  cumulative log-decay
   float* sk = sg + kChunk * LK;     // [64][LK]  k
   float* se = sk + kChunk * LK;     // [64][LK]  e, then E~, then W
@@ -199,6 +197,30 @@ prep_simt_kernel(const PrepArgs<IO, FT> a) {
       for (int i = 0; i < len; ++i) acc = fmaf(sk[i * LK + m], sz[i * LV + j], acc);
       a.Nc[mat_v + idx] = from_f32<FT>(acc);
     }
+  }
+}
+
+template <int DK, int DV, typename IO, typename FT, bool AFFINE>
+__global__ void __launch_bounds__(kPrepSimtThreads)
+prep_simt_kernel(const PrepArgs<IO, FT> a) {
+  extern __shared__ float smem[];
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= a.map.chunk_off[a.map.N]) return;
+  prep_simt_chunk<DK, DV, IO, FT, AFFINE>(a, c, h, smem);
+}
+
+// Exact fallback for the chunks the tensor-core prep hands back (decay too
+// steep for its single in-chunk reference point): list[0] is the count,
+// list[1 + i] = c * H + h.  A fixed grid strides over the list.
+template <int DK, int DV, typename IO, typename FT>
+__global__ void __launch_bounds__(kPrepSimtThreads)
+prep_fixup_kernel(const PrepArgs<IO, FT> a, const int32_t* list) {
+  extern __shared__ float smem[];
+  const int count = list[0];
+  for (int i = blockIdx.x; i < count; i += gridDim.x) {
+    const int e = list[1 + i];
+    prep_simt_chunk<DK, DV, IO, FT, true>(a, e / a.H, e % a.H, smem);
+    __syncthreads();
   }
 }
 

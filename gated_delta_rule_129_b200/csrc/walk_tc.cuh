@@ -84,8 +84,6 @@ __device__ __forceinline__ void set_timeout(int* status, int* s_abort) {
   *reinterpret_cast<volatile int*>(s_abort) = 1;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 template <int DV>
 __global__ void __launch_bounds__(WalkTcCfg<DV>::THREADS, 1)
@@ -205,8 +203,8 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
         for (int i = 0; i < 16; i += 2) {
           const int e = 16 * m + i;
           const uint32_t w2 = ncw[e / 2];
-          S[e] = fmaf(gam, S[e], bf16_lo(w2) - d[i]);
-          S[e + 1] = fmaf(gam, S[e + 1], bf16_hi(w2) - d[i + 1]);
+          S[e] = fmaf(gam, S[e], bf16_lo_f(w2) - d[i]);
+          S[e + 1] = fmaf(gam, S[e + 1], bf16_hi_f(w2) - d[i + 1]);
         }
       }
       store_state((j + 1) & 1);
@@ -232,7 +230,7 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
           uint32_t pw[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            pw[i] = tc::pack_bf16(a.scale * (d[2 * i] + bf16_lo(ow[i])), a.scale * (d[2 * i + 1] + bf16_hi(ow[i])));
+            pw[i] = tc::pack_bf16(a.scale * (d[2 * i] + bf16_lo_f(ow[i])), a.scale * (d[2 * i + 1] + bf16_hi_f(ow[i])));
           uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)(t0 + i_tok) * H + h) * DV + col0 + 16 * m);
           dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
           dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);

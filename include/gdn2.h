@@ -129,6 +129,9 @@ typedef struct gdn2_ws_layout {
   size_t off_Nc;             /* Nc    = Kbar^T U~      [., H, dk, dv]   set 1    */
   size_t off_chunk_offsets;  /* int32 [N + 1]                                    */
   size_t off_status;         /* int32 status word (a gdn2_status value)          */
+  size_t off_fix;            /* int32 [1 + max_chunks * H]: chunks whose decay   */
+                             /* is too steep for the tensor-core prep, redone    */
+                             /* exactly ([0] = count, then chunk * H + head)     */
 } gdn2_ws_layout;
 
 /* Bytes of workspace gdn2_chunk_fwd needs for `desc` (0 if desc is invalid).

@@ -257,3 +257,24 @@ def test_decode_steps_equal_chunk_forward():
         outs.append(gdn2.recurrent_step(s("q"), s("k"), s("v"), s("log_alpha"), s("b"), s("w"), x.scale, state))
     od = torch.stack(outs, dim=1).cpu().numpy()
     assert rel_l2(od, o) <= 1e-5 and rel_l2(state.cpu().numpy(), hT) <= 1e-5
+
+
+def test_steep_decay_falls_back_to_exact_prep():
+    """A chunk whose decay over 32 tokens exceeds the tensor-core prep's range
+    (here log_alpha = -6 on a run of tokens in some channels) is redone by
+    the exact fp32 kernel; the result still matches the oracle and the
+    workspace lists the chunks that were handed back."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    x = make_inputs(1, 300, 2, 128, 128, io="bf16", seed=43, h0_std=0.05)
+    x.log_alpha[0, 70:100, :, :16] = -6.0      # ~180 nats over 30 tokens
+    d = to_device(x)
+    lay = gdn2.workspace_layout(1, 300, 2, 128, 128, 1)
+    ws = torch.zeros(lay["total_bytes"], dtype=torch.uint8, device="cuda")
+    o, hT = gdn2.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], x.scale,
+                           h0=d["h0"], workspace=ws)
+    n_fix = ws[lay["off_fix"]: lay["off_fix"] + 4].view(torch.int32).item()
+    assert n_fix >= 2          # chunk 1 of both heads
+    ro, rh = compare(x, o.float().cpu().numpy(), hT.cpu().numpy())
+    assert ro <= TOL["bf16"] and rh <= TOL["bf16"], (ro, rh)
