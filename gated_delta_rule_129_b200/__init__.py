@@ -19,7 +19,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["chunk_fwd", "chunk_prep", "chunk_walk", "recurrent_step", "workspace_size",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "chunk_prep", "chunk_walk", "recurrent_step", "workspace_size",
            "workspace_layout", "status_string", "GDN2Error", "lib_path", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,7 +34,8 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_NULL", 2: "GDN2_ERR_SHAPE", 3: "GDN2_ERR_DT
           4: "GDN2_ERR_ALIGN", 5: "GDN2_ERR_SEQLENS", 6: "GDN2_ERR_WORKSPACE",
           7: "GDN2_ERR_CUDA", 8: "GDN2_ERR_DEVICE_TIMEOUT", 9: "GDN2_ERR_UNSUPPORTED"}
 
-EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_prep",
+EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_fwd_noalloc",
+            "gdn2_chunk_prep",
             "gdn2_chunk_walk", "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version")
 
 
@@ -87,6 +88,8 @@ def load_library():
         lib.gdn2_workspace_layout.restype = i
         lib.gdn2_chunk_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_fwd.restype = i
+        lib.gdn2_chunk_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
+        lib.gdn2_chunk_fwd_noalloc.restype = i
         lib.gdn2_chunk_prep.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_prep.restype = i
         lib.gdn2_chunk_walk.argtypes = [dp, f, vp, vp, vp, vp, vp, vp]
@@ -205,6 +208,37 @@ def chunk_fwd(q, k, v, log_alpha, b, w, scale=None, h0=None, cu_seqlens=None, *,
                                        _ptr(b), _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens),
                                        _ptr(out), _ptr(hT), _stream(stream))
     _check(st, "gdn2_chunk_fwd")
+    return out, hT
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, scale=None, h0=None, cu_seqlens=None, *,
+                      out=None, hT=None, output_final_state=True, stream=None):
+    """``gdn2_chunk_fwd_noalloc``: like :func:`chunk_fwd`, but the library uses
+    its own fixed device scratch (``NOALLOC_SCRATCH_BYTES``) instead of a
+    workspace, for callers that cannot allocate device memory where they run
+    the operator.  Problems whose workspace would exceed the scratch raise
+    ``GDN2Error`` (``GDN2_ERR_WORKSPACE``).  Calls share the scratch, so calls
+    that overlap on the GPU race; keep them on one stream.  ``out``/``hT``
+    are allocated here only if not given."""
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    io = _io_of(q.dtype)
+    N = ns if cu_seqlens is not None else B
+    if scale is None:
+        scale = dk ** -0.5
+    _need_contig(q, k, v, log_alpha, b, w, h0, cu_seqlens)
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    d = make_desc(B, T, H, dk, dv, io, ns)
+    st = load_library().gdn2_chunk_fwd_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                               _ptr(b), _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens),
+                                               _ptr(out), _ptr(hT), _stream(stream))
+    _check(st, "gdn2_chunk_fwd_noalloc")
     return out, hT
 
 

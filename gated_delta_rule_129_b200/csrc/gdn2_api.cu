@@ -11,6 +11,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -456,5 +457,61 @@ const char* gdn2_status_string(gdn2_status s) {
 }
 
 int gdn2_version(void) { return 100; }
+
+}  // extern "C"
+
+// ------------------------------------------------------- no-alloc variant ----
+// The scratch of gdn2_chunk_fwd_noalloc: part of the library's device image,
+// one copy per device, shared by every call.  In host code the symbol is only
+// a stand-in; the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN2_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) and cached.
+gdn2_status noalloc_scratch(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return GDN2_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN2_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return GDN2_OK;
+}
+}  // namespace
+
+extern "C" {
+
+gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* b, const float* w, float scale,
+                                   const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                                   cudaStream_t stream) {
+  if (!desc) return GDN2_ERR_NULL;
+  gdn2_desc d = *desc;
+  d.workspace = nullptr;
+  d.workspace_bytes = 0;
+  Layout L;
+  gdn2_status st = make_layout(&d, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if (L.l.total_bytes > (size_t)GDN2_NOALLOC_SCRATCH_BYTES) return GDN2_ERR_WORKSPACE;
+  const long long tokens = (long long)d.B * d.T;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, tokens)) != GDN2_OK) return st;
+  if (!out && tokens > 0) return GDN2_ERR_NULL;
+  if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != GDN2_OK) return st;
+  d.workspace = scratch;
+  d.workspace_bytes = (size_t)GDN2_NOALLOC_SCRATCH_BYTES;
+  return gdn2_chunk_fwd(&d, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens, out, hT, stream);
+}
 
 }  // extern "C"

@@ -186,6 +186,38 @@ GDN2_API gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, c
                                 const float* log_alpha, const float* b, const float* w, float scale,
                                 float* state, void* out, cudaStream_t stream);
 
+/* Size of the library's own device scratch used by gdn2_chunk_fwd_noalloc. */
+#define GDN2_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* gdn2_chunk_fwd without a caller-provided workspace (the paper has no
+ * counterpart: this is a deployment convenience, not part of the method).
+ *
+ * Some callers cannot allocate device memory at the point where they run the
+ * operator: a plugin inside a host framework that owns every device
+ * allocation, code running while a CUDA graph is being captured (where
+ * cudaMalloc is not allowed), or a latency-critical path that must not risk
+ * the implicit device synchronisation an allocation can cause.  This entry
+ * point takes the same arguments as gdn2_chunk_fwd and ignores
+ * desc->workspace / workspace_bytes; the scratch is a fixed array of
+ * GDN2_NOALLOC_SCRATCH_BYTES that lives inside the library's device image.
+ * Every GPU that loads the library holds that array until the process exits.
+ *
+ *  - Limit: if gdn2_workspace_size(desc) exceeds GDN2_NOALLOC_SCRATCH_BYTES
+ *    the call returns GDN2_ERR_WORKSPACE and launches nothing; use
+ *    gdn2_chunk_fwd with your own workspace for such sizes.
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current).  Make that
+ *    first call outside any stream capture; later calls make no such lookup.
+ *  - Sharing: all calls use the same array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls whose work
+ *    overlaps on the GPU (other streams, other host threads) race on it:
+ *    order them on one stream or use gdn2_chunk_fwd.
+ * It calls no cudaMalloc, cudaFree or allocating library routine. */
+GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                            const float* log_alpha, const float* b, const float* w, float scale,
+                                            const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                                            cudaStream_t stream);
+
 /* Static description of a status code. */
 GDN2_API const char* gdn2_status_string(gdn2_status status);
 
