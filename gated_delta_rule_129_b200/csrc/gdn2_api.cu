@@ -29,6 +29,7 @@ using bf16 = __nv_bfloat16;
 using gdn2::kChunk;
 
 constexpr size_t kAlign = 256;
+int sm_count();
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -157,10 +158,15 @@ gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, c
   a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
   a.fix_list = at<int32_t>(d->workspace, L.l.off_fix);
   a.status = at<int32_t>(d->workspace, L.l.off_status);
+  a.ready = nullptr;
+  a.task_counter = nullptr;
   auto kern = gdn2::prep_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;
-  dim3 grid(L.l.max_chunks, d->H);
+  // persistent: one CTA per SM (shared memory and TMEM allow no more)
+  const long long tasks = (long long)L.l.max_chunks * d->H;
+  const int grid = (int)std::min<long long>(tasks, sm_count());
+  if (grid <= 0) return GDN2_OK;
   kern<<<grid, C::THREADS, C::SMEM, s>>>(a);
   return launch_status();
 }
@@ -336,6 +342,13 @@ struct DecodeOp {
     return launch_status();
   }
 };
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 1;
+  return n;
+}
 
 bool device_ok() {
   int dev = 0;
