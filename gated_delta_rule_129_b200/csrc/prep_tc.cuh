@@ -530,11 +530,11 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       if (lane == 0) tc::mbar_arrive(rv_ready);
       // Q~ for this thread's output row, while UMMA 3 runs
       const int i_out = 16 * q + lane;
-      uint4 qt_r[8];
+      uint4 qt_r[DK / 8];   // the row's 128 bf16 values of Q~
       if (half == 0 && lane < 16) {
         const uint4* src = reinterpret_cast<const uint4*>(a.Qeff + (tile * kChunk + i_out) * DK);
 #pragma unroll
-        for (int uu = 0; uu < 8; ++uu) qt_r[uu] = src[uu];
+        for (int uu = 0; uu < DK / 8; ++uu) qt_r[uu] = src[uu];
       }
       if (!tc::mbar_wait(mma3_done, ex & 1)) { alive = false; break; }
       // ------------------------------------------- epilogue 3: outputs --
