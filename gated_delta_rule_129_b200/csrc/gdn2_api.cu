@@ -149,6 +149,20 @@ gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, c
       !gdn2::make_tmap(&a.tm_v, v, BF, 3, dv, sv2, bv, NS) || !gdn2::make_tmap(&a.tm_la, la, F32, 3, dk, sk4, bk, NS) ||
       !gdn2::make_tmap(&a.tm_b, b, F32, 3, dk, sk4, bk, NS) || !gdn2::make_tmap(&a.tm_w, w, F32, 3, dv, sv4, bv, NS))
     return GDN2_ERR_CUDA;
+  {
+    const long long rows_k = (long long)std::max(L.l.max_chunks, 1) * d->H * 128;
+    if (rows_k >= (1ll << 31)) return GDN2_ERR_SHAPE;  // TMA coordinates are int32
+    const uint64_t d_mp[2] = {128, (uint64_t)rows_k}, d_nc[2] = {(uint64_t)DV, (uint64_t)rows_k};
+    const uint64_t d_qe[2] = {128, (uint64_t)rows_k / 2}, d_op[2] = {(uint64_t)DV, (uint64_t)rows_k / 2};
+    const uint64_t st_k[1] = {256}, st_v[1] = {(uint64_t)DV * 2};
+    const uint32_t b_k[2] = {64, 128}, b_t[2] = {64, 64};
+    const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!gdn2::make_tmap(&a.tm_Mp, at<void>(d->workspace, L.l.off_Mp), BF, 2, d_mp, st_k, b_k, SW) ||
+        !gdn2::make_tmap(&a.tm_Nc, at<void>(d->workspace, L.l.off_Nc), BF, 2, d_nc, st_v, b_k, SW) ||
+        !gdn2::make_tmap(&a.tm_Qe, at<void>(d->workspace, L.l.off_Qeff), BF, 2, d_qe, st_k, b_t, SW) ||
+        !gdn2::make_tmap(&a.tm_Op, at<void>(d->workspace, L.l.off_Opart), BF, 2, d_op, st_v, b_t, SW))
+      return GDN2_ERR_CUDA;
+  }
   a.map = seq_map(d, L, cu);
   a.H = d->H;
   a.Qeff = at<bf16>(d->workspace, L.l.off_Qeff);

@@ -41,6 +41,8 @@ namespace gdn2 {
 struct PrepTcArgs {
   CUtensorMap tm_q, tm_k, tm_v;    // bf16 [T_total, H, d], box {32 | dv/4, 1, 64}
   CUtensorMap tm_la, tm_b, tm_w;   // fp32 [T_total, H, d], box {32 | dv/4, 1, 64}
+  // outputs, stored by TMA from SW128 staging: box {64, 128} (Mp, Nc), {64, 64} (Q_eff, O_part)
+  CUtensorMap tm_Mp, tm_Nc, tm_Qe, tm_Op;
   SeqMap map;
   int H;
   __nv_bfloat16* Qeff;   // [max_chunks, H, 64, 128]   (holds Q~ between the two phases)
@@ -83,6 +85,9 @@ struct PrepTcCfg {
   static constexpr int OFF_AS = OFF_X, OFF_TS = OFF_X + 17408, OFF_XS = OFF_X + 34816;
   static constexpr int OFF_PB = OFF_X + 38912;  // P as K-major SW128 operand
   static constexpr int OFF_RB = OFF_X, OFF_VB = OFF_X + 16384;  // after UMMA 2
+  // output staging once UMMA 3 has read every operand (SW128 panels of 64 columns)
+  static constexpr int OFF_SMP = OFF_X, OFF_SNC = OFF_X + 32768, OFF_SQE = OFF_X + 65536, OFF_SOP = OFF_X + 81920;
+  static_assert(OFF_SOP + 16384 <= OFF_BAR, "output staging fits in the operand area");
   static constexpr int SMEM = 1024 + OFF_BAR + 2048;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t COL_D1 = 0, COL_R = 64, COL_V = 192, COL_MN = 0, COL_QO = 256;
@@ -264,7 +269,10 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       const int len = pos.len;
       const size_t tile = (size_t)c * H + h;
       volatile int* skipflag = vflag + 2 + (nt & 1);
-      if (tid == 0) *skipflag = 0;
+      if (tid == 0) {
+        *skipflag = 0;
+        tc::tma_store_wait_read();  // previous task's output staging has been read
+      }
       bar_compute();
       // ------------------------------------------------------ slices --
       for (int s = 0; s < C::SLICES; ++s, ++gs) {
@@ -305,9 +313,21 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         {
           const int i = tid >> 2, gq = tid & 3, cl = 8 * gq, cc0 = C::KS * s + cl;
           const bool live = i < len;
-          const float* gi = la + i * 32 + cl;
-          const float* gr = la + 32 * 32 + cl;
-          const float* bb = reinterpret_cast<const float*>(d + C::OFF_B) + i * 32 + cl;
+          // 8 consecutive fp32 values per thread, read as two float4 (scalar
+          // reads of 8 token rows 128 B apart would hit the same banks)
+          float gi[8], gr[8], bb[8];
+          {
+            const float4* g4 = reinterpret_cast<const float4*>(la + i * 32 + cl);
+            const float4* r4 = reinterpret_cast<const float4*>(la + 32 * 32 + cl);
+            const float4* b4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(d + C::OFF_B) + i * 32 + cl);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const float4 x = g4[hh], y = r4[hh], z = b4[hh];
+              gi[4 * hh] = x.x; gi[4 * hh + 1] = x.y; gi[4 * hh + 2] = x.z; gi[4 * hh + 3] = x.w;
+              gr[4 * hh] = y.x; gr[4 * hh + 1] = y.y; gr[4 * hh + 2] = y.z; gr[4 * hh + 3] = y.w;
+              bb[4 * hh] = z.x; bb[4 * hh + 1] = z.y; bb[4 * hh + 2] = z.z; bb[4 * hh + 3] = z.w;
+            }
+          }
           const uint4 kraw = *reinterpret_cast<const uint4*>(d + C::OFF_K + (i * 32 + cl) * 2);
           const uint4 qraw = *reinterpret_cast<const uint4*>(d + C::OFF_Q + (i * 32 + cl) * 2);
           const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
@@ -350,13 +370,29 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
           // Z = w * v for value channels vc0 .. vc0 + VS/4 - 1 (right after E~)
           constexpr int VPT = C::VS / 4;
           const int vl = VPT * gq, vc0 = C::VS * s + vl;
-          const float* ww = reinterpret_cast<const float*>(d + C::OFF_W) + i * C::VS + vl;
-          const __nv_bfloat16* vv = reinterpret_cast<const __nv_bfloat16*>(d + C::OFF_V) + i * C::VS + vl;
+          float ww[VPT];
+          uint32_t vw[VPT / 2];
+          {
+            const float4* w4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(d + C::OFF_W) + i * C::VS + vl);
+#pragma unroll
+            for (int hh = 0; hh < VPT / 4; ++hh) {
+              const float4 x = w4[hh];
+              ww[4 * hh] = x.x; ww[4 * hh + 1] = x.y; ww[4 * hh + 2] = x.z; ww[4 * hh + 3] = x.w;
+            }
+            const uint8_t* vsrc = d + C::OFF_V + (i * C::VS + vl) * 2;
+            if constexpr (VPT == 8) {
+              const uint4 x = *reinterpret_cast<const uint4*>(vsrc);
+              vw[0] = x.x; vw[1] = x.y; vw[2] = x.z; vw[3] = x.w;
+            } else {
+              const uint2 x = *reinterpret_cast<const uint2*>(vsrc);
+              vw[0] = x.x; vw[1] = x.y;
+            }
+          }
           uint32_t zw[VPT / 2];
 #pragma unroll
           for (int p = 0; p < VPT / 2; ++p) {
-            const float z0 = live ? ww[2 * p] * __bfloat162float(vv[2 * p]) : 0.f;
-            const float z1 = live ? ww[2 * p + 1] * __bfloat162float(vv[2 * p + 1]) : 0.f;
+            const float z0 = live ? ww[2 * p] * bf16_lo_f(vw[p]) : 0.f;
+            const float z1 = live ? ww[2 * p + 1] * bf16_hi_f(vw[p]) : 0.f;
             zw[p] = tc::pack_bf16(z0, z1);
           }
           uint8_t* zdst = sm + C::OFF_Z + (vc0 >> 6) * 8192 + sw_unit(i, (vc0 & 63) >> 3) + (vc0 & 7) * 2;
@@ -448,18 +484,34 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         float* X = XS + J * 256;
         for (int I = J + 1; I < 4; ++I) {
           float4 xa = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int kk = 16 * J; kk < 16 * I; ++kk) {
-            const float av = AS[(16 * I + r) * C::LDA + kk];
-            const float4 tv = *reinterpret_cast<const float4*>(TS + kk * C::LDA + 16 * J + 4 * cg);
-            xa.x = fmaf(av, tv.x, xa.x); xa.y = fmaf(av, tv.y, xa.y);
-            xa.z = fmaf(av, tv.z, xa.z); xa.w = fmaf(av, tv.w, xa.w);
+          for (int kb = J; kb < I; ++kb) {
+            const float* arow = AS + (16 * I + r) * C::LDA + 16 * kb;
+            const float* tcol = TS + (16 * kb) * C::LDA + 16 * J + 4 * cg;
+            float av[16];
+#pragma unroll
+            for (int m = 0; m < 16; m += 4) {
+              const float4 a4 = *reinterpret_cast<const float4*>(arow + m);
+              av[m] = a4.x; av[m + 1] = a4.y; av[m + 2] = a4.z; av[m + 3] = a4.w;
+            }
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              const float4 tv = *reinterpret_cast<const float4*>(tcol + m * C::LDA);
+              xa.x = fmaf(av[m], tv.x, xa.x); xa.y = fmaf(av[m], tv.y, xa.y);
+              xa.z = fmaf(av[m], tv.z, xa.z); xa.w = fmaf(av[m], tv.w, xa.w);
+            }
           }
           *reinterpret_cast<float4*>(X + r * 16 + 4 * cg) = xa;
           bar_pair(2 + J);
           float4 ta = make_float4(0.f, 0.f, 0.f, 0.f);
+          float tr[16];
+#pragma unroll
+          for (int m = 0; m < 16; m += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(TS + (16 * I + r) * C::LDA + 16 * I + m);
+            tr[m] = t4.x; tr[m + 1] = t4.y; tr[m + 2] = t4.z; tr[m + 3] = t4.w;
+          }
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            const float tv = TS[(16 * I + r) * C::LDA + 16 * I + m];
+            const float tv = tr[m];
             const float4 xv = *reinterpret_cast<const float4*>(X + m * 16 + 4 * cg);
             ta.x = fmaf(tv, xv.x, ta.x); ta.y = fmaf(tv, xv.y, ta.y);
             ta.z = fmaf(tv, xv.z, ta.z); ta.w = fmaf(tv, xv.w, ta.w);
@@ -474,9 +526,15 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       {
         const int i = tid >> 2, j0 = 16 * (tid & 3);
         uint32_t hw[8], lw[8];
+        float tv[16];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 t4 = *reinterpret_cast<const float4*>(TS + i * C::LDA + j0 + e);
+          tv[e] = t4.x; tv[e + 1] = t4.y; tv[e + 2] = t4.z; tv[e + 3] = t4.w;
+        }
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          const float x0 = TS[i * C::LDA + j0 + e], x1 = TS[i * C::LDA + j0 + e + 1];
+          const float x0 = tv[e], x1 = tv[e + 1];
           const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
           hw[e / 2] = tc::pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
           lw[e / 2] = tc::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
@@ -538,23 +596,28 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       }
       if (!tc::mbar_wait(mma3_done, ex & 1)) { alive = false; break; }
       // ------------------------------------------- epilogue 3: outputs --
+      // Results go to SW128 staging in the (now free) operand area and leave
+      // by TMA bulk stores, so every global write is a whole tile row.
       tc::tc_fence_after();
       {
         const int m = 32 * q + lane;  // key channel row of Mp / Nc
         // half 0: Mp columns 0..127; half 1: Nc columns 0..DV-1 (TMEM 128..)
         const int ncols = half == 0 ? 128 : DV;
+        uint8_t* stg = sm + (half == 0 ? C::OFF_SMP : C::OFF_SNC);
         for (int c0 = 0; c0 < ncols; c0 += 32) {
           uint32_t r[32], pw[16];
           tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0), r);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; e += 2) pw[e / 2] = tc::pack_bf16(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-          __nv_bfloat16* dst = half == 0 ? a.Mp + (tile * DK + m) * DK + c0 : a.Nc + (tile * DK + m) * DV + c0;
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          uint8_t* pnl = stg + (c0 >> 6) * 16384;
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu) d4[uu] = make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
+          for (int uu = 0; uu < 4; ++uu)
+            *reinterpret_cast<uint4*>(pnl + sw_unit(m, ((c0 & 63) >> 3) + uu)) =
+                make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
         }
         // token rows (M = 64 layout): half 0: Q_eff = Q~ - P W; half 1: O_part
+        uint8_t* stt = sm + (half == 0 ? C::OFF_SQE : C::OFF_SOP);
         for (int c0 = 0; c0 < ncols; c0 += 32) {
           uint32_t r[32], pw[16];
           tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_QO + 128 * half + c0), r);
@@ -570,22 +633,35 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
 #pragma unroll
               for (int e = 0; e < 32; e += 2) pw[e / 2] = tc::pack_bf16(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
             }
-            __nv_bfloat16* dst = half == 0 ? a.Qeff + (tile * kChunk + i_out) * DK + c0
-                                           : a.Opart + (tile * kChunk + i_out) * DV + c0;
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            uint8_t* pnl = stt + (c0 >> 6) * 8192;
 #pragma unroll
-            for (int uu = 0; uu < 4; ++uu) d4[uu] = make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
+            for (int uu = 0; uu < 4; ++uu)
+              *reinterpret_cast<uint4*>(pnl + sw_unit(i_out, ((c0 & 63) >> 3) + uu)) =
+                  make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
           }
         }
       }
+      tc::fence_async_smem();
       tc::tc_fence_before();
-      ++ex;
-      if (a.ready) {
-        __threadfence();
-        bar_compute();
-        if (tid == 0) tc::st_release_gpu(a.ready + tile, 1);
+      bar_compute();
+      if (tid == 0) {
+        tc::fence_async_global();  // Q~ went through global with generic stores
+        const int rk = (int)tile * DK, rt = (int)tile * kChunk;
+        for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP + p * 16384, 64 * p, rk);
+        for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC + p * 16384, 64 * p, rk);
+        for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Qe, sm + C::OFF_SQE + p * 8192, 64 * p, rt);
+        for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Op, sm + C::OFF_SOP + p * 8192, 64 * p, rt);
+        tc::tma_store_commit();
+        if (a.ready) {
+          // the factors must be in global memory before the flag says so
+          tc::tma_store_wait_all();
+          __threadfence();
+          tc::st_release_gpu(a.ready + tile, 1);
+        }
       }
+      ++ex;
     }
+    if (tid == 0) tc::tma_store_wait_all();
     if (!alive) {
       atomicExch(a.status, 8);
       vflag[0] = 1;
