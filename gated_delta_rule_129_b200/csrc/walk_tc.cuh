@@ -24,8 +24,10 @@
 //
 // Two TMA rings feed it: ring A (Mp, Q_eff; read only by the UMMAs, released
 // by tcgen05.commit) and ring B (the CTA's Nc and O_part columns and gamma;
-// read by the epilogue warps, released by them).  Warp 4 is the producer: one
-// lane issues the TMA loads and the UMMAs.  Every wait is bounded; on a
+// read by the epilogue warps, released by them).  Warp roles: 0-3 update the
+// state (the serial chain), 4-7 write the outputs, one lane of warp 8 issues
+// the UMMAs, one lane of warp 9 streams the rings by TMA, so nothing but the
+// state update sits between two D_S products.  Every wait is bounded; on a
 // timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT in the status word, drains
 // what it issued and exits.
 #pragma once
@@ -58,8 +60,9 @@ struct WalkTcCfg {
   static constexpr int DK = 128;
   static constexpr int NSL = 32;                 // value columns per CTA
   static constexpr int SLICES = DV / NSL;
-  static constexpr int EPI_WARPS = 4;
-  static constexpr int THREADS = EPI_WARPS * 32 + 32;
+  static constexpr int EPI_WARPS = 4;              // state warps 0-3, output warps 4-7
+  static constexpr int MMA_WARP = 8, TMA_WARP = 9;
+  static constexpr int THREADS = 10 * 32;
   static constexpr int STAGES_A = 3;
   static constexpr int STAGES_B = 4;
   static constexpr int MP_BYTES = DK * DK * 2;             // 32 KiB
@@ -103,7 +106,8 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
   uint64_t* s_done = emptyB + C::STAGES_B;   // D_S of the current chunk is ready
   uint64_t* o_done = s_done + 1;             // D_O of the current chunk is ready
   uint64_t* s_ready = o_done + 1;            // bf16 state operand written
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(s_ready + 1);
+  uint64_t* o_free = s_ready + 1;            // [2] D_O buffer read by the output warps
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(o_free + 2);
   int* s_abort = reinterpret_cast<int*>(tslot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -123,15 +127,17 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     }
     for (int s = 0; s < C::STAGES_B; ++s) {
       tc::mbar_init(&fullB[s], 1);
-      tc::mbar_init(&emptyB[s], C::EPI_WARPS);
+      tc::mbar_init(&emptyB[s], 2 * C::EPI_WARPS);  // state and output warps
     }
     tc::mbar_init(s_done, 1);
     tc::mbar_init(o_done, 1);
     tc::mbar_init(s_ready, C::EPI_WARPS);
+    tc::mbar_init(&o_free[0], C::EPI_WARPS);
+    tc::mbar_init(&o_free[1], C::EPI_WARPS);
     *s_abort = 0;
     tc::fence_mbar_init();
   }
-  if (warp == C::EPI_WARPS) {
+  if (warp == C::MMA_WARP) {
     tc::tmem_alloc(tslot, C::TMEM_COLS);
     tc::tmem_relinquish();
   }
@@ -141,7 +147,7 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
   const uint32_t tbase = *tslot;
 
   if (warp < C::EPI_WARPS) {
-    // ------------------------------------------------------------ epilogue --
+    // ----------------------------------------------------- state update --
     const int row = 32 * warp + lane;  // key channel = TMEM lane
     const size_t sbase = ((size_t)n * H + h) * DK * DV + (size_t)row * DV + col0;
     float S[NSL];
@@ -181,12 +187,11 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
 #pragma unroll
         for (int i = 0; i < NSL; i += 4) *reinterpret_cast<float4*>(cs + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
       }
-      if (!tc::mbar_wait(&fullB[sb], (j / C::STAGES_B) & 1) || !tc::mbar_wait(s_done, j & 1)) {
+      if (!tc::mbar_wait(&fullB[sb], (j / C::STAGES_B) & 1)) {
         set_timeout(a.status, s_abort);
         break;
       }
-      tc::tc_fence_after();
-      // state: S <- gamma * S - Mp S + Nc   (Nc row: 32 bf16 = 64 B)
+      // Nc row (32 bf16) and gamma before the product is ready
       const float gam = reinterpret_cast<const float*>(stB + C::NC_BYTES + C::OP_BYTES)[row];
       uint32_t ncw[NSL / 2];
 #pragma unroll
@@ -194,49 +199,23 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
         const uint4 t = reinterpret_cast<const uint4*>(stB + row * NSL * 2)[u];
         ncw[4 * u] = t.x; ncw[4 * u + 1] = t.y; ncw[4 * u + 2] = t.z; ncw[4 * u + 3] = t.w;
       }
-#pragma unroll
-      for (int m = 0; m < NSL / 16; ++m) {
-        float d[16];
-        tc::tmem_ld16(tc::tmem_addr(tbase, 32 * warp, 16 * m), d);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          const int e = 16 * m + i;
-          const uint32_t w2 = ncw[e / 2];
-          S[e] = fmaf(gam, S[e], bf16_lo_f(w2) - d[i]);
-          S[e + 1] = fmaf(gam, S[e + 1], bf16_hi_f(w2) - d[i + 1]);
-        }
-      }
-      store_state((j + 1) & 1);
-      // output of chunk j: token rows 16 warp + lane (lane < 16) of D_O[j & 1]
-      if (!tc::mbar_wait(o_done, j & 1)) {
+      if (!tc::mbar_wait(s_done, j & 1)) {
         set_timeout(a.status, s_abort);
         break;
       }
       tc::tc_fence_after();
-      const int t0 = s_begin + j * kChunk;
-      const int len = min(kChunk, s_end - t0);
-      const int i_tok = 16 * warp + lane;
-      const uint32_t ocol = (uint32_t)NSL * (1u + (j & 1));
+      // S <- gamma * S - Mp S + Nc
+      uint32_t d[32];
+      tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * warp, 0), d);
+      tc::tmem_wait_ld();
 #pragma unroll
-      for (int m = 0; m < NSL / 16; ++m) {
-        float d[16];
-        tc::tmem_ld16(tc::tmem_addr(tbase, 32 * warp, ocol + 16 * m), d);
-        tc::tmem_wait_ld();
-        if (lane < 16 && i_tok < len) {
-          const uint4* op = reinterpret_cast<const uint4*>(stB + C::NC_BYTES + i_tok * NSL * 2 + 32 * m);
-          const uint4 o0 = op[0], o1 = op[1];
-          const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-          uint32_t pw[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            pw[i] = tc::pack_bf16(a.scale * (d[2 * i] + bf16_lo_f(ow[i])), a.scale * (d[2 * i + 1] + bf16_hi_f(ow[i])));
-          uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)(t0 + i_tok) * H + h) * DV + col0 + 16 * m);
-          dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-          dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-        }
+      for (int e = 0; e < NSL; e += 2) {
+        const uint32_t w2 = ncw[e / 2];
+        S[e] = fmaf(gam, S[e], bf16_lo_f(w2) - __uint_as_float(d[e]));
+        S[e + 1] = fmaf(gam, S[e + 1], bf16_hi_f(w2) - __uint_as_float(d[e + 1]));
       }
-      tc::tc_fence_before();
+      // D_O(j-1) read sS[(j+1)&1]; it was issued before D_S(j), so it is done
+      store_state((j + 1) & 1);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
     }
@@ -245,43 +224,54 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
       for (int i = 0; i < NSL; i += 4)
         *reinterpret_cast<float4*>(a.hT + sbase + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
     }
-  } else if (lane == 0) {
-    // ------------------------------------------------- producer + UMMA issue --
-    tc::prefetch_tmap(&a.tm_Mp);
-    tc::prefetch_tmap(&a.tm_Qe);
-    tc::prefetch_tmap(&a.tm_Nc);
-    tc::prefetch_tmap(&a.tm_Op);
-    tc::prefetch_tmap(&a.tm_g);
-    auto loadA = [&](int j) {
-      const int st = j % C::STAGES_A;
-      const int c = c_begin + j;
-      uint8_t* dst = ringA + st * C::A_BYTES;
-      tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
-      const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
-      tc::tma_load_2d(dst, &a.tm_Mp, &fullA[st], 0, rm);
-      tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &fullA[st], 64, rm);
-      tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
-      tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
-    };
-    auto loadB = [&](int j) {
-      const int st = j % C::STAGES_B;
-      const int c = c_begin + j;
-      uint8_t* dst = ringB + st * C::B_STRIDE;
-      tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
-      tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
-      tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
-      tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
-    };
-    int loadedA = nch < C::STAGES_A ? nch : C::STAGES_A;
-    int loadedB = nch < C::STAGES_B ? nch : C::STAGES_B;
-    for (int j = 0; j < loadedA; ++j) loadA(j);
-    for (int j = 0; j < loadedB; ++j) loadB(j);
+  } else if (warp < 2 * C::EPI_WARPS) {
+    // ---------------------------------------------------------- outputs --
+    const int ow = warp - C::EPI_WARPS;   // TMEM lane quarter of this warp
+    const int i_tok = 16 * ow + lane;     // token row of D_O (M = 64 layout), lane < 16
+    for (int j = 0; j < nch; ++j) {
+      if (*reinterpret_cast<volatile int*>(s_abort)) break;
+      const int sb = j % C::STAGES_B;
+      const uint8_t* stB = ringB + sb * C::B_STRIDE;
+      if (!tc::mbar_wait(&fullB[sb], (j / C::STAGES_B) & 1) || !tc::mbar_wait(o_done, j & 1)) {
+        set_timeout(a.status, s_abort);
+        break;
+      }
+      tc::tc_fence_after();
+      uint32_t d[32];
+      tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * ow, (uint32_t)NSL * (1u + (j & 1))), d);
+      tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&o_free[j & 1]);
+      const int t0 = s_begin + j * kChunk;
+      const int len = min(kChunk, s_end - t0);
+      if (lane < 16 && i_tok < len) {
+        const uint4* op = reinterpret_cast<const uint4*>(stB + C::NC_BYTES + i_tok * NSL * 2);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)(t0 + i_tok) * H + h) * DV + col0);
+#pragma unroll
+        for (int u = 0; u < NSL / 8; ++u) {
+          const uint4 o4 = op[u];
+          const uint32_t ow4[4] = {o4.x, o4.y, o4.z, o4.w};
+          uint32_t pw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            pw[e] = tc::pack_bf16(a.scale * (__uint_as_float(d[8 * u + 2 * e]) + bf16_lo_f(ow4[e])),
+                                  a.scale * (__uint_as_float(d[8 * u + 2 * e + 1]) + bf16_hi_f(ow4[e])));
+          dst[u] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
+    }
+  } else if (warp == C::MMA_WARP && lane == 0) {
+    // --------------------------------------------------------- UMMA issue --
     constexpr uint32_t idS = tc::idesc_bf16(128, NSL, false, true);
     constexpr uint32_t idO = tc::idesc_bf16(64, NSL, false, true);
     int committed = 0;
     for (int j = 0; j < nch; ++j) {
       const int st = j % C::STAGES_A;
-      if (!tc::mbar_wait(&fullA[st], (j / C::STAGES_A) & 1) || !tc::mbar_wait(s_ready, j & 1)) {
+      const bool ok = tc::mbar_wait(&fullA[st], (j / C::STAGES_A) & 1) && tc::mbar_wait(s_ready, j & 1);
+      if (!ok) {
         set_timeout(a.status, s_abort);
         break;
       }
@@ -289,54 +279,84 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
       tc::tc_fence_after();
       const uint32_t mp = tc::smem_u32(ringA + st * C::A_BYTES);
       const uint32_t qe = mp + C::MP_BYTES;
-      const uint32_t sb = tc::smem_u32(sS + (j & 1) * C::S_BYTES);
+      const uint32_t sbuf = tc::smem_u32(sS + (j & 1) * C::S_BYTES);
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s) {
-        const uint64_t bd = tc::sdesc(sb + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
+        const uint64_t bd = tc::sdesc(sbuf + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
         const uint64_t ad = tc::sdesc(mp + (s / 4) * (DK * 128) + (s % 4) * 32, 16, 1024, tc::kLayoutSW128);
         tc::umma_f16(tbase, ad, bd, idS, s > 0);
       }
       tc::umma_commit(s_done);
+      // the output warps have read D_O(j-1): keeps every o_done waiter within
+      // one phase (and frees the D_O buffer D_O(j+1) will use)
+      if (j >= 1 && !tc::mbar_wait(&o_free[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
+        set_timeout(a.status, s_abort);
+        committed = j;
+        break;
+      }
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s) {
-        const uint64_t bd = tc::sdesc(sb + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
+        const uint64_t bd = tc::sdesc(sbuf + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
         const uint64_t ad = tc::sdesc(qe + (s / 4) * (kChunk * 128) + (s % 4) * 32, 16, 1024, tc::kLayoutSW128);
         tc::umma_f16(tbase + (uint32_t)NSL * (1u + (j & 1)), ad, bd, idO, s > 0);
       }
       tc::umma_commit(o_done);
       tc::umma_commit(&emptyA[st]);
       committed = j + 1;
-      // refill ring A with chunk j + STAGES_A once this chunk's UMMAs are done
-      if (loadedA < nch) {
-        if (!tc::mbar_wait(&emptyA[st], (j / C::STAGES_A) & 1)) {
+    }
+    // every issued UMMA has finished before TMEM is released
+    if (committed > 0) tc::mbar_wait(&emptyA[(committed - 1) % C::STAGES_A], ((committed - 1) / C::STAGES_A) & 1);
+    if (committed < nch && *reinterpret_cast<volatile int*>(s_abort)) tc::mbar_wait(s_done, committed & 1);
+  } else if (warp == C::TMA_WARP && lane == 0) {
+    // ------------------------------------------------------- TMA producer --
+    tc::prefetch_tmap(&a.tm_Mp);
+    tc::prefetch_tmap(&a.tm_Qe);
+    tc::prefetch_tmap(&a.tm_Nc);
+    tc::prefetch_tmap(&a.tm_Op);
+    tc::prefetch_tmap(&a.tm_g);
+    int loadedA = 0, loadedB = 0;
+    for (int j = 0; j < nch; ++j) {
+      if (*reinterpret_cast<volatile int*>(s_abort)) break;
+      const int c = c_begin + j;
+      {
+        const int st = j % C::STAGES_A;
+        if (j >= C::STAGES_A && !tc::mbar_wait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1)) {
           set_timeout(a.status, s_abort);
           break;
         }
-        loadA(loadedA++);
+        uint8_t* dst = ringA + st * C::A_BYTES;
+        tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
+        const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
+        tc::tma_load_2d(dst, &a.tm_Mp, &fullA[st], 0, rm);
+        tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &fullA[st], 64, rm);
+        tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
+        tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
+        ++loadedA;
       }
-      // refill ring B with chunk (j - 1) + STAGES_B once the epilogue is done with j - 1
-      if (j >= 1 && loadedB < nch) {
-        const int jb = j - 1;
-        if (!tc::mbar_wait(&emptyB[jb % C::STAGES_B], (jb / C::STAGES_B) & 1)) {
+      {
+        const int st = j % C::STAGES_B;
+        if (j >= C::STAGES_B && !tc::mbar_wait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1)) {
           set_timeout(a.status, s_abort);
           break;
         }
-        loadB(loadedB++);
+        uint8_t* dst = ringB + st * C::B_STRIDE;
+        tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
+        tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
+        tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
+        tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
+        ++loadedB;
       }
     }
-    // drain: issued loads have landed and issued UMMAs have finished before
-    // the CTA releases its shared and tensor memory
-    // (each stage holds at most one outstanding load, so waiting on the last
-    // load of every stage covers all of them, including ones already consumed)
+    // every issued load has landed before the CTA releases its shared memory
+    // (each stage holds at most one outstanding load)
     for (int j = loadedA > C::STAGES_A ? loadedA - C::STAGES_A : 0; j < loadedA; ++j)
       tc::mbar_wait(&fullA[j % C::STAGES_A], (j / C::STAGES_A) & 1);
     for (int j = loadedB > C::STAGES_B ? loadedB - C::STAGES_B : 0; j < loadedB; ++j)
       tc::mbar_wait(&fullB[j % C::STAGES_B], (j / C::STAGES_B) & 1);
-    if (committed > 0) tc::mbar_wait(&emptyA[(committed - 1) % C::STAGES_A], ((committed - 1) / C::STAGES_A) & 1);
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == C::EPI_WARPS) {
+  if (warp == C::MMA_WARP) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tbase, C::TMEM_COLS);
   }
