@@ -26,8 +26,8 @@
 // by tcgen05.commit) and ring B (the CTA's Nc and O_part columns and gamma;
 // read by the epilogue warps, released by them).  Warp roles: 0-3 update the
 // state (the serial chain), 4-7 write the outputs, one lane of warp 8 issues
-// the UMMAs, one lane of warp 9 streams the rings by TMA, so nothing but the
-// state update sits between two D_S products.  Every wait is bounded; on a
+// the UMMAs, one lane each of warps 9 and 10 streams ring A and ring B by TMA,
+// so nothing but the state update sits between two D_S products.  Every wait is bounded; on a
 // timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT in the status word, drains
 // what it issued and exits.
 #pragma once
@@ -61,8 +61,8 @@ struct WalkTcCfg {
   static constexpr int NSL = 32;                 // value columns per CTA
   static constexpr int SLICES = DV / NSL;
   static constexpr int EPI_WARPS = 4;              // state warps 0-3, output warps 4-7
-  static constexpr int MMA_WARP = 8, TMA_WARP = 9;
-  static constexpr int THREADS = 10 * 32;
+  static constexpr int MMA_WARP = 8, TMA_A_WARP = 9, TMA_B_WARP = 10;
+  static constexpr int THREADS = 11 * 32;
   static constexpr int STAGES_A = 3;
   static constexpr int STAGES_B = 4;
   static constexpr int MP_BYTES = DK * DK * 2;             // 32 KiB
@@ -267,6 +267,8 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     // --------------------------------------------------------- UMMA issue --
     constexpr uint32_t idS = tc::idesc_bf16(128, NSL, false, true);
     constexpr uint32_t idO = tc::idesc_bf16(64, NSL, false, true);
+    const uint64_t mp_d0 = tc::sdesc(tc::smem_u32(ringA), 16, 1024, tc::kLayoutSW128);
+    const uint64_t sb_d0 = tc::sdesc(tc::smem_u32(sS), C::S_LBO, 128, tc::kLayoutNone);
     int committed = 0;
     for (int j = 0; j < nch; ++j) {
       const int st = j % C::STAGES_A;
@@ -277,15 +279,15 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
       }
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       tc::tc_fence_after();
-      const uint32_t mp = tc::smem_u32(ringA + st * C::A_BYTES);
-      const uint32_t qe = mp + C::MP_BYTES;
-      const uint32_t sbuf = tc::smem_u32(sS + (j & 1) * C::S_BYTES);
+      // descriptors: the start address sits in the low bits (16-byte units),
+      // so a K-step is a 64-bit add of (byte offset >> 4)
+      const uint64_t mp_d = mp_d0 + (uint64_t)((st * C::A_BYTES) >> 4);
+      const uint64_t qe_d = mp_d + (uint64_t)(C::MP_BYTES >> 4);
+      const uint64_t sb_d = sb_d0 + (uint64_t)(((j & 1) * C::S_BYTES) >> 4);
 #pragma unroll
-      for (int s = 0; s < DK / 16; ++s) {
-        const uint64_t bd = tc::sdesc(sbuf + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
-        const uint64_t ad = tc::sdesc(mp + (s / 4) * (DK * 128) + (s % 4) * 32, 16, 1024, tc::kLayoutSW128);
-        tc::umma_f16(tbase, ad, bd, idS, s > 0);
-      }
+      for (int s = 0; s < DK / 16; ++s)
+        tc::umma_f16(tbase, mp_d + (uint64_t)(((s / 4) * (DK * 128) + (s % 4) * 32) >> 4),
+                     sb_d + (uint64_t)((s * 2 * C::S_LBO) >> 4), idS, s > 0);
       tc::umma_commit(s_done);
       // the output warps have read D_O(j-1): keeps every o_done waiter within
       // one phase (and frees the D_O buffer D_O(j+1) will use)
@@ -295,11 +297,10 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
         break;
       }
 #pragma unroll
-      for (int s = 0; s < DK / 16; ++s) {
-        const uint64_t bd = tc::sdesc(sbuf + s * 2 * C::S_LBO, C::S_LBO, 128, tc::kLayoutNone);
-        const uint64_t ad = tc::sdesc(qe + (s / 4) * (kChunk * 128) + (s % 4) * 32, 16, 1024, tc::kLayoutSW128);
-        tc::umma_f16(tbase + (uint32_t)NSL * (1u + (j & 1)), ad, bd, idO, s > 0);
-      }
+      for (int s = 0; s < DK / 16; ++s)
+        tc::umma_f16(tbase + (uint32_t)NSL * (1u + (j & 1)),
+                     qe_d + (uint64_t)(((s / 4) * (kChunk * 128) + (s % 4) * 32) >> 4),
+                     sb_d + (uint64_t)((s * 2 * C::S_LBO) >> 4), idO, s > 0);
       tc::umma_commit(o_done);
       tc::umma_commit(&emptyA[st]);
       committed = j + 1;
@@ -307,51 +308,52 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     // every issued UMMA has finished before TMEM is released
     if (committed > 0) tc::mbar_wait(&emptyA[(committed - 1) % C::STAGES_A], ((committed - 1) / C::STAGES_A) & 1);
     if (committed < nch && *reinterpret_cast<volatile int*>(s_abort)) tc::mbar_wait(s_done, committed & 1);
-  } else if (warp == C::TMA_WARP && lane == 0) {
-    // ------------------------------------------------------- TMA producer --
+  } else if (warp == C::TMA_A_WARP && lane == 0) {
+    // ------------------------------------------------ ring A producer (TMA) --
     tc::prefetch_tmap(&a.tm_Mp);
     tc::prefetch_tmap(&a.tm_Qe);
-    tc::prefetch_tmap(&a.tm_Nc);
-    tc::prefetch_tmap(&a.tm_Op);
-    tc::prefetch_tmap(&a.tm_g);
-    int loadedA = 0, loadedB = 0;
+    int loaded = 0;
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
-      const int c = c_begin + j;
-      {
-        const int st = j % C::STAGES_A;
-        if (j >= C::STAGES_A && !tc::mbar_wait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1)) {
-          set_timeout(a.status, s_abort);
-          break;
-        }
-        uint8_t* dst = ringA + st * C::A_BYTES;
-        tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
-        const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
-        tc::tma_load_2d(dst, &a.tm_Mp, &fullA[st], 0, rm);
-        tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &fullA[st], 64, rm);
-        tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
-        tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
-        ++loadedA;
+      const int c = c_begin + j, st = j % C::STAGES_A;
+      if (j >= C::STAGES_A && !tc::mbar_wait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1)) {
+        set_timeout(a.status, s_abort);
+        break;
       }
-      {
-        const int st = j % C::STAGES_B;
-        if (j >= C::STAGES_B && !tc::mbar_wait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1)) {
-          set_timeout(a.status, s_abort);
-          break;
-        }
-        uint8_t* dst = ringB + st * C::B_STRIDE;
-        tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
-        tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
-        tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
-        tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
-        ++loadedB;
-      }
+      uint8_t* dst = ringA + st * C::A_BYTES;
+      tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
+      const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
+      tc::tma_load_2d(dst, &a.tm_Mp, &fullA[st], 0, rm);
+      tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &fullA[st], 64, rm);
+      tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
+      tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
+      ++loaded;
     }
     // every issued load has landed before the CTA releases its shared memory
     // (each stage holds at most one outstanding load)
-    for (int j = loadedA > C::STAGES_A ? loadedA - C::STAGES_A : 0; j < loadedA; ++j)
+    for (int j = loaded > C::STAGES_A ? loaded - C::STAGES_A : 0; j < loaded; ++j)
       tc::mbar_wait(&fullA[j % C::STAGES_A], (j / C::STAGES_A) & 1);
-    for (int j = loadedB > C::STAGES_B ? loadedB - C::STAGES_B : 0; j < loadedB; ++j)
+  } else if (warp == C::TMA_B_WARP && lane == 0) {
+    // ------------------------------------------------ ring B producer (TMA) --
+    tc::prefetch_tmap(&a.tm_Nc);
+    tc::prefetch_tmap(&a.tm_Op);
+    tc::prefetch_tmap(&a.tm_g);
+    int loaded = 0;
+    for (int j = 0; j < nch; ++j) {
+      if (*reinterpret_cast<volatile int*>(s_abort)) break;
+      const int c = c_begin + j, st = j % C::STAGES_B;
+      if (j >= C::STAGES_B && !tc::mbar_wait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1)) {
+        set_timeout(a.status, s_abort);
+        break;
+      }
+      uint8_t* dst = ringB + st * C::B_STRIDE;
+      tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
+      tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
+      tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
+      tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
+      ++loaded;
+    }
+    for (int j = loaded > C::STAGES_B ? loaded - C::STAGES_B : 0; j < loaded; ++j)
       tc::mbar_wait(&fullB[j % C::STAGES_B], (j / C::STAGES_B) & 1);
   }
   tc::tc_fence_before();
