@@ -281,6 +281,7 @@ def run_ours(args, rank, world, local):
     barrier_sync(world)
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / ne, world)
 
+    decode = measure_decode(dev, stream, flush) if rank == 0 else None
     if rank != 0:
         return
     hbm, tflops, src = peaks()
@@ -311,12 +312,48 @@ def run_ours(args, rank, world, local):
     }
     clk = sampler.summary() if sampler else None
     line["clocks"] = clk
+    if decode:
+        decode["roofline"] = {"bound": "hbm", "achieved": decode["gbs"], "peak": hbm, "unit": "GB/s",
+                              "frac": decode["gbs"] / hbm}
+        line["decode_step"] = decode
     if world == 1 and not args.no_cpu_baseline:
         tps, cores, t_tok, dt = cpu_oracle_sample(x, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"fp64 C oracle, tokens [0,{t_tok}) of all 16 heads "
                                           f"({dt:.1f} s)"}
     print(json.dumps(line), flush=True)
+
+
+def measure_decode(dev, stream, flush, reps=20):
+    """gdn2_recurrent_step on the 256-state decode batch (B=256, H=16,
+    dk=dv=128, bf16 q/k/v/out, fp32 gates and states): its compulsory traffic
+    is one read and one write of every fp32 state (2 x 256 x 16 x 128 x 128 x
+    4 B) plus the token vectors."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    from workloads import decode_inputs
+    di = decode_inputs(B=256, H=16, dk=128, dv=128, io="bf16", seed=41)
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
+    bf, f32 = torch.bfloat16, torch.float32
+    args = (t(di.q, bf), t(di.k, bf), t(di.v, bf), t(di.log_alpha, f32), t(di.b, f32), t(di.w, f32))
+    state = t(di.state, f32)
+    out = torch.empty((256, 16, 128), dtype=bf, device=dev)
+    nbytes = 2 * state.numel() * 4 + sum(a.numel() * a.element_size() for a in args) + out.numel() * 2
+    for _ in range(3):
+        gdn2.recurrent_step(*args, di.scale, state, out=out, stream=stream)
+    tot = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn2.recurrent_step(*args, di.scale, state, out=out, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    us = tot / reps * 1e3
+    return {"workload": "decode B=256 H=16 dk=dv=128 (one token per state)", "us": us,
+            "tokens_per_s": 256 / (us * 1e-6), "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9}
 
 
 def main():
