@@ -10,6 +10,8 @@ Public functions mirror the C entry points:
 * :func:`chunk_fwd`        -- ``gdn2_chunk_fwd``
 * :func:`chunk_prep`       -- ``gdn2_chunk_prep`` (gate prep + intra-chunk WY)
 * :func:`chunk_walk`       -- ``gdn2_chunk_walk`` (state walk + output)
+* :func:`chunk_plan`, :func:`chunk_fused` -- ``gdn2_chunk_plan``, ``gdn2_chunk_fused``
+  (the fused prep + walk launch on its own, for timing and tests)
 * :func:`recurrent_step`   -- ``gdn2_recurrent_step`` (one decode token)
 * :func:`workspace_size`, :func:`workspace_layout`, :func:`status_string`
 """
@@ -19,7 +21,8 @@ import ctypes
 import os
 import threading
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "chunk_prep", "chunk_walk", "recurrent_step", "workspace_size",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
+           "recurrent_step", "workspace_size",
            "workspace_layout", "status_string", "GDN2Error", "lib_path", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,8 +38,8 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_NULL", 2: "GDN2_ERR_SHAPE", 3: "GDN2_ERR_DT
           7: "GDN2_ERR_CUDA", 8: "GDN2_ERR_DEVICE_TIMEOUT", 9: "GDN2_ERR_UNSUPPORTED"}
 
 EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_fwd_noalloc",
-            "gdn2_chunk_prep",
-            "gdn2_chunk_walk", "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version")
+            "gdn2_chunk_prep", "gdn2_chunk_walk", "gdn2_chunk_plan", "gdn2_chunk_fused",
+            "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version")
 
 
 class GDN2Error(RuntimeError):
@@ -60,7 +63,8 @@ class WsLayout(ctypes.Structure):
                 ("off_Qeff", ctypes.c_size_t), ("off_Opart", ctypes.c_size_t),
                 ("off_gamma_last", ctypes.c_size_t), ("off_Mp", ctypes.c_size_t),
                 ("off_Nc", ctypes.c_size_t), ("off_chunk_offsets", ctypes.c_size_t),
-                ("off_status", ctypes.c_size_t), ("off_fix", ctypes.c_size_t)]
+                ("off_status", ctypes.c_size_t), ("off_fix", ctypes.c_size_t),
+                ("off_sync", ctypes.c_size_t)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -94,6 +98,10 @@ def load_library():
         lib.gdn2_chunk_prep.restype = i
         lib.gdn2_chunk_walk.argtypes = [dp, f, vp, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_walk.restype = i
+        lib.gdn2_chunk_plan.argtypes = [dp, vp, vp]
+        lib.gdn2_chunk_plan.restype = i
+        lib.gdn2_chunk_fused.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
+        lib.gdn2_chunk_fused.restype = i
         lib.gdn2_recurrent_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp]
         lib.gdn2_recurrent_step.restype = i
         lib.gdn2_status_string.argtypes = [i]
@@ -208,6 +216,31 @@ def chunk_fwd(q, k, v, log_alpha, b, w, scale=None, h0=None, cu_seqlens=None, *,
                                        _ptr(b), _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens),
                                        _ptr(out), _ptr(hT), _stream(stream))
     _check(st, "gdn2_chunk_fwd")
+    return out, hT
+
+
+def chunk_plan(shape, dtype, workspace, cu_seqlens=None, *, stream=None):
+    """``gdn2_chunk_plan`` for ``shape = (B, T, H, dk, dv)`` into ``workspace``."""
+    B, T, H, dk, dv = shape
+    ns = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    d = make_desc(B, T, H, dk, dv, _io_of(dtype), ns, workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size())
+    _check(load_library().gdn2_chunk_plan(ctypes.byref(d), _ptr(cu_seqlens), _stream(stream)), "gdn2_chunk_plan")
+
+
+def chunk_fused(q, k, v, log_alpha, b, w, scale, workspace, h0=None, cu_seqlens=None, *, out, hT=None,
+                stream=None):
+    """``gdn2_chunk_fused``: the fused prep + walk launch alone (run
+    :func:`chunk_plan` on the same workspace first).  Raises ``GDN2Error``
+    (``GDN2_ERR_UNSUPPORTED``) when the problem does not take the fused path."""
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    _need_contig(q, k, v, log_alpha, b, w, h0, cu_seqlens)
+    d = make_desc(B, T, H, dk, dv, _io_of(q.dtype), ns, workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_fused(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                                         _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens), _ptr(out), _ptr(hT),
+                                         _stream(stream))
+    _check(st, "gdn2_chunk_fused")
     return out, hT
 
 

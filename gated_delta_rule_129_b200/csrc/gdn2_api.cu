@@ -19,6 +19,7 @@
 #include "plan.cuh"
 #include "prep_simt.cuh"
 #include "prep_tc.cuh"
+#include "fused_tc.cuh"
 #include "tmap.cuh"
 #include "walk_simt.cuh"
 #include "walk_tc.cuh"
@@ -89,6 +90,7 @@ gdn2_status make_layout(const gdn2_desc* d, bool packed, Layout* out) {
   L.off_chunk_offsets = off; off = align_up(off + (size_t)(N + 1) * sizeof(int32_t));
   L.off_status = off;     off = align_up(off + sizeof(int32_t));
   L.off_fix = off;        off = align_up(off + (wy ? 0 : (size_t)(1 + (size_t)max_chunks * d->H) * sizeof(int32_t)));
+  L.off_sync = off;       off = align_up(off + (wy ? 0 : (size_t)(2 + (size_t)max_chunks * d->H) * sizeof(int32_t)));
   L.total_bytes = off;
   out->N = N;
   return GDN2_OK;
@@ -121,10 +123,12 @@ gdn2::SeqMap seq_map(const gdn2_desc* d, const Layout& L, const int32_t* cu) {
 }
 
 gdn2_status launch_plan(const gdn2_desc* d, const Layout& L, const int32_t* cu, cudaStream_t s) {
+  const bool affine = L.l.factor_set == 1;
   gdn2::plan_kernel<<<1, gdn2::kPlanThreads, 0, s>>>(
       cu, L.N, d->T, d->B * d->T, at<int32_t>(d->workspace, L.l.off_chunk_offsets),
       at<int32_t>(d->workspace, L.l.off_status), (int)GDN2_ERR_SEQLENS,
-      L.l.factor_set == 1 ? at<int32_t>(d->workspace, L.l.off_fix) : nullptr);
+      affine ? at<int32_t>(d->workspace, L.l.off_fix) : nullptr,
+      affine ? at<int32_t>(d->workspace, L.l.off_sync) : nullptr, affine ? 2 + L.l.max_chunks * d->H : 0);
   return launch_status();
 }
 
@@ -132,13 +136,11 @@ gdn2_status launch_plan(const gdn2_desc* d, const Layout& L, const int32_t* cu, 
 // bf16 I/O with dk = 128: gate prep, intra-chunk WY and the affine state map
 // on the tensor cores.
 template <int DV>
-gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
-                           const float* la, const float* b, const float* w, const int32_t* cu, cudaStream_t s) {
+gdn2_status fill_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
+                         const float* la, const float* b, const float* w, const int32_t* cu, gdn2::PrepTcArgs& a) {
   using C = gdn2::PrepTcCfg<DV>;
-  gdn2::PrepTcArgs a;
   std::memset(&a, 0, sizeof(a));
   const uint64_t T_total = (uint64_t)d->B * d->T;
-  if (T_total == 0) return GDN2_OK;
   const uint64_t dk[3] = {128, (uint64_t)d->H, T_total}, dv[3] = {(uint64_t)DV, (uint64_t)d->H, T_total};
   const uint64_t sk2[2] = {128 * 2, (uint64_t)d->H * 128 * 2}, sk4[2] = {128 * 4, (uint64_t)d->H * 128 * 4};
   const uint64_t sv2[2] = {(uint64_t)DV * 2, (uint64_t)d->H * DV * 2}, sv4[2] = {(uint64_t)DV * 4, (uint64_t)d->H * DV * 4};
@@ -146,8 +148,10 @@ gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, c
   const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const CUtensorMapSwizzle NS = CU_TENSOR_MAP_SWIZZLE_NONE;
   if (!gdn2::make_tmap(&a.tm_q, q, BF, 3, dk, sk2, bk, NS) || !gdn2::make_tmap(&a.tm_k, k, BF, 3, dk, sk2, bk, NS) ||
-      !gdn2::make_tmap(&a.tm_v, v, BF, 3, dv, sv2, bv, NS) || !gdn2::make_tmap(&a.tm_la, la, F32, 3, dk, sk4, bk, NS) ||
-      !gdn2::make_tmap(&a.tm_b, b, F32, 3, dk, sk4, bk, NS) || !gdn2::make_tmap(&a.tm_w, w, F32, 3, dv, sv4, bv, NS))
+      !gdn2::make_tmap(&a.tm_v, v, BF, 3, dv, sv2, bv, NS) ||
+      !gdn2::make_tmap(&a.tm_la, la, F32, 3, dk, sk4, bk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !gdn2::make_tmap(&a.tm_b, b, F32, 3, dk, sk4, bk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !gdn2::make_tmap(&a.tm_w, w, F32, 3, dv, sv4, bv, C::W_SWIZZLED ? CU_TENSOR_MAP_SWIZZLE_128B : NS))
     return GDN2_ERR_CUDA;
   {
     const long long rows_k = (long long)std::max(L.l.max_chunks, 1) * d->H * 128;
@@ -174,6 +178,17 @@ gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, c
   a.status = at<int32_t>(d->workspace, L.l.off_status);
   a.ready = nullptr;
   a.task_counter = nullptr;
+  return GDN2_OK;
+}
+
+template <int DV>
+gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
+                           const float* la, const float* b, const float* w, const int32_t* cu, cudaStream_t s) {
+  using C = gdn2::PrepTcCfg<DV>;
+  if ((uint64_t)d->B * d->T == 0) return GDN2_OK;
+  gdn2::PrepTcArgs a;
+  gdn2_status st = fill_prep_tc<DV>(d, L, q, k, v, la, b, w, cu, a);
+  if (st != GDN2_OK) return st;
   auto kern = gdn2::prep_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;
@@ -187,9 +202,9 @@ gdn2_status launch_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, c
 
 // ---------------------------------------------------------------- prep ----
 template <int DK, int DV, typename IO, typename FT>
-gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, const void* k,
-                          const void* v, const float* la, const float* b, const float* w,
-                          const int32_t* cu, cudaStream_t s) {
+gdn2::PrepArgs<IO, FT> prep_args(const gdn2_desc* d, const Layout& L, const void* q, const void* k,
+                                 const void* v, const float* la, const float* b, const float* w,
+                                 const int32_t* cu) {
   gdn2::PrepArgs<IO, FT> a;
   a.q = static_cast<const IO*>(q);
   a.k = static_cast<const IO*>(k);
@@ -207,19 +222,36 @@ gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, co
   a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
   a.Mp = at<FT>(d->workspace, L.l.off_Mp);
   a.Nc = at<FT>(d->workspace, L.l.off_Nc);
+  return a;
+}
+
+// Exact redo of the chunks the tensor-core prep handed back (the kernel
+// reads the list's length on the device; an empty list costs one launch).
+template <int DK, int DV, typename IO, typename FT>
+gdn2_status launch_fixup(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
+                         const float* la, const float* b, const float* w, const int32_t* cu, cudaStream_t s) {
+  const auto a = prep_args<DK, DV, IO, FT>(d, L, q, k, v, la, b, w, cu);
+  constexpr size_t smem = gdn2::prep_simt_smem_bytes<DK, DV>();
+  auto fix = gdn2::prep_fixup_kernel<DK, DV, IO, FT>;
+  if (cudaFuncSetAttribute(fix, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  const int grid = std::min(L.l.max_chunks * d->H, sm_count());
+  fix<<<grid, gdn2::kPrepSimtThreads, smem, s>>>(a, at<const int32_t>(d->workspace, L.l.off_fix));
+  return launch_status();
+}
+
+template <int DK, int DV, typename IO, typename FT>
+gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, const void* k,
+                          const void* v, const float* la, const float* b, const float* w,
+                          const int32_t* cu, cudaStream_t s) {
+  const auto a = prep_args<DK, DV, IO, FT>(d, L, q, k, v, la, b, w, cu);
   if (L.l.max_chunks == 0) return GDN2_OK;
   constexpr size_t smem = gdn2::prep_simt_smem_bytes<DK, DV>();
   if constexpr (DK == 128 && std::is_same<IO, bf16>::value) {
     if (L.l.factor_set == 1) {
       const gdn2_status st = launch_prep_tc<DV>(d, L, q, k, v, la, b, w, cu, s);
       if (st != GDN2_OK) return st;
-      // exact redo of the chunks the tensor-core prep handed back
-      auto fix = gdn2::prep_fixup_kernel<DK, DV, IO, FT>;
-      if (cudaFuncSetAttribute(fix, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return GDN2_ERR_CUDA;
-      const int grid = std::min(L.l.max_chunks * d->H, 148);
-      fix<<<grid, gdn2::kPrepSimtThreads, smem, s>>>(a, at<const int32_t>(d->workspace, L.l.off_fix));
-      return launch_status();
+      return launch_fixup<DK, DV, IO, FT>(d, L, q, k, v, la, b, w, cu, s);
     }
   }
   auto kern = L.l.factor_set == 1 ? gdn2::prep_simt_kernel<DK, DV, IO, FT, true>
@@ -234,10 +266,9 @@ gdn2_status launch_prep_t(const gdn2_desc* d, const Layout& L, const void* q, co
 // ------------------------------------------------------- walk (tensor) ----
 // bf16 I/O with dk = 128: the affine walk on the tensor cores.
 template <int DV>
-gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const float* h0,
-                           const int32_t* cu, void* out, float* hT, float* chunk_states, cudaStream_t s) {
+gdn2_status fill_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const float* h0, const int32_t* cu,
+                         void* out, float* hT, float* chunk_states, gdn2::WalkTcArgs& a) {
   using C = gdn2::WalkTcCfg<DV>;
-  gdn2::WalkTcArgs a;
   std::memset(&a, 0, sizeof(a));
   const long long rows_mp = (long long)std::max(L.l.max_chunks, 1) * d->H * 128;
   if (rows_mp >= (1ll << 31)) return GDN2_ERR_SHAPE;  // TMA coordinates are int32
@@ -246,11 +277,13 @@ gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, con
   const uint64_t d_mp[2] = {128, rows_k}, d_qe[2] = {128, rows_t};
   const uint64_t d_nc[2] = {(uint64_t)DV, rows_k}, d_op[2] = {(uint64_t)DV, rows_t}, d_g[2] = {128, rows_g};
   const uint64_t st_k[1] = {256}, st_v[1] = {(uint64_t)DV * 2}, st_g[1] = {512};
-  const uint32_t b_mp[2] = {64, 128}, b_qe[2] = {64, 64}, b_nc[2] = {32, 128}, b_op[2] = {32, 64}, b_g[2] = {128, 1};
-  if (!gdn2::make_tmap(&a.tm_Mp, at<void>(d->workspace, L.l.off_Mp), BF, 2, d_mp, st_k, b_mp, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !gdn2::make_tmap(&a.tm_Qe, at<void>(d->workspace, L.l.off_Qeff), BF, 2, d_qe, st_k, b_qe, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !gdn2::make_tmap(&a.tm_Nc, at<void>(d->workspace, L.l.off_Nc), BF, 2, d_nc, st_v, b_nc, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !gdn2::make_tmap(&a.tm_Op, at<void>(d->workspace, L.l.off_Opart), BF, 2, d_op, st_v, b_op, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  const uint32_t b_mp[2] = {64, 128}, b_qe[2] = {64, 64}, b_nc[2] = {(uint32_t)C::NSL, 128},
+                 b_op[2] = {(uint32_t)C::NSL, 64}, b_g[2] = {128, 1};
+  const CUtensorMapSwizzle SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!gdn2::make_tmap(&a.tm_Mp, at<void>(d->workspace, L.l.off_Mp), BF, 2, d_mp, st_k, b_mp, SW) ||
+      !gdn2::make_tmap(&a.tm_Qe, at<void>(d->workspace, L.l.off_Qeff), BF, 2, d_qe, st_k, b_qe, SW) ||
+      !gdn2::make_tmap(&a.tm_Nc, at<void>(d->workspace, L.l.off_Nc), BF, 2, d_nc, st_v, b_nc, SW) ||
+      !gdn2::make_tmap(&a.tm_Op, at<void>(d->workspace, L.l.off_Opart), BF, 2, d_op, st_v, b_op, SW) ||
       !gdn2::make_tmap(&a.tm_g, at<void>(d->workspace, L.l.off_gamma_last), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d_g, st_g,
                        b_g, CU_TENSOR_MAP_SWIZZLE_NONE))
     return GDN2_ERR_CUDA;
@@ -262,7 +295,19 @@ gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, con
   a.hT = hT;
   a.chunk_states = chunk_states;
   a.status = at<int32_t>(d->workspace, L.l.off_status);
+  return GDN2_OK;
+}
+
+template <int DV>
+gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const float* h0,
+                           const int32_t* cu, void* out, float* hT, float* chunk_states, cudaStream_t s,
+                           const int* gate = nullptr) {
+  using C = gdn2::WalkTcCfg<DV>;
   if (L.N == 0) return GDN2_OK;
+  gdn2::WalkTcArgs a;
+  gdn2_status st = fill_walk_tc<DV>(d, L, scale, h0, cu, out, hT, chunk_states, a);
+  if (st != GDN2_OK) return st;
+  a.gate = gate;
   auto kern = gdn2::walk_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;
@@ -303,6 +348,51 @@ gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, cons
   if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
   kern<<<(unsigned)blocks, gdn2::kWalkSimtThreads, smem, s>>>(a);
   return launch_status();
+}
+
+// ------------------------------------------------------------- fused ----
+// Prep and walk in one launch when the walk needs few CTAs (long sequences,
+// few heads); then the fixup of handed-back chunks and, only if one of them
+// cut the walk short, the walk again.
+template <int DV>
+bool fused_fits(const gdn2_desc* d, const Layout& L) {
+  const long long n_walk = (long long)L.N * d->H * gdn2::WalkTcCfg<DV>::SLICES;
+  return L.l.factor_set == 1 && L.N > 0 && (long long)d->B * d->T > 0 &&
+         n_walk + gdn2::FusedTcCfg<DV>::MIN_PREP_CTAS <= sm_count();
+}
+
+template <int DV>
+gdn2_status launch_fused_tc(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
+                            const float* la, const float* b, const float* w, const int32_t* cu, float scale,
+                            const float* h0, void* out, float* hT, cudaStream_t s) {
+  using F = gdn2::FusedTcCfg<DV>;
+  gdn2::PrepTcArgs pa;
+  gdn2::WalkTcArgs wa;
+  gdn2_status st = fill_prep_tc<DV>(d, L, q, k, v, la, b, w, cu, pa);
+  if (st != GDN2_OK) return st;
+  if ((st = fill_walk_tc<DV>(d, L, scale, h0, cu, out, hT, nullptr, wa)) != GDN2_OK) return st;
+  int* sync = at<int>(d->workspace, L.l.off_sync);
+  pa.task_counter = sync;
+  pa.ready = sync + 2;
+  wa.ready = sync + 2;
+  wa.redo = sync + 1;
+  const int n_sm = sm_count();
+  const int n_walk = L.N * d->H * gdn2::WalkTcCfg<DV>::SLICES;
+  auto kern = gdn2::fused_tc_kernel<DV>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  kern<<<n_sm, F::THREADS, F::SMEM, s>>>(pa, wa, n_sm - n_walk);
+  return launch_status();
+}
+
+template <int DV>
+gdn2_status launch_fused_full(const gdn2_desc* d, const Layout& L, const void* q, const void* k, const void* v,
+                              const float* la, const float* b, const float* w, const int32_t* cu, float scale,
+                              const float* h0, void* out, float* hT, cudaStream_t s) {
+  gdn2_status st = launch_fused_tc<DV>(d, L, q, k, v, la, b, w, cu, scale, h0, out, hT, s);
+  if (st != GDN2_OK) return st;
+  if ((st = launch_fixup<128, DV, bf16, bf16>(d, L, q, k, v, la, b, w, cu, s)) != GDN2_OK) return st;
+  return launch_walk_tc<DV>(d, L, scale, h0, cu, out, hT, nullptr, s, at<int>(d->workspace, L.l.off_sync) + 1);
 }
 
 // ----------------------------------------------------------- dispatch ----
@@ -447,9 +537,46 @@ gdn2_status gdn2_chunk_fwd(const gdn2_desc* desc, const void* q, const void* k, 
   if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return GDN2_ERR_ALIGN;
   if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
   if ((st = launch_plan(desc, L, cu_seqlens, stream)) != GDN2_OK) return st;
+  if (desc->io == GDN2_IO_BF16 && desc->dk == 128) {
+    if (desc->dv == 128 && fused_fits<128>(desc, L))
+      return launch_fused_full<128>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
+    if (desc->dv == 64 && fused_fits<64>(desc, L))
+      return launch_fused_full<64>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
+  }
   if ((st = dispatch<PrepOp>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, stream)) != GDN2_OK)
     return st;
   return dispatch<WalkOp>(desc, L, scale, h0, cu_seqlens, out, hT, (float*)nullptr, stream);
+}
+
+gdn2_status gdn2_chunk_plan(const gdn2_desc* desc, const int32_t* cu_seqlens, cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  return launch_plan(desc, L, cu_seqlens, stream);
+}
+
+gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                             const float* log_alpha, const float* b, const float* w, float scale,
+                             const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                             cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  const long long tokens = (long long)desc->B * desc->T;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, tokens)) != GDN2_OK) return st;
+  if (!out && tokens > 0) return GDN2_ERR_NULL;
+  if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if (desc->io == GDN2_IO_BF16 && desc->dk == 128) {
+    if (desc->dv == 128 && fused_fits<128>(desc, L))
+      return launch_fused_tc<128>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
+    if (desc->dv == 64 && fused_fits<64>(desc, L))
+      return launch_fused_tc<64>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
+  }
+  return GDN2_ERR_UNSUPPORTED;
 }
 
 gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, const void* k, const void* v,

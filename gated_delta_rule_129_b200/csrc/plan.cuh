@@ -7,7 +7,8 @@
 // turns the counts into chunk_off[0..N].  A malformed cu_seqlens (first entry
 // not 0, a decreasing pair, or a last entry other than the total token count)
 // stores GDN2_ERR_SEQLENS in the status word and zero chunks for every
-// sequence, so no later kernel touches the token arrays.
+// sequence, so no later kernel touches the token arrays.  It also clears the
+// handed-back list and the flags the fused prep + walk synchronise on.
 #pragma once
 
 #include "common.cuh"
@@ -19,7 +20,7 @@ constexpr int kPlanThreads = 1024;
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int32_t* __restrict__ cu, int N, int T_dense, int T_total,
             int32_t* __restrict__ chunk_off, int32_t* __restrict__ status, int err_code,
-            int32_t* __restrict__ fix_count) {
+            int32_t* __restrict__ fix_count, int32_t* __restrict__ sync, int n_sync) {
   __shared__ int s_scan[kPlanThreads];
   __shared__ int s_bad;
   const int tid = threadIdx.x;
@@ -61,6 +62,8 @@ plan_kernel(const int32_t* __restrict__ cu, int N, int T_dense, int T_total,
     *status = any_bad ? err_code : 0;
     if (fix_count) *fix_count = 0;
   }
+  // task counter, redo flag and ready flags of the fused prep + walk
+  for (int i = tid; i < n_sync; i += kPlanThreads) sync[i] = 0;
 }
 
 }  // namespace gdn2

@@ -1,32 +1,45 @@
 // prep_tc.cuh -- gate preparation + intra-chunk WY + the chunk's affine state
 // map on the tensor cores (bf16 I/O, dk = 128, dv in {64, 128}).
 //
-// Persistent CTAs walk a list of (chunk, head) tasks.  Warps 0-7 compute,
-// warp 8 streams the inputs by TMA, warp 9 issues the UMMAs.  Per chunk of
-// n <= 64 tokens (page "Gated DeltaNet-2：将擦除与写入分开", sections
-// "在两个维度上独立控制" and "词元路径与并行训练"; the algebra is the recurrence
-// unrolled over one chunk, written as products):
+// Persistent CTAs walk a list of (chunk, head) tasks.  Warp roles:
+//   warp 8      TMA producer: streams each task's inputs in four 32-channel
+//               slices through a 3-slot ring that runs ahead across tasks;
+//   warp 10     scan: per slice, the in-chunk cumulative sum g of log_alpha
+//               (in place), the per-channel constants exp(g_r), exp(g_n - g_r),
+//               exp(g_n), and the decay-range check;
+//   warp 9      UMMA issue (one elected lane);
+//   warps 0-7   build the operands of each slice, then run the epilogues and
+//               the triangular solve of the task.
+// Per chunk of n <= 64 tokens (page "Gated DeltaNet-2：将擦除与写入分开",
+// sections "在两个维度上独立控制" and "词元路径与并行训练"; the algebra is the
+// recurrence unrolled over one chunk, written as products):
 //
-//  1. Gate prep (fp32).  The inputs stream in 32-channel slices through a
-//     3-slot TMA ring that runs ahead across tasks; per slice: g = in-chunk
-//     cumulative sum of log_alpha, and the bf16 operands, all with the decay
-//     folded in around one reference token r = 32 of the chunk:
+//  1. Gate prep (fp32), with the decay folded in around one reference token
+//     r = 32 of the chunk:
 //        E^_i = b_i k_i exp(g_i - g_r),  Q^_i = q_i exp(g_i - g_r),
-//        K^_j = k_j exp(g_r - g_j),      E~_i = b_i k_i exp(g_i),
-//        Kbar_j = k_j exp(g_n - g_j),    Q~_i = q_i exp(g_i),  Z_i = w_i v_i.
+//        K^_j = k_j exp(g_r - g_j),      Z_i = w_i v_i.
 //     For j <= i the product of the two factors is exp(g_i - g_j) <= 1; each
-//     factor alone stays inside exp(+-80) as long as no 32-token stretch of a
-//     channel decays by more than 80 nats.  A chunk that breaks this bound is
-//     handed back for the exact fp32 kernel (prep_fixup_kernel).
-//  2. UMMA 1: [E^; Q^] . K^T  (M = 128, N = 64, K = 128) -> A (strictly lower
-//     part of rows 0..63) and P (lower part with diagonal, rows 64..127).
+//     factor alone stays inside exp(+-60) as long as no 32-token stretch of a
+//     channel decays by more than 60 nats (which keeps every fp32 product
+//     below the accumulator's range).  A chunk that breaks this bound is
+//     handed back for the exact fp32 kernel (prep_fixup_kernel).  The other
+//     decayed operands are the same tensors scaled per channel,
+//        E~ = E^ diag(exp(g_r)),  Q~ = Q^ diag(exp(g_r)),
+//        Kbar = K^ diag(exp(g_n - g_r)),
+//     so they are never built: the scales are applied to rows or columns of
+//     the fp32 products in the epilogues.
+//  2. UMMA 1, accumulated slice by slice as the operands are built:
+//     [E^; Q^] . K^T (M = 128, N = 64, K = 128) -> A (strictly lower part of
+//     rows 0..63) and P (lower part with diagonal, rows 64..127).
 //  3. T = (I + A)^-1 in fp32 on the CUDA cores: the four 16 x 16 diagonal
-//     blocks by forward substitution, then each block column below the
-//     diagonal by a warp pair; T is split into bf16 hi + lo, stored side by
-//     side as one operand so one UMMA applies both (~16 bits of T kept).
-//  4. UMMA 2: [R_hi | R_lo] = Kbar^T [T_hi | T_lo], [V_hi | V_lo] = P [T_hi | T_lo].
-//  5. UMMA 3: [Mp | Nc] = R [E~ | Z], [P W | O_part] = V [E~ | Z]; the epilogue
-//     writes Mp, Nc, Q_eff = Q~ - P W, O_part (bf16) and exp(g_n) (fp32).
+//     blocks by forward substitution, then two levels of block merges
+//     [[T1, 0], [-T2 A21 T1, T2]] (16 -> 32 -> 64).  T is split into bf16
+//     hi + lo, stored side by side as one operand (~16 bits of T kept).
+//  4. UMMA 2: [R'_hi | R'_lo] = K^^T [T_hi | T_lo], [V_hi | V_lo] = P [T_hi | T_lo];
+//     R = Kbar^T T = diag(exp(g_n - g_r)) R'.
+//  5. UMMA 3: [Mp' | Nc] = R [E^ | Z], [P W' | O_part] = V [E^ | Z]; the
+//     epilogue writes Mp = Mp' diag(exp(g_r)), Nc, Q_eff = (Q^ - P W')
+//     diag(exp(g_r)) and O_part (bf16) by TMA stores.
 // Rows past the chunk's last token are zero in every operand, so they add
 // nothing; the padded rows of Q_eff and O_part come out as exact zeros.
 #pragma once
@@ -45,13 +58,13 @@ struct PrepTcArgs {
   CUtensorMap tm_Mp, tm_Nc, tm_Qe, tm_Op;
   SeqMap map;
   int H;
-  __nv_bfloat16* Qeff;   // [max_chunks, H, 64, 128]   (holds Q~ between the two phases)
+  __nv_bfloat16* Qeff;   // [max_chunks, H, 64, 128]
   __nv_bfloat16* Opart;  // [max_chunks, H, 64, DV]
   __nv_bfloat16* Mp;     // [max_chunks, H, 128, 128]
   __nv_bfloat16* Nc;     // [max_chunks, H, 128, DV]
   float* gamma_last;     // [max_chunks, H, 128]
   int32_t* fix_list;     // [0] = count, then c * H + h of handed-back chunks
-  int* ready;            // optional [max_chunks * H]: 1 = factors written, 2 = handed back
+  int* ready;            // optional [max_chunks * H], zeroed: 2 = factors written, 3 = handed back
   int* task_counter;     // optional: tasks taken dynamically (else static striding)
   int* status;
 };
@@ -64,40 +77,53 @@ struct PrepTcCfg {
   static constexpr int SLICES = 4;
   static constexpr int NSLOT = 3;
   static constexpr int COMPUTE_WARPS = 8;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
-  static constexpr int THREADS = 10 * 32;
-  // raw slot: la, b fp32 [64][32]; q, k bf16 [64][32]; v bf16 [64][VS]; w fp32 [64][VS]
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, SCAN_WARP = 10;
+  static constexpr int THREADS = 11 * 32;
+  // raw slot: la (-> g in place), b fp32 [64][32]; q, k bf16 [64][32]; v bf16 [64][VS]; w fp32 [64][VS].
+  // The fp32 rows of 128 bytes (la, b, and w when VS = 32) arrive SW128-swizzled
+  // (16-byte unit u of token row t at u ^ (t & 7)), so that the 8 lanes of a
+  // float4 access, which span two token rows, hit distinct banks.
   static constexpr int OFF_LA = 0, OFF_B = 8192, OFF_Q = 16384, OFF_K = 20480, OFF_V = 24576;
   static constexpr int OFF_W = OFF_V + kChunk * VS * 2;
   static constexpr int SLOT_BYTES = OFF_W + kChunk * VS * 4;
   static constexpr int SLOT_STRIDE = 36864;
+  static constexpr bool W_SWIZZLED = VS == 32;
   static constexpr int RING = NSLOT * SLOT_STRIDE;
-  // operands (1024-aligned)
-  static constexpr int OFF_X = RING;            // [E^; Q^] K-major SW128, 2 panels x 128 rows
-  static constexpr int OFF_KH = OFF_X + 32768;  // K^ K-major SW128, 2 panels x 64 rows
-  static constexpr int OFF_ET = OFF_KH + 16384; // E~ MN-major SW128 (rows = tokens), 2 panels
-  static constexpr int OFF_Z = OFF_ET + 16384;  // Z right after E~: [E~ | Z] is one operand
-  static constexpr int OFF_KB = OFF_Z + 16384;  // Kbar^T MN-major SW128 A operand, 2 panels
-  static constexpr int OFF_T = OFF_KB + 16384;  // [T_hi | T_lo] MN-major SW128, 2 panels
-  static constexpr int OFF_BAR = OFF_T + 16384;
-  // reuse of [E^; Q^] and K^ (48 KiB) once UMMA 1 has read them
-  static constexpr int LDA = 68;                // fp32 row stride of A and T
-  static constexpr int OFF_AS = OFF_X, OFF_TS = OFF_X + 17408, OFF_XS = OFF_X + 34816;
-  static constexpr int OFF_PB = OFF_X + 38912;  // P as K-major SW128 operand
-  static constexpr int OFF_RB = OFF_X, OFF_VB = OFF_X + 16384;  // after UMMA 2
-  // output staging once UMMA 3 has read every operand (SW128 panels of 64 columns)
-  static constexpr int OFF_SMP = OFF_X, OFF_SNC = OFF_X + 32768, OFF_SQE = OFF_X + 65536, OFF_SOP = OFF_X + 81920;
-  static_assert(OFF_SOP + 16384 <= OFF_BAR, "output staging fits in the operand area");
-  static constexpr int SMEM = 1024 + OFF_BAR + 2048;
+  // Operands: four SW128 panel slots of 16 KiB (128 rows of 64 bf16), 1024-aligned.
+  //   slot 0 / 1: rows 0..63 E^, rows 64..127 Q^ (channels 0..63 / 64..127)
+  //   slot 2 / 3: rows 0..63 Z (value channels 0..63 / 64..127), rows 64..127 K^
+  // so that [E^; Q^] (UMMA 1 A, M = 128), K^ (UMMA 1 B and, MN-major, the
+  // UMMA 2 A operand) and [E^ | Z] (UMMA 3 B, MN-major) each have one panel
+  // stride (16 KiB).
+  static constexpr int OFF_X = RING;
+  static constexpr int PANEL = 16384;
+  static constexpr int OFF_Z = OFF_X + 2 * PANEL;
+  static constexpr int OFF_KH = OFF_Z + 8192;
+  // free area (48 KiB): solve scratch, then T, then R and V
+  static constexpr int OFF_F = OFF_X + 4 * PANEL;
+  static constexpr int OFF_BAR = OFF_F + 49152;
+  static constexpr int LDA = 68;                // fp32 row stride of A and T: float4 rows, and a
+  static constexpr int LDT = 68;                // column of 8 rows spans all 32 banks
+  static constexpr int OFF_AS = OFF_F, OFF_TS = OFF_F + 17408, OFF_PB = OFF_F + 34816, OFF_XS = OFF_F + 43008;
+  static constexpr int OFF_T = OFF_F;           // [T_hi | T_lo] MN-major SW128, over A once A is dead
+  static constexpr int OFF_RB = OFF_F, OFF_VB = OFF_F + 16384;  // after UMMA 2: [R; V] K-major
+  // output staging once UMMA 3 has read its operands (SW128 panels of 64
+  // columns); Q_eff is formed in place over Q^ (rows 64..127 of slots 0, 1)
+  static constexpr int OFF_SMP0 = OFF_F, OFF_SMP1 = OFF_F + 16384;
+  static constexpr int OFF_SNC0 = OFF_F + 32768, OFF_SNC1 = OFF_X + 2 * PANEL;
+  static constexpr int OFF_SOP0 = OFF_X + 3 * PANEL, OFF_SOP1 = OFF_X + 3 * PANEL + 8192;
+  static constexpr int OFF_SQE = OFF_X + 8192;  // + p * PANEL
+  static_assert(OFF_XS + 4096 <= OFF_BAR, "solve scratch fits in the free area");
+  static_assert(64 * LDA * 4 <= OFF_TS - OFF_AS && 64 * LDT * 4 <= OFF_PB - OFF_TS, "A and T scratch");
+  static constexpr int SMEM = 1024 + OFF_BAR + 3072;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t COL_D1 = 0, COL_R = 64, COL_V = 192, COL_MN = 0, COL_QO = 256;
   static_assert(SLOT_BYTES <= SLOT_STRIDE, "slot fits");
-  static_assert(OFF_PB + 8192 <= OFF_X + 49152, "solve scratch fits in the freed operands");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-__device__ __forceinline__ void bar_pair(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void bar_half(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
 // byte offset of the 16-byte unit holding elements [8u, 8u+8) of row `row`
 // in an SW128 panel (rows of 64 bf16)
@@ -107,26 +133,42 @@ __device__ __forceinline__ void store8(uint8_t* p, const uint32_t (&w)[8], int a
   *reinterpret_cast<uint4*>(p) = make_uint4(w[at], w[at + 1], w[at + 2], w[at + 3]);
 }
 
+__device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
+  const float4 x = reinterpret_cast<const float4*>(p)[0], y = reinterpret_cast<const float4*>(p)[1];
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+
+// float index of channel c (0..31) of token row t in an SW128 fp32 tile
+__device__ __forceinline__ int swf(int t, int c) { return t * 32 + ((((c >> 2) ^ (t & 7))) << 2) + (c & 3); }
+
+// channels 8g .. 8g+7 of token row t of an SW128 fp32 tile (two 16-byte units)
+__device__ __forceinline__ void load8f_sw(const float* tile, int t, int g, float (&v)[8]) {
+  const float4 x = *reinterpret_cast<const float4*>(tile + t * 32 + (((2 * g) ^ (t & 7)) << 2));
+  const float4 y = *reinterpret_cast<const float4*>(tile + t * 32 + (((2 * g + 1) ^ (t & 7)) << 2));
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+
 template <int DV>
 __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int cta_count) {
   using C = PrepTcCfg<DV>;
   constexpr int DK = C::DK;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);  // [NSLOT]
-  uint64_t* empty = full + C::NSLOT;                                // [NSLOT]
-  uint64_t* ops_ready = empty + C::NSLOT;
-  uint64_t* mma1_done = ops_ready + 1;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);  // [NSLOT] producer -> scan
+  uint64_t* gready = full + C::NSLOT;                               // [NSLOT] scan -> build
+  uint64_t* empty = gready + C::NSLOT;                              // [NSLOT] build -> producer
+  uint64_t* built = empty + C::NSLOT;                               // [SLICES] build -> UMMA 1
+  uint64_t* mma1_done = built + C::SLICES;
   uint64_t* t_ready = mma1_done + 1;
   uint64_t* mma2_done = t_ready + 1;
   uint64_t* rv_ready = mma2_done + 1;
   uint64_t* mma3_done = rv_ready + 1;
-  uint64_t* task_full = mma3_done + 1;   // [2] task ids handed from producer to compute
-  uint64_t* task_empty = task_full + 2;  // [2]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(task_empty + 2);
-  int* s_flag = reinterpret_cast<int*>(tslot + 1);   // [0] abort, [1] done, [2 + (task & 1)] hand back
-  int* s_task = s_flag + 4;                          // [2] task ids
-  float* s_tot = reinterpret_cast<float*>(s_task + 2);  // [8][32] segment totals
-  float* s_er = s_tot + 256;                             // [32] exp(g_r)
-  float* s_enr = s_er + 32;                              // [32] exp(g_n - g_r)
+  uint64_t* fin = mma3_done + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::OFF_BAR + 256);
+  int* s_flag = reinterpret_cast<int*>(tslot + 1);    // [0] abort, [1] done
+  int* slot_task = s_flag + 2;                        // [NSLOT] task id of the slot's slice
+  int* slot_skip = slot_task + C::NSLOT;              // [NSLOT] decay range exceeded
+  float* s_gr = reinterpret_cast<float*>(sm + C::OFF_BAR + 512);  // [NSLOT][32] g_r
+  float* s_er = s_gr + C::NSLOT * 32;                             // [2][128] exp(g_r), by task parity
+  float* s_enr = s_er + 2 * DK;                                   // [2][128] exp(g_n - g_r)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
@@ -135,19 +177,17 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   if (tid == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
       tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&gready[s], 1);
       tc::mbar_init(&empty[s], C::COMPUTE_WARPS);
     }
-    tc::mbar_init(ops_ready, C::COMPUTE_WARPS);
+    for (int s = 0; s < C::SLICES; ++s) tc::mbar_init(&built[s], C::COMPUTE_WARPS);
     tc::mbar_init(mma1_done, 1);
     tc::mbar_init(t_ready, C::COMPUTE_WARPS);
     tc::mbar_init(mma2_done, 1);
     tc::mbar_init(rv_ready, C::COMPUTE_WARPS);
     tc::mbar_init(mma3_done, 1);
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&task_full[s], 1);
-      tc::mbar_init(&task_empty[s], C::COMPUTE_WARPS);
-    }
-    s_flag[0] = s_flag[1] = s_flag[2] = s_flag[3] = 0;
+    tc::mbar_init(fin, 1);
+    s_flag[0] = s_flag[1] = 0;
     tc::fence_mbar_init();
   }
   if (warp == C::MMA_WARP) {
@@ -159,31 +199,38 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   tc::tc_fence_after();
   const uint32_t tbase = *tslot;
   volatile int* vflag = s_flag;
+  volatile int* vtask = slot_task;
 
   if (warp == C::PRODUCER_WARP) {
     // ---------------------------------------------------- input producer --
-    // Takes tasks (dynamic counter or static stride), hands each task id to
-    // the compute warps through a 2-entry mailbox, and streams its four input
-    // slices through the ring.  A task id of -1 ends the CTA's work.
+    // Takes tasks (dynamic counter or static stride) and streams the four
+    // input slices of each through the ring, the task id beside each slice.
+    // A slot holding task id -1 (no data) ends the CTA's work.
     if (lane == 0) {
-      int gs = 0, nt = 0, k_static = 0;
+      int gs = 0, k_static = 0;
       bool ok = true;
-      while (ok) {
+      for (bool more = true; more && ok;) {
         int task;
         if (a.task_counter) task = atomicAdd(a.task_counter, 1);
         else task = cta_rank + cta_count * (k_static++);
         if (task >= ntasks) task = -1;
-        const int mb = nt & 1;
-        if (nt >= 2 && !tc::mbar_wait(&task_empty[mb], ((nt - 2) >> 1) & 1)) { ok = false; break; }
-        s_task[mb] = task;
-        tc::mbar_arrive(&task_full[mb]);
-        ++nt;
-        if (task < 0 || vflag[0]) break;
-        const int c = task / H, h = task % H;
-        const int t0 = chunk_pos(a.map, c).t0;
-        for (int s = 0; s < C::SLICES; ++s, ++gs) {
+        int h = 0, t0 = 0;
+        if (task >= 0) {
+          h = task % H;
+          t0 = chunk_pos(a.map, task / H).t0;
+        }
+        const int nsl = task < 0 ? 1 : C::SLICES;
+        for (int s = 0; s < nsl; ++s, ++gs) {
           const int slot = gs % C::NSLOT, use = gs / C::NSLOT;
           if (use > 0 && !tc::mbar_wait(&empty[slot], (use - 1) & 1)) { ok = false; break; }
+          if (vflag[0]) { more = false; break; }
+          vtask[slot] = task;
+          if (task < 0) {
+            tc::mbar_arrive(&full[slot]);
+            more = false;
+            ++gs;
+            break;
+          }
           uint8_t* d = sm + slot * C::SLOT_STRIDE;
           tc::mbar_arrive_expect_tx(&full[slot], C::SLOT_BYTES);
           tc::tma_load_3d(d + C::OFF_LA, &a.tm_la, &full[slot], C::KS * s, h, t0);
@@ -202,13 +249,55 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       for (int g = gs > C::NSLOT ? gs - C::NSLOT : 0; g < gs; ++g)
         tc::mbar_wait(&full[g % C::NSLOT], (g / C::NSLOT) & 1);
     }
+  } else if (warp == C::SCAN_WARP) {
+    // -------------------------------------------------------------- scan --
+    // lane = channel of the slice; g_t = sum of log_alpha over tokens <= t of
+    // the chunk (tokens past its end count as 0), written over log_alpha.
+    int s_in = 0, tpar = 0;
+    for (int gs = 0;; ++gs) {
+      const int slot = gs % C::NSLOT, use = gs / C::NSLOT;
+      if (!tc::mbar_wait(&full[slot], use & 1)) {
+        atomicExch(a.status, 8);
+        vflag[0] = 1;
+        break;
+      }
+      const int task = vtask[slot];
+      if (task >= 0 && !vflag[0]) {
+        const int c = task / H;
+        const int len = chunk_pos(a.map, c).len;
+        const size_t tile = (size_t)c * H + task % H;
+        float* la = reinterpret_cast<float*>(sm + slot * C::SLOT_STRIDE + C::OFF_LA);
+        float v[kChunk];
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) v[t] = la[swf(t, lane)];
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) {
+          acc += t < len ? v[t] : 0.f;
+          v[t] = acc;
+        }
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) la[swf(t, lane)] = v[t];
+        const float g0 = v[0], gr = v[32], gn = v[kChunk - 1];
+        const bool bad = (g0 - gr > 60.f) || (gr - gn > 60.f);
+        s_gr[slot * 32 + lane] = gr;
+        s_er[tpar * DK + C::KS * s_in + lane] = __expf(gr);
+        s_enr[tpar * DK + C::KS * s_in + lane] = __expf(gn - gr);
+        a.gamma_last[tile * DK + C::KS * s_in + lane] = expf(gn);
+        if (a.ready) __threadfence();  // published with the chunk's other factors
+        const unsigned any = __ballot_sync(0xffffffffu, bad);
+        if (lane == 0) slot_skip[slot] = any != 0u;
+        s_in = (s_in + 1) & (C::SLICES - 1);
+        if (s_in == 0) tpar ^= 1;
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&gready[slot]);
+      if (task < 0 || vflag[0]) break;
+    }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------- UMMA issue --
-    // One round of three UMMA groups per task the compute warps did not hand
-    // back; the compute warps arrive once more with s_flag[2] set when done.
     if (lane == 0) {
       const uint32_t X = tc::smem_u32(sm + C::OFF_X), KH = tc::smem_u32(sm + C::OFF_KH);
-      const uint32_t EZ = tc::smem_u32(sm + C::OFF_ET), KB = tc::smem_u32(sm + C::OFF_KB);
       const uint32_t TT = tc::smem_u32(sm + C::OFF_T), PB = tc::smem_u32(sm + C::OFF_PB);
       const uint32_t RB = tc::smem_u32(sm + C::OFF_RB), VB = tc::smem_u32(sm + C::OFF_VB);
       const uint32_t SW = tc::kLayoutSW128;
@@ -217,23 +306,28 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       constexpr uint32_t idV = tc::idesc_bf16(64, 128, false, true);
       constexpr uint32_t idM = tc::idesc_bf16(128, 128 + DV, false, true);
       constexpr uint32_t idQ = tc::idesc_bf16(64, 128 + DV, false, true);
-      for (int ex = 0;; ++ex) {
-        if (!tc::mbar_wait(ops_ready, ex & 1)) break;
-        if (vflag[1] || vflag[0]) break;
-        tc::tc_fence_after();
+      bool ok = true;
+      for (int ex = 0; ok; ++ex) {
+        // UMMA 1, two K-steps of 16 channels per slice as the slices are built
+        for (int s = 0; s < C::SLICES; ++s) {
+          if (!tc::mbar_wait(&built[s], ex & 1) || vflag[0]) { ok = false; break; }
+          if (vflag[1]) break;
+          tc::tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < DK / 16; ++s) {
-          const uint32_t ko = (s >> 2), kk = (s & 3) * 32;
-          tc::umma_f16(tbase + C::COL_D1, tc::sdesc(X + ko * 16384 + kk, 16, 1024, SW),
-                       tc::sdesc(KH + ko * 8192 + kk, 16, 1024, SW), id1, s > 0);
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t k = 2 * s + kk, ko = k >> 2, kb = (k & 3) * 32;
+            tc::umma_f16(tbase + C::COL_D1, tc::sdesc(X + ko * C::PANEL + kb, 16, 1024, SW),
+                         tc::sdesc(KH + ko * C::PANEL + kb, 16, 1024, SW), id1, k > 0);
+          }
         }
+        if (!ok || vflag[1]) break;
         tc::umma_commit(mma1_done);
         if (!tc::mbar_wait(t_ready, ex & 1) || vflag[0]) break;
         tc::tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const uint64_t t_d = tc::sdesc(TT + s * 2048, 8192, 1024, SW);
-          tc::umma_f16(tbase + C::COL_R, tc::sdesc(KB + s * 2048, 8192, 1024, SW), t_d, idR, s > 0);
+          tc::umma_f16(tbase + C::COL_R, tc::sdesc(KH + s * 2048, C::PANEL, 1024, SW), t_d, idR, s > 0);
           tc::umma_f16(tbase + C::COL_V, tc::sdesc(PB + s * 32, 16, 1024, SW), t_d, idV, s > 0);
         }
         tc::umma_commit(mma2_done);
@@ -241,101 +335,74 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         tc::tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint64_t ez_d = tc::sdesc(EZ + s * 2048, 8192, 1024, SW);
+          const uint64_t ez_d = tc::sdesc(X + s * 2048, C::PANEL, 1024, SW);
           tc::umma_f16(tbase + C::COL_MN, tc::sdesc(RB + s * 32, 16, 1024, SW), ez_d, idM, s > 0);
           tc::umma_f16(tbase + C::COL_QO, tc::sdesc(VB + s * 32, 16, 1024, SW), ez_d, idQ, s > 0);
         }
         tc::umma_commit(mma3_done);
       }
+      // nothing of ours is left in the tensor pipe when TMEM is released
+      tc::umma_commit(fin);
+      tc::mbar_wait(fin, 0);
     }
   } else {
     // ----------------------------------------------------------- compute --
     const int q = warp & 3, half = warp >> 2;
-    int gs = 0, ex = 0;
+    float* AS = reinterpret_cast<float*>(sm + C::OFF_AS);
+    float* TS = reinterpret_cast<float*>(sm + C::OFF_TS);
+    float* XS = reinterpret_cast<float*>(sm + C::OFF_XS);
+    int gs = 0;
     bool alive = true;
-    for (int nt = 0; alive; ++nt) {
-      const int mb = nt & 1;
-      if (!tc::mbar_wait(&task_full[mb], (nt >> 1) & 1)) {
-        atomicExch(a.status, 8);
-        vflag[0] = 1;
-        break;
+    // The two storing threads (tid 0 and 128) publish a task's ready flag
+    // once its tiles are in global memory: checked when they next store, so
+    // the check never waits on stores still in flight.
+    int pend = -1;
+    auto publish = [&]() {
+      tc::tma_store_wait_all();
+      if (a.ready && pend >= 0) {
+        tc::fence_async_global();
+        __threadfence();
+        tc::red_add_release_gpu(a.ready + pend, 1);
       }
-      const int task = s_task[mb];
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&task_empty[mb]);
-      if (task < 0 || vflag[0]) break;
-      const int c = task / H, h = task % H;
-      const ChunkPos pos = chunk_pos(a.map, c);
-      const int len = pos.len;
-      const size_t tile = (size_t)c * H + h;
-      volatile int* skipflag = vflag + 2 + (nt & 1);
-      if (tid == 0) {
-        *skipflag = 0;
-        tc::tma_store_wait_read();  // previous task's output staging has been read
-      }
-      bar_compute();
+      pend = -1;
+    };
+    for (int ex = 0;; ++ex) {
+      int task = -1, len = 0;
+      size_t tile = 0;
+      bool skip = false;
       // ------------------------------------------------------ slices --
       for (int s = 0; s < C::SLICES; ++s, ++gs) {
         const int slot = gs % C::NSLOT;
+        if (!tc::mbar_wait(&gready[slot], (gs / C::NSLOT) & 1)) { alive = false; break; }
+        task = vtask[slot];
+        if (task < 0 || vflag[0]) break;
+        if (s == 0) {
+          const int c = task / H;
+          len = chunk_pos(a.map, c).len;
+          tile = (size_t)c * H + task % H;
+          // the previous task's output stores have read the operand area and Q_eff
+          if ((tid & 127) == 0) tc::tma_store_wait_read();
+          bar_compute();
+        }
+        skip |= reinterpret_cast<volatile int*>(slot_skip)[slot] != 0;
         uint8_t* d = sm + slot * C::SLOT_STRIDE;
-        float* la = reinterpret_cast<float*>(d + C::OFF_LA);   // becomes g
-        if (!tc::mbar_wait(&full[slot], (gs / C::NSLOT) & 1)) {
-          atomicExch(a.status, 8);
-          vflag[0] = 1;
-          alive = false;
-          break;
-        }
-        // cumulative log-decay: lane = channel, warp = 8-token segment
-        float loc[8];
-        float acc = 0.f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int tok = 8 * warp + t;
-          acc += tok < len ? la[tok * 32 + lane] : 0.f;
-          loc[t] = acc;
-        }
-        s_tot[warp * 32 + lane] = acc;
-        bar_compute();
-        float off = 0.f;
-        for (int w2 = 0; w2 < warp; ++w2) off += s_tot[w2 * 32 + lane];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) la[(8 * warp + t) * 32 + lane] = loc[t] + off;
-        bar_compute();
-        if (warp == 0) {
-          const float g0 = la[lane], gr = la[32 * 32 + lane], gn = la[63 * 32 + lane];
-          if (g0 - gr > 80.f || gr - gn > 80.f) *skipflag = 1;
-          s_er[lane] = __expf(gr);
-          s_enr[lane] = __expf(gn - gr);
-          a.gamma_last[tile * DK + C::KS * s + lane] = expf(gn);
-        }
-        bar_compute();
+        const float* g = reinterpret_cast<const float*>(d + C::OFF_LA);
         // operands for token i, key channels cc0 .. cc0 + 7
+        const int i = tid >> 2, gq = tid & 3, cl = 8 * gq, cc0 = C::KS * s + cl;
+        const bool live = i < len;
         {
-          const int i = tid >> 2, gq = tid & 3, cl = 8 * gq, cc0 = C::KS * s + cl;
-          const bool live = i < len;
-          // 8 consecutive fp32 values per thread, read as two float4 (scalar
-          // reads of 8 token rows 128 B apart would hit the same banks)
           float gi[8], gr[8], bb[8];
-          {
-            const float4* g4 = reinterpret_cast<const float4*>(la + i * 32 + cl);
-            const float4* r4 = reinterpret_cast<const float4*>(la + 32 * 32 + cl);
-            const float4* b4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(d + C::OFF_B) + i * 32 + cl);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const float4 x = g4[hh], y = r4[hh], z = b4[hh];
-              gi[4 * hh] = x.x; gi[4 * hh + 1] = x.y; gi[4 * hh + 2] = x.z; gi[4 * hh + 3] = x.w;
-              gr[4 * hh] = y.x; gr[4 * hh + 1] = y.y; gr[4 * hh + 2] = y.z; gr[4 * hh + 3] = y.w;
-              bb[4 * hh] = z.x; bb[4 * hh + 1] = z.y; bb[4 * hh + 2] = z.z; bb[4 * hh + 3] = z.w;
-            }
-          }
+          load8f_sw(g, i, gq, gi);
+          load8f(s_gr + slot * 32 + cl, gr);
+          load8f_sw(reinterpret_cast<const float*>(d + C::OFF_B), i, gq, bb);
           const uint4 kraw = *reinterpret_cast<const uint4*>(d + C::OFF_K + (i * 32 + cl) * 2);
           const uint4 qraw = *reinterpret_cast<const uint4*>(d + C::OFF_Q + (i * 32 + cl) * 2);
           const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
           const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
-          uint32_t eh[8], kh[8], et[4], kb[4], qt[4];
+          uint32_t eh[8], kh[4];
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
-            float o_eh[2], o_qh[2], o_kh[2], o_et[2], o_kb[2], o_qt[2];
+            float o_eh[2], o_qh[2], o_kh[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int m = 2 * p + e;
@@ -344,40 +411,36 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
               const float bv = live ? bb[m] : 0.f;
               const float x = gi[m] - gr[m];
               const float E = __expf(x), F = __expf(-x);
-              const float gam = s_er[cl + m] * E, kbf = s_enr[cl + m] * F;
               o_eh[e] = bv * kv * E;
               o_qh[e] = qv * E;
               o_kh[e] = kv * F;
-              o_et[e] = bv * kv * gam;
-              o_kb[e] = kv * kbf;
-              o_qt[e] = qv * gam;
             }
             eh[p] = tc::pack_bf16(o_eh[0], o_eh[1]);
             eh[4 + p] = tc::pack_bf16(o_qh[0], o_qh[1]);
             kh[p] = tc::pack_bf16(o_kh[0], o_kh[1]);
-            et[p] = tc::pack_bf16(o_et[0], o_et[1]);
-            kb[p] = tc::pack_bf16(o_kb[0], o_kb[1]);
-            qt[p] = tc::pack_bf16(o_qt[0], o_qt[1]);
           }
           const uint32_t pnl = cc0 >> 6, u = (cc0 & 63) >> 3;
-          store8(sm + C::OFF_X + pnl * 16384 + sw_unit(i, u), eh, 0);
-          store8(sm + C::OFF_X + pnl * 16384 + sw_unit(64 + i, u), eh, 4);
-          *reinterpret_cast<uint4*>(sm + C::OFF_KH + pnl * 8192 + sw_unit(i, u)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-          *reinterpret_cast<uint4*>(sm + C::OFF_ET + pnl * 8192 + sw_unit(i, u)) = make_uint4(et[0], et[1], et[2], et[3]);
-          *reinterpret_cast<uint4*>(sm + C::OFF_KB + pnl * 8192 + sw_unit(i, u)) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
-          // Q~ waits in the Q_eff buffer until the last epilogue
-          *reinterpret_cast<uint4*>(a.Qeff + (tile * kChunk + i) * DK + cc0) = make_uint4(qt[0], qt[1], qt[2], qt[3]);
+          store8(sm + C::OFF_X + pnl * C::PANEL + sw_unit(i, u), eh, 0);
+          store8(sm + C::OFF_X + pnl * C::PANEL + sw_unit(64 + i, u), eh, 4);
+          *reinterpret_cast<uint4*>(sm + C::OFF_KH + pnl * C::PANEL + sw_unit(i, u)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
+        }
+        {
           // Z = w * v for value channels vc0 .. vc0 + VS/4 - 1 (right after E~)
           constexpr int VPT = C::VS / 4;
           const int vl = VPT * gq, vc0 = C::VS * s + vl;
           float ww[VPT];
           uint32_t vw[VPT / 2];
           {
-            const float4* w4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(d + C::OFF_W) + i * C::VS + vl);
+            const float* wt = reinterpret_cast<const float*>(d + C::OFF_W);
+            if constexpr (C::W_SWIZZLED) {
+              load8f_sw(wt, i, gq, *reinterpret_cast<float(*)[8]>(ww));
+            } else {
+              const float4* w4 = reinterpret_cast<const float4*>(wt + i * C::VS + vl);
 #pragma unroll
-            for (int hh = 0; hh < VPT / 4; ++hh) {
-              const float4 x = w4[hh];
-              ww[4 * hh] = x.x; ww[4 * hh + 1] = x.y; ww[4 * hh + 2] = x.z; ww[4 * hh + 3] = x.w;
+              for (int hh = 0; hh < VPT / 4; ++hh) {
+                const float4 x = w4[hh];
+                ww[4 * hh] = x.x; ww[4 * hh + 1] = x.y; ww[4 * hh + 2] = x.z; ww[4 * hh + 3] = x.w;
+              }
             }
             const uint8_t* vsrc = d + C::OFF_V + (i * C::VS + vl) * 2;
             if constexpr (VPT == 8) {
@@ -395,31 +458,18 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
             const float z1 = live ? ww[2 * p + 1] * bf16_hi_f(vw[p]) : 0.f;
             zw[p] = tc::pack_bf16(z0, z1);
           }
-          uint8_t* zdst = sm + C::OFF_Z + (vc0 >> 6) * 8192 + sw_unit(i, (vc0 & 63) >> 3) + (vc0 & 7) * 2;
+          uint8_t* zdst = sm + C::OFF_Z + (vc0 >> 6) * C::PANEL + sw_unit(i, (vc0 & 63) >> 3) + (vc0 & 7) * 2;
           if constexpr (VPT == 8) *reinterpret_cast<uint4*>(zdst) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
           else *reinterpret_cast<uint2*>(zdst) = make_uint2(zw[0], zw[1]);
         }
+        tc::fence_async_smem();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&empty[slot]);
-      }
-      if (!alive) break;
-      tc::fence_async_smem();
-      tc::tc_fence_before();
-      bar_compute();
-      if (*skipflag) {
-        // decay too steep for one reference point: hand the chunk back
-        if (tid == 0) {
-          const int idx = atomicAdd(a.fix_list, 1);
-          a.fix_list[1 + idx] = (int)tile;
-          if (a.ready) tc::st_release_gpu(a.ready + tile, 2);
+        if (lane == 0) {
+          tc::mbar_arrive(&empty[slot]);
+          tc::mbar_arrive(&built[s]);
         }
-        continue;
       }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(ops_ready);
-      float* AS = reinterpret_cast<float*>(sm + C::OFF_AS);
-      float* TS = reinterpret_cast<float*>(sm + C::OFF_TS);
-      float* XS = reinterpret_cast<float*>(sm + C::OFF_XS);
+      if (!alive || task < 0 || vflag[0]) break;
       if (!tc::mbar_wait(mma1_done, ex & 1)) { alive = false; break; }
       // -------------------------------------------- epilogue 1: A and P --
       tc::tc_fence_after();
@@ -431,14 +481,10 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         if (q < 2) {
           const int i = 32 * q + lane;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 v4;
-            v4.x = (j0 + e < i) ? __uint_as_float(r[e]) : 0.f;
-            v4.y = (j0 + e + 1 < i) ? __uint_as_float(r[e + 1]) : 0.f;
-            v4.z = (j0 + e + 2 < i) ? __uint_as_float(r[e + 2]) : 0.f;
-            v4.w = (j0 + e + 3 < i) ? __uint_as_float(r[e + 3]) : 0.f;
-            *reinterpret_cast<float4*>(AS + i * C::LDA + j0 + e) = v4;
-          }
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(AS + i * C::LDA + j0 + e) =
+                make_float4(j0 + e < i ? __uint_as_float(r[e]) : 0.f, j0 + e + 1 < i ? __uint_as_float(r[e + 1]) : 0.f,
+                            j0 + e + 2 < i ? __uint_as_float(r[e + 2]) : 0.f, j0 + e + 3 < i ? __uint_as_float(r[e + 3]) : 0.f);
         } else {
           const int i = 32 * q + lane - 64;
           uint32_t pw[16];
@@ -454,83 +500,113 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       }
       bar_compute();
       // ------------------------------------------- T = (I + A)^-1, fp32 --
+      // (a) diagonal 16 x 16 blocks by forward substitution (warps 0-3,
+      //     lane l < 16 owns column l of block `warp`); warps 4-7 zero the
+      //     two upper blocks the merges below read.
       if (warp < 4) {
-        // diagonal block I = warp; lane l < 16 owns column l
         const int I = warp, l = lane;
         float t[16];
+        t[0] = l == 0 ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float accv = 0.f;
+        for (int i = 1; i < 16; ++i) {
+          float arow[16];
+          load8f(AS + (16 * I + i) * C::LDA + 16 * I, *reinterpret_cast<float(*)[8]>(arow));
+          load8f(AS + (16 * I + i) * C::LDA + 16 * I + 8, *reinterpret_cast<float(*)[8]>(arow + 8));
+          // t[m] = 0 for m < l, so the sum may run over every m < i
+          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int m = 0; m < i; ++m)
-            if (m >= l) accv = fmaf(AS[(16 * I + i) * C::LDA + 16 * I + m], t[m], accv);
-          t[i] = i < l ? 0.f : (i == l ? 1.f : -accv);
+          for (int m = 0; m < i; ++m) {
+            if (m & 1) s1 = fmaf(arow[m], t[m], s1);
+            else s0 = fmaf(arow[m], t[m], s0);
+          }
+          t[i] = i < l ? 0.f : (i == l ? 1.f : -(s0 + s1));
         }
         if (l < 16)
 #pragma unroll
-          for (int i = 0; i < 16; ++i) TS[(16 * I + i) * C::LDA + 16 * I + l] = t[i];
+          for (int i = 0; i < 16; ++i) TS[(16 * I + i) * C::LDT + 16 * I + l] = t[i];
       } else {
-        for (int idx = tid - 128; idx < 64 * 64; idx += 128) {
-          const int rr = idx >> 6, cc = idx & 63;
-          if ((cc >> 4) > (rr >> 4)) TS[rr * C::LDA + cc] = 0.f;
-        }
+        const int z = tid - 128;  // 0..127: two 16 x 16 blocks, 4 values each
+        const int blk = z >> 6, rr = (z >> 2) & 15, cc = 4 * (z & 3);
+        const int r0 = 32 * blk + rr, c0 = 32 * blk + 16 + cc;
+        *reinterpret_cast<float4*>(TS + r0 * C::LDT + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       bar_compute();
-      // block column J below the diagonal, by warps J and J + 4 (64 threads):
-      // thread (r = row in block, cg = 4-column group)
-      if ((warp & 3) < 3) {
-        const int J = warp & 3, pt = (warp >> 2) * 32 + lane;   // 0..63 within the pair
-        const int r = pt >> 2, cg = pt & 3;
-        float* X = XS + J * 256;
-        for (int I = J + 1; I < 4; ++I) {
-          float4 xa = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int kb = J; kb < I; ++kb) {
-            const float* arow = AS + (16 * I + r) * C::LDA + 16 * kb;
-            const float* tcol = TS + (16 * kb) * C::LDA + 16 * J + 4 * cg;
-            float av[16];
+      // (b) 16 -> 32: blocks (1,0) and (3,2); warps 0-3 and 4-7.
+      {
+        const int m = warp >> 2, ba = 2 * m, bb = 2 * m + 1;
+        const int t = tid & 127, r = t >> 3, c = 2 * (t & 7);
+        float* X2 = XS + m * 256;
+        float x0 = 0.f, x1 = 0.f;
+        float arow[16];
+        load8f(AS + (16 * bb + r) * C::LDA + 16 * ba, *reinterpret_cast<float(*)[8]>(arow));
+        load8f(AS + (16 * bb + r) * C::LDA + 16 * ba + 8, *reinterpret_cast<float(*)[8]>(arow + 8));
+        const float* tcol = TS + (16 * ba) * C::LDT + 16 * ba + c;
 #pragma unroll
-            for (int m = 0; m < 16; m += 4) {
-              const float4 a4 = *reinterpret_cast<const float4*>(arow + m);
-              av[m] = a4.x; av[m + 1] = a4.y; av[m + 2] = a4.z; av[m + 3] = a4.w;
-            }
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-              const float4 tv = *reinterpret_cast<const float4*>(tcol + m * C::LDA);
-              xa.x = fmaf(av[m], tv.x, xa.x); xa.y = fmaf(av[m], tv.y, xa.y);
-              xa.z = fmaf(av[m], tv.z, xa.z); xa.w = fmaf(av[m], tv.w, xa.w);
-            }
-          }
-          *reinterpret_cast<float4*>(X + r * 16 + 4 * cg) = xa;
-          bar_pair(2 + J);
-          float4 ta = make_float4(0.f, 0.f, 0.f, 0.f);
-          float tr[16];
-#pragma unroll
-          for (int m = 0; m < 16; m += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(TS + (16 * I + r) * C::LDA + 16 * I + m);
-            tr[m] = t4.x; tr[m + 1] = t4.y; tr[m + 2] = t4.z; tr[m + 3] = t4.w;
-          }
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const float tv = tr[m];
-            const float4 xv = *reinterpret_cast<const float4*>(X + m * 16 + 4 * cg);
-            ta.x = fmaf(tv, xv.x, ta.x); ta.y = fmaf(tv, xv.y, ta.y);
-            ta.z = fmaf(tv, xv.z, ta.z); ta.w = fmaf(tv, xv.w, ta.w);
-          }
-          *reinterpret_cast<float4*>(TS + (16 * I + r) * C::LDA + 16 * J + 4 * cg) =
-              make_float4(-ta.x, -ta.y, -ta.z, -ta.w);
-          bar_pair(2 + J);
+        for (int k = 0; k < 16; ++k) {
+          const float2 tv = *reinterpret_cast<const float2*>(tcol + k * C::LDT);
+          x0 = fmaf(arow[k], tv.x, x0);
+          x1 = fmaf(arow[k], tv.y, x1);
         }
+        *reinterpret_cast<float2*>(X2 + r * 16 + c) = make_float2(x0, x1);
+        bar_half(2 + m);
+        float y0 = 0.f, y1 = 0.f;
+        float trow[16];
+        load8f(TS + (16 * bb + r) * C::LDT + 16 * bb, *reinterpret_cast<float(*)[8]>(trow));
+        load8f(TS + (16 * bb + r) * C::LDT + 16 * bb + 8, *reinterpret_cast<float(*)[8]>(trow + 8));
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 xv = *reinterpret_cast<const float2*>(X2 + k * 16 + c);
+          y0 = fmaf(trow[k], xv.x, y0);
+          y1 = fmaf(trow[k], xv.y, y1);
+        }
+        *reinterpret_cast<float2*>(TS + (16 * bb + r) * C::LDT + 16 * ba + c) = make_float2(-y0, -y1);
       }
       bar_compute();
-      // T -> [T_hi | T_lo], MN-major SW128 (row i, 64 columns j per panel)
+      // (c) 32 -> 64: block (1,0) of 32 x 32 blocks; thread = row r, columns c..c+3.
+      {
+        const int r = tid >> 3, c = 4 * (tid & 7);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+          float av[8];
+          load8f(AS + (32 + r) * C::LDA + k0, av);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 tv = *reinterpret_cast<const float4*>(TS + (k0 + k) * C::LDT + c);
+            x.x = fmaf(av[k], tv.x, x.x); x.y = fmaf(av[k], tv.y, x.y);
+            x.z = fmaf(av[k], tv.z, x.z); x.w = fmaf(av[k], tv.w, x.w);
+          }
+        }
+        *reinterpret_cast<float4*>(XS + r * 32 + c) = x;
+        bar_compute();
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+          float tv[8];
+          load8f(TS + (32 + r) * C::LDT + 32 + k0, tv);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 xv = *reinterpret_cast<const float4*>(XS + (k0 + k) * 32 + c);
+            y.x = fmaf(tv[k], xv.x, y.x); y.y = fmaf(tv[k], xv.y, y.y);
+            y.z = fmaf(tv[k], xv.z, y.z); y.w = fmaf(tv[k], xv.w, y.w);
+          }
+        }
+        *reinterpret_cast<float4*>(TS + (32 + r) * C::LDT + c) = make_float4(-y.x, -y.y, -y.z, -y.w);
+      }
+      bar_compute();
+      // T -> [T_hi | T_lo], MN-major SW128 (row i, 64 columns j per panel);
+      // entries above the diagonal are zero.
       {
         const int i = tid >> 2, j0 = 16 * (tid & 3);
         uint32_t hw[8], lw[8];
         float tv[16];
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
-          const float4 t4 = *reinterpret_cast<const float4*>(TS + i * C::LDA + j0 + e);
-          tv[e] = t4.x; tv[e + 1] = t4.y; tv[e + 2] = t4.z; tv[e + 3] = t4.w;
+          const float4 t4 = *reinterpret_cast<const float4*>(TS + i * C::LDT + j0 + e);
+          tv[e] = j0 + e <= i ? t4.x : 0.f;
+          tv[e + 1] = j0 + e + 1 <= i ? t4.y : 0.f;
+          tv[e + 2] = j0 + e + 2 <= i ? t4.z : 0.f;
+          tv[e + 3] = j0 + e + 3 <= i ? t4.w : 0.f;
         }
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
@@ -550,19 +626,20 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(t_ready);
       if (!tc::mbar_wait(mma2_done, ex & 1)) { alive = false; break; }
-      // ---------------------------------- epilogue 2: R, V = hi + lo -> bf16 --
+      // ------------- epilogue 2: R = exp(g_n - g_r) (R'_hi + R'_lo), V = V_hi + V_lo -> bf16 --
       tc::tc_fence_after();
       {
         const int j0 = 32 * half;
+        const int m = 32 * q + lane;
+        const float sc = s_enr[(ex & 1) * DK + m];
         uint32_t rh[32], rl[32], pw[16];
         tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_R + j0), rh);
         tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_R + 64 + j0), rl);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
-          pw[e / 2] = tc::pack_bf16(__uint_as_float(rh[e]) + __uint_as_float(rl[e]),
-                                    __uint_as_float(rh[e + 1]) + __uint_as_float(rl[e + 1]));
-        const int m = 32 * q + lane;
+          pw[e / 2] = tc::pack_bf16(sc * (__uint_as_float(rh[e]) + __uint_as_float(rl[e])),
+                                    sc * (__uint_as_float(rh[e + 1]) + __uint_as_float(rl[e + 1])));
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu)
           *reinterpret_cast<uint4*>(sm + C::OFF_RB + sw_unit(m, (j0 >> 3) + uu)) =
@@ -586,90 +663,131 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(rv_ready);
-      // Q~ for this thread's output row, while UMMA 3 runs
-      const int i_out = 16 * q + lane;
-      uint4 qt_r[DK / 8];   // the row's 128 bf16 values of Q~
-      if (half == 0 && lane < 16) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.Qeff + (tile * kChunk + i_out) * DK);
-#pragma unroll
-        for (int uu = 0; uu < DK / 8; ++uu) qt_r[uu] = src[uu];
-      }
       if (!tc::mbar_wait(mma3_done, ex & 1)) { alive = false; break; }
       // ------------------------------------------- epilogue 3: outputs --
       // Results go to SW128 staging in the (now free) operand area and leave
       // by TMA bulk stores, so every global write is a whole tile row.
       tc::tc_fence_after();
+      const float* er = s_er + (ex & 1) * DK;   // exp(g_r) by key channel
       {
         const int m = 32 * q + lane;  // key channel row of Mp / Nc
-        // half 0: Mp columns 0..127; half 1: Nc columns 0..DV-1 (TMEM 128..)
+        // half 0: Mp = Mp' diag(exp(g_r)), columns 0..127; half 1: Nc columns
+        // 0..DV-1 (TMEM 128..)
         const int ncols = half == 0 ? 128 : DV;
-        uint8_t* stg = sm + (half == 0 ? C::OFF_SMP : C::OFF_SNC);
-        for (int c0 = 0; c0 < ncols; c0 += 32) {
-          uint32_t r[32], pw[16];
-          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0), r);
-          tc::tmem_wait_ld();
+        for (int c0 = 0; c0 < ncols; c0 += 64) {
+          uint32_t r0[32], r1[32];
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0), r0);
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0 + 32), r1);
+          tc::tmem_wait_ld_regs(r0);
+          tc::tmem_wait_ld_regs(r1);
+          uint8_t* pnl = sm + (half == 0 ? (c0 ? C::OFF_SMP1 : C::OFF_SMP0) : (c0 ? C::OFF_SNC1 : C::OFF_SNC0));
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) pw[e / 2] = tc::pack_bf16(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-          uint8_t* pnl = stg + (c0 >> 6) * 16384;
+          for (int uu = 0; uu < 8; ++uu) {
+            const uint32_t* r = uu < 4 ? r0 + 8 * uu : r1 + 8 * (uu - 4);
+            float sc[8];
+            if (half == 0) load8f(er + c0 + 8 * uu, sc);
+            else
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu)
-            *reinterpret_cast<uint4*>(pnl + sw_unit(m, ((c0 & 63) >> 3) + uu)) =
-                make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
+              for (int e = 0; e < 8; ++e) sc[e] = 1.f;
+            *reinterpret_cast<uint4*>(pnl + sw_unit(m, uu)) =
+                make_uint4(tc::pack_bf16(sc[0] * __uint_as_float(r[0]), sc[1] * __uint_as_float(r[1])),
+                           tc::pack_bf16(sc[2] * __uint_as_float(r[2]), sc[3] * __uint_as_float(r[3])),
+                           tc::pack_bf16(sc[4] * __uint_as_float(r[4]), sc[5] * __uint_as_float(r[5])),
+                           tc::pack_bf16(sc[6] * __uint_as_float(r[6]), sc[7] * __uint_as_float(r[7])));
+          }
         }
-        // token rows (M = 64 layout): half 0: Q_eff = Q~ - P W; half 1: O_part
-        uint8_t* stt = sm + (half == 0 ? C::OFF_SQE : C::OFF_SOP);
-        for (int c0 = 0; c0 < ncols; c0 += 32) {
-          uint32_t r[32], pw[16];
-          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_QO + 128 * half + c0), r);
-          tc::tmem_wait_ld();
-          if (lane < 16) {
-            if (half == 0) {
-              const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qt_r[c0 / 8]);
+      }
+      // this half's tile (Mp or Nc) leaves while the token rows are finished
+      tc::fence_async_smem();
+      bar_half(2 + half);
+      if ((tid & 127) == 0 && !skip) {
+        if (pend >= 0) publish();
+        const int rk = (int)tile * DK;
+        if (half == 0) {
+          tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP0, 0, rk);
+          tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP1, 64, rk);
+        } else {
+          tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC0, 0, rk);
+          if (DV == 128) tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC1, 64, rk);
+        }
+        tc::tma_store_commit();
+      }
+      {
+        // token rows (M = 64 layout): half 0: Q_eff = (Q^ - P W') diag(exp(g_r)),
+        // in place over Q^; half 1: O_part.  The next 32 columns load while
+        // one is packed.
+        const int ncols = half == 0 ? 128 : DV;
+        const int i_out = 16 * q + lane;
+        uint8_t* base = sm + (half == 0 ? C::OFF_SQE : C::OFF_SOP0);
+        const int pstride = half == 0 ? C::PANEL : 8192;
+        auto pack_rows = [&](const uint32_t (&r)[32], int c0) {
+          if (lane >= 16) return;
+          uint8_t* pnl = base + (c0 >> 6) * pstride;
 #pragma unroll
-              for (int e = 0; e < 32; e += 2)
-                pw[e / 2] = tc::pack_bf16(bf16_lo_f(qw[e / 2]) - __uint_as_float(r[e]),
-                                          bf16_hi_f(qw[e / 2]) - __uint_as_float(r[e + 1]));
+          for (int uu = 0; uu < 4; ++uu) {
+            uint4* dst = reinterpret_cast<uint4*>(pnl + sw_unit(i_out, ((c0 & 63) >> 3) + uu));
+            uint32_t pw[4];
+            if (half == 0) {
+              const uint4 qv = *dst;
+              const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+              float sc[8];
+              load8f(er + c0 + 8 * uu, sc);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                pw[e] = tc::pack_bf16(sc[2 * e] * (bf16_lo_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e])),
+                                      sc[2 * e + 1] * (bf16_hi_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e + 1])));
             } else {
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) pw[e / 2] = tc::pack_bf16(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+              for (int e = 0; e < 4; ++e)
+                pw[e] = tc::pack_bf16(__uint_as_float(r[8 * uu + 2 * e]), __uint_as_float(r[8 * uu + 2 * e + 1]));
             }
-            uint8_t* pnl = stt + (c0 >> 6) * 8192;
-#pragma unroll
-            for (int uu = 0; uu < 4; ++uu)
-              *reinterpret_cast<uint4*>(pnl + sw_unit(i_out, ((c0 & 63) >> 3) + uu)) =
-                  make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
+            *dst = make_uint4(pw[0], pw[1], pw[2], pw[3]);
           }
+        };
+        uint32_t ra[32], rb[32];
+        const uint32_t col = C::COL_QO + 128 * half;
+        tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col), ra);
+        tc::tmem_wait_ld_regs(ra);
+        for (int c0 = 0; c0 < ncols; c0 += 64) {
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col + c0 + 32), rb);
+          pack_rows(ra, c0);
+          tc::tmem_wait_ld_regs(rb);
+          if (c0 + 64 < ncols) tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col + c0 + 64), ra);
+          pack_rows(rb, c0 + 32);
+          if (c0 + 64 < ncols) tc::tmem_wait_ld_regs(ra);
         }
       }
       tc::fence_async_smem();
       tc::tc_fence_before();
       bar_compute();
-      if (tid == 0) {
-        tc::fence_async_global();  // Q~ went through global with generic stores
-        const int rk = (int)tile * DK, rt = (int)tile * kChunk;
-        for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP + p * 16384, 64 * p, rk);
-        for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC + p * 16384, 64 * p, rk);
-        for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Qe, sm + C::OFF_SQE + p * 8192, 64 * p, rt);
-        for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Op, sm + C::OFF_SOP + p * 8192, 64 * p, rt);
-        tc::tma_store_commit();
-        if (a.ready) {
-          // the factors must be in global memory before the flag says so
-          tc::tma_store_wait_all();
-          __threadfence();
-          tc::st_release_gpu(a.ready + tile, 1);
+      if ((tid & 127) == 0) {
+        if (skip) {
+          // decay too steep for one reference point: hand the chunk back
+          if (tid == 0) {
+            const int idx = atomicAdd(a.fix_list, 1);
+            a.fix_list[1 + idx] = (int)tile;
+            if (a.ready) tc::st_release_gpu(a.ready + tile, 3);
+          }
+        } else {
+          const int rt = (int)tile * kChunk;
+          if (half == 0)
+            for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Qe, sm + C::OFF_SQE + p * C::PANEL, 64 * p, rt);
+          else
+            for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Op, sm + C::OFF_SOP0 + p * 8192, 64 * p, rt);
+          tc::tma_store_commit();
+          if (a.ready) pend = (int)tile;  // each storing thread adds 1: 2 = factors written
         }
       }
-      ++ex;
     }
-    if (tid == 0) tc::tma_store_wait_all();
+    if ((tid & 127) == 0) publish();
     if (!alive) {
       atomicExch(a.status, 8);
       vflag[0] = 1;
     }
-    // release the UMMA warp
+    // release the UMMA warp (it waits for slice 0 of a next task)
     vflag[1] = 1;
     __syncwarp();
-    if (lane == 0) tc::mbar_arrive(ops_ready);
+    if (lane == 0) tc::mbar_arrive(&built[0]);
   }
   tc::tc_fence_before();
   __syncthreads();

@@ -1,16 +1,16 @@
 // walk_tc.cuh -- inter-chunk state walk + chunk output on the tensor cores
 // (bf16 I/O, dk = 128, dv in {64, 128}).
 //
-// One CTA per (sequence, head, 32-column value slice).  The columns of the
+// One CTA per (sequence, head, 64-column value slice).  The columns of the
 // state evolve independently (every update is a left product), so a head's
-// dv columns are split over dv/32 CTAs; each CTA keeps its 128 x 32 slice of
+// dv columns are split over dv/64 CTAs; each CTA keeps its 128 x 64 slice of
 // the state in fp32 registers for the whole walk (4 epilogue warps: warp w
 // owns key rows 32w .. 32w+31, the TMEM lane quarter it may read; each thread
-// one key row x 32 columns).  A bf16 copy of the slice in shared memory is the
+// one key row x 64 columns).  A bf16 copy of the slice in shared memory is the
 // B operand of two UMMAs per chunk:
 //
-//   D_S = Mp . S        (M = 128 key rows,  K = 128, N = 32)
-//   D_O = Q_eff . S     (M = 64 tokens,     K = 128, N = 32)
+//   D_S = Mp . S        (M = 128 key rows,  K = 128, N = 64)
+//   D_O = Q_eff . S     (M = 64 tokens,     K = 128, N = 64)
 //
 // and then   S <- diag(gamma) S - D_S + Nc      (fp32, in registers)
 //            O  = scale * (D_O + O_part)        (query reads the updated state)
@@ -30,6 +30,11 @@
 // so nothing but the state update sits between two D_S products.  Every wait is bounded; on a
 // timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT in the status word, drains
 // what it issued and exits.
+//
+// Run beside the prep CTAs in one launch (gdn2_fused_kernel), the two TMA
+// warps wait for each chunk's ready flag before loading its factors; a chunk
+// the prep handed back to the exact kernel ends the walk early and raises the
+// redo flag, and the host-side sequence then re-runs the walk after the fixup.
 #pragma once
 
 #include <cuda.h>
@@ -42,8 +47,8 @@ namespace gdn2 {
 struct WalkTcArgs {
   CUtensorMap tm_Mp;   // Mp    [rows = max_chunks*H*128, 128] bf16, box {64, 128}, SW128
   CUtensorMap tm_Qe;   // Q_eff [rows = max_chunks*H*64,  128] bf16, box {64, 64},  SW128
-  CUtensorMap tm_Nc;   // Nc    [rows = max_chunks*H*128, dv]  bf16, box {32, 128}
-  CUtensorMap tm_Op;   // O_part[rows = max_chunks*H*64,  dv]  bf16, box {32, 64}
+  CUtensorMap tm_Nc;   // Nc    [rows = max_chunks*H*128, dv]  bf16, box {64, 128}, SW128
+  CUtensorMap tm_Op;   // O_part[rows = max_chunks*H*64,  dv]  bf16, box {64, 64},  SW128
   CUtensorMap tm_g;    // gamma [rows = max_chunks*H,     128] fp32, box {128, 1}
   SeqMap map;
   int H;
@@ -53,23 +58,26 @@ struct WalkTcArgs {
   float* hT;
   float* chunk_states;
   int* status;
+  const int* ready;    // optional [max_chunks * H]: wait for 2 (written); 3 = handed back
+  int* redo;           // set when a handed-back chunk ended the walk early
+  const int* gate;     // optional: the kernel does nothing unless *gate != 0
 };
 
 template <int DV>
 struct WalkTcCfg {
   static constexpr int DK = 128;
-  static constexpr int NSL = 32;                 // value columns per CTA
+  static constexpr int NSL = 64;                 // value columns per CTA
   static constexpr int SLICES = DV / NSL;
   static constexpr int EPI_WARPS = 4;              // state warps 0-3, output warps 4-7
   static constexpr int MMA_WARP = 8, TMA_A_WARP = 9, TMA_B_WARP = 10;
   static constexpr int THREADS = 11 * 32;
-  static constexpr int STAGES_A = 3;
-  static constexpr int STAGES_B = 4;
+  static constexpr int STAGES_A = 2;
+  static constexpr int STAGES_B = 3;
   static constexpr int MP_BYTES = DK * DK * 2;             // 32 KiB
   static constexpr int QE_BYTES = kChunk * DK * 2;         // 16 KiB
   static constexpr int A_BYTES = MP_BYTES + QE_BYTES;
-  static constexpr int NC_BYTES = DK * NSL * 2;            // 8 KiB
-  static constexpr int OP_BYTES = kChunk * NSL * 2;        // 4 KiB
+  static constexpr int NC_BYTES = DK * NSL * 2;            // 16 KiB, SW128 rows of 64
+  static constexpr int OP_BYTES = kChunk * NSL * 2;        // 8 KiB, SW128 rows of 64
   static constexpr int G_BYTES = DK * 4;                   // 512 B
   static constexpr int B_BYTES = NC_BYTES + OP_BYTES + G_BYTES;
   static constexpr int B_STRIDE = (B_BYTES + 1023) / 1024 * 1024;
@@ -79,7 +87,9 @@ struct WalkTcCfg {
   static constexpr int S_BYTES = DK * NSL * 2;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + STAGES_A * A_BYTES + STAGES_B * B_STRIDE + 2 * S_BYTES + BAR_BYTES;
-  static constexpr int TMEM_COLS = 128;  // D_S [0,32), D_O[0] [32,64), D_O[1] [64,96)
+  static constexpr int TMEM_COLS = 256;  // D_S [0,64), D_O[0] [64,128), D_O[1] [128,192)
+  static_assert(NSL == 64, "SW128 Nc / O_part rows hold 64 columns");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ void set_timeout(int* status, int* s_abort) {
@@ -88,14 +98,48 @@ __device__ __forceinline__ void set_timeout(int* status, int* s_abort) {
 }
 
 
+// Bounded wait that also ends when the CTA winds down (abort flag): true once
+// the phase has completed; a timeout is recorded in the status word.
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, int* status, int* s_abort) {
+  if (tc::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = tc::global_ns();
+  for (;;) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(s_abort)) return false;
+    if (tc::global_ns() - t0 > 2000000000ull) {
+      set_timeout(status, s_abort);
+      return false;
+    }
+  }
+}
+
+// Bounded wait until chunk tile `t` is ready; false on a timeout or when the
+// prep handed the chunk back (then the redo flag is raised).
+__device__ __forceinline__ bool wait_chunk_ready(const WalkTcArgs& a, int t, int* s_abort) {
+  const uint64_t t0 = tc::global_ns();
+  for (;;) {
+    const int r = tc::ld_acquire_gpu(a.ready + t);
+    if (r == 2) break;
+    if (r == 3) {
+      atomicExch(a.redo, 1);
+      *reinterpret_cast<volatile int*>(s_abort) = 1;
+      return false;
+    }
+    if (*reinterpret_cast<volatile int*>(s_abort)) return false;
+    if (tc::global_ns() - t0 > 2000000000ull) {
+      set_timeout(a.status, s_abort);
+      return false;
+    }
+  }
+  // the TMA loads that follow read what the flag published
+  tc::fence_async_global();
+  return true;
+}
+
 template <int DV>
-__global__ void __launch_bounds__(WalkTcCfg<DV>::THREADS, 1)
-walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
+__device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
   using C = WalkTcCfg<DV>;
   constexpr int DK = C::DK, NSL = C::NSL;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = tc::smem_u32(smem_raw);
-  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* ringA = sm;
   uint8_t* ringB = ringA + C::STAGES_A * C::A_BYTES;
   uint8_t* sS = ringB + C::STAGES_B * C::B_STRIDE;          // [2][S_BYTES]
@@ -107,14 +151,15 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
   uint64_t* o_done = s_done + 1;             // D_O of the current chunk is ready
   uint64_t* s_ready = o_done + 1;            // bf16 state operand written
   uint64_t* o_free = s_ready + 1;            // [2] D_O buffer read by the output warps
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(o_free + 2);
+  uint64_t* fin = o_free + 2;                // every issued UMMA has finished
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(fin + 1);
   int* s_abort = reinterpret_cast<int*>(tslot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const int sl = blockIdx.x % C::SLICES;
-  const int h = (blockIdx.x / C::SLICES) % H;
-  const int n = blockIdx.x / (C::SLICES * H);
+  const int sl = cta % C::SLICES;
+  const int h = (cta / C::SLICES) % H;
+  const int n = cta / (C::SLICES * H);
   const int col0 = sl * NSL;
   const int c_begin = a.map.chunk_off[n];
   const int nch = a.map.chunk_off[n + 1] - c_begin;
@@ -134,6 +179,7 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     tc::mbar_init(s_ready, C::EPI_WARPS);
     tc::mbar_init(&o_free[0], C::EPI_WARPS);
     tc::mbar_init(&o_free[1], C::EPI_WARPS);
+    tc::mbar_init(fin, 1);
     *s_abort = 0;
     tc::fence_mbar_init();
   }
@@ -187,32 +233,36 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
 #pragma unroll
         for (int i = 0; i < NSL; i += 4) *reinterpret_cast<float4*>(cs + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
       }
-      if (!tc::mbar_wait(&fullB[sb], (j / C::STAGES_B) & 1)) {
-        set_timeout(a.status, s_abort);
-        break;
-      }
-      // Nc row (32 bf16) and gamma before the product is ready
+      if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort)) break;
+      // Nc row (64 bf16, SW128) and gamma before the product is ready
       const float gam = reinterpret_cast<const float*>(stB + C::NC_BYTES + C::OP_BYTES)[row];
       uint32_t ncw[NSL / 2];
 #pragma unroll
       for (int u = 0; u < NSL / 8; ++u) {
-        const uint4 t = reinterpret_cast<const uint4*>(stB + row * NSL * 2)[u];
+        const uint4 t = *reinterpret_cast<const uint4*>(stB + row * 128 + ((u ^ (row & 7)) << 4));
         ncw[4 * u] = t.x; ncw[4 * u + 1] = t.y; ncw[4 * u + 2] = t.z; ncw[4 * u + 3] = t.w;
       }
-      if (!tc::mbar_wait(s_done, j & 1)) {
-        set_timeout(a.status, s_abort);
-        break;
-      }
+      if (!wwait(s_done, j & 1, a.status, s_abort)) break;
       tc::tc_fence_after();
       // S <- gamma * S - Mp S + Nc
-      uint32_t d[32];
-      tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * warp, 0), d);
-      tc::tmem_wait_ld();
+      {
+        uint32_t d0[32], d1[32];
+        tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * warp, 0), d0);
+        tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * warp, 32), d1);
+        tc::tmem_wait_ld_regs(d0);
+        tc::tmem_wait_ld_regs(d1);
 #pragma unroll
-      for (int e = 0; e < NSL; e += 2) {
-        const uint32_t w2 = ncw[e / 2];
-        S[e] = fmaf(gam, S[e], bf16_lo_f(w2) - __uint_as_float(d[e]));
-        S[e + 1] = fmaf(gam, S[e + 1], bf16_hi_f(w2) - __uint_as_float(d[e + 1]));
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t w2 = ncw[e / 2];
+          S[e] = fmaf(gam, S[e], bf16_lo_f(w2) - __uint_as_float(d0[e]));
+          S[e + 1] = fmaf(gam, S[e + 1], bf16_hi_f(w2) - __uint_as_float(d0[e + 1]));
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t w2 = ncw[16 + e / 2];
+          S[32 + e] = fmaf(gam, S[32 + e], bf16_lo_f(w2) - __uint_as_float(d1[e]));
+          S[32 + e + 1] = fmaf(gam, S[32 + e + 1], bf16_hi_f(w2) - __uint_as_float(d1[e + 1]));
+        }
       }
       // D_O(j-1) read sS[(j+1)&1]; it was issued before D_S(j), so it is done
       store_state((j + 1) & 1);
@@ -232,31 +282,32 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int sb = j % C::STAGES_B;
       const uint8_t* stB = ringB + sb * C::B_STRIDE;
-      if (!tc::mbar_wait(&fullB[sb], (j / C::STAGES_B) & 1) || !tc::mbar_wait(o_done, j & 1)) {
-        set_timeout(a.status, s_abort);
+      if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort) || !wwait(o_done, j & 1, a.status, s_abort))
         break;
-      }
       tc::tc_fence_after();
-      uint32_t d[32];
-      tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * ow, (uint32_t)NSL * (1u + (j & 1))), d);
-      tc::tmem_wait_ld();
+      uint32_t d0[32], d1[32];
+      tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * ow, (uint32_t)NSL * (1u + (j & 1))), d0);
+      tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * ow, (uint32_t)NSL * (1u + (j & 1)) + 32), d1);
+      tc::tmem_wait_ld_regs(d0);
+      tc::tmem_wait_ld_regs(d1);
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&o_free[j & 1]);
       const int t0 = s_begin + j * kChunk;
       const int len = min(kChunk, s_end - t0);
       if (lane < 16 && i_tok < len) {
-        const uint4* op = reinterpret_cast<const uint4*>(stB + C::NC_BYTES + i_tok * NSL * 2);
+        const uint8_t* op = stB + C::NC_BYTES + i_tok * 128;
         uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)(t0 + i_tok) * H + h) * DV + col0);
 #pragma unroll
         for (int u = 0; u < NSL / 8; ++u) {
-          const uint4 o4 = op[u];
+          const uint4 o4 = *reinterpret_cast<const uint4*>(op + ((u ^ (i_tok & 7)) << 4));
           const uint32_t ow4[4] = {o4.x, o4.y, o4.z, o4.w};
+          const uint32_t* dd = u < 4 ? d0 + 8 * u : d1 + 8 * (u - 4);
           uint32_t pw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            pw[e] = tc::pack_bf16(a.scale * (__uint_as_float(d[8 * u + 2 * e]) + bf16_lo_f(ow4[e])),
-                                  a.scale * (__uint_as_float(d[8 * u + 2 * e + 1]) + bf16_hi_f(ow4[e])));
+            pw[e] = tc::pack_bf16(a.scale * (__uint_as_float(dd[2 * e]) + bf16_lo_f(ow4[e])),
+                                  a.scale * (__uint_as_float(dd[2 * e + 1]) + bf16_hi_f(ow4[e])));
           dst[u] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
       }
@@ -269,14 +320,10 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     constexpr uint32_t idO = tc::idesc_bf16(64, NSL, false, true);
     const uint64_t mp_d0 = tc::sdesc(tc::smem_u32(ringA), 16, 1024, tc::kLayoutSW128);
     const uint64_t sb_d0 = tc::sdesc(tc::smem_u32(sS), C::S_LBO, 128, tc::kLayoutNone);
-    int committed = 0;
     for (int j = 0; j < nch; ++j) {
       const int st = j % C::STAGES_A;
-      const bool ok = tc::mbar_wait(&fullA[st], (j / C::STAGES_A) & 1) && tc::mbar_wait(s_ready, j & 1);
-      if (!ok) {
-        set_timeout(a.status, s_abort);
+      if (!wwait(&fullA[st], (j / C::STAGES_A) & 1, a.status, s_abort) || !wwait(s_ready, j & 1, a.status, s_abort))
         break;
-      }
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       tc::tc_fence_after();
       // descriptors: the start address sits in the low bits (16-byte units),
@@ -291,11 +338,7 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
       tc::umma_commit(s_done);
       // the output warps have read D_O(j-1): keeps every o_done waiter within
       // one phase (and frees the D_O buffer D_O(j+1) will use)
-      if (j >= 1 && !tc::mbar_wait(&o_free[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
-        set_timeout(a.status, s_abort);
-        committed = j;
-        break;
-      }
+      if (j >= 1 && !wwait(&o_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, s_abort)) break;
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s)
         tc::umma_f16(tbase + (uint32_t)NSL * (1u + (j & 1)),
@@ -303,11 +346,10 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
                      sb_d + (uint64_t)((s * 2 * C::S_LBO) >> 4), idO, s > 0);
       tc::umma_commit(o_done);
       tc::umma_commit(&emptyA[st]);
-      committed = j + 1;
     }
     // every issued UMMA has finished before TMEM is released
-    if (committed > 0) tc::mbar_wait(&emptyA[(committed - 1) % C::STAGES_A], ((committed - 1) / C::STAGES_A) & 1);
-    if (committed < nch && *reinterpret_cast<volatile int*>(s_abort)) tc::mbar_wait(s_done, committed & 1);
+    tc::umma_commit(fin);
+    tc::mbar_wait(fin, 0);
   } else if (warp == C::TMA_A_WARP && lane == 0) {
     // ------------------------------------------------ ring A producer (TMA) --
     tc::prefetch_tmap(&a.tm_Mp);
@@ -316,10 +358,8 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int c = c_begin + j, st = j % C::STAGES_A;
-      if (j >= C::STAGES_A && !tc::mbar_wait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1)) {
-        set_timeout(a.status, s_abort);
-        break;
-      }
+      if (j >= C::STAGES_A && !wwait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1, a.status, s_abort)) break;
+      if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringA + st * C::A_BYTES;
       tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
       const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
@@ -342,10 +382,8 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int c = c_begin + j, st = j % C::STAGES_B;
-      if (j >= C::STAGES_B && !tc::mbar_wait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1)) {
-        set_timeout(a.status, s_abort);
-        break;
-      }
+      if (j >= C::STAGES_B && !wwait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1, a.status, s_abort)) break;
+      if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringB + st * C::B_STRIDE;
       tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
       tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
@@ -362,6 +400,16 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tbase, C::TMEM_COLS);
   }
+}
+
+template <int DV>
+__global__ void __launch_bounds__(WalkTcCfg<DV>::THREADS, 1)
+walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
+  if (a.gate && *a.gate == 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  walk_tc_cta<DV>(a, sm, blockIdx.x);
 }
 
 }  // namespace gdn2

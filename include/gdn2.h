@@ -132,6 +132,9 @@ typedef struct gdn2_ws_layout {
   size_t off_fix;            /* int32 [1 + max_chunks * H]: chunks whose decay   */
                              /* is too steep for the tensor-core prep, redone    */
                              /* exactly ([0] = count, then chunk * H + head)     */
+  size_t off_sync;           /* int32 [2 + max_chunks * H] (set 1): [0] next     */
+                             /* prep task, [1] walk redo flag, then one ready    */
+                             /* flag per (chunk, head) for the fused prep + walk */
 } gdn2_ws_layout;
 
 /* Bytes of workspace gdn2_chunk_fwd needs for `desc` (0 if desc is invalid).
@@ -152,7 +155,11 @@ GDN2_API gdn2_status gdn2_workspace_layout(const gdn2_desc* desc, gdn2_ws_layout
  *   cu_seqlens : int32 [num_seqs + 1] (device) or NULL for B dense sequences
  *   out        : [B, T, H, dv]  io dtype
  *   hT         : [N, H, dk, dv] fp32 final state, or NULL to skip; may alias h0
- * Asynchronous on `stream`.  Runs gdn2_chunk_prep then gdn2_chunk_walk. */
+ * Asynchronous on `stream`.  For bf16 I/O with dk = 128, when the walk needs
+ * at most (SM count - 32) CTAs (sequences x H x dv/64), the prep and the walk
+ * run in one launch and the walk takes each chunk's factors as soon as they
+ * are written (gdn2_chunk_fused); otherwise it runs gdn2_chunk_prep then
+ * gdn2_chunk_walk.  Both orders compute the same values. */
 GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
                            const float* log_alpha, const float* b, const float* w, float scale,
                            const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
@@ -172,6 +179,23 @@ GDN2_API gdn2_status gdn2_chunk_prep(const gdn2_desc* desc, const void* q, const
 GDN2_API gdn2_status gdn2_chunk_walk(const gdn2_desc* desc, float scale, const float* h0,
                             const int32_t* cu_seqlens, void* out, float* hT,
                             float* chunk_states, cudaStream_t stream);
+
+/* The bookkeeping every chunked call starts with: chunk offsets of the
+ * sequences (from cu_seqlens on the device), the status word, and the lists
+ * and flags of the affine path, all in the workspace.  gdn2_chunk_fwd and
+ * gdn2_chunk_prep run it themselves; gdn2_chunk_fused needs it first. */
+GDN2_API gdn2_status gdn2_chunk_plan(const gdn2_desc* desc, const int32_t* cu_seqlens, cudaStream_t stream);
+
+/* The single launch of gdn2_chunk_fwd's fused path (see there), without the
+ * plan before it or the exact redo after it of chunks whose decay is too steep
+ * for the tensor-core prep; call gdn2_chunk_plan first.  A call then gives the
+ * full result unless such a chunk exists, which gdn2_chunk_fwd handles.
+ * Returns GDN2_ERR_UNSUPPORTED when the problem does not take the fused path
+ * (not bf16 with dk = 128, or the walk needs too many CTAs). */
+GDN2_API gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                             const float* log_alpha, const float* b, const float* w, float scale,
+                             const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                             cudaStream_t stream);
 
 /* One decode token for a batch of states, updated in place.
  * desc: B = batch, H, dk, dv, io (T, num_seqs and the workspace are ignored).
