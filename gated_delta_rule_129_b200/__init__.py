@@ -64,7 +64,7 @@ class WsLayout(ctypes.Structure):
                 ("off_gamma_last", ctypes.c_size_t), ("off_Mp", ctypes.c_size_t),
                 ("off_Nc", ctypes.c_size_t), ("off_chunk_offsets", ctypes.c_size_t),
                 ("off_status", ctypes.c_size_t), ("off_fix", ctypes.c_size_t),
-                ("off_sync", ctypes.c_size_t)]
+                ("off_sync", ctypes.c_size_t), ("off_colscale", ctypes.c_size_t)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}

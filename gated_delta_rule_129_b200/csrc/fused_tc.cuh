@@ -4,7 +4,9 @@
 // the prep could use all of them, and run back to back the two add up.  Here
 // one persistent grid of one CTA per SM holds both: the last n_walk CTAs walk
 // (one per sequence, head and 64-column value slice), the others take prep
-// tasks in chunk-major order from a shared counter.  A prep CTA publishes a
+// tasks in chunk-major order from a shared counter.  The walk CTAs take prep
+// tasks too until the counter reaches stop_at, chosen on the host so that
+// the walk, started then, ends about when the prep does.  A prep CTA publishes a
 // chunk's ready flag once its factors are in global memory (where they are
 // still in L2 when the walk reads them); the walk's TMA warps wait for the
 // flag before loading.  Only the walk waits, and only for work that the prep
@@ -32,8 +34,14 @@ fused_tc_kernel(const __grid_constant__ PrepTcArgs pa, const __grid_constant__ W
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  if ((int)blockIdx.x < n_prep) prep_tc_cta<DV>(pa, sm, blockIdx.x, n_prep);
-  else walk_tc_cta<DV>(wa, sm, (int)blockIdx.x - n_prep);
+  if ((int)blockIdx.x < n_prep) {
+    prep_tc_cta<DV>(pa, sm, blockIdx.x, n_prep);
+  } else {
+    // early on, the walk would only wait for the prep wavefront: take prep
+    // tasks until the counter reaches pa.stop_at, then walk
+    prep_tc_cta<DV>(pa, sm, blockIdx.x, gridDim.x, true);
+    walk_tc_cta<DV>(wa, sm, (int)blockIdx.x - n_prep);
+  }
 }
 
 }  // namespace gdn2

@@ -91,6 +91,7 @@ gdn2_status make_layout(const gdn2_desc* d, bool packed, Layout* out) {
   L.off_status = off;     off = align_up(off + sizeof(int32_t));
   L.off_fix = off;        off = align_up(off + (wy ? 0 : (size_t)(1 + (size_t)max_chunks * d->H) * sizeof(int32_t)));
   L.off_sync = off;       off = align_up(off + (wy ? 0 : (size_t)(2 + (size_t)max_chunks * d->H) * sizeof(int32_t)));
+  L.off_colscale = off;   off = align_up(off + (wy ? 0 : (size_t)max_chunks * d->H * d->dk * sizeof(float)));
   L.total_bytes = off;
   out->N = N;
   return GDN2_OK;
@@ -174,6 +175,7 @@ gdn2_status fill_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, con
   a.Mp = at<bf16>(d->workspace, L.l.off_Mp);
   a.Nc = at<bf16>(d->workspace, L.l.off_Nc);
   a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
+  a.colscale = at<float>(d->workspace, L.l.off_colscale);
   a.fix_list = at<int32_t>(d->workspace, L.l.off_fix);
   a.status = at<int32_t>(d->workspace, L.l.off_status);
   a.ready = nullptr;
@@ -222,6 +224,7 @@ gdn2::PrepArgs<IO, FT> prep_args(const gdn2_desc* d, const Layout& L, const void
   a.gamma_last = at<float>(d->workspace, L.l.off_gamma_last);
   a.Mp = at<FT>(d->workspace, L.l.off_Mp);
   a.Nc = at<FT>(d->workspace, L.l.off_Nc);
+  a.colscale = L.l.factor_set == 1 ? at<float>(d->workspace, L.l.off_colscale) : nullptr;
   return a;
 }
 
@@ -285,7 +288,9 @@ gdn2_status fill_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const
       !gdn2::make_tmap(&a.tm_Nc, at<void>(d->workspace, L.l.off_Nc), BF, 2, d_nc, st_v, b_nc, SW) ||
       !gdn2::make_tmap(&a.tm_Op, at<void>(d->workspace, L.l.off_Opart), BF, 2, d_op, st_v, b_op, SW) ||
       !gdn2::make_tmap(&a.tm_g, at<void>(d->workspace, L.l.off_gamma_last), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d_g, st_g,
-                       b_g, CU_TENSOR_MAP_SWIZZLE_NONE))
+                       b_g, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !gdn2::make_tmap(&a.tm_cs, at<void>(d->workspace, L.l.off_colscale), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d_g,
+                       st_g, b_g, CU_TENSOR_MAP_SWIZZLE_NONE))
     return GDN2_ERR_CUDA;
   a.map = seq_map(d, L, cu);
   a.H = d->H;
@@ -378,6 +383,18 @@ gdn2_status launch_fused_tc(const gdn2_desc* d, const Layout& L, const void* q, 
   wa.redo = sync + 1;
   const int n_sm = sm_count();
   const int n_walk = L.N * d->H * gdn2::WalkTcCfg<DV>::SLICES;
+  // When the walk CTAs stop taking prep tasks: beside the prep, a walk step
+  // costs about a ninth of a prep task on one SM (measured at 16K x 1:
+  // ~1.4 us per chunk against ~12 us per task), so a walk of nch chunks
+  // started when nch * (n_sm - n_walk) / 9 tasks are left ends about with
+  // the prep (a sweep of the switch point at 16K x 1 has its flat optimum
+  // there).
+  {
+    const long long tasks = (long long)L.l.max_chunks * d->H;
+    const long long nch = ((long long)d->B * d->T + (long long)kChunk * L.N - 1) / ((long long)kChunk * L.N);
+    const long long left = nch * (n_sm - n_walk) / 9;
+    pa.stop_at = (int)std::max(0ll, tasks - left);
+  }
   auto kern = gdn2::fused_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;

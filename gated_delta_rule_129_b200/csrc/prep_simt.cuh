@@ -39,6 +39,7 @@ struct PrepArgs {
   FT* Qeff;
   FT* Opart;
   float* gamma_last;
+  float* colscale;   // affine set: column scale of Mp and Q_eff (1 here: stored unscaled)
   FT* Mp;  // affine factor set only: Kbar^T W   [., H, DK, DK]
   FT* Nc;  // affine factor set only: Kbar^T U~  [., H, DK, DV]
 };
@@ -149,6 +150,7 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     sk[i * LK + cc] = i < len ? sk[i * LK + cc] * expf(sg[(kChunk - 1) * LK + cc] - sg[i * LK + cc]) : 0.f;
   }
   if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
+  if (AFFINE && a.colscale && tid < DK) a.colscale[((size_t)c * H + h) * DK + tid] = 1.f;
   __syncthreads();
   // Forward substitution, row by row: W_i = E~_i - sum_{j<i} A_ij W_j, and the
   // same for U~ with Z.  One thread per column of [W | U~].

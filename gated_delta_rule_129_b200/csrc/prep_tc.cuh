@@ -26,8 +26,10 @@
 //     decayed operands are the same tensors scaled per channel,
 //        E~ = E^ diag(exp(g_r)),  Q~ = Q^ diag(exp(g_r)),
 //        Kbar = K^ diag(exp(g_n - g_r)),
-//     so they are never built: the scales are applied to rows or columns of
-//     the fp32 products in the epilogues.
+//     so they are never built: exp(g_n - g_r) scales the rows of R in an
+//     epilogue, and exp(g_r), a column scale of Mp and of Q_eff, is stored
+//     beside them (colscale) and applied by the walk to the rows of the state
+//     operand (Mp S = Mp' (diag(exp(g_r)) S), and likewise Q_eff S).
 //  2. UMMA 1, accumulated slice by slice as the operands are built:
 //     [E^; Q^] . K^T (M = 128, N = 64, K = 128) -> A (strictly lower part of
 //     rows 0..63) and P (lower part with diagonal, rows 64..127).
@@ -38,8 +40,8 @@
 //  4. UMMA 2: [R'_hi | R'_lo] = K^^T [T_hi | T_lo], [V_hi | V_lo] = P [T_hi | T_lo];
 //     R = Kbar^T T = diag(exp(g_n - g_r)) R'.
 //  5. UMMA 3: [Mp' | Nc] = R [E^ | Z], [P W' | O_part] = V [E^ | Z]; the
-//     epilogue writes Mp = Mp' diag(exp(g_r)), Nc, Q_eff = (Q^ - P W')
-//     diag(exp(g_r)) and O_part (bf16) by TMA stores.
+//     epilogue writes Mp', Nc, Q_eff' = Q^ - P W' and O_part (bf16) by TMA
+//     stores; Mp = Mp' diag(exp(g_r)) and Q_eff = Q_eff' diag(exp(g_r)).
 // Rows past the chunk's last token are zero in every operand, so they add
 // nothing; the padded rows of Q_eff and O_part come out as exact zeros.
 #pragma once
@@ -63,9 +65,11 @@ struct PrepTcArgs {
   __nv_bfloat16* Mp;     // [max_chunks, H, 128, 128]
   __nv_bfloat16* Nc;     // [max_chunks, H, 128, DV]
   float* gamma_last;     // [max_chunks, H, 128]
+  float* colscale;       // [max_chunks, H, 128]: exp(g_r), the column scale of the stored Mp and Q_eff
   int32_t* fix_list;     // [0] = count, then c * H + h of handed-back chunks
   int* ready;            // optional [max_chunks * H], zeroed: 2 = factors written, 3 = handed back
   int* task_counter;     // optional: tasks taken dynamically (else static striding)
+  int stop_at;           // with task_counter: a CTA given a later role stops taking tasks here
   int* status;
 };
 
@@ -148,8 +152,10 @@ __device__ __forceinline__ void load8f_sw(const float* tile, int t, int g, float
   v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
 }
 
+// `stopper`: this CTA takes no task once the shared counter has reached
+// a.stop_at (it has another role to play after this one).
 template <int DV>
-__device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int cta_count) {
+__device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int cta_count, bool stopper = false) {
   using C = PrepTcCfg<DV>;
   constexpr int DK = C::DK;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);  // [NSLOT] producer -> scan
@@ -167,8 +173,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   int* slot_task = s_flag + 2;                        // [NSLOT] task id of the slot's slice
   int* slot_skip = slot_task + C::NSLOT;              // [NSLOT] decay range exceeded
   float* s_gr = reinterpret_cast<float*>(sm + C::OFF_BAR + 512);  // [NSLOT][32] g_r
-  float* s_er = s_gr + C::NSLOT * 32;                             // [2][128] exp(g_r), by task parity
-  float* s_enr = s_er + 2 * DK;                                   // [2][128] exp(g_n - g_r)
+  float* s_enr = s_gr + C::NSLOT * 32;                            // [2][128] exp(g_n - g_r), by task parity
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
@@ -192,7 +197,8 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   }
   if (warp == C::MMA_WARP) {
     tc::tmem_alloc(tslot, C::TMEM_COLS);
-    tc::tmem_relinquish();
+    // a CTA with a later role allocates again, so it keeps the permit
+    if (!stopper) tc::tmem_relinquish();
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -211,7 +217,10 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       bool ok = true;
       for (bool more = true; more && ok;) {
         int task;
-        if (a.task_counter) task = atomicAdd(a.task_counter, 1);
+        if (a.task_counter) {
+          task = (stopper && *reinterpret_cast<volatile int*>(a.task_counter) >= a.stop_at)
+                     ? ntasks : atomicAdd(a.task_counter, 1);
+        }
         else task = cta_rank + cta_count * (k_static++);
         if (task >= ntasks) task = -1;
         int h = 0, t0 = 0;
@@ -281,9 +290,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         const float g0 = v[0], gr = v[32], gn = v[kChunk - 1];
         const bool bad = (g0 - gr > 60.f) || (gr - gn > 60.f);
         s_gr[slot * 32 + lane] = gr;
-        s_er[tpar * DK + C::KS * s_in + lane] = __expf(gr);
         s_enr[tpar * DK + C::KS * s_in + lane] = __expf(gn - gr);
         a.gamma_last[tile * DK + C::KS * s_in + lane] = expf(gn);
+        a.colscale[tile * DK + C::KS * s_in + lane] = __expf(gr);
         if (a.ready) __threadfence();  // published with the chunk's other factors
         const unsigned any = __ballot_sync(0xffffffffu, bad);
         if (lane == 0) slot_skip[slot] = any != 0u;
@@ -562,36 +571,43 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         *reinterpret_cast<float2*>(TS + (16 * bb + r) * C::LDT + 16 * ba + c) = make_float2(-y0, -y1);
       }
       bar_compute();
-      // (c) 32 -> 64: block (1,0) of 32 x 32 blocks; thread = row r, columns c..c+3.
+      // (c) 32 -> 64: block (1,0) of 32 x 32 blocks, T21 = -T22 (A21 T11).
+      // Both products skip the zero triangle of their T factor, with the
+      // triangle's bound uniform per warp: X = A21 T11 by (lane = row r,
+      // warp = columns 4w..4w+3, k >= 4w), then T21 by (lane = column,
+      // warp = rows 4w..4w+3, k <= 4w+3).  A row of A21 and of T22 is read
+      // as float4 by one lane; the T11 / X values every lane needs are
+      // broadcasts.
       {
-        const int r = tid >> 3, c = 4 * (tid & 7);
+        const int r = lane, c0 = 4 * warp;
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k0 = c0; k0 < 32; k0 += 4) {
+          const float4 av = *reinterpret_cast<const float4*>(AS + (32 + r) * C::LDA + k0);
+          const float a4[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
-        for (int k0 = 0; k0 < 32; k0 += 8) {
-          float av[8];
-          load8f(AS + (32 + r) * C::LDA + k0, av);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float4 tv = *reinterpret_cast<const float4*>(TS + (k0 + k) * C::LDT + c);
-            x.x = fmaf(av[k], tv.x, x.x); x.y = fmaf(av[k], tv.y, x.y);
-            x.z = fmaf(av[k], tv.z, x.z); x.w = fmaf(av[k], tv.w, x.w);
+          for (int k = 0; k < 4; ++k) {
+            const float4 tv = *reinterpret_cast<const float4*>(TS + (k0 + k) * C::LDT + c0);
+            x.x = fmaf(a4[k], tv.x, x.x); x.y = fmaf(a4[k], tv.y, x.y);
+            x.z = fmaf(a4[k], tv.z, x.z); x.w = fmaf(a4[k], tv.w, x.w);
           }
         }
-        *reinterpret_cast<float4*>(XS + r * 32 + c) = x;
+        *reinterpret_cast<float4*>(XS + r * 32 + c0) = x;
         bar_compute();
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int col = lane, r0 = 4 * warp;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 0; k0 <= r0; k0 += 4) {
+          float xv[4];
 #pragma unroll
-        for (int k0 = 0; k0 < 32; k0 += 8) {
-          float tv[8];
-          load8f(TS + (32 + r) * C::LDT + 32 + k0, tv);
+          for (int k = 0; k < 4; ++k) xv[k] = XS[(k0 + k) * 32 + col];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float4 xv = *reinterpret_cast<const float4*>(XS + (k0 + k) * 32 + c);
-            y.x = fmaf(tv[k], xv.x, y.x); y.y = fmaf(tv[k], xv.y, y.y);
-            y.z = fmaf(tv[k], xv.z, y.z); y.w = fmaf(tv[k], xv.w, y.w);
+          for (int i = 0; i < 4; ++i) {
+            const float4 tv = *reinterpret_cast<const float4*>(TS + (32 + r0 + i) * C::LDT + 32 + k0);
+            y[i] = fmaf(tv.x, xv[0], y[i]); y[i] = fmaf(tv.y, xv[1], y[i]);
+            y[i] = fmaf(tv.z, xv[2], y[i]); y[i] = fmaf(tv.w, xv[3], y[i]);
           }
         }
-        *reinterpret_cast<float4*>(TS + (32 + r) * C::LDT + c) = make_float4(-y.x, -y.y, -y.z, -y.w);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) TS[(32 + r0 + i) * C::LDT + col] = -y[i];
       }
       bar_compute();
       // T -> [T_hi | T_lo], MN-major SW128 (row i, 64 columns j per panel);
@@ -668,11 +684,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       // Results go to SW128 staging in the (now free) operand area and leave
       // by TMA bulk stores, so every global write is a whole tile row.
       tc::tc_fence_after();
-      const float* er = s_er + (ex & 1) * DK;   // exp(g_r) by key channel
       {
         const int m = 32 * q + lane;  // key channel row of Mp / Nc
-        // half 0: Mp = Mp' diag(exp(g_r)), columns 0..127; half 1: Nc columns
-        // 0..DV-1 (TMEM 128..)
+        // half 0: Mp' columns 0..127; half 1: Nc columns 0..DV-1 (TMEM 128..)
         const int ncols = half == 0 ? 128 : DV;
         for (int c0 = 0; c0 < ncols; c0 += 64) {
           uint32_t r0[32], r1[32];
@@ -684,16 +698,11 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
 #pragma unroll
           for (int uu = 0; uu < 8; ++uu) {
             const uint32_t* r = uu < 4 ? r0 + 8 * uu : r1 + 8 * (uu - 4);
-            float sc[8];
-            if (half == 0) load8f(er + c0 + 8 * uu, sc);
-            else
-#pragma unroll
-              for (int e = 0; e < 8; ++e) sc[e] = 1.f;
             *reinterpret_cast<uint4*>(pnl + sw_unit(m, uu)) =
-                make_uint4(tc::pack_bf16(sc[0] * __uint_as_float(r[0]), sc[1] * __uint_as_float(r[1])),
-                           tc::pack_bf16(sc[2] * __uint_as_float(r[2]), sc[3] * __uint_as_float(r[3])),
-                           tc::pack_bf16(sc[4] * __uint_as_float(r[4]), sc[5] * __uint_as_float(r[5])),
-                           tc::pack_bf16(sc[6] * __uint_as_float(r[6]), sc[7] * __uint_as_float(r[7])));
+                make_uint4(tc::pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                           tc::pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                           tc::pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                           tc::pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7])));
           }
         }
       }
@@ -713,9 +722,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         tc::tma_store_commit();
       }
       {
-        // token rows (M = 64 layout): half 0: Q_eff = (Q^ - P W') diag(exp(g_r)),
-        // in place over Q^; half 1: O_part.  The next 32 columns load while
-        // one is packed.
+        // token rows (M = 64 layout): half 0: Q_eff' = Q^ - P W', in place
+        // over Q^; half 1: O_part.  The next 32 columns load while one is
+        // packed.
         const int ncols = half == 0 ? 128 : DV;
         const int i_out = 16 * q + lane;
         uint8_t* base = sm + (half == 0 ? C::OFF_SQE : C::OFF_SOP0);
@@ -730,12 +739,10 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
             if (half == 0) {
               const uint4 qv = *dst;
               const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-              float sc[8];
-              load8f(er + c0 + 8 * uu, sc);
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                pw[e] = tc::pack_bf16(sc[2 * e] * (bf16_lo_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e])),
-                                      sc[2 * e + 1] * (bf16_hi_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e + 1])));
+                pw[e] = tc::pack_bf16(bf16_lo_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e]),
+                                      bf16_hi_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e + 1]));
             } else {
 #pragma unroll
               for (int e = 0; e < 4; ++e)
@@ -795,6 +802,23 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
     tc::tc_fence_after();
     tc::tmem_dealloc(tbase, C::TMEM_COLS);
   }
+  if (stopper && tid == 0) {
+    // the shared memory is about to be laid out for the next role
+    for (int s = 0; s < C::NSLOT; ++s) {
+      tc::mbar_inval(&full[s]);
+      tc::mbar_inval(&gready[s]);
+      tc::mbar_inval(&empty[s]);
+    }
+    for (int s = 0; s < C::SLICES; ++s) tc::mbar_inval(&built[s]);
+    tc::mbar_inval(mma1_done);
+    tc::mbar_inval(t_ready);
+    tc::mbar_inval(mma2_done);
+    tc::mbar_inval(rv_ready);
+    tc::mbar_inval(mma3_done);
+    tc::mbar_inval(fin);
+    tc::fence_async_smem();
+  }
+  if (stopper) __syncthreads();
 }
 
 template <int DV>

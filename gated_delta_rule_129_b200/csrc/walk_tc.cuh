@@ -9,8 +9,11 @@
 // one key row x 64 columns).  A bf16 copy of the slice in shared memory is the
 // B operand of two UMMAs per chunk:
 //
-//   D_S = Mp . S        (M = 128 key rows,  K = 128, N = 64)
-//   D_O = Q_eff . S     (M = 64 tokens,     K = 128, N = 64)
+//   D_S = Mp' . S'      (M = 128 key rows,  K = 128, N = 64)
+//   D_O = Q_eff' . S'   (M = 64 tokens,     K = 128, N = 64)
+//
+// where S' = diag(colscale) S is the bf16 operand (the prep stores Mp and
+// Q_eff with their columns divided by colscale, so Mp S = Mp' S'),
 //
 // and then   S <- diag(gamma) S - D_S + Nc      (fp32, in registers)
 //            O  = scale * (D_O + O_part)        (query reads the updated state)
@@ -23,10 +26,11 @@
 // the output epilogue of chunk j overlaps the critical path of chunk j+1.
 //
 // Two TMA rings feed it: ring A (Mp, Q_eff; read only by the UMMAs, released
-// by tcgen05.commit) and ring B (the CTA's Nc and O_part columns and gamma;
-// read by the epilogue warps, released by them).  Warp roles: 0-3 update the
-// state (the serial chain), 4-7 write the outputs, one lane of warp 8 issues
-// the UMMAs, one lane each of warps 9 and 10 streams ring A and ring B by TMA,
+// by tcgen05.commit) and ring B (the CTA's Nc and O_part columns, gamma and
+// colscale; read by the epilogue warps, released by them).  Warp roles: 0-3
+// update the state (the serial chain), 4-7 write the outputs, one lane of
+// warp 8 issues the UMMAs, one lane each of warps 9 and 10 streams ring A
+// (and prefetches the chunks ahead into L2) and ring B by TMA,
 // so nothing but the state update sits between two D_S products.  Every wait is bounded; on a
 // timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT in the status word, drains
 // what it issued and exits.
@@ -50,6 +54,7 @@ struct WalkTcArgs {
   CUtensorMap tm_Nc;   // Nc    [rows = max_chunks*H*128, dv]  bf16, box {64, 128}, SW128
   CUtensorMap tm_Op;   // O_part[rows = max_chunks*H*64,  dv]  bf16, box {64, 64},  SW128
   CUtensorMap tm_g;    // gamma [rows = max_chunks*H,     128] fp32, box {128, 1}
+  CUtensorMap tm_cs;   // colscale, same shape and box
   SeqMap map;
   int H;
   float scale;
@@ -73,13 +78,14 @@ struct WalkTcCfg {
   static constexpr int THREADS = 11 * 32;
   static constexpr int STAGES_A = 2;
   static constexpr int STAGES_B = 3;
+  static constexpr int PF = 4;                   // L2 prefetch distance in chunks
   static constexpr int MP_BYTES = DK * DK * 2;             // 32 KiB
   static constexpr int QE_BYTES = kChunk * DK * 2;         // 16 KiB
   static constexpr int A_BYTES = MP_BYTES + QE_BYTES;
   static constexpr int NC_BYTES = DK * NSL * 2;            // 16 KiB, SW128 rows of 64
   static constexpr int OP_BYTES = kChunk * NSL * 2;        // 8 KiB, SW128 rows of 64
-  static constexpr int G_BYTES = DK * 4;                   // 512 B
-  static constexpr int B_BYTES = NC_BYTES + OP_BYTES + G_BYTES;
+  static constexpr int G_BYTES = DK * 4;                   // 512 B each: gamma, colscale
+  static constexpr int B_BYTES = NC_BYTES + OP_BYTES + 2 * G_BYTES;
   static constexpr int B_STRIDE = (B_BYTES + 1023) / 1024 * 1024;
   // bf16 state operand, MN-major interleaved core matrices (8 key rows x 8
   // columns, 128 B): offset(kg, ng) = kg * S_LBO + ng * 128
@@ -205,15 +211,16 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     // this thread's row in the interleaved operand: core matrix (row/8, g),
     // 16-byte line row%8
     const uint32_t srow = (row >> 3) * C::S_LBO + (row & 7) * 16;
-    auto store_state = [&](int buf) {
+    // the bf16 operand of the chunk that reads it: this row times its colscale
+    auto store_state = [&](int buf, float cs) {
       uint8_t* base = sS + buf * C::S_BYTES + srow;
 #pragma unroll
       for (int g = 0; g < NSL / 8; ++g) {
         uint4 pk;
-        pk.x = tc::pack_bf16(S[8 * g + 0], S[8 * g + 1]);
-        pk.y = tc::pack_bf16(S[8 * g + 2], S[8 * g + 3]);
-        pk.z = tc::pack_bf16(S[8 * g + 4], S[8 * g + 5]);
-        pk.w = tc::pack_bf16(S[8 * g + 6], S[8 * g + 7]);
+        pk.x = tc::pack_bf16(cs * S[8 * g + 0], cs * S[8 * g + 1]);
+        pk.y = tc::pack_bf16(cs * S[8 * g + 2], cs * S[8 * g + 3]);
+        pk.z = tc::pack_bf16(cs * S[8 * g + 4], cs * S[8 * g + 5]);
+        pk.w = tc::pack_bf16(cs * S[8 * g + 6], cs * S[8 * g + 7]);
         *reinterpret_cast<uint4*>(base + g * 128) = pk;
       }
       tc::fence_async_smem();
@@ -221,7 +228,13 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_ready);
     };
-    store_state(0);
+    auto colscale_of = [&](int j) {   // row's colscale for chunk j (its ring B stage has landed)
+      return reinterpret_cast<const float*>(ringB + (j % C::STAGES_B) * C::B_STRIDE + C::NC_BYTES + C::OP_BYTES +
+                                            C::G_BYTES)[row];
+    };
+    if (nch > 0) {
+      if (wwait(&fullB[0], 0, a.status, s_abort)) store_state(0, colscale_of(0));
+    }
 
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
@@ -264,8 +277,15 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
           S[32 + e + 1] = fmaf(gam, S[32 + e + 1], bf16_hi_f(w2) - __uint_as_float(d1[e + 1]));
         }
       }
-      // D_O(j-1) read sS[(j+1)&1]; it was issued before D_S(j), so it is done
-      store_state((j + 1) & 1);
+      // D_O(j-1) read sS[(j+1)&1]; it was issued before D_S(j), so it is done.
+      // The operand is for chunk j+1 (its stage lands before this one is released).
+      float cs_next = 1.f;
+      if (j + 1 < nch) {
+        const int sn = (j + 1) % C::STAGES_B;
+        if (!wwait(&fullB[sn], ((j + 1) / C::STAGES_B) & 1, a.status, s_abort)) break;
+        cs_next = colscale_of(j + 1);
+      }
+      store_state((j + 1) & 1, cs_next);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
     }
@@ -358,6 +378,23 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int c = c_begin + j, st = j % C::STAGES_A;
+      // Pull chunk j + PF's factors into L2 (all of them: the ring B warp
+      // only reads what this brings), if they are written by now; the rings
+      // are shallow and the factors may have left L2.
+      if (j + C::PF < nch) {
+        const int cp = c + C::PF, tp = cp * H + h;
+        if (!a.ready || tc::ld_acquire_gpu(a.ready + tp) == 2) {
+          const int rm = tp * DK, rq = tp * kChunk;
+          tc::tma_prefetch_2d(&a.tm_Mp, 0, rm);
+          tc::tma_prefetch_2d(&a.tm_Mp, 64, rm);
+          tc::tma_prefetch_2d(&a.tm_Qe, 0, rq);
+          tc::tma_prefetch_2d(&a.tm_Qe, 64, rq);
+          tc::tma_prefetch_2d(&a.tm_Nc, col0, rm);
+          tc::tma_prefetch_2d(&a.tm_Op, col0, rq);
+          tc::tma_prefetch_2d(&a.tm_g, 0, tp);
+          tc::tma_prefetch_2d(&a.tm_cs, 0, tp);
+        }
+      }
       if (j >= C::STAGES_A && !wwait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1, a.status, s_abort)) break;
       if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringA + st * C::A_BYTES;
@@ -378,6 +415,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     tc::prefetch_tmap(&a.tm_Nc);
     tc::prefetch_tmap(&a.tm_Op);
     tc::prefetch_tmap(&a.tm_g);
+    tc::prefetch_tmap(&a.tm_cs);
     int loaded = 0;
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
@@ -389,6 +427,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
       tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
       tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
+      tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES + C::G_BYTES, &a.tm_cs, &fullB[st], 0, c * H + h);
       ++loaded;
     }
     for (int j = loaded > C::STAGES_B ? loaded - C::STAGES_B : 0; j < loaded; ++j)

@@ -111,7 +111,11 @@ typedef struct gdn2_desc {
  *    walk computes U = U~ - W S and S' = diag(gamma) S + Kbar^T U.
  *  factor_set 1 ("affine", bf16 I/O with dk = 128): the chunk's affine state
  *    map, Mp = Kbar^T W [dk, dk] and Nc = Kbar^T U~ [dk, dv], so that
- *    S' = diag(gamma) S - Mp S + Nc (one matrix product per chunk).
+ *    S' = diag(gamma) S - Mp S + Nc (one matrix product per chunk).  In this
+ *    set Mp and Q_eff are stored with their columns divided by colscale
+ *    ([., H, dk] fp32, exp of the in-chunk cumulative log-decay at token 32,
+ *    1 for chunks from the exact kernel): the factors are Mp diag(colscale)
+ *    and Q_eff diag(colscale).
  * Tensors of the other set have zero size. */
 typedef struct gdn2_ws_layout {
   size_t total_bytes;
@@ -135,6 +139,7 @@ typedef struct gdn2_ws_layout {
   size_t off_sync;           /* int32 [2 + max_chunks * H] (set 1): [0] next     */
                              /* prep task, [1] walk redo flag, then one ready    */
                              /* flag per (chunk, head) for the fused prep + walk */
+  size_t off_colscale;       /* column scale of Mp, Q_eff [., H, dk] fp32 set 1 */
 } gdn2_ws_layout;
 
 /* Bytes of workspace gdn2_chunk_fwd needs for `desc` (0 if desc is invalid).

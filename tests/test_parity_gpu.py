@@ -65,6 +65,13 @@ def _factors(ws, lay, H, dk, dv, io):
         f.update(Mp=view(lay["off_Mp"], mc, H, dk, dk), Nc=view(lay["off_Nc"], mc, H, dk, dv))
     g = ws[lay["off_gamma_last"]: lay["off_gamma_last"] + mc * H * dk * 4].view(torch.float32)
     f["gamma_last"] = g.view(mc, H, dk).cpu().numpy()
+    if lay["factor_set"] == 1:
+        # Mp and Q_eff are stored with their columns divided by colscale
+        cs = ws[lay["off_colscale"]: lay["off_colscale"] + mc * H * dk * 4].view(torch.float32)
+        cs = cs.view(mc, H, 1, dk).cpu().numpy().astype(np.float64)
+        with np.errstate(invalid="ignore", over="ignore"):   # unused chunk slots hold no data
+            f["Mp"] = f["Mp"] * cs
+            f["Q_eff"] = f["Q_eff"] * cs
     return f
 
 
