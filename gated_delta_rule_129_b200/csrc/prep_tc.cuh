@@ -4,9 +4,9 @@
 // Persistent CTAs walk a list of (chunk, head) tasks.  Warp roles:
 //   warp 8      TMA producer: streams each task's inputs in four 32-channel
 //               slices through a 3-slot ring that runs ahead across tasks;
-//   warp 10     scan: per slice, the in-chunk cumulative sum g of log_alpha
-//               (in place), the per-channel constants exp(g_r), exp(g_n - g_r),
-//               exp(g_n), and the decay-range check;
+//   warp 10     scan: per slice, the in-chunk cumulative sum g of log_alpha,
+//               written in place as g - g_r, the per-channel constants
+//               exp(g_r), exp(g_n - g_r), exp(g_n), and the decay-range check;
 //   warp 9      UMMA issue (one elected lane);
 //   warps 0-7   build the operands of each slice, then run the epilogues and
 //               the triangular solve of the task.
@@ -118,6 +118,7 @@ struct PrepTcCfg {
   static constexpr int OFF_SOP0 = OFF_X + 3 * PANEL, OFF_SOP1 = OFF_X + 3 * PANEL + 8192;
   static constexpr int OFF_SQE = OFF_X + 8192;  // + p * PANEL
   static_assert(OFF_XS + 4096 <= OFF_BAR, "solve scratch fits in the free area");
+  static_assert(OFF_VB + 16384 <= OFF_BAR, "the M = 128 read of V stays inside the free area");
   static_assert(64 * LDA * 4 <= OFF_TS - OFF_AS && 64 * LDT * 4 <= OFF_PB - OFF_TS, "A and T scratch");
   static constexpr int SMEM = 1024 + OFF_BAR + 3072;
   static constexpr int TMEM_COLS = 512;
@@ -172,8 +173,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   int* s_flag = reinterpret_cast<int*>(tslot + 1);    // [0] abort, [1] done
   int* slot_task = s_flag + 2;                        // [NSLOT] task id of the slot's slice
   int* slot_skip = slot_task + C::NSLOT;              // [NSLOT] decay range exceeded
-  float* s_gr = reinterpret_cast<float*>(sm + C::OFF_BAR + 512);  // [NSLOT][32] g_r
-  float* s_enr = s_gr + C::NSLOT * 32;                            // [2][128] exp(g_n - g_r), by task parity
+  float* s_enr = reinterpret_cast<float*>(sm + C::OFF_BAR + 512);  // [2][128] exp(g_n - g_r), by task parity
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
@@ -279,17 +279,28 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         float v[kChunk];
 #pragma unroll
         for (int t = 0; t < kChunk; ++t) v[t] = la[swf(t, lane)];
-        float acc = 0.f;
+        // four 16-token running sums side by side, then the block offsets
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int t = 0; t < kChunk; ++t) {
-          acc += t < len ? v[t] : 0.f;
-          v[t] = acc;
+        for (int t = 0; t < 16; ++t)
+#pragma unroll
+          for (int bq = 0; bq < 4; ++bq) {
+            const int tt = 16 * bq + t;
+            acc[bq] += tt < len ? v[tt] : 0.f;
+            v[tt] = acc[bq];
+          }
+        const float off1 = acc[0], off2 = off1 + acc[1], off3 = off2 + acc[2];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          v[16 + t] += off1;
+          v[32 + t] += off2;
+          v[48 + t] += off3;
         }
-#pragma unroll
-        for (int t = 0; t < kChunk; ++t) la[swf(t, lane)] = v[t];
         const float g0 = v[0], gr = v[32], gn = v[kChunk - 1];
         const bool bad = (g0 - gr > 60.f) || (gr - gn > 60.f);
-        s_gr[slot * 32 + lane] = gr;
+        // what the build needs: x_t = g_t - g_r, over log_alpha
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) la[swf(t, lane)] = v[t] - gr;
         s_enr[tpar * DK + C::KS * s_in + lane] = __expf(gn - gr);
         a.gamma_last[tile * DK + C::KS * s_in + lane] = expf(gn);
         a.colscale[tile * DK + C::KS * s_in + lane] = __expf(gr);
@@ -314,7 +325,10 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       constexpr uint32_t idR = tc::idesc_bf16(128, 128, true, true);
       constexpr uint32_t idV = tc::idesc_bf16(64, 128, false, true);
       constexpr uint32_t idM = tc::idesc_bf16(128, 128 + DV, false, true);
-      constexpr uint32_t idQ = tc::idesc_bf16(64, 128 + DV, false, true);
+      // M = 128 although V has 64 rows: rows 64..127 read the (dead) bytes
+      // after V and land in TMEM lanes nobody reads, so the 64 real rows sit
+      // in lanes 0..63 (two full lane quarters) for the epilogue
+      constexpr uint32_t idQ = tc::idesc_bf16(128, 128 + DV, false, true);
       bool ok = true;
       for (int ex = 0; ok; ++ex) {
         // UMMA 1, two K-steps of 16 channels per slice as the slices are built
@@ -400,9 +414,8 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         const int i = tid >> 2, gq = tid & 3, cl = 8 * gq, cc0 = C::KS * s + cl;
         const bool live = i < len;
         {
-          float gi[8], gr[8], bb[8];
+          float gi[8], bb[8];   // gi: g_i - g_r
           load8f_sw(g, i, gq, gi);
-          load8f(s_gr + slot * 32 + cl, gr);
           load8f_sw(reinterpret_cast<const float*>(d + C::OFF_B), i, gq, bb);
           const uint4 kraw = *reinterpret_cast<const uint4*>(d + C::OFF_K + (i * 32 + cl) * 2);
           const uint4 qraw = *reinterpret_cast<const uint4*>(d + C::OFF_Q + (i * 32 + cl) * 2);
@@ -418,7 +431,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
               const float kv = live ? (e ? bf16_hi_f(kw[p]) : bf16_lo_f(kw[p])) : 0.f;
               const float qv = live ? (e ? bf16_hi_f(qw[p]) : bf16_lo_f(qw[p])) : 0.f;
               const float bv = live ? bb[m] : 0.f;
-              const float x = gi[m] - gr[m];
+              const float x = gi[m];
               const float E = __expf(x), F = __expf(-x);
               o_eh[e] = bv * kv * E;
               o_qh[e] = qv * E;
@@ -721,16 +734,15 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         }
         tc::tma_store_commit();
       }
-      {
-        // token rows (M = 64 layout): half 0: Q_eff' = Q^ - P W', in place
-        // over Q^; half 1: O_part.  The next 32 columns load while one is
-        // packed.
+      if (q < 2) {
+        // token rows (lanes 0..63, warps of lane quarters 0 and 1): half 0:
+        // Q_eff' = Q^ - P W', in place over Q^; half 1: O_part.  The next
+        // 32 columns load while one is packed.
         const int ncols = half == 0 ? 128 : DV;
-        const int i_out = 16 * q + lane;
+        const int i_out = 32 * q + lane;
         uint8_t* base = sm + (half == 0 ? C::OFF_SQE : C::OFF_SOP0);
         const int pstride = half == 0 ? C::PANEL : 8192;
         auto pack_rows = [&](const uint32_t (&r)[32], int c0) {
-          if (lane >= 16) return;
           uint8_t* pnl = base + (c0 >> 6) * pstride;
 #pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
