@@ -300,6 +300,7 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / ne, world)
 
     decode = measure_decode(dev, stream, flush) if rank == 0 else None
+    others = measure_other_configs(dev, stream, flush, peaks()[0]) if (rank == 0 and not args.no_other_configs) else None
     if rank != 0:
         return
     hbm, tflops, src = peaks()
@@ -336,6 +337,8 @@ def run_ours(args, rank, world, local):
         decode["roofline"] = {"bound": "hbm", "achieved": decode["gbs"], "peak": hbm, "unit": "GB/s",
                               "frac": decode["gbs"] / hbm}
         line["decode_step"] = decode
+    if others:
+        line["other_configs"] = others
     if world == 1 and not args.no_cpu_baseline:
         tps, cores, t_tok, dt = cpu_oracle_sample(x, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -376,6 +379,54 @@ def measure_decode(dev, stream, flush, reps=20):
             "tokens_per_s": 256 / (us * 1e-6), "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9}
 
 
+def measure_other_configs(dev, stream, flush, hbm, steps=10):
+    """gdn2_chunk_fwd on the other bf16 workloads (2K x 8, 4K x 4 with
+    b = w = beta, 32 packed sequences): tokens/s and the step roofline
+    fraction, same timing rules as the headline number."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    from workloads import config
+    out_cfg = {}
+    for cid, variant in ((1, "a"), (3, "a"), (4, "a")):
+        x = config(cid, variant)
+        t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
+        bf, f32 = torch.bfloat16, torch.float32
+        q, k, v = t(x.q, bf), t(x.k, bf), t(x.v, bf)
+        la, b, w = t(x.log_alpha, f32), t(x.b, f32), t(x.w, f32)
+        h0 = None if x.h0 is None else t(x.h0, f32)
+        cu = None if x.cu_seqlens is None else t(x.cu_seqlens, torch.int32)
+        Bc, Tc, Hc = x.q.shape[0], x.q.shape[1], x.q.shape[2]
+        ns = 0 if cu is None else len(x.cu_seqlens) - 1
+        nseq = ns if cu is not None else Bc
+        ws = torch.empty(gdn2.workspace_size(Bc, Tc, Hc, DK, DV, gdn2.GDN2_IO_BF16, ns), dtype=torch.uint8,
+                         device=dev)
+        o = torch.empty_like(v)
+        hT = torch.empty((nseq, Hc, DK, DV), dtype=f32, device=dev)
+
+        def run():
+            gdn2.chunk_fwd(q, k, v, la, b, w, x.scale, h0=h0, cu_seqlens=cu, out=o, hT=hT, workspace=ws,
+                           stream=stream)
+        for _ in range(3):
+            run()
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run()
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        ms = tot / steps
+        tokens = Bc * Tc
+        alg = tokens * Hc * ALG_BYTES_PER_TH + nseq * Hc * DK * DV * 4 * (2 if h0 is not None else 1)
+        out_cfg[x.name] = {"tokens_per_s": tokens / (ms / 1e3), "ms_per_step": ms,
+                           "roofline_frac": (alg / (hbm * 1e9)) / (ms / 1e3)}
+        del q, k, v, la, b, w, h0, cu, ws, o, hT
+    return out_cfg
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -384,6 +435,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
