@@ -26,6 +26,7 @@ MUTANTS = {
     "erase gate read from head 0": ("const double* bt = J->b + ((size_t)t * H + h) * dk;",
                                     "const double* bt = J->b + ((size_t)t * H) * dk;"),
     "erase uses the query": ("e[c] = bt[c] * kt[c];", "e[c] = bt[c] * qt[c];"),
+    "erase gate clamped to [0, 1]": ("e[c] = bt[c] * kt[c];", "e[c] = fmin(bt[c], 1.0) * kt[c];"),
 }
 
 PIN_TESTS = [
@@ -33,6 +34,7 @@ PIN_TESTS = [
     pins.test_reduction_to_gated_deltanet,
     pins.test_reduction_to_deltanet,
     pins.test_delta_rule_overwrite_invariant,
+    pins.test_full_range_erase_repeated_token_is_identity,
     pins.test_no_erase_is_decayed_linear_attention,
     pins.test_no_erase_no_write_is_pure_decay,
     pins.test_basis_keys_exact_example,

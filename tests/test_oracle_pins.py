@@ -5,7 +5,9 @@ None of these compares the oracle with a retyped copy of itself.  They use
     against a separately written scalar-gate oracle;
   * the delta-rule overwrite invariant (with unit keys, alpha = 1 and
     b = w = 1 the state maps k_t exactly to v_t, and a query equal to k_t
-    reads scale * v_t from the updated state);
+    reads scale * v_t from the updated state), and its reflection form at
+    the top of the widened erase range (b = 2: a repeated token is the
+    identity on the state);
   * closed forms of the degenerate cases b = 0 (decayed linear attention) and
     b = w = 0 (pure decay), written as cumulative sums, not as a loop;
   * an exact rational example with one-hot keys (tests/golden/basis_keys.json);
@@ -96,6 +98,45 @@ def test_delta_rule_overwrite_invariant():
     # and the final state maps the last key to the last value
     for h in range(2):
         np.testing.assert_allclose(hT[0, h].T @ k[0, -1, h], x.v[0, -1, h], rtol=0, atol=1e-12)
+
+
+def test_full_range_erase_repeated_token_is_identity():
+    """At the top of the widened erase range (b = 2 in every channel), with
+    alpha = 1, w = 1 and a unit key, one token applies the reflection
+    I - 2 k k^T to the state and writes k v^T.  The same token twice in a row
+    therefore leaves the state as it was, and with q = k the two outputs are
+    scale * (v - S^T k) and scale * S^T k, S the state before the pair.  A
+    dropped erase, a wrong sign of the correction or a query that reads the
+    old state breaks one of the three."""
+    x = make_inputs(1, 24, 2, 16, 8, io="f32", seed=16, h0_std=0.5)
+    k = x.k.astype(np.float64)
+    k = k / np.linalg.norm(k, axis=-1, keepdims=True)
+    k[:, 1::2] = k[:, 0::2]                                   # tokens come in identical pairs
+    v = x.v.astype(np.float64)
+    v[:, 1::2] = v[:, 0::2]
+    zeros = np.zeros_like(x.log_alpha, dtype=np.float64)
+    twos, ones_v = np.full(x.b.shape, 2.0), np.ones(x.w.shape)
+    o, hT = oracle.recurrent(k, k, v, zeros, twos, ones_v, 0.5, h0=x.h0)
+    np.testing.assert_allclose(hT, x.h0, rtol=0, atol=1e-12)
+    h0 = x.h0[0].astype(np.float64)                           # [H, dk, dv]
+    read = np.einsum("hkv,thk->thv", h0, k[0])                # S^T k with S = h0
+    np.testing.assert_allclose(o[0, 0::2], 0.5 * (v[0, 0::2] - read[0::2]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o[0, 1::2], 0.5 * read[1::2], rtol=0, atol=1e-12)
+
+
+def test_gate_ablation_inputs():
+    """The ablation inputs keep the plain call's draws: b scaled into (0, 2),
+    or b / w replaced by their channel mean."""
+    base = make_inputs(2, 30, 3, 16, 8, io="f32", seed=17)
+    wide = make_inputs(2, 30, 3, 16, 8, io="f32", seed=17, erase_range=2.0)
+    assert np.array_equal(wide.b, 2.0 * base.b) and np.array_equal(wide.w, base.w)
+    assert wide.b.max() < 2.0 and wide.b.min() > 0.0
+    me = make_inputs(2, 30, 3, 16, 8, io="f32", seed=17, mean_gate="erase")
+    np.testing.assert_allclose(me.b, np.broadcast_to(base.b.mean(-1, keepdims=True), base.b.shape), rtol=1e-6)
+    assert np.array_equal(me.w, base.w) and np.array_equal(me.k, base.k)
+    mw = make_inputs(2, 30, 3, 16, 8, io="f32", seed=17, mean_gate="write")
+    np.testing.assert_allclose(mw.w, np.broadcast_to(base.w.mean(-1, keepdims=True), base.w.shape), rtol=1e-6)
+    assert np.array_equal(mw.b, base.b)
 
 
 # --- closed forms of the degenerate gates --------------------------------------------

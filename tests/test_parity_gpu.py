@@ -46,6 +46,33 @@ def test_strong_decay(io):
     assert ro <= TOL[io] and rh <= TOL[io], (ro, rh)
 
 
+# The gate ablations of page "Gated DeltaNet-2：将擦除与写入分开", section
+# "消融实验与训练吞吐量": erase range widened to [0, 2], and one gate averaged
+# over its channels at run time (same kernels, other inputs).
+GATE_VARIANTS = [dict(erase_range=2.0), dict(mean_gate="erase"), dict(mean_gate="write"),
+                 dict(erase_range=2.0, mean_gate="erase")]
+
+
+@pytest.mark.parametrize("io,dk,dv", [("bf16", 128, 128), ("f32", 64, 64), ("bf16", 128, 64)])
+@pytest.mark.parametrize("kw", GATE_VARIANTS, ids=lambda k: "-".join(f"{a}={b}" for a, b in k.items()))
+def test_gate_ablation_inputs(io, dk, dv, kw):
+    x = make_inputs(2, 333, 3, dk, dv, io=io, seed=51 + dk + dv, h0_std=0.05, **kw)
+    o, hT = run_gpu(x)
+    ro, rh = compare(x, o, hT)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(hT))
+    assert ro <= TOL[io] and rh <= TOL[io], (ro, rh)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_gate_ablation_strong_decay_varlen(io):
+    lengths = [300, 65, 1, 190]
+    x = make_inputs(1, sum(lengths), 4, 128, 128, io=io, seed=57, decay="strong", h0_std=0.05,
+                    lengths=lengths, erase_range=2.0)
+    o, hT = run_gpu(x)
+    ro, rh = compare(x, o, hT)
+    assert ro <= TOL[io] and rh <= TOL[io], (ro, rh)
+
+
 # --- the stages, one at a time ------------------------------------------------
 
 def _factors(ws, lay, H, dk, dv, io):
@@ -246,6 +273,23 @@ def test_recurrent_step_matches_oracle(io, dk, dv, B):
                               t(di.b, torch.float32), t(di.w, torch.float32), di.scale, state)
     o_ref, s_ref = oracle.recurrent_step(di.q, di.k, di.v, di.log_alpha, di.b, di.w, di.scale, di.state)
     assert rel_l2(out.float().cpu().numpy(), o_ref) <= TOL[io]
+    assert rel_l2(state.cpu().numpy(), s_ref) <= 1e-5
+
+
+@pytest.mark.parametrize("kw", GATE_VARIANTS[:3], ids=lambda k: "-".join(f"{a}={b}" for a, b in k.items()))
+def test_recurrent_step_gate_ablations(kw):
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    import oracle
+    di = decode_inputs(B=7, H=3, dk=128, dv=128, io="bf16", seed=61, **kw)
+    t = lambda a, ty: torch.from_numpy(a).to("cuda", ty)  # noqa: E731
+    state = t(di.state, torch.float32)
+    out = gdn2.recurrent_step(t(di.q, torch.bfloat16), t(di.k, torch.bfloat16), t(di.v, torch.bfloat16),
+                              t(di.log_alpha, torch.float32), t(di.b, torch.float32), t(di.w, torch.float32),
+                              di.scale, state)
+    o_ref, s_ref = oracle.recurrent_step(di.q, di.k, di.v, di.log_alpha, di.b, di.w, di.scale, di.state)
+    assert rel_l2(out.float().cpu().numpy(), o_ref) <= TOL["bf16"]
     assert rel_l2(state.cpu().numpy(), s_ref) <= 1e-5
 
 

@@ -24,7 +24,9 @@ standard normals, drawn in the order q, k, v, log_alpha, b, w, h0):
   v     : N(0,1) (workload 0) or SiLU(N(0,1)) (bf16 workloads)
   log_alpha : -0.1 * softplus(N(0,1))   (mild), or
               -softplus(N(-2, 1.5))     (strong: per-channel decay from ~1 to ~0)
-  b, w  : sigmoid(N(0,1)) per (token, head, channel)
+  b, w  : sigmoid(N(0,1)) per (token, head, channel); the ablation variants
+          scale b by 2 (erase range [0, 2]) or replace b or w by its channel
+          mean (make_inputs: erase_range, mean_gate)
   h0    : N(0, sigma) with sigma the standard deviation (0.01), fp32
 "N(mu, s)" is read as mean and standard deviation.  bf16 tensors are rounded
 to nearest-even from float32 and returned as float32 arrays holding exactly
@@ -93,7 +95,7 @@ class Inputs:
 
 
 def make_inputs(B, T, H, dk, dv, io="bf16", seed=0, decay="mild", gates="channel",
-                h0_std=None, lengths=None, v_act=None) -> Inputs:
+                h0_std=None, lengths=None, v_act=None, erase_range=1.0, mean_gate=None) -> Inputs:
     """General generator.
 
     ``decay``: "mild" (-0.1*softplus(N(0,1))) or "strong" (-softplus(N(-2,1.5))).
@@ -103,6 +105,13 @@ def make_inputs(B, T, H, dk, dv, io="bf16", seed=0, decay="mild", gates="channel
     ``lengths``: if given, B must be 1 and T == sum(lengths); sequences are
     packed and ``cu_seqlens`` is set.
     ``v_act``: "silu" or None; defaults to "silu" for bf16 and None for f32.
+    ``erase_range``: b = erase_range * sigmoid(N(0,1)) (the ablation widening
+    the erase gate's range from [0, 1] to [0, 2] uses 2).
+    ``mean_gate``: None, "erase" or "write": the ablation that averages one
+    gate (b, the erase gate, or w, the write gate) over its channels at run
+    time, broadcast back over them.  Page "Gated DeltaNet-2：将擦除与写入分开",
+    section "消融实验与训练吞吐量".  Neither option changes the draws, so the
+    other tensors are those of the plain call with the same seed.
     """
     rng = np.random.default_rng(seed)
     shp_k = (B, T, H, dk)
@@ -140,6 +149,14 @@ def make_inputs(B, T, H, dk, dv, io="bf16", seed=0, decay="mild", gates="channel
         w = np.broadcast_to(beta[..., None], shp_v).astype(np.float32)
     else:
         raise ValueError(gates)
+    if erase_range != 1.0:
+        b = (np.float32(erase_range) * b).astype(np.float32)
+    if mean_gate == "erase":
+        b = np.broadcast_to(b.mean(axis=-1, dtype=np.float32)[..., None], shp_k).astype(np.float32)
+    elif mean_gate == "write":
+        w = np.broadcast_to(w.mean(axis=-1, dtype=np.float32)[..., None], shp_v).astype(np.float32)
+    elif mean_gate is not None:
+        raise ValueError(mean_gate)
     cu = None
     if lengths is not None:
         assert B == 1 and T == int(np.sum(lengths))
@@ -205,9 +222,10 @@ class DecodeInputs:
     io: str
 
 
-def decode_inputs(B=256, H=16, dk=128, dv=128, io="bf16", seed=41, state_std=0.01) -> DecodeInputs:
-    """Single-token decode batch: one token per state, same distributions as above."""
-    x = make_inputs(B, 1, H, dk, dv, io=io, seed=seed, decay="mild")
+def decode_inputs(B=256, H=16, dk=128, dv=128, io="bf16", seed=41, state_std=0.01, **gate_kw) -> DecodeInputs:
+    """Single-token decode batch: one token per state, same distributions as
+    above (``gate_kw``: make_inputs' erase_range / mean_gate)."""
+    x = make_inputs(B, 1, H, dk, dv, io=io, seed=seed, decay="mild", **gate_kw)
     rng = np.random.default_rng(seed + 1000)
     state = (state_std * rng.standard_normal((B, H, dk, dv), dtype=np.float32)).astype(np.float32)
     sq = lambda a: np.ascontiguousarray(a[:, 0])  # noqa: E731
