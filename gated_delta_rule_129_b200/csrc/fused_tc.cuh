@@ -21,8 +21,9 @@ namespace gdn2 {
 
 template <int DV>
 struct FusedTcCfg {
+  // the walk leaves the prep's extra (store) warp idle
   static constexpr int THREADS = PrepTcCfg<DV>::THREADS;
-  static_assert(THREADS == WalkTcCfg<DV>::THREADS, "one block shape for both roles");
+  static_assert(THREADS >= WalkTcCfg<DV>::THREADS, "one block shape for both roles");
   static constexpr int SMEM =
       PrepTcCfg<DV>::SMEM > WalkTcCfg<DV>::SMEM ? PrepTcCfg<DV>::SMEM : WalkTcCfg<DV>::SMEM;
   static constexpr int MIN_PREP_CTAS = 32;
@@ -39,7 +40,7 @@ fused_tc_kernel(const __grid_constant__ PrepTcArgs pa, const __grid_constant__ W
   } else {
     // early on, the walk would only wait for the prep wavefront: take prep
     // tasks until the counter reaches pa.stop_at, then walk
-    prep_tc_cta<DV>(pa, sm, blockIdx.x, gridDim.x, true);
+    if (pa.stop_at > 0) prep_tc_cta<DV>(pa, sm, blockIdx.x, gridDim.x, true);
     walk_tc_cta<DV>(wa, sm, (int)blockIdx.x - n_prep);
   }
 }

@@ -180,6 +180,7 @@ gdn2_status fill_prep_tc(const gdn2_desc* d, const Layout& L, const void* q, con
   a.status = at<int32_t>(d->workspace, L.l.off_status);
   a.ready = nullptr;
   a.task_counter = nullptr;
+  a.l2_prefetch = 1;
   return GDN2_OK;
 }
 
@@ -379,20 +380,21 @@ gdn2_status launch_fused_tc(const gdn2_desc* d, const Layout& L, const void* q, 
   int* sync = at<int>(d->workspace, L.l.off_sync);
   pa.task_counter = sync;
   pa.ready = sync + 2;
+  pa.l2_prefetch = 0;
   wa.ready = sync + 2;
   wa.redo = sync + 1;
   const int n_sm = sm_count();
   const int n_walk = L.N * d->H * gdn2::WalkTcCfg<DV>::SLICES;
-  // When the walk CTAs stop taking prep tasks: beside the prep, a walk step
-  // costs about a ninth of a prep task on one SM (measured at 16K x 1:
-  // ~1.4 us per chunk against ~12 us per task), so a walk of nch chunks
-  // started when nch * (n_sm - n_walk) / 9 tasks are left ends about with
-  // the prep (a sweep of the switch point at 16K x 1 has its flat optimum
-  // there).
+  // When the walk CTAs stop taking prep tasks: a walk of nch chunks started
+  // when nch * (n_sm - n_walk) / 7 tasks are left ends about with the prep
+  // (beside the prep, a walk step costs about a seventh of a prep task on
+  // one SM).  With the prep's stores off its critical path this leaves the
+  // walk CTAs no prep work on the workloads measured (a sweep of the switch
+  // point at 16K x 1 has its optimum at 0), and then they skip the prep role.
   {
     const long long tasks = (long long)L.l.max_chunks * d->H;
     const long long nch = ((long long)d->B * d->T + (long long)kChunk * L.N - 1) / ((long long)kChunk * L.N);
-    const long long left = nch * (n_sm - n_walk) / 9;
+    const long long left = nch * (n_sm - n_walk) / 7;
     pa.stop_at = (int)std::max(0ll, tasks - left);
   }
   auto kern = gdn2::fused_tc_kernel<DV>;

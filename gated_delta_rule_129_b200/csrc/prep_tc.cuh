@@ -9,7 +9,11 @@
 //               exp(g_r), exp(g_n - g_r), exp(g_n), and the decay-range check;
 //   warp 9      UMMA issue (one elected lane);
 //   warps 0-7   build the operands of each slice, then run the epilogues and
-//               the triangular solve of the task.
+//               the triangular solve of the task;
+//   warp 11     output stores (one lane): takes each task's staged tiles,
+//               stores them by TMA, frees the staging for the next task's
+//               builds once read, and publishes the task's ready flag once
+//               its stores are complete, off the compute warps' path.
 // Per chunk of n <= 64 tokens (page "Gated DeltaNet-2：将擦除与写入分开",
 // sections "在两个维度上独立控制" and "词元路径与并行训练"; the algebra is the
 // recurrence unrolled over one chunk, written as products):
@@ -70,6 +74,7 @@ struct PrepTcArgs {
   int* ready;            // optional [max_chunks * H], zeroed: 2 = factors written, 3 = handed back
   int* task_counter;     // optional: tasks taken dynamically (else static striding)
   int stop_at;           // with task_counter: a CTA given a later role stops taking tasks here
+  int l2_prefetch;       // start each task's last input slice towards L2 when the task is taken
   int* status;
 };
 
@@ -81,8 +86,8 @@ struct PrepTcCfg {
   static constexpr int SLICES = 4;
   static constexpr int NSLOT = 3;
   static constexpr int COMPUTE_WARPS = 8;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, SCAN_WARP = 10;
-  static constexpr int THREADS = 11 * 32;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, SCAN_WARP = 10, STORE_WARP = 11;
+  static constexpr int THREADS = 12 * 32;
   // raw slot: la (-> g in place), b fp32 [64][32]; q, k bf16 [64][32]; v bf16 [64][VS]; w fp32 [64][VS].
   // The fp32 rows of 128 bytes (la, b, and w when VS = 32) arrive SW128-swizzled
   // (16-byte unit u of token row t at u ^ (t & 7)), so that the 8 lanes of a
@@ -112,11 +117,15 @@ struct PrepTcCfg {
   static constexpr int OFF_T = OFF_F;           // [T_hi | T_lo] MN-major SW128, over A once A is dead
   static constexpr int OFF_RB = OFF_F, OFF_VB = OFF_F + 16384;  // after UMMA 2: [R; V] K-major
   // output staging once UMMA 3 has read its operands (SW128 panels of 64
-  // columns); Q_eff is formed in place over Q^ (rows 64..127 of slots 0, 1)
+  // columns).  The first stores of a task (Mp, Nc) use the free area and
+  // slot 2, the last ones (Q_eff, O_part) slots 1 and 3 only: the next
+  // task's first two slices (which write slots 0 and 2) need only the first
+  // stores to have left shared memory, its last two slices all of them.
   static constexpr int OFF_SMP0 = OFF_F, OFF_SMP1 = OFF_F + 16384;
   static constexpr int OFF_SNC0 = OFF_F + 32768, OFF_SNC1 = OFF_X + 2 * PANEL;
   static constexpr int OFF_SOP0 = OFF_X + 3 * PANEL, OFF_SOP1 = OFF_X + 3 * PANEL + 8192;
-  static constexpr int OFF_SQE = OFF_X + 8192;  // + p * PANEL
+  static constexpr int OFF_SQE = OFF_X + PANEL;  // + p * 8192 (slot 1)
+  static constexpr int OFF_QH = OFF_X + 8192;    // Q^, + p * PANEL
   static_assert(OFF_XS + 4096 <= OFF_BAR, "solve scratch fits in the free area");
   static_assert(OFF_VB + 16384 <= OFF_BAR, "the M = 128 read of V stays inside the free area");
   static_assert(64 * LDA * 4 <= OFF_TS - OFF_AS && 64 * LDT * 4 <= OFF_PB - OFF_TS, "A and T scratch");
@@ -169,10 +178,17 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   uint64_t* rv_ready = mma2_done + 1;
   uint64_t* mma3_done = rv_ready + 1;
   uint64_t* fin = mma3_done + 1;
+  uint64_t* mma2a_done = fin + 1;   // the R half of UMMA 2
+  uint64_t* mma3a_done = mma2a_done + 1;  // the [Mp' | Nc] half of UMMA 3
+  uint64_t* st_a = mma3a_done + 1;  // Mp and Nc staged (both half leaders)
+  uint64_t* st_b = st_a + 1;        // Q_eff and O_part staged
+  uint64_t* rd_a = st_b + 1;        // the store warp: Mp / Nc staging read
+  uint64_t* rd_b = rd_a + 1;        // the store warp: all staging read
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::OFF_BAR + 256);
   int* s_flag = reinterpret_cast<int*>(tslot + 1);    // [0] abort, [1] done
   int* slot_task = s_flag + 2;                        // [NSLOT] task id of the slot's slice
   int* slot_skip = slot_task + C::NSLOT;              // [NSLOT] decay range exceeded
+  int* s_store = slot_skip + C::NSLOT;                // [2] tile being stored (-1: none left), skip
   float* s_enr = reinterpret_cast<float*>(sm + C::OFF_BAR + 512);  // [2][128] exp(g_n - g_r), by task parity
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -192,6 +208,12 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
     tc::mbar_init(rv_ready, C::COMPUTE_WARPS);
     tc::mbar_init(mma3_done, 1);
     tc::mbar_init(fin, 1);
+    tc::mbar_init(mma2a_done, 1);
+    tc::mbar_init(mma3a_done, 1);
+    tc::mbar_init(st_a, 2);
+    tc::mbar_init(st_b, 1);
+    tc::mbar_init(rd_a, 1);
+    tc::mbar_init(rd_b, 1);
     s_flag[0] = s_flag[1] = 0;
     tc::fence_mbar_init();
   }
@@ -227,6 +249,19 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         if (task >= 0) {
           h = task % H;
           t0 = chunk_pos(a.map, task / H).t0;
+        }
+        if (task >= 0 && a.l2_prefetch) {
+          // the last slice is loaded only once this task's first slice has
+          // been built (three slots, four slices): start it towards L2 now.
+          // (Beside the walk in the fused launch this costs more than it
+          // saves, and is left off there.)
+          constexpr int s3 = C::SLICES - 1;
+          tc::tma_prefetch_3d(&a.tm_la, C::KS * s3, h, t0);
+          tc::tma_prefetch_3d(&a.tm_b, C::KS * s3, h, t0);
+          tc::tma_prefetch_3d(&a.tm_q, C::KS * s3, h, t0);
+          tc::tma_prefetch_3d(&a.tm_k, C::KS * s3, h, t0);
+          tc::tma_prefetch_3d(&a.tm_v, C::VS * s3, h, t0);
+          tc::tma_prefetch_3d(&a.tm_w, C::VS * s3, h, t0);
         }
         const int nsl = task < 0 ? 1 : C::SLICES;
         for (int s = 0; s < nsl; ++s, ++gs) {
@@ -325,9 +360,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       constexpr uint32_t idR = tc::idesc_bf16(128, 128, true, true);
       constexpr uint32_t idV = tc::idesc_bf16(64, 128, false, true);
       constexpr uint32_t idM = tc::idesc_bf16(128, 128 + DV, false, true);
-      // M = 128 although V has 64 rows: rows 64..127 read the (dead) bytes
-      // after V and land in TMEM lanes nobody reads, so the 64 real rows sit
-      // in lanes 0..63 (two full lane quarters) for the epilogue
+      // M = 128 over [V; V] (epilogue 2 writes V twice): the 64 token rows
+      // land in lanes 0..63 and again in 64..127, so all four TMEM lane
+      // quarters hold them and all eight epilogue warps share the token rows
       constexpr uint32_t idQ = tc::idesc_bf16(128, 128 + DV, false, true);
       bool ok = true;
       for (int ex = 0; ok; ++ex) {
@@ -347,26 +382,89 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         tc::umma_commit(mma1_done);
         if (!tc::mbar_wait(t_ready, ex & 1) || vflag[0]) break;
         tc::tc_fence_after();
+        // R first, committed on its own: its epilogue starts while V runs
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint64_t t_d = tc::sdesc(TT + s * 2048, 8192, 1024, SW);
-          tc::umma_f16(tbase + C::COL_R, tc::sdesc(KH + s * 2048, C::PANEL, 1024, SW), t_d, idR, s > 0);
-          tc::umma_f16(tbase + C::COL_V, tc::sdesc(PB + s * 32, 16, 1024, SW), t_d, idV, s > 0);
-        }
+        for (int s = 0; s < 4; ++s)
+          tc::umma_f16(tbase + C::COL_R, tc::sdesc(KH + s * 2048, C::PANEL, 1024, SW),
+                       tc::sdesc(TT + s * 2048, 8192, 1024, SW), idR, s > 0);
+        tc::umma_commit(mma2a_done);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          tc::umma_f16(tbase + C::COL_V, tc::sdesc(PB + s * 32, 16, 1024, SW), tc::sdesc(TT + s * 2048, 8192, 1024, SW),
+                       idV, s > 0);
         tc::umma_commit(mma2_done);
         if (!tc::mbar_wait(rv_ready, ex & 1) || vflag[0]) break;
         tc::tc_fence_after();
+        // [Mp' | Nc] first (its epilogue starts while the token rows run)
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint64_t ez_d = tc::sdesc(X + s * 2048, C::PANEL, 1024, SW);
-          tc::umma_f16(tbase + C::COL_MN, tc::sdesc(RB + s * 32, 16, 1024, SW), ez_d, idM, s > 0);
-          tc::umma_f16(tbase + C::COL_QO, tc::sdesc(VB + s * 32, 16, 1024, SW), ez_d, idQ, s > 0);
-        }
+        for (int s = 0; s < 4; ++s)
+          tc::umma_f16(tbase + C::COL_MN, tc::sdesc(RB + s * 32, 16, 1024, SW), tc::sdesc(X + s * 2048, C::PANEL, 1024, SW),
+                       idM, s > 0);
+        tc::umma_commit(mma3a_done);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          tc::umma_f16(tbase + C::COL_QO, tc::sdesc(VB + s * 32, 16, 1024, SW), tc::sdesc(X + s * 2048, C::PANEL, 1024, SW),
+                       idQ, s > 0);
         tc::umma_commit(mma3_done);
       }
       // nothing of ours is left in the tensor pipe when TMEM is released
       tc::umma_commit(fin);
       tc::mbar_wait(fin, 0);
+    }
+  } else if (warp == C::STORE_WARP) {
+    // ----------------------------------------------------------- stores --
+    // Per task: the Mp / Nc tiles once both half leaders have staged them,
+    // the Q_eff / O_part tiles once the epilogue is done; the staging is
+    // handed back as soon as the stores have read it, and the task's ready
+    // flag (2 = factors written) is raised once its stores are complete,
+    // which is checked one task later so that it never holds up a store.
+    if (lane == 0) {
+      volatile int* vst = s_store;
+      int pend = -1;
+      bool ok = true;
+      auto publish = [&](int t) {
+        tc::fence_async_global();
+        __threadfence();
+        tc::red_add_release_gpu(a.ready + t, 2);
+      };
+      for (int ex = 0;; ++ex) {
+        if (!tc::mbar_wait(st_a, ex & 1)) { ok = false; break; }
+        const int tile = vst[0];
+        const bool skip = vst[1] != 0;
+        if (tile < 0) break;
+        if (!skip) {
+          const int rk = tile * DK;
+          tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP0, 0, rk);
+          tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP1, 64, rk);
+          tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC0, 0, rk);
+          if (DV == 128) tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC1, 64, rk);
+          tc::tma_store_commit();
+        }
+        if (!tc::mbar_wait(st_b, ex & 1)) { ok = false; break; }
+        if (!skip) {
+          const int rt = tile * kChunk;
+          for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Qe, sm + C::OFF_SQE + p * 8192, 64 * p, rt);
+          for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Op, sm + C::OFF_SOP0 + p * 8192, 64 * p, rt);
+          tc::tma_store_commit();
+        }
+        tc::tma_store_wait_read_but_newest();
+        tc::mbar_arrive(rd_a);
+        tc::tma_store_wait_read();
+        tc::mbar_arrive(rd_b);
+        if (pend >= 0) {
+          // the previous stored task's two groups are complete
+          if (skip) tc::tma_store_wait_all();
+          else tc::tma_store_wait_all_but_two();
+          if (a.ready) publish(pend);
+        }
+        pend = skip ? -1 : tile;
+      }
+      tc::tma_store_wait_all();
+      if (pend >= 0 && a.ready) publish(pend);
+      if (!ok) {
+        atomicExch(a.status, 8);
+        vflag[0] = 1;
+      }
     }
   } else {
     // ----------------------------------------------------------- compute --
@@ -376,20 +474,8 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
     float* XS = reinterpret_cast<float*>(sm + C::OFF_XS);
     int gs = 0;
     bool alive = true;
-    // The two storing threads (tid 0 and 128) publish a task's ready flag
-    // once its tiles are in global memory: checked when they next store, so
-    // the check never waits on stores still in flight.
-    int pend = -1;
-    auto publish = [&]() {
-      tc::tma_store_wait_all();
-      if (a.ready && pend >= 0) {
-        tc::fence_async_global();
-        __threadfence();
-        tc::red_add_release_gpu(a.ready + pend, 1);
-      }
-      pend = -1;
-    };
-    for (int ex = 0;; ++ex) {
+    int ex = 0;
+    for (;; ++ex) {
       int task = -1, len = 0;
       size_t tile = 0;
       bool skip = false;
@@ -403,9 +489,11 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
           const int c = task / H;
           len = chunk_pos(a.map, c).len;
           tile = (size_t)c * H + task % H;
-          // the previous task's output stores have read the operand area and Q_eff
-          if ((tid & 127) == 0) tc::tma_store_wait_read();
-          bar_compute();
+          // the previous task's first stores (Mp, Nc) have left slot 2
+          if (ex > 0 && !tc::mbar_wait(rd_a, (ex - 1) & 1)) { alive = false; break; }
+        } else if (s == 2) {
+          // and its last ones (Q_eff, O_part) slots 1 and 3
+          if (ex > 0 && !tc::mbar_wait(rd_b, (ex - 1) & 1)) { alive = false; break; }
         }
         skip |= reinterpret_cast<volatile int*>(slot_skip)[slot] != 0;
         uint8_t* d = sm + slot * C::SLOT_STRIDE;
@@ -654,7 +742,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(t_ready);
-      if (!tc::mbar_wait(mma2_done, ex & 1)) { alive = false; break; }
+      if (!tc::mbar_wait(mma2a_done, ex & 1)) { alive = false; break; }
       // ------------- epilogue 2: R = exp(g_n - g_r) (R'_hi + R'_lo), V = V_hi + V_lo -> bf16 --
       tc::tc_fence_after();
       {
@@ -669,6 +757,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         for (int e = 0; e < 32; e += 2)
           pw[e / 2] = tc::pack_bf16(sc * (__uint_as_float(rh[e]) + __uint_as_float(rl[e])),
                                     sc * (__uint_as_float(rh[e + 1]) + __uint_as_float(rl[e + 1])));
+        // R goes over T, which the V half of UMMA 2 reads
+        if (!tc::mbar_wait(mma2_done, ex & 1)) alive = false;
+        tc::tc_fence_after();
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu)
           *reinterpret_cast<uint4*>(sm + C::OFF_RB + sw_unit(m, (j0 >> 3) + uu)) =
@@ -682,17 +773,21 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
           for (int e = 0; e < 32; e += 2)
             pw[e / 2] = tc::pack_bf16(__uint_as_float(rh[e]) + __uint_as_float(rl[e]),
                                       __uint_as_float(rh[e + 1]) + __uint_as_float(rl[e + 1]));
+          // and again as rows 64..127, so the token rows of the M = 128
+          // product below fill all four TMEM lane quarters
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu)
-            *reinterpret_cast<uint4*>(sm + C::OFF_VB + sw_unit(i, (j0 >> 3) + uu)) =
-                make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
+          for (int uu = 0; uu < 4; ++uu) {
+            const uint4 v4 = make_uint4(pw[4 * uu], pw[4 * uu + 1], pw[4 * uu + 2], pw[4 * uu + 3]);
+            *reinterpret_cast<uint4*>(sm + C::OFF_VB + sw_unit(i, (j0 >> 3) + uu)) = v4;
+            *reinterpret_cast<uint4*>(sm + C::OFF_VB + 8192 + sw_unit(i, (j0 >> 3) + uu)) = v4;
+          }
         }
       }
       tc::fence_async_smem();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(rv_ready);
-      if (!tc::mbar_wait(mma3_done, ex & 1)) { alive = false; break; }
+      if (!alive || !tc::mbar_wait(mma3a_done, ex & 1)) { alive = false; break; }
       // ------------------------------------------- epilogue 3: outputs --
       // Results go to SW128 staging in the (now free) operand area and leave
       // by TMA bulk stores, so every global write is a whole tile row.
@@ -707,6 +802,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
           tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0 + 32), r1);
           tc::tmem_wait_ld_regs(r0);
           tc::tmem_wait_ld_regs(r1);
+          // the second panels (over V and Z) wait for the token-row half of
+          // UMMA 3, which reads both
+          if (c0 && !tc::mbar_wait(mma3_done, ex & 1)) alive = false;
           uint8_t* pnl = sm + (half == 0 ? (c0 ? C::OFF_SMP1 : C::OFF_SMP0) : (c0 ? C::OFF_SNC1 : C::OFF_SNC0));
 #pragma unroll
           for (int uu = 0; uu < 8; ++uu) {
@@ -719,86 +817,81 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
           }
         }
       }
-      // this half's tile (Mp or Nc) leaves while the token rows are finished
+      // this half's tile (Mp or Nc) is staged: it leaves (store warp) while
+      // the token rows are finished
       tc::fence_async_smem();
       bar_half(2 + half);
-      if ((tid & 127) == 0 && !skip) {
-        if (pend >= 0) publish();
-        const int rk = (int)tile * DK;
-        if (half == 0) {
-          tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP0, 0, rk);
-          tc::tma_store_2d(&a.tm_Mp, sm + C::OFF_SMP1, 64, rk);
-        } else {
-          tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC0, 0, rk);
-          if (DV == 128) tc::tma_store_2d(&a.tm_Nc, sm + C::OFF_SNC1, 64, rk);
+      if ((tid & 127) == 0) {
+        if (tid == 0) {
+          s_store[0] = (int)tile;
+          s_store[1] = skip ? 1 : 0;
         }
-        tc::tma_store_commit();
+        tc::mbar_arrive(st_a);
       }
-      if (q < 2) {
-        // token rows (lanes 0..63, warps of lane quarters 0 and 1): half 0:
-        // Q_eff' = Q^ - P W', in place over Q^; half 1: O_part.  The next
-        // 32 columns load while one is packed.
-        const int ncols = half == 0 ? 128 : DV;
-        const int i_out = 32 * q + lane;
-        uint8_t* base = sm + (half == 0 ? C::OFF_SQE : C::OFF_SOP0);
-        const int pstride = half == 0 ? C::PANEL : 8192;
-        auto pack_rows = [&](const uint32_t (&r)[32], int c0) {
-          uint8_t* pnl = base + (c0 >> 6) * pstride;
+      {
+        // token rows: lane quarters 0, 1 form Q_eff' = Q^ - P W' (columns
+        // 0..127, in slot 1 from Q^ in slot 0 / 1), lane quarters 2, 3
+        // (the same rows again) O_part (columns 128..); each half takes one
+        // 64-column panel.
+        const bool qside = q < 2;
+        if (qside || DV == 128 || half == 0) {
+          const int i_out = 32 * (q & 1) + lane;
+          uint8_t* pnl = sm + (qside ? C::OFF_SQE : C::OFF_SOP0) + half * 8192;
+          const uint8_t* qh = sm + C::OFF_QH + half * C::PANEL;
+          auto pack_rows = [&](const uint32_t (&r)[32], int cc) {
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu) {
-            uint4* dst = reinterpret_cast<uint4*>(pnl + sw_unit(i_out, ((c0 & 63) >> 3) + uu));
-            uint32_t pw[4];
-            if (half == 0) {
-              const uint4 qv = *dst;
-              const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+            for (int uu = 0; uu < 4; ++uu) {
+              const uint32_t off = sw_unit(i_out, (cc >> 3) + uu);
+              uint32_t pw[4];
+              if (qside) {
+                const uint4 qv = *reinterpret_cast<const uint4*>(qh + off);
+                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                pw[e] = tc::pack_bf16(bf16_lo_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e]),
-                                      bf16_hi_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e + 1]));
-            } else {
+                for (int e = 0; e < 4; ++e)
+                  pw[e] = tc::pack_bf16(bf16_lo_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e]),
+                                        bf16_hi_f(qw[e]) - __uint_as_float(r[8 * uu + 2 * e + 1]));
+              } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                pw[e] = tc::pack_bf16(__uint_as_float(r[8 * uu + 2 * e]), __uint_as_float(r[8 * uu + 2 * e + 1]));
+                for (int e = 0; e < 4; ++e)
+                  pw[e] = tc::pack_bf16(__uint_as_float(r[8 * uu + 2 * e]), __uint_as_float(r[8 * uu + 2 * e + 1]));
+              }
+              *reinterpret_cast<uint4*>(pnl + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
             }
-            *dst = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-          }
-        };
-        uint32_t ra[32], rb[32];
-        const uint32_t col = C::COL_QO + 128 * half;
-        tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col), ra);
-        tc::tmem_wait_ld_regs(ra);
-        for (int c0 = 0; c0 < ncols; c0 += 64) {
-          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col + c0 + 32), rb);
-          pack_rows(ra, c0);
+          };
+          uint32_t ra[32], rb[32];
+          const uint32_t col = C::COL_QO + (qside ? 0u : 128u) + 64u * half;
+          if (!tc::mbar_wait(mma3_done, ex & 1)) alive = false;
+          tc::tc_fence_after();
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col), ra);
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col + 32), rb);
+          tc::tmem_wait_ld_regs(ra);
+          pack_rows(ra, 0);
           tc::tmem_wait_ld_regs(rb);
-          if (c0 + 64 < ncols) tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, col + c0 + 64), ra);
-          pack_rows(rb, c0 + 32);
-          if (c0 + 64 < ncols) tc::tmem_wait_ld_regs(ra);
+          pack_rows(rb, 32);
         }
       }
       tc::fence_async_smem();
       tc::tc_fence_before();
       bar_compute();
-      if ((tid & 127) == 0) {
+      if (tid == 0) {
         if (skip) {
           // decay too steep for one reference point: hand the chunk back
-          if (tid == 0) {
-            const int idx = atomicAdd(a.fix_list, 1);
-            a.fix_list[1 + idx] = (int)tile;
-            if (a.ready) tc::st_release_gpu(a.ready + tile, 3);
-          }
-        } else {
-          const int rt = (int)tile * kChunk;
-          if (half == 0)
-            for (int p = 0; p < 2; ++p) tc::tma_store_2d(&a.tm_Qe, sm + C::OFF_SQE + p * C::PANEL, 64 * p, rt);
-          else
-            for (int p = 0; p < DV / 64; ++p) tc::tma_store_2d(&a.tm_Op, sm + C::OFF_SOP0 + p * 8192, 64 * p, rt);
-          tc::tma_store_commit();
-          if (a.ready) pend = (int)tile;  // each storing thread adds 1: 2 = factors written
+          const int idx = atomicAdd(a.fix_list, 1);
+          a.fix_list[1 + idx] = (int)tile;
+          if (a.ready) tc::st_release_gpu(a.ready + tile, 3);
         }
+        tc::mbar_arrive(st_b);
       }
     }
-    if ((tid & 127) == 0) publish();
+    // no task left: the store warp finishes what it holds and ends (once it
+    // has taken the last task's tile index)
+    if ((tid & 127) == 0) {
+      if (tid == 0) {
+        if (ex > 0) tc::mbar_wait(rd_a, (ex - 1) & 1);
+        s_store[0] = -1;
+      }
+      tc::mbar_arrive(st_a);
+    }
     if (!alive) {
       atomicExch(a.status, 8);
       vflag[0] = 1;
@@ -828,6 +921,12 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
     tc::mbar_inval(rv_ready);
     tc::mbar_inval(mma3_done);
     tc::mbar_inval(fin);
+    tc::mbar_inval(mma2a_done);
+    tc::mbar_inval(mma3a_done);
+    tc::mbar_inval(st_a);
+    tc::mbar_inval(st_b);
+    tc::mbar_inval(rd_a);
+    tc::mbar_inval(rd_b);
     tc::fence_async_smem();
   }
   if (stopper) __syncthreads();

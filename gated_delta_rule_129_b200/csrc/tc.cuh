@@ -96,10 +96,23 @@ __device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int c0, int c1
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(c0), "r"(c1)
                : "memory");
 }
+__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(c0), "r"(c1),
+               "r"(c2)
+               : "memory");
+}
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // The shared-memory sources of all committed stores may be reused.
 __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// As tma_store_wait_read, for every committed group but the newest.
+__device__ __forceinline__ void tma_store_wait_read_but_newest() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// All committed stores but the two newest groups have been performed.
+__device__ __forceinline__ void tma_store_wait_all_but_two() {
+  asm volatile("cp.async.bulk.wait_group 2;" ::: "memory");
 }
 // All committed stores have been performed (visible in global memory).
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }

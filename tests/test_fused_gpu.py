@@ -54,6 +54,8 @@ CASES = [
     dict(B=1, T=777, H=3, dv=64, lengths=None, h0=0.05),
     dict(B=2, T=300, H=2, dv=128, lengths=None, h0=0.05),
     dict(B=1, T=None, H=3, dv=128, lengths=[130, 0, 64, 1, 500], h0=0.05),
+    # 20 heads: the walk CTAs take prep tasks first (switch point above 0)
+    dict(B=1, T=300, H=20, dv=128, lengths=None, h0=0.05),
 ]
 
 
