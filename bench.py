@@ -45,6 +45,12 @@ ALG_FLOPS = TH * (6 * DK * DV + 5 * 64 * 128 + 64 * 64 / 3)
 # the affine set (bf16 Mp, Nc = 2 x 128 x 128 x 2 B per 64 tokens, Q_eff,
 # O_part = 2 x 64 x 128 x 2 B: 1536 B per token-head; exp(g_n) fp32 8 B).
 FACTOR_BYTES_PER_TH = 1536 + 8
+# DRAM bytes (read + write) of one fused launch at 16K x 1, from one ncu
+# capture (dram__bytes_read.sum 629,582,336 + dram__bytes_write.sum
+# 424,988,928) of this build's fused kernel under this script's own command;
+# profiles/ holds the command.  It must be taken again (or set to None)
+# whenever the fused kernel changes.
+FUSED_TRAFFIC_BYTES = 629582336 + 424988928
 PREP_BYTES = TH * (2304 + FACTOR_BYTES_PER_TH)
 WALK_BYTES = TH * (FACTOR_BYTES_PER_TH + 256) + B * H * DK * DV * 4
 L2_FLUSH_BYTES = 256 << 20
@@ -320,7 +326,7 @@ def run_ours(args, rank, world, local):
                    "global_batch": world * B, "seq_len": T, "parallelism": f"replicas x{world}",
                    "l2": "flushed between timed steps (256 MiB write)"},
         "roofline": {"bound": "hbm", "achieved": dom_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": dom_gbs / hbm, "traffic": None, "kernel": dom,
+                     "frac": dom_gbs / hbm, "traffic": FUSED_TRAFFIC_BYTES, "kernel": dom,
                      "kernel_ms": kern_ms[dom], "alg_bytes_per_launch": dom_bytes,
                      "peak_source": f"{src} (MEASURED_PEAKS hbm_gbs)" if src == "measured" else src},
         "roofline_step": {"alg_bytes": ALG_BYTES, "alg_flops": ALG_FLOPS, "t_roof_us": t_roof * 1e6,
