@@ -46,11 +46,10 @@ ALG_FLOPS = TH * (6 * DK * DV + 5 * 64 * 128 + 64 * 64 / 3)
 # O_part = 2 x 64 x 128 x 2 B: 1536 B per token-head; exp(g_n) fp32 8 B).
 FACTOR_BYTES_PER_TH = 1536 + 8
 # DRAM bytes (read + write) of one fused launch at 16K x 1, from one ncu
-# capture (dram__bytes_read.sum 629,582,336 + dram__bytes_write.sum
-# 424,988,928) of this build's fused kernel under this script's own command;
-# profiles/ holds the command.  It must be taken again (or set to None)
-# whenever the fused kernel changes.
-FUSED_TRAFFIC_BYTES = 629582336 + 424988928
+# capture of this build's fused kernel under this script's own command
+# (profiles/ holds the command), or None until that capture exists.  It is
+# taken again whenever the fused kernel changes.
+FUSED_TRAFFIC_BYTES = None
 PREP_BYTES = TH * (2304 + FACTOR_BYTES_PER_TH)
 WALK_BYTES = TH * (FACTOR_BYTES_PER_TH + 256) + B * H * DK * DV * 4
 L2_FLUSH_BYTES = 256 << 20

@@ -416,11 +416,9 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
     // Per task: the Mp / Nc tiles once both half leaders have staged them,
     // the Q_eff / O_part tiles once the epilogue is done; the staging is
     // handed back as soon as the stores have read it, and the task's ready
-    // flag (2 = factors written) is raised once its stores are complete,
-    // which is checked one task later so that it never holds up a store.
+    // flag (2 = factors written) is raised once its stores are complete.
     if (lane == 0) {
       volatile int* vst = s_store;
-      int pend = -1;
       bool ok = true;
       auto publish = [&](int t) {
         tc::fence_async_global();
@@ -451,16 +449,14 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         tc::mbar_arrive(rd_a);
         tc::tma_store_wait_read();
         tc::mbar_arrive(rd_b);
-        if (pend >= 0) {
-          // the previous stored task's two groups are complete
-          if (skip) tc::tma_store_wait_all();
-          else tc::tma_store_wait_all_but_two();
-          if (a.ready) publish(pend);
+        if (!skip && a.ready) {
+          // the compute warps are building the next task by now and need
+          // nothing more from this warp until its epilogue
+          tc::tma_store_wait_all();
+          publish(tile);
         }
-        pend = skip ? -1 : tile;
       }
       tc::tma_store_wait_all();
-      if (pend >= 0 && a.ready) publish(pend);
       if (!ok) {
         atomicExch(a.status, 8);
         vflag[0] = 1;
