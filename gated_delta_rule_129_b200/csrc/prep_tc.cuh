@@ -189,6 +189,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   int* slot_task = s_flag + 2;                        // [NSLOT] task id of the slot's slice
   int* slot_skip = slot_task + C::NSLOT;              // [NSLOT] decay range exceeded
   int* s_store = slot_skip + C::NSLOT;                // [2] tile being stored (-1: none left), skip
+  int* slot_len = s_store + 2;                        // [NSLOT] valid tokens of the slot's chunk
   float* s_enr = reinterpret_cast<float*>(sm + C::OFF_BAR + 512);  // [2][128] exp(g_n - g_r), by task parity
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -228,6 +229,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
   const uint32_t tbase = *tslot;
   volatile int* vflag = s_flag;
   volatile int* vtask = slot_task;
+  volatile int* vlen = slot_len;
 
   if (warp == C::PRODUCER_WARP) {
     // ---------------------------------------------------- input producer --
@@ -245,10 +247,12 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         }
         else task = cta_rank + cta_count * (k_static++);
         if (task >= ntasks) task = -1;
-        int h = 0, t0 = 0;
+        int h = 0, t0 = 0, tlen = 0;
         if (task >= 0) {
           h = task % H;
-          t0 = chunk_pos(a.map, task / H).t0;
+          const ChunkPos cp = chunk_pos(a.map, task / H);
+          t0 = cp.t0;
+          tlen = cp.len;
         }
         if (task >= 0 && a.l2_prefetch) {
           // the last slice is loaded only once this task's first slice has
@@ -269,6 +273,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
           if (use > 0 && !tc::mbar_wait(&empty[slot], (use - 1) & 1)) { ok = false; break; }
           if (vflag[0]) { more = false; break; }
           vtask[slot] = task;
+          vlen[slot] = tlen;  // the consumers need not look the chunk up again
           if (task < 0) {
             tc::mbar_arrive(&full[slot]);
             more = false;
@@ -308,7 +313,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       const int task = vtask[slot];
       if (task >= 0 && !vflag[0]) {
         const int c = task / H;
-        const int len = chunk_pos(a.map, c).len;
+        const int len = vlen[slot];
         const size_t tile = (size_t)c * H + task % H;
         float* la = reinterpret_cast<float*>(sm + slot * C::SLOT_STRIDE + C::OFF_LA);
         float v[kChunk];
@@ -338,8 +343,10 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         for (int t = 0; t < kChunk; ++t) la[swf(t, lane)] = v[t] - gr;
         s_enr[tpar * DK + C::KS * s_in + lane] = __expf(gn - gr);
         a.gamma_last[tile * DK + C::KS * s_in + lane] = expf(gn);
+        // published with the chunk's other factors: the store warp's fence
+        // and release of the ready flag come after these writes through the
+        // CTA's mbarrier chain (releases are cumulative)
         a.colscale[tile * DK + C::KS * s_in + lane] = __expf(gr);
-        if (a.ready) __threadfence();  // published with the chunk's other factors
         const unsigned any = __ballot_sync(0xffffffffu, bad);
         if (lane == 0) slot_skip[slot] = any != 0u;
         s_in = (s_in + 1) & (C::SLICES - 1);
@@ -483,7 +490,7 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         if (task < 0 || vflag[0]) break;
         if (s == 0) {
           const int c = task / H;
-          len = chunk_pos(a.map, c).len;
+          len = vlen[slot];
           tile = (size_t)c * H + task % H;
           // the previous task's first stores (Mp, Nc) have left slot 2
           if (ex > 0 && !tc::mbar_wait(rd_a, (ex - 1) & 1)) { alive = false; break; }
