@@ -300,8 +300,8 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
     }
   } else if (warp == C::SCAN_WARP) {
     // -------------------------------------------------------------- scan --
-    // lane = channel of the slice; g_t = sum of log_alpha over tokens <= t of
-    // the chunk (tokens past its end count as 0), written over log_alpha.
+    // g_t = sum of log_alpha over tokens <= t of the chunk (tokens past its
+    // end count as 0), written over log_alpha as g_t - g_r.
     int s_in = 0, tpar = 0;
     for (int gs = 0;; ++gs) {
       const int slot = gs % C::NSLOT, use = gs / C::NSLOT;
@@ -316,37 +316,68 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
         const int len = vlen[slot];
         const size_t tile = (size_t)c * H + task % H;
         float* la = reinterpret_cast<float*>(sm + slot * C::SLOT_STRIDE + C::OFF_LA);
-        float v[kChunk];
+        // lane = (token quarter tq, channel group cg): tokens 16 tq .. 16 tq + 15
+        // of channels 4 cg .. 4 cg + 3, one 16-byte unit of each SW128 row
+        const int tq = lane >> 3, cg = lane & 7;
+        auto unit = [&](int i) {
+          const int t = 16 * tq + i;
+          return reinterpret_cast<float4*>(la + t * 32 + ((cg ^ (t & 7)) << 2));
+        };
+        float4 v[16];
 #pragma unroll
-        for (int t = 0; t < kChunk; ++t) v[t] = la[swf(t, lane)];
-        // four 16-token running sums side by side, then the block offsets
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = 0; i < 16; ++i) v[i] = *unit(i);
+        // running sums within the quarter (tokens past the chunk's end add 0)
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-#pragma unroll
-          for (int bq = 0; bq < 4; ++bq) {
-            const int tt = 16 * bq + t;
-            acc[bq] += tt < len ? v[tt] : 0.f;
-            v[tt] = acc[bq];
+        for (int i = 0; i < 16; ++i) {
+          if (16 * tq + i < len) {
+            acc.x += v[i].x; acc.y += v[i].y; acc.z += v[i].z; acc.w += v[i].w;
           }
-        const float off1 = acc[0], off2 = off1 + acc[1], off3 = off2 + acc[2];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          v[16 + t] += off1;
-          v[32 + t] += off2;
-          v[48 + t] += off3;
+          v[i] = acc;
         }
-        const float g0 = v[0], gr = v[32], gn = v[kChunk - 1];
-        const bool bad = (g0 - gr > 60.f) || (gr - gn > 60.f);
+        // the quarters' offsets: inclusive scan of the totals over tq, then
+        // the previous quarter's value
+        auto shfl_up4 = [](float4 a, int d) {
+          return make_float4(__shfl_up_sync(0xffffffffu, a.x, d), __shfl_up_sync(0xffffffffu, a.y, d),
+                             __shfl_up_sync(0xffffffffu, a.z, d), __shfl_up_sync(0xffffffffu, a.w, d));
+        };
+        auto shfl4 = [](float4 a, int src) {
+          return make_float4(__shfl_sync(0xffffffffu, a.x, src), __shfl_sync(0xffffffffu, a.y, src),
+                             __shfl_sync(0xffffffffu, a.z, src), __shfl_sync(0xffffffffu, a.w, src));
+        };
+        float4 inc = acc;
+        {
+          const float4 y = shfl_up4(inc, 8);
+          if (tq >= 1) { inc.x += y.x; inc.y += y.y; inc.z += y.z; inc.w += y.w; }
+          const float4 z = shfl_up4(inc, 16);
+          if (tq >= 2) { inc.x += z.x; inc.y += z.y; inc.z += z.z; inc.w += z.w; }
+        }
+        float4 off = shfl_up4(inc, 8);
+        if (tq == 0) off = make_float4(0.f, 0.f, 0.f, 0.f);
+        // g at token 0 (quarter 0), r = 32 (quarter 2) and 63 (quarter 3)
+        const float4 first = make_float4(v[0].x + off.x, v[0].y + off.y, v[0].z + off.z, v[0].w + off.w);
+        const float4 last = make_float4(v[15].x + off.x, v[15].y + off.y, v[15].z + off.z, v[15].w + off.w);
+        const float4 g0 = shfl4(first, cg), gr = shfl4(first, 16 + cg), gn = shfl4(last, 24 + cg);
+        const bool bad = (g0.x - gr.x > 60.f) || (g0.y - gr.y > 60.f) || (g0.z - gr.z > 60.f) ||
+                         (g0.w - gr.w > 60.f) || (gr.x - gn.x > 60.f) || (gr.y - gn.y > 60.f) ||
+                         (gr.z - gn.z > 60.f) || (gr.w - gn.w > 60.f);
         // what the build needs: x_t = g_t - g_r, over log_alpha
 #pragma unroll
-        for (int t = 0; t < kChunk; ++t) la[swf(t, lane)] = v[t] - gr;
-        s_enr[tpar * DK + C::KS * s_in + lane] = __expf(gn - gr);
-        a.gamma_last[tile * DK + C::KS * s_in + lane] = expf(gn);
-        // published with the chunk's other factors: the store warp's fence
-        // and release of the ready flag come after these writes through the
-        // CTA's mbarrier chain (releases are cumulative)
-        a.colscale[tile * DK + C::KS * s_in + lane] = __expf(gr);
+        for (int i = 0; i < 16; ++i)
+          *unit(i) = make_float4((v[i].x + off.x) - gr.x, (v[i].y + off.y) - gr.y, (v[i].z + off.z) - gr.z,
+                                 (v[i].w + off.w) - gr.w);
+        if (tq == 0) {
+          const int ch = C::KS * s_in + 4 * cg;
+          *reinterpret_cast<float4*>(s_enr + tpar * DK + ch) =
+              make_float4(__expf(gn.x - gr.x), __expf(gn.y - gr.y), __expf(gn.z - gr.z), __expf(gn.w - gr.w));
+          *reinterpret_cast<float4*>(a.gamma_last + tile * DK + ch) =
+              make_float4(expf(gn.x), expf(gn.y), expf(gn.z), expf(gn.w));
+          // published with the chunk's other factors: the store warp's fence
+          // and release of the ready flag come after these writes through the
+          // CTA's mbarrier chain (releases are cumulative)
+          *reinterpret_cast<float4*>(a.colscale + tile * DK + ch) =
+              make_float4(__expf(gr.x), __expf(gr.y), __expf(gr.z), __expf(gr.w));
+        }
         const unsigned any = __ballot_sync(0xffffffffu, bad);
         if (lane == 0) slot_skip[slot] = any != 0u;
         s_in = (s_in + 1) & (C::SLICES - 1);
@@ -798,26 +829,42 @@ __device__ void prep_tc_cta(const PrepTcArgs& a, uint8_t* sm, int cta_rank, int 
       {
         const int m = 32 * q + lane;  // key channel row of Mp / Nc
         // half 0: Mp' columns 0..127; half 1: Nc columns 0..DV-1 (TMEM 128..)
-        const int ncols = half == 0 ? 128 : DV;
-        for (int c0 = 0; c0 < ncols; c0 += 64) {
-          uint32_t r0[32], r1[32];
-          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0), r0);
-          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, C::COL_MN + 128 * half + c0 + 32), r1);
+        const uint32_t colb = C::COL_MN + 128 * half;
+        auto stage = [&](uint8_t* pnl, const uint32_t (&pk)[32]) {
+#pragma unroll
+          for (int uu = 0; uu < 8; ++uu)
+            *reinterpret_cast<uint4*>(pnl + sw_unit(m, uu)) =
+                make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
+        };
+        uint32_t r0[32], r1[32], pk[32];
+        tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, colb), r0);
+        tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, colb + 32), r1);
+        tc::tmem_wait_ld_regs(r0);
+        tc::tmem_wait_ld_regs(r1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          pk[e] = tc::pack_bf16(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+          pk[16 + e] = tc::pack_bf16(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+        }
+        const bool second = half == 0 || DV == 128;
+        if (second) {
+          // the second 64 columns load while the first are staged
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, colb + 64), r0);
+          tc::tmem_ld32_nowait(tc::tmem_addr(tbase, 32 * q, colb + 96), r1);
+        }
+        stage(sm + (half == 0 ? C::OFF_SMP0 : C::OFF_SNC0), pk);
+        if (second) {
           tc::tmem_wait_ld_regs(r0);
           tc::tmem_wait_ld_regs(r1);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            pk[e] = tc::pack_bf16(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+            pk[16 + e] = tc::pack_bf16(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+          }
           // the second panels (over V and Z) wait for the token-row half of
           // UMMA 3, which reads both
-          if (c0 && !tc::mbar_wait(mma3_done, ex & 1)) alive = false;
-          uint8_t* pnl = sm + (half == 0 ? (c0 ? C::OFF_SMP1 : C::OFF_SMP0) : (c0 ? C::OFF_SNC1 : C::OFF_SNC0));
-#pragma unroll
-          for (int uu = 0; uu < 8; ++uu) {
-            const uint32_t* r = uu < 4 ? r0 + 8 * uu : r1 + 8 * (uu - 4);
-            *reinterpret_cast<uint4*>(pnl + sw_unit(m, uu)) =
-                make_uint4(tc::pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                           tc::pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                           tc::pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                           tc::pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7])));
-          }
+          if (!tc::mbar_wait(mma3_done, ex & 1)) alive = false;
+          stage(sm + (half == 0 ? C::OFF_SMP1 : C::OFF_SNC1), pk);
         }
       }
       // this half's tile (Mp or Nc) is staged: it leaves (store warp) while
