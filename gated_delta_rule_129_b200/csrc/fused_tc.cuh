@@ -3,10 +3,8 @@
 // On a long sequence with few heads the walk runs on a few dozen SMs while
 // the prep could use all of them, and run back to back the two add up.  Here
 // one persistent grid of one CTA per SM holds both: the last n_walk CTAs walk
-// (one per head and 64-column value slice, through the sequences one after
-// the other), the others take prep tasks in chunk-major order from a shared
-// counter, so the chunks of every head come ready in the order its walk CTAs
-// use them.  The walk CTAs take prep
+// (one per sequence, head and 64-column value slice), the others take prep
+// tasks in chunk-major order from a shared counter.  The walk CTAs take prep
 // tasks too until the counter reaches stop_at, chosen on the host so that
 // the walk, started then, ends about when the prep does.  A prep CTA publishes a
 // chunk's ready flag once its factors are in global memory (where they are
@@ -43,9 +41,7 @@ fused_tc_kernel(const __grid_constant__ PrepTcArgs pa, const __grid_constant__ W
     // early on, the walk would only wait for the prep wavefront: take prep
     // tasks until the counter reaches pa.stop_at, then walk
     if (pa.stop_at > 0) prep_tc_cta<DV>(pa, sm, blockIdx.x, gridDim.x, true);
-    // one walk CTA per (head, value slice), through every sequence in turn
-    const int w = (int)blockIdx.x - n_prep;
-    walk_tc_cta<DV>(wa, sm, w / WalkTcCfg<DV>::SLICES, w % WalkTcCfg<DV>::SLICES, 0, wa.map.N);
+    walk_tc_cta<DV>(wa, sm, (int)blockIdx.x - n_prep);
   }
 }
 

@@ -362,13 +362,8 @@ gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, cons
 // cut the walk short, the walk again.
 template <int DV>
 bool fused_fits(const gdn2_desc* d, const Layout& L) {
-  // The walk CTAs (one per head and value slice) take the sequences one after
-  // the other; each sequence change costs a read of its initial state on the
-  // walk's serial path, so many short sequences (under 4 chunks on average)
-  // keep the two-kernel path, which walks all sequences at once.
-  const long long n_walk = (long long)d->H * gdn2::WalkTcCfg<DV>::SLICES;
-  const long long tokens = (long long)d->B * d->T;
-  return L.l.factor_set == 1 && L.N > 0 && tokens > 0 && tokens >= 4ll * kChunk * L.N &&
+  const long long n_walk = (long long)L.N * d->H * gdn2::WalkTcCfg<DV>::SLICES;
+  return L.l.factor_set == 1 && L.N > 0 && (long long)d->B * d->T > 0 &&
          n_walk + gdn2::FusedTcCfg<DV>::MIN_PREP_CTAS <= sm_count();
 }
 
@@ -389,7 +384,7 @@ gdn2_status launch_fused_tc(const gdn2_desc* d, const Layout& L, const void* q, 
   wa.ready = sync + 2;
   wa.redo = sync + 1;
   const int n_sm = sm_count();
-  const int n_walk = d->H * gdn2::WalkTcCfg<DV>::SLICES;
+  const int n_walk = L.N * d->H * gdn2::WalkTcCfg<DV>::SLICES;
   // When the walk CTAs stop taking prep tasks: a walk of nch chunks started
   // when nch * (n_sm - n_walk) / 7 tasks are left ends about with the prep
   // (beside the prep, a walk step costs about a seventh of a prep task on
@@ -398,7 +393,7 @@ gdn2_status launch_fused_tc(const gdn2_desc* d, const Layout& L, const void* q, 
   // point at 16K x 1 has its optimum at 0), and then they skip the prep role.
   {
     const long long tasks = (long long)L.l.max_chunks * d->H;
-    const long long nch = L.l.max_chunks;  // the walk's length: every sequence's chunks
+    const long long nch = ((long long)d->B * d->T + (long long)kChunk * L.N - 1) / ((long long)kChunk * L.N);
     const long long left = nch * (n_sm - n_walk) / 7;
     pa.stop_at = (int)std::max(0ll, tasks - left);
   }

@@ -142,13 +142,8 @@ __device__ __forceinline__ bool wait_chunk_ready(const WalkTcArgs& a, int t, int
   return true;
 }
 
-// Walks value slice `sl` of head `h` through sequences n0 .. n1-1 one after
-// the other (their chunks are consecutive in the chunk numbering): the rings
-// and the UMMA issue run over the chunks without a break, and at the end of
-// each sequence the state warps store its final state and load the next
-// sequence's initial one.
 template <int DV>
-__device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int h, int sl, int n0, int n1) {
+__device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
   using C = WalkTcCfg<DV>;
   constexpr int DK = C::DK, NSL = C::NSL;
   uint8_t* ringA = sm;
@@ -168,9 +163,13 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int h, int sl, int
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
+  const int sl = cta % C::SLICES;
+  const int h = (cta / C::SLICES) % H;
+  const int n = cta / (C::SLICES * H);
   const int col0 = sl * NSL;
-  const int c_begin = a.map.chunk_off[n0];
-  const int nch = a.map.chunk_off[n1] - c_begin;
+  const int c_begin = a.map.chunk_off[n];
+  const int nch = a.map.chunk_off[n + 1] - c_begin;
+  const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
 
   if (tid == 0) {
     for (int s = 0; s < C::STAGES_A; ++s) {
@@ -202,47 +201,13 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int h, int sl, int
   if (warp < C::EPI_WARPS) {
     // ----------------------------------------------------- state update --
     const int row = 32 * warp + lane;  // key channel = TMEM lane
-    auto sbase_of = [&](int n) { return ((size_t)n * H + h) * DK * DV + (size_t)row * DV + col0; };
+    const size_t sbase = ((size_t)n * H + h) * DK * DV + (size_t)row * DV + col0;
     float S[NSL];
-    auto load_h0 = [&](int n) {
 #pragma unroll
-      for (int i = 0; i < NSL; i += 4) {
-        const float4 v =
-            a.h0 ? *reinterpret_cast<const float4*>(a.h0 + sbase_of(n) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-        S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
-      }
-    };
-    auto store_hT = [&](int n) {
-      if (a.hT)
-#pragma unroll
-        for (int i = 0; i < NSL; i += 4)
-          *reinterpret_cast<float4*>(a.hT + sbase_of(n) + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
-    };
-    // sequence n is being walked; sequences without chunks keep their
-    // initial state
-    int n = n0;
-    auto skip_empty = [&]() {
-      while (n < n1 && a.map.chunk_off[n + 1] == a.map.chunk_off[n]) {
-        if (a.hT) {
-          load_h0(n);
-          store_hT(n);
-        }
-        ++n;
-      }
-    };
-    // the next sequence's initial state is read on the walk's serial path:
-    // start it towards L2 while this one is walked
-    auto prefetch_h0 = [&](int m) {
-      if (a.h0 && m < n1) {
-        const float* p = a.h0 + sbase_of(m);
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 32));
-      }
-    };
-    skip_empty();
-    if (n < n1) load_h0(n);
-    prefetch_h0(n + 1);
-    int c_next_seq = n < n1 ? a.map.chunk_off[n + 1] : 0;  // first chunk after sequence n
+    for (int i = 0; i < NSL; i += 4) {
+      const float4 v = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + sbase + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
+    }
     // this thread's row in the interleaved operand: core matrix (row/8, g),
     // 16-byte line row%8
     const uint32_t srow = (row >> 3) * C::S_LBO + (row & 7) * 16;
@@ -320,39 +285,21 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int h, int sl, int
         if (!wwait(&fullB[sn], ((j + 1) / C::STAGES_B) & 1, a.status, s_abort)) break;
         cs_next = colscale_of(j + 1);
       }
-      if (c + 1 == c_next_seq) {
-        // sequence n is done: its final state out, the next one's initial
-        // state in (the operand stored below is the next chunk's)
-        store_hT(n);
-        ++n;
-        skip_empty();
-        if (n < n1) {
-          load_h0(n);
-          prefetch_h0(n + 1);
-          c_next_seq = a.map.chunk_off[n + 1];
-        }
-      }
       store_state((j + 1) & 1, cs_next);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
+    }
+    if (a.hT && !*reinterpret_cast<volatile int*>(s_abort)) {
+#pragma unroll
+      for (int i = 0; i < NSL; i += 4)
+        *reinterpret_cast<float4*>(a.hT + sbase + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
     }
   } else if (warp < 2 * C::EPI_WARPS) {
     // ---------------------------------------------------------- outputs --
     const int ow = warp - C::EPI_WARPS;   // TMEM lane quarter of this warp
     const int i_tok = 16 * ow + lane;     // token row of D_O (M = 64 layout), lane < 16
-    // the sequence of the current chunk, its first chunk and its tokens
-    int no = n0, c_first = c_begin, c_after = a.map.chunk_off[n0 + 1];
-    int s_begin = a.map.seq_begin(n0), s_end = a.map.seq_end(n0);
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
-      const int c = c_begin + j;
-      while (c >= c_after) {
-        ++no;
-        c_first = c_after;
-        c_after = a.map.chunk_off[no + 1];
-        s_begin = a.map.seq_begin(no);
-        s_end = a.map.seq_end(no);
-      }
       const int sb = j % C::STAGES_B;
       const uint8_t* stB = ringB + sb * C::B_STRIDE;
       if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort) || !wwait(o_done, j & 1, a.status, s_abort))
@@ -366,7 +313,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int h, int sl, int
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&o_free[j & 1]);
-      const int t0 = s_begin + (c - c_first) * kChunk;
+      const int t0 = s_begin + j * kChunk;
       const int len = min(kChunk, s_end - t0);
       if (lane < 16 && i_tok < len) {
         const uint8_t* op = stB + C::NC_BYTES + i_tok * 128;
@@ -501,10 +448,7 @@ walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  // one CTA per (sequence, head, value slice)
-  const int cta = blockIdx.x, H = a.H;
-  const int n = cta / (WalkTcCfg<DV>::SLICES * H);
-  walk_tc_cta<DV>(a, sm, (cta / WalkTcCfg<DV>::SLICES) % H, cta % WalkTcCfg<DV>::SLICES, n, n + 1);
+  walk_tc_cta<DV>(a, sm, blockIdx.x);
 }
 
 }  // namespace gdn2
