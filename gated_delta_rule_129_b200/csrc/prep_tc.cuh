@@ -2,8 +2,10 @@
 // map on the tensor cores (bf16 I/O, dk = 128, dv in {64, 128}).
 //
 // Persistent CTAs walk a list of (chunk, head) tasks.  Warp roles:
-//   warp 8      TMA producer: streams each task's inputs in four 32-channel
-//               slices through a 3-slot ring that runs ahead across tasks;
+//   warp 8      TMA producer: takes the tasks, streams each task's inputs
+//               in four 32-channel slices through a 3-slot ring that runs
+//               ahead across tasks, and puts the task id and its chunk's
+//               length beside each slice (nobody else looks the chunk up);
 //   warp 10     scan: per slice, the in-chunk cumulative sum g of log_alpha,
 //               written in place as g - g_r, the per-channel constants
 //               exp(g_r), exp(g_n - g_r), exp(g_n), and the decay-range check;
@@ -43,9 +45,11 @@
 //     hi + lo, stored side by side as one operand (~16 bits of T kept).
 //  4. UMMA 2: [R'_hi | R'_lo] = K^^T [T_hi | T_lo], [V_hi | V_lo] = P [T_hi | T_lo];
 //     R = Kbar^T T = diag(exp(g_n - g_r)) R'.
-//  5. UMMA 3: [Mp' | Nc] = R [E^ | Z], [P W' | O_part] = V [E^ | Z]; the
-//     epilogue writes Mp', Nc, Q_eff' = Q^ - P W' and O_part (bf16) by TMA
-//     stores; Mp = Mp' diag(exp(g_r)) and Q_eff = Q_eff' diag(exp(g_r)).
+//  5. UMMA 3: [Mp' | Nc] = R [E^ | Z], then [P W' | O_part] = [V; V] [E^ | Z]
+//     (the 64 token rows twice, so they fill all four TMEM lane quarters);
+//     the epilogue stages Mp', Nc, Q_eff' = Q^ - P W' and O_part (bf16) and
+//     the store warp writes them by TMA; Mp = Mp' diag(exp(g_r)) and
+//     Q_eff = Q_eff' diag(exp(g_r)).
 // Rows past the chunk's last token are zero in every operand, so they add
 // nothing; the padded rows of Q_eff and O_part come out as exact zeros.
 #pragma once
