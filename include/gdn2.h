@@ -139,6 +139,8 @@ typedef struct gdn2_ws_layout {
   size_t off_sync;           /* int32 [2 + max_chunks * H] (set 1): [0] next     */
                              /* prep task, [1] walk redo flag, then one ready    */
                              /* flag per (chunk, head) for the fused prep + walk */
+                             /* (0 = not yet, 2 = factors written, 3 = handed    */
+                             /* back for the exact redo)                         */
   size_t off_colscale;       /* column scale of Mp, Q_eff [., H, dk] fp32 set 1 */
 } gdn2_ws_layout;
 
