@@ -19,6 +19,9 @@ Contents
   recurrence with every sequence one token long.
 * :mod:`oracle.chunk_wy` -- the 64-token chunkwise WY restatement in fp64
   (numpy), used to check the chunk algebra and to give per-chunk intermediates.
+* :mod:`oracle.backward` -- the gradients of O and hT with respect to every
+  input, reverse mode through the token recurrence in fp64 (numpy; small cases),
+  pinned by finite differences of :func:`recurrent`.
 
 Arrays use the token-major layout ``[B, T, H, D]`` (or ``[1, T_total, H, D]``
 with ``cu_seqlens``).  Inputs of any float dtype are upcast to fp64 exactly.
