@@ -22,6 +22,9 @@ Contents
 * :mod:`oracle.backward` -- the gradients of O and hT with respect to every
   input, reverse mode through the token recurrence in fp64 (numpy; small cases),
   pinned by finite differences of :func:`recurrent`.
+* :mod:`oracle.chunk_backward` -- the same gradients through the 64-token chunk
+  form (the algebra a backward over chunks evaluates), checked against
+  :mod:`oracle.backward`.
 
 Arrays use the token-major layout ``[B, T, H, D]`` (or ``[1, T_total, H, D]``
 with ``cu_seqlens``).  Inputs of any float dtype are upcast to fp64 exactly.

@@ -112,3 +112,49 @@ def test_finite_differences_catch_mutant(name):
     grads = _grads(x, arrs, dO, dhT, module=mod)
     with pytest.raises(AssertionError):
         _fd_check(x, arrs, dO, dhT, grads, _all_elements(arrs))
+
+
+# --- the chunkwise backward against the token backward ------------------------------
+
+def _rel(a, b):
+    return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
+
+
+@pytest.mark.parametrize("T,chunk,decay,lengths", [(23, 8, "mild", None), (150, 64, "strong", None),
+                                                    (None, 16, "strong", [40, 0, 1, 33])])
+def test_chunk_backward_equals_token_backward(T, chunk, decay, lengths):
+    from oracle.chunk_backward import backward as chunk_backward
+    if lengths is not None:
+        T = sum(lengths)
+    x, arrs, dO, dhT = _case(1 if lengths else 2, T, 2, 6, 5, seed=84, decay=decay, lengths=lengths)
+    ref = _grads(x, arrs, dO, dhT)
+    got = chunk_backward(*(arrs[n] for n in NAMES), x.scale, dO, dhT=dhT, h0=arrs["h0"],
+                         cu_seqlens=x.cu_seqlens, chunk=chunk)
+    for name in NAMES + ("h0",):
+        assert _rel(got[name], ref[name]) <= 1e-9, (name, _rel(got[name], ref[name]))
+
+
+CHUNK_MUTANTS = {
+    "start-state gradient misses the W S0 path": (
+        "dS0 = scale * Qt.T @ dO + np.exp(gn)[:, None] * dS1 - W.T @ dU",
+        "dS0 = scale * Qt.T @ dO + np.exp(gn)[:, None] * dS1"),
+    "pairwise decay not differentiated": ("dg = M.sum(axis=1) - M.sum(axis=0)", "dg = np.zeros_like(g)"),
+    "query mask without the diagonal": ("dP = np.where(lower_incl, scale * dO @ U.T, 0.0)",
+                                        "dP = np.where(lower_strict, scale * dO @ U.T, 0.0)"),
+    "inverse's gradient not transposed": ("dA = np.where(lower_strict, -T.T @ dT @ T.T, 0.0)",
+                                          "dA = np.where(lower_strict, -T @ dT @ T, 0.0)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CHUNK_MUTANTS))
+def test_token_backward_catches_chunk_mutant(name):
+    from oracle import chunk_backward as cb_mod
+    old, new = CHUNK_MUTANTS[name]
+    src = open(cb_mod.__file__).read()
+    assert src.count(old) == 1, old
+    mod = types.ModuleType("chunk_backward_mutant")
+    exec(compile(src.replace(old, new), "chunk_backward_mutant", "exec"), mod.__dict__)
+    x, arrs, dO, dhT = _case(2, 23, 2, 6, 5, seed=84)
+    ref = _grads(x, arrs, dO, dhT)
+    got = mod.backward(*(arrs[n] for n in NAMES), x.scale, dO, dhT=dhT, h0=arrs["h0"], chunk=8)
+    assert max(_rel(got[n], ref[n]) for n in NAMES + ("h0",)) > 1e-6
