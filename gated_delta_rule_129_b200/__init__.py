@@ -39,7 +39,8 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_NULL", 2: "GDN2_ERR_SHAPE", 3: "GDN2_ERR_DT
 
 EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_fwd_noalloc",
             "gdn2_chunk_prep", "gdn2_chunk_walk", "gdn2_chunk_plan", "gdn2_chunk_fused",
-            "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version")
+            "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version", "gdn2_backward_workspace_size",
+            "gdn2_chunk_bwd")
 
 
 class GDN2Error(RuntimeError):
@@ -103,6 +104,10 @@ def load_library():
         lib.gdn2_chunk_fused.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_fused.restype = i
         lib.gdn2_recurrent_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp]
+        lib.gdn2_backward_workspace_size.argtypes = [dp]
+        lib.gdn2_backward_workspace_size.restype = sz
+        lib.gdn2_chunk_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.gdn2_chunk_bwd.restype = i
         lib.gdn2_recurrent_step.restype = i
         lib.gdn2_status_string.argtypes = [i]
         lib.gdn2_status_string.restype = ctypes.c_char_p
@@ -310,6 +315,40 @@ def chunk_walk(workspace, shape, io_dtype, scale, h0=None, cu_seqlens=None, *, o
                                         _ptr(out), _ptr(hT), _ptr(chunk_states), _stream(stream))
     _check(st, "gdn2_chunk_walk")
     return out, hT
+
+
+def backward_workspace_size(B, T, H, dk, dv, io=GDN2_IO_BF16, num_seqs=0) -> int:
+    d = make_desc(B, T, H, dk, dv, io, num_seqs)
+    return int(load_library().gdn2_backward_workspace_size(ctypes.byref(d)))
+
+
+def chunk_bwd(q, k, v, log_alpha, b, w, scale, dO, h0=None, dhT=None, cu_seqlens=None, *, workspace=None,
+              stream=None):
+    """``gdn2_chunk_bwd``: gradients of :func:`chunk_fwd`'s ``(out, hT)``
+    contracted with ``dO`` (``[B, T, H, dv]``, the dtype of ``q``) and ``dhT``
+    (``[N, H, dk, dv]`` fp32 or None).  Returns a dict of fp32 tensors
+    ``q, k, v, log_alpha, b, w`` (input shapes) and ``h0`` ``[N, H, dk, dv]``."""
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    io = _io_of(q.dtype)
+    N = ns if cu_seqlens is not None else B
+    _need_contig(q, k, v, log_alpha, b, w, h0, cu_seqlens, dO, dhT)
+    if workspace is None:
+        nbytes = backward_workspace_size(B, T, H, dk, dv, io, ns)
+        if nbytes == 0:
+            raise GDN2Error(2, "gdn2_backward_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {n: torch.empty(t.shape, **f32) for n, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha),
+                                                       ("b", b), ("w", w))}
+    g["h0"] = torch.empty((N, H, dk, dv), **f32)
+    d = make_desc(B, T, H, dk, dv, io, ns, workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                                       _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens), _ptr(dO), _ptr(dhT),
+                                       _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["log_alpha"]), _ptr(g["b"]),
+                                       _ptr(g["w"]), _ptr(g["h0"]), _stream(stream))
+    _check(st, "gdn2_chunk_bwd")
+    return g
 
 
 def recurrent_step(q, k, v, log_alpha, b, w, scale, state, *, out=None, stream=None):

@@ -14,6 +14,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "bwd_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "plan.cuh"
@@ -466,6 +467,64 @@ struct DecodeOp {
   }
 };
 
+// ------------------------------------------------------------- backward ----
+// Workspace of gdn2_chunk_bwd: the status word, then one fp32 state per
+// (checkpoint slot, head); a sequence's chunk m uses slot seq_begin / 64 + m + n,
+// so T_total / 64 + N + 1 slots cover every sequence without overlap.
+gdn2_status bwd_layout(const gdn2_desc* d, bool packed, size_t* total, size_t* off_ckpt) {
+  gdn2_status st = check_dims(d, packed);
+  if (st != GDN2_OK) return st;
+  const long long N = packed ? d->num_seqs : d->B;
+  const long long slots = (long long)d->B * d->T / kChunk + N + 1;
+  *off_ckpt = kAlign;
+  *total = kAlign + align_up((size_t)slots * d->H * d->dk * d->dv * sizeof(float));
+  return GDN2_OK;
+}
+
+template <int DK, int DV, typename IO, typename FT>
+struct BwdOp {
+  static gdn2_status run(const gdn2_desc* d, int N, const void* q, const void* k, const void* v, const float* la,
+                         const float* b, const float* w, float scale, const float* h0, const int32_t* cu,
+                         const void* dO, const float* dhT, float* dq, float* dk, float* dv, float* dla, float* db,
+                         float* dw, float* dh0, int* status, float* ckpt, cudaStream_t s) {
+    gdn2::BwdArgs<IO> a;
+    a.q = static_cast<const IO*>(q);
+    a.k = static_cast<const IO*>(k);
+    a.v = static_cast<const IO*>(v);
+    a.dO = static_cast<const IO*>(dO);
+    a.la = la;
+    a.b = b;
+    a.w = w;
+    a.h0 = h0;
+    a.dhT = dhT;
+    a.cu = cu;
+    a.N = N;
+    a.T = d->T;
+    a.T_total = d->B * d->T;
+    a.H = d->H;
+    a.scale = scale;
+    a.ckpt = ckpt;
+    a.dq = dq;
+    a.dk = dk;
+    a.dla = dla;
+    a.db = db;
+    a.dv = dv;
+    a.dw = dw;
+    a.dh0 = dh0;
+    a.status = status;
+    a.seqlens_err = (int)GDN2_ERR_SEQLENS;
+    const long long blocks = (long long)N * d->H * (DV / gdn2::kBwdCols);
+    if (blocks == 0) return GDN2_OK;
+    if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+    constexpr size_t smem = (size_t)gdn2::bwd_smem_floats<DK, DV>() * sizeof(float);
+    auto kern = gdn2::bwd_simt_kernel<DK, DV, IO>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return GDN2_ERR_CUDA;
+    kern<<<(unsigned)blocks, DK, smem, s>>>(a);
+    return launch_status();
+  }
+};
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
@@ -630,6 +689,52 @@ const char* gdn2_status_string(gdn2_status s) {
 }
 
 int gdn2_version(void) { return 100; }
+
+size_t gdn2_backward_workspace_size(const gdn2_desc* desc) {
+  if (!desc) return 0;
+  size_t total = 0, off = 0;
+  if (bwd_layout(desc, desc->num_seqs > 0, &total, &off) != GDN2_OK) return 0;
+  return total;
+}
+
+gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* b, const float* w, float scale, const float* h0,
+                           const int32_t* cu_seqlens, const void* dO, const float* dhT, float* dq, float* dk,
+                           float* dv, float* dlog_alpha, float* db, float* dw, float* dh0, cudaStream_t stream) {
+  if (!desc) return GDN2_ERR_NULL;
+  const bool packed = cu_seqlens != nullptr;
+  size_t total = 0, off_ckpt = 0;
+  gdn2_status st = bwd_layout(desc, packed, &total, &off_ckpt);
+  if (st != GDN2_OK) return st;
+  if (!desc->workspace) return GDN2_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(desc->workspace) & (kAlign - 1)) != 0) return GDN2_ERR_ALIGN;
+  if (desc->workspace_bytes < total) return GDN2_ERR_WORKSPACE;
+  const long long tokens = (long long)desc->B * desc->T;
+  const int N = packed ? desc->num_seqs : desc->B;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, tokens)) != GDN2_OK) return st;
+  if (tokens > 0 && (!dO || !dq || !dk || !dv || !dlog_alpha || !db || !dw)) return GDN2_ERR_NULL;
+  if (!dh0) return GDN2_ERR_NULL;
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dlog_alpha) ||
+      !aligned16(db) || !aligned16(dw) || !aligned16(dh0) || (h0 && !aligned16(h0)) || (dhT && !aligned16(dhT)))
+    return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  int* status = at<int32_t>(desc->workspace, 0);
+  const size_t kbytes = (size_t)tokens * desc->H * desc->dk * sizeof(float);
+  const size_t vbytes = (size_t)tokens * desc->H * desc->dv * sizeof(float);
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), stream) != cudaSuccess) return GDN2_ERR_CUDA;
+  if (tokens > 0) {
+    // the key-side gradients are sums over every CTA of a head; the
+    // value-side ones are cleared too, so tokens outside every sequence of a
+    // malformed cu_seqlens read as zero
+    float* zero_k[4] = {dq, dk, dlog_alpha, db};
+    for (float* p : zero_k)
+      if (cudaMemsetAsync(p, 0, kbytes, stream) != cudaSuccess) return GDN2_ERR_CUDA;
+    if (cudaMemsetAsync(dv, 0, vbytes, stream) != cudaSuccess || cudaMemsetAsync(dw, 0, vbytes, stream) != cudaSuccess)
+      return GDN2_ERR_CUDA;
+  }
+  return dispatch<BwdOp>(desc, N, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens, dO, dhT, dq, dk, dv, dlog_alpha,
+                         db, dw, dh0, status, at<float>(desc->workspace, off_ckpt), stream);
+}
 
 }  // extern "C"
 

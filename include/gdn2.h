@@ -204,6 +204,35 @@ GDN2_API gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, cons
                              const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
                              cudaStream_t stream);
 
+/* Bytes of workspace gdn2_chunk_bwd needs for `desc` (0 if desc is invalid):
+ * a status word and one fp32 dk x dv state per head for every 64-token chunk
+ * start (T_total / 64 + sequences + 1 of them). */
+GDN2_API size_t gdn2_backward_workspace_size(const gdn2_desc* desc);
+
+/* Gradients of gdn2_chunk_fwd's outputs: given dO (the gradient of out) and
+ * dhT (of hT), the gradients of every input.  Reverse mode through the token
+ * recurrence (page "Gated DeltaNet-2：将擦除与写入分开", section
+ * "在两个维度上独立控制"; the pages train with the operator, section
+ * "词元路径与并行训练"), fp32 on the CUDA cores: per (sequence, head) the
+ * forward states at every 64-token chunk start are stored in the workspace,
+ * and each chunk's token states are recomputed from there on the way back.
+ * desc, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens: as for
+ *   gdn2_chunk_fwd (the same call's inputs); desc->workspace holds at least
+ *   gdn2_backward_workspace_size(desc) bytes, 256-byte aligned;
+ * dO  : [B, T, H, dv] io dtype;  dhT : [N, H, dk, dv] fp32, NULL = zero;
+ * dq, dk, dlog_alpha, db : [B, T, H, dk] fp32;  dv, dw : [B, T, H, dv] fp32;
+ * dh0 : [N, H, dk, dv] fp32 (the gradient of h0, also when h0 is NULL).
+ * Every gradient is written (the call clears them on `stream` first).
+ * Device pointers, 16-byte aligned, owned by the caller.  A malformed
+ * cu_seqlens sets GDN2_ERR_SEQLENS in the workspace's first int32 and leaves
+ * the gradients of the affected sequences zero; nothing outside the arrays is
+ * touched.  Asynchronous on `stream`. */
+GDN2_API gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* b, const float* w, float scale,
+                                    const float* h0, const int32_t* cu_seqlens, const void* dO, const float* dhT,
+                                    float* dq, float* dk, float* dv, float* dlog_alpha, float* db, float* dw,
+                                    float* dh0, cudaStream_t stream);
+
 /* One decode token for a batch of states, updated in place.
  * desc: B = batch, H, dk, dv, io (T, num_seqs and the workspace are ignored).
  *   q, k, log_alpha, b : [B, H, dk]   (q, k in io dtype; the rest fp32)
