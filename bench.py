@@ -318,6 +318,12 @@ def run_ours(args, rank, world, local):
 
     decode = measure_decode(dev, stream, flush) if rank == 0 else None
     others = measure_other_configs(dev, stream, flush, peaks()[0]) if (rank == 0 and not args.no_other_configs) else None
+    backward = None
+    if rank == 0 and not args.no_backward:
+        try:
+            backward = measure_backward(dev, stream, peaks()[0])
+        except Exception as exc:  # the forward's line must print whatever happens here
+            backward = {"error": str(exc)[:300]}
     if rank != 0:
         return
     hbm, tflops, src = peaks()
@@ -356,6 +362,8 @@ def run_ours(args, rank, world, local):
         line["decode_step"] = decode
     if others:
         line["other_configs"] = others
+    if backward:
+        line["backward_step"] = backward
     if world == 1 and not args.no_cpu_baseline:
         tps, cores, t_tok, dt = cpu_oracle_sample(x, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -394,6 +402,39 @@ def measure_decode(dev, stream, flush, reps=20):
     us = tot / reps * 1e3
     return {"workload": "decode B=256 H=16 dk=dv=128 (one token per state)", "us": us,
             "tokens_per_s": 256 / (us * 1e-6), "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9}
+
+
+def measure_backward(dev, stream, hbm, reps=3):
+    """gdn2_chunk_bwd (the gradients of every input, a CUDA-core baseline) on
+    the 16K x 1 workload with a random bf16 dO.  Its algorithmic traffic per
+    token-head: the inputs (768 + 1536 B), dO (256 B) and the six fp32
+    gradients (4 x 512 + 2 x 512 B), plus dh0."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    from workloads import config
+    x = config(WORKLOAD_ID)
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
+    q, k, v = (t(a, torch.bfloat16) for a in (x.q, x.k, x.v))
+    la, b, w = (t(a, torch.float32) for a in (x.log_alpha, x.b, x.w))
+    gen = torch.Generator(device=dev).manual_seed(5)
+    dO = torch.randn(v.shape, generator=gen, dtype=torch.float32, device=dev).to(torch.bfloat16)
+    ws = torch.empty(gdn2.backward_workspace_size(B, T, H, DK, DV, gdn2.GDN2_IO_BF16), dtype=torch.uint8, device=dev)
+    gdn2.chunk_bwd(q, k, v, la, b, w, x.scale, dO, workspace=ws, stream=stream)
+    tot = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gdn2.chunk_bwd(q, k, v, la, b, w, x.scale, dO, workspace=ws, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms = tot / reps
+    alg = TH * (768 + 1536 + 256 + 6 * 512) + B * H * DK * DV * 4
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"workload": "16Kx1 backward (gdn2_chunk_bwd, CUDA-core baseline), bf16 inputs, fp32 gradients",
+            "ms": ms, "tokens_per_s": B * T / (ms / 1e3), "alg_bytes": alg,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
 
 
 def measure_other_configs(dev, stream, flush, hbm, steps=10):
@@ -476,6 +517,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-configs", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--ncu-case", action="store_true",
                     help="run the small fused-kernel case for ncu captures and exit")
     args = ap.parse_args()
