@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -74,7 +75,8 @@ class ClockSampler:
 
     def __init__(self, device_index):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        fd, self.path = tempfile.mkstemp(prefix="gdn2_clocks_", suffix=".csv")
+        os.close(fd)
         try:
             import torch
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -86,7 +88,6 @@ class ClockSampler:
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(self.cmd, stdout=self.f, stderr=subprocess.DEVNULL)
             # the first sample is out before the timed region starts
@@ -123,6 +124,11 @@ class ClockSampler:
                     continue
         except OSError:
             return None
+        finally:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -250,46 +256,51 @@ def run_ours(args, rank, world, local):
     for _ in range(args.warmup):
         step()
         flush.zero_()
+    # The timed steps; after each one (outside its events, like the L2 flush)
+    # the fused launch alone is timed once, after its plan, so that the
+    # kernel's and the step's medians come from the same loop.
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier_sync(world)
     for i in range(args.steps):
         flush.zero_()
         starts[i].record(stream)
         step()
         ends[i].record(stream)
+        flush.zero_()
+        gdn2.chunk_plan((B, T, H, DK, DV), bf, ws, stream=stream)
+        k0[i].record(stream)
+        gdn2.chunk_fused(q, k, v, la, b, w, x.scale, ws, out=out, hT=hT, stream=stream)
+        k1[i].record(stream)
     barrier_sync(world)
     if sampler:
         sampler.__exit__(None, None, None)
-    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
-    ms = max_over_ranks(ms, world)
+    step_ms = [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)]
+    fused_ms = [a_.elapsed_time(b_) for a_, b_ in zip(k0, k1)]
+    ms_mean = sum(step_ms) / args.steps
+    ms = max_over_ranks(statistics.median(step_ms), world)
     # chunk_fwd here: plan, the fused prep + walk launch, and the two guards
     # after it (exact redo of steep-decay chunks; walk again if one occurred)
     launches_per_step = 4
 
-    # per-kernel durations: the fused launch alone (after its plan), and the
-    # two stages run back to back through their own entry points
-    kt = {"fused": [], "prep": [], "walk": []}
+    # the two stages run back to back through their own entry points
+    kt = {"prep": [], "walk": []}
     nk = max(3, min(args.steps, 50))
     for i in range(nk):
         flush.zero_()
-        gdn2.chunk_plan((B, T, H, DK, DV), bf, ws, stream=stream)
-        e0, e1, e2, e3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
-        e0.record(stream)
-        gdn2.chunk_fused(q, k, v, la, b, w, x.scale, ws, out=out, hT=hT, stream=stream)
-        e1.record(stream)
-        flush.zero_()
+        e2, e3, e4 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         e2.record(stream)
         gdn2.chunk_prep(q, k, v, la, b, w, workspace=ws, stream=stream)
         e3.record(stream)
-        e4 = torch.cuda.Event(enable_timing=True)
         gdn2.chunk_walk(ws, (B, T, H, DK, DV), bf, x.scale, out=out, hT=hT, stream=stream)
         e4.record(stream)
-        kt["fused"].append((e0, e1))
         kt["prep"].append((e2, e3))
         kt["walk"].append((e3, e4))
     torch.cuda.synchronize()
-    kern_ms = {kname: sum(a.elapsed_time(bb) for a, bb in ev) / len(ev) for kname, ev in kt.items()}
+    kern_ms = {kname: statistics.median(a.elapsed_time(bb) for a, bb in ev) for kname, ev in kt.items()}
+    kern_ms["fused"] = statistics.median(fused_ms)
 
     # end to end: pinned host inputs -> device -> chunk_fwd -> O, hT back to pinned host
     host = {n: getattr(x, n) for n in ("q", "k", "v", "log_alpha", "b", "w")}
@@ -337,7 +348,8 @@ def run_ours(args, rank, world, local):
     dom_gbs = dom_bytes / (kern_ms[dom] / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_mean": ms_mean, "higher_is_better": True,
+        "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "16Kx1 B=1 T=16384 H=16 dk=dv=128 bf16 I/O, fp32 gates (strong decay)",
                    "global_batch": world * B, "seq_len": T, "parallelism": f"replicas x{world}",
@@ -350,6 +362,8 @@ def run_ours(args, rank, world, local):
                           "t_meas_us": ms * 1e3, "frac": t_roof / (ms / 1e3),
                           "achieved_gbs": ALG_BYTES / (ms / 1e3) / 1e9},
         "kernels_ms": kern_ms,
+        "timing": "medians over the timed steps; the fused kernel alone is timed once after each timed step, "
+                  "in the same loop",
         "e2e": {"value": job_tokens_per_s(world, tokens, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ne},
         "gpu_launches": launches_per_step * args.steps,
@@ -439,15 +453,30 @@ def measure_backward(dev, stream, hbm, reps=3):
 
 def measure_other_configs(dev, stream, flush, hbm, steps=10):
     """gdn2_chunk_fwd on the other bf16 workloads (2K x 8, 4K x 4 with
-    b = w = beta, 32 packed sequences): tokens/s and the step roofline
-    fraction, same timing rules as the headline number."""
+    b = w = beta, 32 packed sequences) and on the gate ablations of the 16K x 1
+    inputs (erase range [0, 2], channel-mean erase or write gate): tokens/s
+    and the step roofline fraction, same timing rules as the headline number
+    (median of the timed steps)."""
     import torch
 
     import gated_delta_rule_129_b200 as gdn2
     from workloads import config
+    from workloads import make_inputs
     out_cfg = {}
-    for cid, variant in ((1, "a"), (3, "a"), (4, "a")):
-        x = config(cid, variant)
+    ablations = [
+        ("16Kx1 erase range [0,2] (b scaled by 2)", dict(erase_range=2.0)),
+        ("16Kx1 channel-mean erase gate", dict(mean_gate="erase")),
+        ("16Kx1 channel-mean write gate", dict(mean_gate="write")),
+    ]
+    cases = [lambda c=c, v_=v_: config(c, v_) for c, v_ in ((1, "a"), (3, "a"), (4, "a"))]
+    for name, kw in ablations:
+        def mk(name=name, kw=kw):
+            xi = make_inputs(1, 16384, 16, 128, 128, io="bf16", seed=2, decay="strong", **kw)
+            xi.name = name
+            return xi
+        cases.append(mk)
+    for make in cases:
+        x = make()
         t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
         bf, f32 = torch.bfloat16, torch.float32
         q, k, v = t(x.q, bf), t(x.k, bf), t(x.v, bf)
@@ -467,7 +496,7 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
                            stream=stream)
         for _ in range(3):
             run()
-        tot = 0.0
+        times = []
         for _ in range(steps):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -475,8 +504,8 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
             run()
             e1.record(stream)
             e1.synchronize()
-            tot += e0.elapsed_time(e1)
-        ms = tot / steps
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
         tokens = Bc * Tc
         alg = tokens * Hc * ALG_BYTES_PER_TH + nseq * Hc * DK * DV * 4 * (2 if h0 is not None else 1)
         out_cfg[x.name] = {"tokens_per_s": tokens / (ms / 1e3), "ms_per_step": ms,

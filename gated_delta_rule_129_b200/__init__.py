@@ -21,7 +21,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "noalloc_status", "chunk_walk_flagged", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
            "recurrent_step", "workspace_size",
            "workspace_layout", "status_string", "GDN2Error", "lib_path", "load_library"]
 
@@ -40,7 +40,7 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_NULL", 2: "GDN2_ERR_SHAPE", 3: "GDN2_ERR_DT
 EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_fwd_noalloc",
             "gdn2_chunk_prep", "gdn2_chunk_walk", "gdn2_chunk_plan", "gdn2_chunk_fused",
             "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version", "gdn2_backward_workspace_size",
-            "gdn2_chunk_bwd")
+            "gdn2_chunk_bwd", "gdn2_noalloc_status", "gdn2_chunk_walk_flagged")
 
 
 class GDN2Error(RuntimeError):
@@ -95,6 +95,10 @@ def load_library():
         lib.gdn2_chunk_fwd.restype = i
         lib.gdn2_chunk_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_fwd_noalloc.restype = i
+        lib.gdn2_noalloc_status.argtypes = [dp, vp, vp]
+        lib.gdn2_noalloc_status.restype = i
+        lib.gdn2_chunk_walk_flagged.argtypes = [dp, f, vp, vp, vp, vp, ctypes.c_ulonglong, vp]
+        lib.gdn2_chunk_walk_flagged.restype = i
         lib.gdn2_chunk_prep.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_prep.restype = i
         lib.gdn2_chunk_walk.argtypes = [dp, f, vp, vp, vp, vp, vp, vp]
@@ -280,6 +284,20 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, scale=None, h0=None, cu_seqlens=
     return out, hT
 
 
+def noalloc_status(q, v, cu_seqlens=None, *, stream=None):
+    """``gdn2_noalloc_status``: the device status word of the last
+    :func:`chunk_fwd_noalloc` call on inputs shaped like ``q``, ``v``
+    (``cu_seqlens`` for a packed call), as an int32 CUDA tensor of one element
+    filled on ``stream`` (0 = ok, 5 = malformed cu_seqlens, 8 = a bounded
+    device wait gave up)."""
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    out = torch.empty(4, dtype=torch.int32, device=q.device)
+    d = make_desc(B, T, H, dk, dv, _io_of(q.dtype), ns)
+    _check(load_library().gdn2_noalloc_status(ctypes.byref(d), _ptr(out), _stream(stream)), "gdn2_noalloc_status")
+    return out[:1]
+
+
 def chunk_prep(q, k, v, log_alpha, b, w, cu_seqlens=None, *, workspace=None, stream=None):
     """Stage 1 only.  Returns the workspace tensor holding the chunk factors."""
     B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
@@ -314,6 +332,29 @@ def chunk_walk(workspace, shape, io_dtype, scale, h0=None, cu_seqlens=None, *, o
     st = load_library().gdn2_chunk_walk(ctypes.byref(d), float(scale), _ptr(h0), _ptr(cu_seqlens),
                                         _ptr(out), _ptr(hT), _ptr(chunk_states), _stream(stream))
     _check(st, "gdn2_chunk_walk")
+    return out, hT
+
+
+def chunk_walk_flagged(workspace, shape, io_dtype, scale, h0=None, cu_seqlens=None, *, out=None, hT=None,
+                       wait_budget_ns=0, stream=None):
+    """``gdn2_chunk_walk_flagged``: :func:`chunk_walk` that takes each chunk
+    only once its ready flag in the workspace is raised, with every bounded
+    device wait limited to ``wait_budget_ns`` (0 = 2 s).  Returns ``(out, hT)``;
+    a wait that gave up shows in the workspace status word."""
+    torch = _torch()
+    B, T, H, dk, dv = shape
+    ns = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+    N = ns if cu_seqlens is not None else B
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=io_dtype, device=workspace.device)
+    if hT is None:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=workspace.device)
+    d = make_desc(B, T, H, dk, dv, _io_of(io_dtype), ns, workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_walk_flagged(ctypes.byref(d), float(scale), _ptr(h0), _ptr(cu_seqlens),
+                                                _ptr(out), _ptr(hT), ctypes.c_ulonglong(int(wait_budget_ns)),
+                                                _stream(stream))
+    _check(st, "gdn2_chunk_walk_flagged")
     return out, hT
 
 

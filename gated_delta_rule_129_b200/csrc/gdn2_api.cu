@@ -11,7 +11,6 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 #include <type_traits>
 
 #include "bwd_simt.cuh"
@@ -308,13 +307,19 @@ gdn2_status fill_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const
 template <int DV>
 gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, const float* h0,
                            const int32_t* cu, void* out, float* hT, float* chunk_states, cudaStream_t s,
-                           const int* gate = nullptr) {
+                           const int* gate = nullptr, bool flagged = false, unsigned long long wait_ns = 0) {
   using C = gdn2::WalkTcCfg<DV>;
   if (L.N == 0) return GDN2_OK;
   gdn2::WalkTcArgs a;
   gdn2_status st = fill_walk_tc<DV>(d, L, scale, h0, cu, out, hT, chunk_states, a);
   if (st != GDN2_OK) return st;
   a.gate = gate;
+  if (flagged) {
+    int* sync = at<int>(d->workspace, L.l.off_sync);
+    a.ready = sync + 2;
+    a.redo = sync + 1;
+  }
+  a.wait_ns = wait_ns;
   auto kern = gdn2::walk_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;
@@ -401,8 +406,26 @@ gdn2_status launch_fused_tc(const gdn2_desc* d, const Layout& L, const void* q, 
   auto kern = gdn2::fused_tc_kernel<DV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM) != cudaSuccess)
     return GDN2_ERR_CUDA;
-  kern<<<n_sm, F::THREADS, F::SMEM, s>>>(pa, wa, n_sm - n_walk);
-  return launch_status();
+  // The walk CTAs wait on flags the prep CTAs raise, so every CTA must be
+  // resident at once: a cooperative launch guarantees it or fails (fewer SMs
+  // available than the device reports, e.g. under MPS or in a green context),
+  // and then the caller runs the two stage kernels instead.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_sm);
+  cfg.blockDim = dim3(F::THREADS);
+  cfg.dynamicSmemBytes = F::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, pa, wa, n_sm - n_walk);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return GDN2_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? launch_status() : GDN2_ERR_CUDA;
 }
 
 template <int DV>
@@ -410,6 +433,11 @@ gdn2_status launch_fused_full(const gdn2_desc* d, const Layout& L, const void* q
                               const float* la, const float* b, const float* w, const int32_t* cu, float scale,
                               const float* h0, void* out, float* hT, cudaStream_t s) {
   gdn2_status st = launch_fused_tc<DV>(d, L, q, k, v, la, b, w, cu, scale, h0, out, hT, s);
+  if (st == GDN2_ERR_UNSUPPORTED) {
+    // not all CTAs could be resident at once: the two stage kernels
+    if ((st = launch_prep_t<128, DV, bf16, bf16>(d, L, q, k, v, la, b, w, cu, s)) != GDN2_OK) return st;
+    return launch_walk_tc<DV>(d, L, scale, h0, cu, out, hT, nullptr, s);
+  }
   if (st != GDN2_OK) return st;
   if ((st = launch_fixup<128, DV, bf16, bf16>(d, L, q, k, v, la, b, w, cu, s)) != GDN2_OK) return st;
   return launch_walk_tc<DV>(d, L, scale, h0, cu, out, hT, nullptr, s, at<int>(d->workspace, L.l.off_sync) + 1);
@@ -657,6 +685,24 @@ gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, const void* k
   return GDN2_ERR_UNSUPPORTED;
 }
 
+gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale, const float* h0,
+                                    const int32_t* cu_seqlens, void* out, float* hT,
+                                    unsigned long long wait_budget_ns, cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  if (!out && (long long)desc->B * desc->T > 0) return GDN2_ERR_NULL;
+  if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return GDN2_ERR_ALIGN;
+  if (L.l.factor_set != 1) return GDN2_ERR_UNSUPPORTED;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if (desc->dv == 128)
+    return launch_walk_tc<128>(desc, L, scale, h0, cu_seqlens, out, hT, nullptr, stream, nullptr, true,
+                               wait_budget_ns);
+  return launch_walk_tc<64>(desc, L, scale, h0, cu_seqlens, out, hT, nullptr, stream, nullptr, true,
+                            wait_budget_ns);
+}
+
 gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, const void* k, const void* v,
                                 const float* log_alpha, const float* b, const float* w, float scale,
                                 float* state, void* out, cudaStream_t stream) {
@@ -745,23 +791,14 @@ gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN2_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
-
-// Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// Device address of the scratch on the current device.  It is looked up on
+// every call (a host-side query once the module is loaded), so a module that
+// was reloaded at another address (after cudaDeviceReset, or under another
+// context) is never reached through a stale pointer.
 gdn2_status noalloc_scratch(void** addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDN2_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return GDN2_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN2_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
-  }
-  *addr = g_noalloc_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN2_ERR_CUDA;
+  *addr = p;
   return GDN2_OK;
 }
 }  // namespace
@@ -790,6 +827,29 @@ gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_desc* desc, const void* q, const v
   d.workspace = scratch;
   d.workspace_bytes = (size_t)GDN2_NOALLOC_SCRATCH_BYTES;
   return gdn2_chunk_fwd(&d, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens, out, hT, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+gdn2_status gdn2_noalloc_status(const gdn2_desc* desc, int32_t* status, cudaStream_t stream) {
+  if (!desc || !status) return GDN2_ERR_NULL;
+  if (!aligned16(status)) return GDN2_ERR_ALIGN;
+  gdn2_desc d = *desc;
+  d.workspace = nullptr;
+  d.workspace_bytes = 0;
+  Layout L;
+  gdn2_status st = make_layout(&d, d.num_seqs > 0, &L);
+  if (st != GDN2_OK) return st;
+  if (L.l.total_bytes > (size_t)GDN2_NOALLOC_SCRATCH_BYTES) return GDN2_ERR_WORKSPACE;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != GDN2_OK) return st;
+  if (cudaMemcpyAsync(status, static_cast<char*>(scratch) + L.l.off_status, sizeof(int32_t),
+                      cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  return GDN2_OK;
 }
 
 }  // extern "C"

@@ -66,7 +66,13 @@ struct WalkTcArgs {
   const int* ready;    // optional [max_chunks * H]: wait for 2 (written); 3 = handed back
   int* redo;           // set when a handed-back chunk ended the walk early
   const int* gate;     // optional: the kernel does nothing unless *gate != 0
+  unsigned long long wait_ns;  // limit of every bounded wait (0: the default, 2 s)
 };
+
+// The walk's wait limit: the host's choice, or 2 s.
+__device__ __forceinline__ uint64_t walk_budget(const WalkTcArgs& a) {
+  return a.wait_ns ? (uint64_t)a.wait_ns : 2000000000ull;
+}
 
 template <int DV>
 struct WalkTcCfg {
@@ -106,13 +112,14 @@ __device__ __forceinline__ void set_timeout(int* status, int* s_abort) {
 
 // Bounded wait that also ends when the CTA winds down (abort flag): true once
 // the phase has completed; a timeout is recorded in the status word.
-__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, int* status, int* s_abort) {
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, int* status, int* s_abort,
+                                      uint64_t budget_ns = 2000000000ull) {
   if (tc::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = tc::global_ns();
   for (;;) {
     if (tc::mbar_try_wait(bar, parity)) return true;
     if (*reinterpret_cast<volatile int*>(s_abort)) return false;
-    if (tc::global_ns() - t0 > 2000000000ull) {
+    if (tc::global_ns() - t0 > budget_ns) {
       set_timeout(status, s_abort);
       return false;
     }
@@ -132,7 +139,7 @@ __device__ __forceinline__ bool wait_chunk_ready(const WalkTcArgs& a, int t, int
       return false;
     }
     if (*reinterpret_cast<volatile int*>(s_abort)) return false;
-    if (tc::global_ns() - t0 > 2000000000ull) {
+    if (tc::global_ns() - t0 > walk_budget(a)) {
       set_timeout(a.status, s_abort);
       return false;
     }
@@ -160,6 +167,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
   uint64_t* fin = o_free + 2;                // every issued UMMA has finished
   uint32_t* tslot = reinterpret_cast<uint32_t*>(fin + 1);
   int* s_abort = reinterpret_cast<int*>(tslot + 1);
+  const uint64_t wb = walk_budget(a);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
@@ -233,7 +241,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
                                             C::G_BYTES)[row];
     };
     if (nch > 0) {
-      if (wwait(&fullB[0], 0, a.status, s_abort)) store_state(0, colscale_of(0));
+      if (wwait(&fullB[0], 0, a.status, s_abort, wb)) store_state(0, colscale_of(0));
     }
 
     for (int j = 0; j < nch; ++j) {
@@ -246,7 +254,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
 #pragma unroll
         for (int i = 0; i < NSL; i += 4) *reinterpret_cast<float4*>(cs + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
       }
-      if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort)) break;
+      if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort, wb)) break;
       // Nc row (64 bf16, SW128) and gamma before the product is ready
       const float gam = reinterpret_cast<const float*>(stB + C::NC_BYTES + C::OP_BYTES)[row];
       uint32_t ncw[NSL / 2];
@@ -255,7 +263,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
         const uint4 t = *reinterpret_cast<const uint4*>(stB + row * 128 + ((u ^ (row & 7)) << 4));
         ncw[4 * u] = t.x; ncw[4 * u + 1] = t.y; ncw[4 * u + 2] = t.z; ncw[4 * u + 3] = t.w;
       }
-      if (!wwait(s_done, j & 1, a.status, s_abort)) break;
+      if (!wwait(s_done, j & 1, a.status, s_abort, wb)) break;
       tc::tc_fence_after();
       // S <- gamma * S - Mp S + Nc
       {
@@ -282,7 +290,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       float cs_next = 1.f;
       if (j + 1 < nch) {
         const int sn = (j + 1) % C::STAGES_B;
-        if (!wwait(&fullB[sn], ((j + 1) / C::STAGES_B) & 1, a.status, s_abort)) break;
+        if (!wwait(&fullB[sn], ((j + 1) / C::STAGES_B) & 1, a.status, s_abort, wb)) break;
         cs_next = colscale_of(j + 1);
       }
       store_state((j + 1) & 1, cs_next);
@@ -302,7 +310,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int sb = j % C::STAGES_B;
       const uint8_t* stB = ringB + sb * C::B_STRIDE;
-      if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort) || !wwait(o_done, j & 1, a.status, s_abort))
+      if (!wwait(&fullB[sb], (j / C::STAGES_B) & 1, a.status, s_abort, wb) || !wwait(o_done, j & 1, a.status, s_abort, wb))
         break;
       tc::tc_fence_after();
       uint32_t d0[32], d1[32];
@@ -342,7 +350,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     const uint64_t sb_d0 = tc::sdesc(tc::smem_u32(sS), C::S_LBO, 128, tc::kLayoutNone);
     for (int j = 0; j < nch; ++j) {
       const int st = j % C::STAGES_A;
-      if (!wwait(&fullA[st], (j / C::STAGES_A) & 1, a.status, s_abort) || !wwait(s_ready, j & 1, a.status, s_abort))
+      if (!wwait(&fullA[st], (j / C::STAGES_A) & 1, a.status, s_abort, wb) || !wwait(s_ready, j & 1, a.status, s_abort, wb))
         break;
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       tc::tc_fence_after();
@@ -358,7 +366,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       tc::umma_commit(s_done);
       // the output warps have read D_O(j-1): keeps every o_done waiter within
       // one phase (and frees the D_O buffer D_O(j+1) will use)
-      if (j >= 1 && !wwait(&o_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, s_abort)) break;
+      if (j >= 1 && !wwait(&o_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, s_abort, wb)) break;
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s)
         tc::umma_f16(tbase + (uint32_t)NSL * (1u + (j & 1)),
@@ -395,7 +403,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
           tc::tma_prefetch_2d(&a.tm_cs, 0, tp);
         }
       }
-      if (j >= C::STAGES_A && !wwait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1, a.status, s_abort)) break;
+      if (j >= C::STAGES_A && !wwait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1, a.status, s_abort, wb)) break;
       if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringA + st * C::A_BYTES;
       tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
@@ -420,7 +428,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     for (int j = 0; j < nch; ++j) {
       if (*reinterpret_cast<volatile int*>(s_abort)) break;
       const int c = c_begin + j, st = j % C::STAGES_B;
-      if (j >= C::STAGES_B && !wwait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1, a.status, s_abort)) break;
+      if (j >= C::STAGES_B && !wwait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1, a.status, s_abort, wb)) break;
       if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringB + st * C::B_STRIDE;
       tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);

@@ -165,8 +165,11 @@ GDN2_API gdn2_status gdn2_workspace_layout(const gdn2_desc* desc, gdn2_ws_layout
  * Asynchronous on `stream`.  For bf16 I/O with dk = 128, when the walk needs
  * at most (SM count - 32) CTAs (sequences x H x dv/64), the prep and the walk
  * run in one launch and the walk takes each chunk's factors as soon as they
- * are written (gdn2_chunk_fused); otherwise it runs gdn2_chunk_prep then
- * gdn2_chunk_walk.  Both orders compute the same values. */
+ * are written (gdn2_chunk_fused, a cooperative launch: all its CTAs are
+ * resident at once, or it is not launched); otherwise, or when the
+ * cooperative launch is refused (fewer SMs available than the device has),
+ * it runs gdn2_chunk_prep then gdn2_chunk_walk.  Both orders compute the same
+ * values. */
 GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
                            const float* log_alpha, const float* b, const float* w, float scale,
                            const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
@@ -198,11 +201,24 @@ GDN2_API gdn2_status gdn2_chunk_plan(const gdn2_desc* desc, const int32_t* cu_se
  * for the tensor-core prep; call gdn2_chunk_plan first.  A call then gives the
  * full result unless such a chunk exists, which gdn2_chunk_fwd handles.
  * Returns GDN2_ERR_UNSUPPORTED when the problem does not take the fused path
- * (not bf16 with dk = 128, or the walk needs too many CTAs). */
+ * (not bf16 with dk = 128, or the walk needs too many CTAs) or when the
+ * cooperative launch cannot make every CTA resident at once. */
 GDN2_API gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, const void* k, const void* v,
                              const float* log_alpha, const float* b, const float* w, float scale,
                              const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
                              cudaStream_t stream);
+
+/* gdn2_chunk_walk with the walk taking each chunk only once its ready flag in
+ * the workspace (off_sync, the flags gdn2_chunk_fused's prep raises) reads 2,
+ * and with every bounded device-side wait limited to wait_budget_ns (0 = the
+ * default of 2 s).  For tests and diagnostics of the fused path's hand-off: a
+ * walk whose flags nobody raises ends after the limit with
+ * GDN2_ERR_DEVICE_TIMEOUT in the workspace status word and its outputs
+ * unspecified, instead of hanging.  Affine factor set only (bf16 I/O with
+ * dk = 128); GDN2_ERR_UNSUPPORTED otherwise.  Asynchronous on `stream`. */
+GDN2_API gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale, const float* h0,
+                                             const int32_t* cu_seqlens, void* out, float* hT,
+                                             unsigned long long wait_budget_ns, cudaStream_t stream);
 
 /* Bytes of workspace gdn2_chunk_bwd needs for `desc` (0 if desc is invalid):
  * a status word and one fp32 dk x dv state per head for every 64-token chunk
@@ -265,18 +281,32 @@ GDN2_API gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, c
  *  - Limit: if gdn2_workspace_size(desc) exceeds GDN2_NOALLOC_SCRATCH_BYTES
  *    the call returns GDN2_ERR_WORKSPACE and launches nothing; use
  *    gdn2_chunk_fwd with your own workspace for such sizes.
- *  - Set-up: the first call on each device looks up the array's device
- *    address (cudaGetSymbolAddress, with that device current).  Make that
- *    first call outside any stream capture; later calls make no such lookup.
+ *  - Set-up: every call looks up the array's device address on the current
+ *    device (cudaGetSymbolAddress, a host-side query).  The first call on a
+ *    device may load the library's device code there, so make that first
+ *    call outside any stream capture.
  *  - Sharing: all calls use the same array and it keeps the last call's
  *    contents (nothing in it needs to start at zero).  Calls whose work
  *    overlaps on the GPU (other streams, other host threads) race on it:
  *    order them on one stream or use gdn2_chunk_fwd.
+ *  - Device-side errors (a malformed cu_seqlens, a bounded wait that gave
+ *    up) land in a status word inside the array, as they do in a workspace;
+ *    gdn2_noalloc_status copies it out.
  * It calls no cudaMalloc, cudaFree or allocating library routine. */
 GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_desc* desc, const void* q, const void* k, const void* v,
                                             const float* log_alpha, const float* b, const float* w, float scale,
                                             const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
                                             cudaStream_t stream);
+
+/* The status word the last gdn2_chunk_fwd_noalloc call for the same `desc`
+ * left in the library's scratch (GDN2_OK, or an error found on the device:
+ * GDN2_ERR_SEQLENS, GDN2_ERR_DEVICE_TIMEOUT), copied into the caller's
+ * device int32 *status (16-byte aligned) on `stream`, so it is read after that
+ * call's work when both are on one stream.  desc must describe the same
+ * problem (num_seqs > 0 for a packed call); its workspace fields are ignored.
+ * Returns GDN2_ERR_WORKSPACE for problems the no-alloc call rejects.  It
+ * allocates nothing. */
+GDN2_API gdn2_status gdn2_noalloc_status(const gdn2_desc* desc, int32_t* status, cudaStream_t stream);
 
 /* Static description of a status code. */
 GDN2_API const char* gdn2_status_string(gdn2_status status);
