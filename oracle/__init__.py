@@ -25,6 +25,9 @@ Contents
 * :mod:`oracle.chunk_backward` -- the same gradients through the 64-token chunk
   form (the algebra a backward over chunks evaluates), checked against
   :mod:`oracle.backward`.
+* :mod:`oracle.state_map` -- the affine state map (Phi, Psi) of a token range
+  and the composition of consecutive maps (the two-level chunk scan and the
+  state passing between ranges of one sequence), fp64 numpy.
 
 Arrays use the token-major layout ``[B, T, H, D]`` (or ``[1, T_total, H, D]``
 with ``cu_seqlens``).  Inputs of any float dtype are upcast to fp64 exactly.
