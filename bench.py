@@ -456,7 +456,8 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
     b = w = beta, 32 packed sequences) and on the gate ablations of the 16K x 1
     inputs (erase range [0, 2], channel-mean erase or write gate): tokens/s
     and the step roofline fraction, same timing rules as the headline number
-    (median of the timed steps)."""
+    (median of the timed steps); and the 16K x 1 workload through the two-level
+    chunk scan (gdn2_chunk_fwd_segmented)."""
     import torch
 
     import gated_delta_rule_129_b200 as gdn2
@@ -468,14 +469,20 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
         ("16Kx1 channel-mean erase gate", dict(mean_gate="erase")),
         ("16Kx1 channel-mean write gate", dict(mean_gate="write")),
     ]
-    cases = [lambda c=c, v_=v_: config(c, v_) for c, v_ in ((1, "a"), (3, "a"), (4, "a"))]
+    cases = [(lambda c=c, v_=v_: config(c, v_), False) for c, v_ in ((1, "a"), (3, "a"), (4, "a"))]
     for name, kw in ablations:
         def mk(name=name, kw=kw):
             xi = make_inputs(1, 16384, 16, 128, 128, io="bf16", seed=2, decay="strong", **kw)
             xi.name = name
             return xi
-        cases.append(mk)
-    for make in cases:
+        cases.append((mk, False))
+
+    def mk_seg():
+        xi = config(WORKLOAD_ID)
+        xi.name = "16Kx1 through the two-level chunk scan (gdn2_chunk_fwd_segmented, 64-chunk segments)"
+        return xi
+    cases.append((mk_seg, True))
+    for make, segmented in cases:
         x = make()
         t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
         bf, f32 = torch.bfloat16, torch.float32
@@ -491,9 +498,17 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
         o = torch.empty_like(v)
         hT = torch.empty((nseq, Hc, DK, DV), dtype=f32, device=dev)
 
+        if segmented:
+            ws = torch.empty(gdn2.segmented_workspace_size(Bc, Tc, Hc, DK, DV, gdn2.GDN2_IO_BF16, ns), dtype=torch.uint8,
+                             device=dev)
+
         def run():
-            gdn2.chunk_fwd(q, k, v, la, b, w, x.scale, h0=h0, cu_seqlens=cu, out=o, hT=hT, workspace=ws,
-                           stream=stream)
+            if segmented:
+                gdn2.chunk_fwd_segmented(q, k, v, la, b, w, x.scale, h0=h0, cu_seqlens=cu, out=o, hT=hT,
+                                         workspace=ws, stream=stream)
+            else:
+                gdn2.chunk_fwd(q, k, v, la, b, w, x.scale, h0=h0, cu_seqlens=cu, out=o, hT=hT, workspace=ws,
+                               stream=stream)
         for _ in range(3):
             run()
         times = []

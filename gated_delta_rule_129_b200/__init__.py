@@ -21,7 +21,8 @@ import ctypes
 import os
 import threading
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "noalloc_status", "chunk_walk_flagged", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "noalloc_status", "chunk_walk_flagged", "chunk_fwd_segmented",
+           "segmented_workspace_size", "state_map", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
            "recurrent_step", "workspace_size",
            "workspace_layout", "status_string", "GDN2Error", "lib_path", "load_library"]
 
@@ -40,7 +41,8 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_NULL", 2: "GDN2_ERR_SHAPE", 3: "GDN2_ERR_DT
 EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "gdn2_chunk_fwd_noalloc",
             "gdn2_chunk_prep", "gdn2_chunk_walk", "gdn2_chunk_plan", "gdn2_chunk_fused",
             "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version", "gdn2_backward_workspace_size",
-            "gdn2_chunk_bwd", "gdn2_noalloc_status", "gdn2_chunk_walk_flagged")
+            "gdn2_chunk_bwd", "gdn2_noalloc_status", "gdn2_chunk_walk_flagged",
+            "gdn2_segmented_workspace_size", "gdn2_chunk_fwd_segmented", "gdn2_state_map")
 
 
 class GDN2Error(RuntimeError):
@@ -99,6 +101,12 @@ def load_library():
         lib.gdn2_noalloc_status.restype = i
         lib.gdn2_chunk_walk_flagged.argtypes = [dp, f, vp, vp, vp, vp, ctypes.c_ulonglong, vp]
         lib.gdn2_chunk_walk_flagged.restype = i
+        lib.gdn2_segmented_workspace_size.argtypes = [dp, i]
+        lib.gdn2_segmented_workspace_size.restype = sz
+        lib.gdn2_chunk_fwd_segmented.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, vp, i, vp]
+        lib.gdn2_chunk_fwd_segmented.restype = i
+        lib.gdn2_state_map.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.gdn2_state_map.restype = i
         lib.gdn2_chunk_prep.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_prep.restype = i
         lib.gdn2_chunk_walk.argtypes = [dp, f, vp, vp, vp, vp, vp, vp]
@@ -356,6 +364,61 @@ def chunk_walk_flagged(workspace, shape, io_dtype, scale, h0=None, cu_seqlens=No
                                                 _stream(stream))
     _check(st, "gdn2_chunk_walk_flagged")
     return out, hT
+
+
+def segmented_workspace_size(B, T, H, dk, dv, io=GDN2_IO_BF16, num_seqs=0, segment_chunks=0) -> int:
+    d = make_desc(B, T, H, dk, dv, io, num_seqs)
+    return int(load_library().gdn2_segmented_workspace_size(ctypes.byref(d), int(segment_chunks)))
+
+
+def chunk_fwd_segmented(q, k, v, log_alpha, b, w, scale=None, h0=None, cu_seqlens=None, *, segment_chunks=0,
+                        out=None, hT=None, workspace=None, output_final_state=True, stream=None):
+    """``gdn2_chunk_fwd_segmented``: :func:`chunk_fwd` through the two-level
+    chunk scan, each sequence split into segments of ``segment_chunks``
+    64-token chunks (0 = the library's choice).  Returns ``(out, hT)``."""
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    io = _io_of(q.dtype)
+    N = ns if cu_seqlens is not None else B
+    if scale is None:
+        scale = dk ** -0.5
+    _need_contig(q, k, v, log_alpha, b, w, h0, cu_seqlens)
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = segmented_workspace_size(B, T, H, dk, dv, io, ns, segment_chunks)
+        if nbytes == 0:
+            raise GDN2Error(9, "gdn2_segmented_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    d = make_desc(B, T, H, dk, dv, io, ns, workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_chunk_fwd_segmented(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                                 _ptr(b), _ptr(w), float(scale), _ptr(h0), _ptr(cu_seqlens),
+                                                 _ptr(out), _ptr(hT), int(segment_chunks), _stream(stream))
+    _check(st, "gdn2_chunk_fwd_segmented")
+    return out, hT
+
+
+def state_map(q, k, v, log_alpha, b, w, cu_seqlens=None, *, phi=None, psi=None, workspace=None, stream=None):
+    """``gdn2_state_map``: the affine map of every sequence, ``(phi [N, H, dk,
+    dk], psi [N, H, dk, dv])`` fp32, with final state = phi @ S_start + psi."""
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q, v, cu_seqlens)
+    io = _io_of(q.dtype)
+    N = ns if cu_seqlens is not None else B
+    _need_contig(q, k, v, log_alpha, b, w, cu_seqlens)
+    if phi is None:
+        phi = torch.empty((N, H, dk, dk), dtype=torch.float32, device=q.device)
+    if psi is None:
+        psi = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _alloc_workspace((B, T, H, dk, dv, io, ns), q.device)
+    d = make_desc(B, T, H, dk, dv, io, ns, workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    st = load_library().gdn2_state_map(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                                       _ptr(w), _ptr(cu_seqlens), _ptr(phi), _ptr(psi), _stream(stream))
+    _check(st, "gdn2_state_map")
+    return phi, psi
 
 
 def backward_workspace_size(B, T, H, dk, dv, io=GDN2_IO_BF16, num_seqs=0) -> int:

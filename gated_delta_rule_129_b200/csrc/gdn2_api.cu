@@ -20,6 +20,7 @@
 #include "prep_simt.cuh"
 #include "prep_tc.cuh"
 #include "fused_tc.cuh"
+#include "segscan.cuh"
 #include "tmap.cuh"
 #include "walk_simt.cuh"
 #include "walk_tc.cuh"
@@ -329,6 +330,30 @@ gdn2_status launch_walk_tc(const gdn2_desc* d, const Layout& L, float scale, con
   return launch_status();
 }
 
+// The walk over other ranges than the call's sequences (the segments of the
+// two-level scan), in map mode (MAP: [Phi | Psi] from [I | 0]) or with
+// outputs from per-range start states.
+template <int DV, bool MAP>
+gdn2_status launch_walk_ranges(const gdn2_desc* d, const Layout& L, float scale, const gdn2::SeqMap& ranges,
+                               const float* h0, void* out, float* phi, float* psi, cudaStream_t s) {
+  using C = gdn2::WalkTcCfg<DV>;
+  if (ranges.N == 0) return GDN2_OK;
+  gdn2::WalkTcArgs a;
+  gdn2_status st = fill_walk_tc<DV>(d, L, scale, h0, nullptr, out, nullptr, nullptr, a);
+  if (st != GDN2_OK) return st;
+  a.map = ranges;
+  a.phi = phi;
+  a.psi = psi;
+  auto kern = gdn2::walk_tc_kernel<DV, MAP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    return GDN2_ERR_CUDA;
+  const long long slices = MAP ? (128 + DV) / C::NSL : C::SLICES;
+  const long long blocks = (long long)ranges.N * d->H * slices;
+  if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+  kern<<<(unsigned)blocks, C::THREADS, C::SMEM, s>>>(a);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------- walk ----
 template <int DK, int DV, typename IO, typename FT>
 gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, const float* h0,
@@ -553,6 +578,72 @@ struct BwdOp {
   }
 };
 
+// ------------------------------------------------- two-level chunk scan ----
+// Extra workspace of gdn2_chunk_fwd_segmented, after the usual layout: the
+// virtual segments, their maps (Phi, Psi, fp32) and start states (fp32).
+struct SegLayout {
+  int L = 0, ns_max = 0;
+  size_t off_seg_cu = 0, off_seg_chunk = 0, off_seq_seg = 0, off_phi = 0, off_psi = 0, off_seg_h0 = 0, total = 0;
+};
+
+gdn2_status seg_layout(const gdn2_desc* d, const Layout& L, int segment_chunks, SegLayout* g) {
+  if (segment_chunks < 0) return GDN2_ERR_SHAPE;
+  const long long tokens = (long long)d->B * d->T;
+  // chunks per sequence (on average, for a packed row)
+  const long long nch = L.N > 0 ? (tokens / L.N + kChunk - 1) / kChunk : 0;
+  const long long Lc = segment_chunks > 0 ? segment_chunks : std::max(8ll, (nch + 3) / 4);
+  const bool packed = d->num_seqs > 0;
+  const long long ns = packed ? L.l.max_chunks / Lc + L.N
+                              : (long long)d->B * ((((long long)d->T + kChunk - 1) / kChunk + Lc - 1) / Lc);
+  if (ns > INT32_MAX / 4 || Lc > INT32_MAX / 4) return GDN2_ERR_SHAPE;
+  g->L = (int)Lc;
+  g->ns_max = (int)ns;
+  size_t off = align_up(L.l.total_bytes);
+  g->off_seg_cu = off;    off = align_up(off + (size_t)(ns + 1) * sizeof(int32_t));
+  g->off_seg_chunk = off; off = align_up(off + (size_t)(ns + 1) * sizeof(int32_t));
+  g->off_seq_seg = off;   off = align_up(off + (size_t)(L.N + 1) * sizeof(int32_t));
+  g->off_phi = off;       off = align_up(off + (size_t)ns * d->H * d->dk * d->dk * sizeof(float));
+  g->off_psi = off;       off = align_up(off + (size_t)ns * d->H * d->dk * d->dv * sizeof(float));
+  g->off_seg_h0 = off;    off = align_up(off + (size_t)ns * d->H * d->dk * d->dv * sizeof(float));
+  g->total = off;
+  return GDN2_OK;
+}
+
+template <int DV>
+gdn2_status launch_segmented(const gdn2_desc* d, const Layout& L, const SegLayout& g, const void* q, const void* k,
+                             const void* v, const float* la, const float* b, const float* w, const int32_t* cu,
+                             float scale, const float* h0, void* out, float* hT, cudaStream_t s) {
+  gdn2_status st;
+  if ((st = launch_prep_t<128, DV, bf16, bf16>(d, L, q, k, v, la, b, w, cu, s)) != GDN2_OK) return st;
+  int32_t* seg_cu = at<int32_t>(d->workspace, g.off_seg_cu);
+  int32_t* seg_chunk = at<int32_t>(d->workspace, g.off_seg_chunk);
+  int32_t* seq_seg = at<int32_t>(d->workspace, g.off_seq_seg);
+  float* phi = at<float>(d->workspace, g.off_phi);
+  float* psi = at<float>(d->workspace, g.off_psi);
+  float* seg_h0 = at<float>(d->workspace, g.off_seg_h0);
+  gdn2::segplan_kernel<<<1, gdn2::kSegPlanThreads, 0, s>>>(cu, L.N, d->T, d->B * d->T,
+                                                           at<const int32_t>(d->workspace, L.l.off_chunk_offsets),
+                                                           g.L, g.ns_max, seg_cu, seg_chunk, seq_seg);
+  if ((st = launch_status()) != GDN2_OK) return st;
+  gdn2::SeqMap segs;
+  segs.cu = seg_cu;
+  segs.chunk_off = seg_chunk;
+  segs.N = g.ns_max;
+  segs.T = d->T;
+  // 1. every segment's affine map
+  if ((st = launch_walk_ranges<DV, true>(d, L, scale, segs, nullptr, nullptr, phi, psi, s)) != GDN2_OK) return st;
+  // 2. the scan of the maps: start states of the segments, final states
+  const long long blocks = (long long)L.N * d->H * (DV / gdn2::kScanCols);
+  if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+  if (blocks > 0) {
+    gdn2::segscan_kernel<128, DV><<<(unsigned)blocks, gdn2::kScanThreads, 0, s>>>(phi, psi, seq_seg, d->H, h0,
+                                                                                  seg_h0, hT);
+    if ((st = launch_status()) != GDN2_OK) return st;
+  }
+  // 3. the segments again, with outputs, from their start states
+  return launch_walk_ranges<DV, false>(d, L, scale, segs, seg_h0, out, nullptr, nullptr, s);
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
@@ -683,6 +774,63 @@ gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, const void* k
       return launch_fused_tc<64>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
   }
   return GDN2_ERR_UNSUPPORTED;
+}
+
+size_t gdn2_segmented_workspace_size(const gdn2_desc* desc, int segment_chunks) {
+  if (!desc) return 0;
+  Layout L;
+  if (make_layout(desc, desc->num_seqs > 0, &L) != GDN2_OK || L.l.factor_set != 1) return 0;
+  SegLayout g;
+  if (seg_layout(desc, L, segment_chunks, &g) != GDN2_OK) return 0;
+  return g.total;
+}
+
+gdn2_status gdn2_chunk_fwd_segmented(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                     const float* log_alpha, const float* b, const float* w, float scale,
+                                     const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                                     int segment_chunks, cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if (L.l.factor_set != 1) return GDN2_ERR_UNSUPPORTED;
+  SegLayout g;
+  if ((st = seg_layout(desc, L, segment_chunks, &g)) != GDN2_OK) return st;
+  if (!desc->workspace) return GDN2_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(desc->workspace) & (kAlign - 1)) != 0) return GDN2_ERR_ALIGN;
+  if (desc->workspace_bytes < g.total) return GDN2_ERR_WORKSPACE;
+  const long long tokens = (long long)desc->B * desc->T;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, tokens)) != GDN2_OK) return st;
+  if (!out && tokens > 0) return GDN2_ERR_NULL;
+  if (!aligned16(out) || (h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if ((st = launch_plan(desc, L, cu_seqlens, stream)) != GDN2_OK) return st;
+  if (desc->dv == 128)
+    return launch_segmented<128>(desc, L, g, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
+  return launch_segmented<64>(desc, L, g, q, k, v, log_alpha, b, w, cu_seqlens, scale, h0, out, hT, stream);
+}
+
+gdn2_status gdn2_state_map(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* b, const float* w, const int32_t* cu_seqlens,
+                           float* phi, float* psi, cudaStream_t stream) {
+  Layout L;
+  gdn2_status st = make_layout(desc, cu_seqlens != nullptr, &L);
+  if (st != GDN2_OK) return st;
+  if (L.l.factor_set != 1) return GDN2_ERR_UNSUPPORTED;
+  if ((st = check_workspace(desc, L)) != GDN2_OK) return st;
+  if ((st = check_inputs(q, k, v, log_alpha, b, w, (long long)desc->B * desc->T)) != GDN2_OK) return st;
+  if (!phi || !psi) return GDN2_ERR_NULL;
+  if (!aligned16(phi) || !aligned16(psi)) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if ((st = launch_plan(desc, L, cu_seqlens, stream)) != GDN2_OK) return st;
+  gdn2::SeqMap seqs = seq_map(desc, L, cu_seqlens);
+  if (desc->dv == 128) {
+    if ((st = launch_prep_t<128, 128, bf16, bf16>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, stream)) != GDN2_OK)
+      return st;
+    return launch_walk_ranges<128, true>(desc, L, 1.f, seqs, nullptr, nullptr, phi, psi, stream);
+  }
+  if ((st = launch_prep_t<128, 64, bf16, bf16>(desc, L, q, k, v, log_alpha, b, w, cu_seqlens, stream)) != GDN2_OK)
+    return st;
+  return launch_walk_ranges<64, true>(desc, L, 1.f, seqs, nullptr, nullptr, phi, psi, stream);
 }
 
 gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale, const float* h0,

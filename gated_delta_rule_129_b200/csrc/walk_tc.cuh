@@ -35,6 +35,13 @@
 // timeout the CTA records GDN2_ERR_DEVICE_TIMEOUT in the status word, drains
 // what it issued and exits.
 //
+// Map mode (MAP = true, the first level of the two-level chunk scan): the
+// same walk over a range of chunks, started from [I | 0] instead of a state,
+// on the dk + dv columns of [Phi | Psi] (the chunk's Nc is added to the Psi
+// columns only), without outputs; at the end of the range the CTA writes its
+// columns of Phi (dk x dk) and Psi (dk x dv), the range's affine state map
+// S_end = Phi S_start + Psi.
+//
 // Run beside the prep CTAs in one launch (gdn2_fused_kernel), the two TMA
 // warps wait for each chunk's ready flag before loading its factors; a chunk
 // the prep handed back to the exact kernel ends the walk early and raises the
@@ -67,6 +74,8 @@ struct WalkTcArgs {
   int* redo;           // set when a handed-back chunk ended the walk early
   const int* gate;     // optional: the kernel does nothing unless *gate != 0
   unsigned long long wait_ns;  // limit of every bounded wait (0: the default, 2 s)
+  float* phi;          // map mode: [ranges, H, dk, dk] fp32
+  float* psi;          // map mode: [ranges, H, dk, dv] fp32
 };
 
 // The walk's wait limit: the host's choice, or 2 s.
@@ -153,10 +162,12 @@ __device__ __forceinline__ bool wait_chunk_ready(const WalkTcArgs& a, int t, int
   return true;
 }
 
-template <int DV>
+template <int DV, bool MAP = false>
 __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
   using C = WalkTcCfg<DV>;
   constexpr int DK = C::DK, NSL = C::NSL;
+  // column slices per range: dv / 64 of the state, or (dk + dv) / 64 of [Phi | Psi]
+  constexpr int SLC = MAP ? (DK + DV) / NSL : C::SLICES;
   uint8_t* ringA = sm;
   uint8_t* ringB = ringA + C::STAGES_A * C::A_BYTES;
   uint8_t* sS = ringB + C::STAGES_B * C::B_STRIDE;          // [2][S_BYTES]
@@ -175,10 +186,14 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const int sl = cta % C::SLICES;
-  const int h = (cta / C::SLICES) % H;
-  const int n = cta / (C::SLICES * H);
-  const int col0 = sl * NSL;
+  const int sl = cta % SLC;
+  const int h = (cta / SLC) % H;
+  const int n = cta / (SLC * H);
+  // map mode: slices 0 .. dk/64 - 1 hold Phi (key columns), the rest Psi
+  const bool phi_slice = MAP && sl < DK / NSL;
+  const int col0 = MAP && !phi_slice ? (sl - DK / NSL) * NSL : sl * NSL;
+  const bool use_nc = !phi_slice;
+  constexpr uint32_t A_TX = MAP ? C::MP_BYTES : C::A_BYTES;
   const int c_begin = a.map.chunk_off[n];
   const int nch = a.map.chunk_off[n + 1] - c_begin;
   const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
@@ -190,7 +205,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     }
     for (int s = 0; s < C::STAGES_B; ++s) {
       tc::mbar_init(&fullB[s], 1);
-      tc::mbar_init(&emptyB[s], 2 * C::EPI_WARPS);  // state and output warps
+      tc::mbar_init(&emptyB[s], (MAP ? 1 : 2) * C::EPI_WARPS);  // state (and output) warps
     }
     tc::mbar_init(s_done, 1);
     tc::mbar_init(o_done, 1);
@@ -215,10 +230,16 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
     const int row = 32 * warp + lane;  // key channel = TMEM lane
     const size_t sbase = ((size_t)n * H + h) * DK * DV + (size_t)row * DV + col0;
     float S[NSL];
+    if (MAP) {
+      // [I | 0]: this thread's row of the identity (Phi) or zeros (Psi)
 #pragma unroll
-    for (int i = 0; i < NSL; i += 4) {
-      const float4 v = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + sbase + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-      S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
+      for (int i = 0; i < NSL; ++i) S[i] = phi_slice && row == col0 + i ? 1.f : 0.f;
+    } else {
+#pragma unroll
+      for (int i = 0; i < NSL; i += 4) {
+        const float4 v = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + sbase + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        S[i] = v.x; S[i + 1] = v.y; S[i + 2] = v.z; S[i + 3] = v.w;
+      }
     }
     // this thread's row in the interleaved operand: core matrix (row/8, g),
     // 16-byte line row%8
@@ -264,7 +285,9 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       uint32_t ncw[NSL / 2];
 #pragma unroll
       for (int u = 0; u < NSL / 8; ++u) {
-        const uint4 t = *reinterpret_cast<const uint4*>(stB + row * 128 + ((u ^ (row & 7)) << 4));
+        // (Phi columns of map mode take no Nc: zero words)
+        const uint4 t = use_nc ? *reinterpret_cast<const uint4*>(stB + row * 128 + ((u ^ (row & 7)) << 4))
+                               : make_uint4(0u, 0u, 0u, 0u);
         ncw[4 * u] = t.x; ncw[4 * u + 1] = t.y; ncw[4 * u + 2] = t.z; ncw[4 * u + 3] = t.w;
       }
       if (!wwait(s_done, j & 1, a.status, s_abort, wb)) break;
@@ -301,12 +324,18 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
     }
-    if (a.hT && !*reinterpret_cast<volatile int*>(s_abort)) {
+    if (MAP && !*reinterpret_cast<volatile int*>(s_abort)) {
+      float* dst = phi_slice ? a.phi + (((size_t)n * H + h) * DK + row) * DK + col0
+                             : a.psi + (((size_t)n * H + h) * DK + row) * DV + col0;
+#pragma unroll
+      for (int i = 0; i < NSL; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
+    } else if (a.hT && !*reinterpret_cast<volatile int*>(s_abort)) {
 #pragma unroll
       for (int i = 0; i < NSL; i += 4)
         *reinterpret_cast<float4*>(a.hT + sbase + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
     }
   } else if (warp < 2 * C::EPI_WARPS) {
+    if constexpr (!MAP) {  // no outputs in map mode
     // ---------------------------------------------------------- outputs --
     const int ow = warp - C::EPI_WARPS;   // TMEM lane quarter of this warp
     const int i_tok = 16 * ow + lane;     // token row of D_O (M = 64 layout), lane < 16
@@ -346,6 +375,7 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&emptyB[sb]);
     }
+    }
   } else if (warp == C::MMA_WARP && lane == 0) {
     // --------------------------------------------------------- UMMA issue --
     constexpr uint32_t idS = tc::idesc_bf16(128, NSL, false, true);
@@ -368,6 +398,10 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
         tc::umma_f16(tbase, mp_d + (uint64_t)(((s / 4) * (DK * 128) + (s % 4) * 32) >> 4),
                      sb_d + (uint64_t)((s * 2 * C::S_LBO) >> 4), idS, s > 0);
       tc::umma_commit(s_done);
+      if (MAP) {
+        tc::umma_commit(&emptyA[st]);
+        continue;
+      }
       // the output warps have read D_O(j-1): keeps every o_done waiter within
       // one phase (and frees the D_O buffer D_O(j+1) will use)
       if (j >= 1 && !wwait(&o_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, s_abort, wb)) break;
@@ -399,10 +433,12 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
           const int rm = tp * DK, rq = tp * kChunk;
           tc::tma_prefetch_2d(&a.tm_Mp, 0, rm);
           tc::tma_prefetch_2d(&a.tm_Mp, 64, rm);
-          tc::tma_prefetch_2d(&a.tm_Qe, 0, rq);
-          tc::tma_prefetch_2d(&a.tm_Qe, 64, rq);
-          tc::tma_prefetch_2d(&a.tm_Nc, col0, rm);
-          tc::tma_prefetch_2d(&a.tm_Op, col0, rq);
+          if (!MAP) {
+            tc::tma_prefetch_2d(&a.tm_Qe, 0, rq);
+            tc::tma_prefetch_2d(&a.tm_Qe, 64, rq);
+            tc::tma_prefetch_2d(&a.tm_Op, col0, rq);
+          }
+          if (use_nc) tc::tma_prefetch_2d(&a.tm_Nc, col0, rm);
           tc::tma_prefetch_2d(&a.tm_g, 0, tp);
           tc::tma_prefetch_2d(&a.tm_cs, 0, tp);
         }
@@ -410,12 +446,14 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       if (j >= C::STAGES_A && !wwait(&emptyA[st], ((j - C::STAGES_A) / C::STAGES_A) & 1, a.status, s_abort, wb)) break;
       if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringA + st * C::A_BYTES;
-      tc::mbar_arrive_expect_tx(&fullA[st], C::A_BYTES);
+      tc::mbar_arrive_expect_tx(&fullA[st], A_TX);
       const int rm = (c * H + h) * DK, rq = (c * H + h) * kChunk;
       tc::tma_load_2d(dst, &a.tm_Mp, &fullA[st], 0, rm);
       tc::tma_load_2d(dst + DK * 128, &a.tm_Mp, &fullA[st], 64, rm);
-      tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
-      tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
+      if (!MAP) {
+        tc::tma_load_2d(dst + C::MP_BYTES, &a.tm_Qe, &fullA[st], 0, rq);
+        tc::tma_load_2d(dst + C::MP_BYTES + kChunk * 128, &a.tm_Qe, &fullA[st], 64, rq);
+      }
       ++loaded;
     }
     // every issued load has landed before the CTA releases its shared memory
@@ -435,9 +473,9 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
       if (j >= C::STAGES_B && !wwait(&emptyB[st], ((j - C::STAGES_B) / C::STAGES_B) & 1, a.status, s_abort, wb)) break;
       if (a.ready && !wait_chunk_ready(a, c * H + h, s_abort)) break;
       uint8_t* dst = ringB + st * C::B_STRIDE;
-      tc::mbar_arrive_expect_tx(&fullB[st], C::B_BYTES);
-      tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
-      tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
+      tc::mbar_arrive_expect_tx(&fullB[st], (use_nc ? C::NC_BYTES : 0) + (MAP ? 0 : C::OP_BYTES) + 2 * C::G_BYTES);
+      if (use_nc) tc::tma_load_2d(dst, &a.tm_Nc, &fullB[st], col0, (c * H + h) * DK);
+      if (!MAP) tc::tma_load_2d(dst + C::NC_BYTES, &a.tm_Op, &fullB[st], col0, (c * H + h) * kChunk);
       tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES, &a.tm_g, &fullB[st], 0, c * H + h);
       tc::tma_load_2d(dst + C::NC_BYTES + C::OP_BYTES + C::G_BYTES, &a.tm_cs, &fullB[st], 0, c * H + h);
       ++loaded;
@@ -453,14 +491,14 @@ __device__ void walk_tc_cta(const WalkTcArgs& a, uint8_t* sm, int cta) {
   }
 }
 
-template <int DV>
+template <int DV, bool MAP = false>
 __global__ void __launch_bounds__(WalkTcCfg<DV>::THREADS, 1)
 walk_tc_kernel(const __grid_constant__ WalkTcArgs a) {
   if (a.gate && *a.gate == 0) return;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  walk_tc_cta<DV>(a, sm, blockIdx.x);
+  walk_tc_cta<DV, MAP>(a, sm, blockIdx.x);
 }
 
 }  // namespace gdn2

@@ -208,6 +208,55 @@ GDN2_API gdn2_status gdn2_chunk_fused(const gdn2_desc* desc, const void* q, cons
                              const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
                              cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Two-level chunk scan (state passing between ranges of a sequence).
+ *
+ * Over any range of tokens the recurrence is affine in the state: the state at
+ * the end of the range is Phi S_start + Psi, with Phi (dk x dk) the product of
+ * the per-token linear parts (I - k_t e_t^T) diag(alpha_t) and Psi (dk x dv)
+ * the state the range reaches from zero (page "Gated DeltaNet-2：将擦除与写入分开",
+ * section "在两个维度上独立控制", applied token after token).  Maps of
+ * consecutive ranges compose: (Phi2 Phi1, Phi2 Psi1 + Psi2).  The walk over a
+ * long sequence is a chain of T/64 dependent chunk steps; splitting it into
+ * segments of L chunks turns it into (1) every segment's map, in parallel,
+ * (2) a short fp32 scan of the maps that gives each segment its start state,
+ * (3) every segment's walk with outputs, in parallel.  Ranks that each hold a
+ * range of one long sequence pass state the same way: each computes its
+ * range's map (gdn2_state_map), the maps of the earlier ranges give its start
+ * state, and it runs gdn2_chunk_fwd from there.
+ * Affine factor set only (bf16 I/O with dk = 128); GDN2_ERR_UNSUPPORTED
+ * otherwise.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes of gdn2_chunk_fwd_segmented: gdn2_workspace_size(desc) plus
+ * the segments, their maps and start states (0 if desc is invalid or not the
+ * affine set).  segment_chunks = L, the chunks per segment; 0 chooses
+ * max(8, ceil(chunks per sequence / 4)) (from desc alone). */
+GDN2_API size_t gdn2_segmented_workspace_size(const gdn2_desc* desc, int segment_chunks);
+
+/* gdn2_chunk_fwd through the two-level chunk scan (arguments and results as
+ * there; desc->workspace holds gdn2_segmented_workspace_size(desc,
+ * segment_chunks) bytes).  Each sequence is split into segments of
+ * segment_chunks 64-token chunks (0: see above); the outputs equal
+ * gdn2_chunk_fwd's up to rounding (the start state of a segment is the fp32
+ * product of the earlier segments' maps instead of a chunk-by-chunk walk).
+ * Asynchronous on `stream`. */
+GDN2_API gdn2_status gdn2_chunk_fwd_segmented(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                              const float* log_alpha, const float* b, const float* w, float scale,
+                                              const float* h0, const int32_t* cu_seqlens, void* out, float* hT,
+                                              int segment_chunks, cudaStream_t stream);
+
+/* The affine state map of every sequence of the call (the whole range of its
+ * tokens): phi [N, H, dk, dk] and psi [N, H, dk, dv], fp32, device, so that
+ * the final state from a start state S is phi S + psi.  q is needed by the
+ * chunk preparation it shares with gdn2_chunk_fwd; the workspace is
+ * gdn2_workspace_size(desc) bytes.  An empty sequence (or a malformed
+ * cu_seqlens, reported in the status word) gives the identity map.
+ * Asynchronous on `stream`. */
+GDN2_API gdn2_status gdn2_state_map(const gdn2_desc* desc, const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* b, const float* w,
+                                    const int32_t* cu_seqlens, float* phi, float* psi, cudaStream_t stream);
+
 /* gdn2_chunk_walk with the walk taking each chunk only once its ready flag in
  * the workspace (off_sync, the flags gdn2_chunk_fused's prep raises) reads 2,
  * and with every bounded device-side wait limited to wait_budget_ns (0 = the
