@@ -25,6 +25,9 @@ Contents
 * :mod:`oracle.chunk_backward` -- the same gradients through the 64-token chunk
   form (the algebra a backward over chunks evaluates), checked against
   :mod:`oracle.backward`.
+* :mod:`oracle.token_path` -- the token path around the operator (short causal
+  convolution, SiLU, L2 normalisation of q and k; RMS normalisation and the
+  output gate of the operator's output), fp64 numpy.
 * :mod:`oracle.state_map` -- the affine state map (Phi, Psi) of a token range
   and the composition of consecutive maps (the two-level chunk scan and the
   state passing between ranges of one sequence), fp64 numpy.
