@@ -328,6 +328,7 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / ne, world)
 
     decode = measure_decode(dev, stream, flush) if rank == 0 else None
+    token_path = measure_token_path(dev, stream, flush, peaks()[0]) if rank == 0 else None
     others = measure_other_configs(dev, stream, flush, peaks()[0]) if (rank == 0 and not args.no_other_configs) else None
     backward = None
     if rank == 0 and not args.no_backward:
@@ -374,6 +375,8 @@ def run_ours(args, rank, world, local):
         decode["roofline"] = {"bound": "hbm", "achieved": decode["gbs"], "peak": hbm, "unit": "GB/s",
                               "frac": decode["gbs"] / hbm}
         line["decode_step"] = decode
+    if token_path:
+        line["token_path"] = token_path
     if others:
         line["other_configs"] = others
     if backward:
@@ -449,6 +452,51 @@ def measure_backward(dev, stream, hbm, reps=3):
     return {"workload": "16Kx1 backward (gdn2_chunk_bwd, CUDA-core baseline), bf16 inputs, fp32 gradients",
             "ms": ms, "tokens_per_s": B * T / (ms / 1e3), "alg_bytes": alg,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
+
+
+def measure_token_path(dev, stream, flush, hbm, reps=20):
+    """The token path around the operator at 16K x 1 (H=16, d=128, bf16):
+    gdn2_token_prologue (reads q, k, v from the projections, writes the
+    operator's q, k, v: 6 x 256 B per token-head) and gdn2_token_epilogue
+    (reads o and the gate, writes the gated output: 3 x 256 B per token-head),
+    each timed alone with CUDA events, L2 flushed, with its HBM roofline."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    gen = torch.Generator(device=dev).manual_seed(7)
+    r = lambda *s: torch.randn(*s, generator=gen, device=dev)  # noqa: E731
+    bf = torch.bfloat16
+    q_raw, k_raw, v_raw = (r(B, T, H, DK).to(bf) for _ in range(3))
+    wq, wk, wv = (0.5 * r(H * DK, 4) for _ in range(3))
+    gate = r(B, T, H, DV).to(bf)
+    wt = torch.ones(DV, device=dev)
+    q, k, v = (torch.empty_like(q_raw) for _ in range(3))
+    out = torch.empty_like(v_raw)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+    res = {}
+    for name, fn, per_th in (
+            ("prologue", lambda: gdn2.token_prologue(q_raw, k_raw, v_raw, wq, wk, wv, q=q, k=k, v=v, stream=stream),
+             6 * 256),
+            ("epilogue", lambda: gdn2.token_epilogue(v_raw, gate, wt, out=out, stream=stream), 3 * 256)):
+        ms = timed(fn)
+        nbytes = TH * per_th
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[name] = {"ms": ms, "alg_bytes": nbytes, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+                                                                  "unit": "GB/s", "frac": gbs / hbm}}
+    return res
 
 
 def measure_other_configs(dev, stream, flush, hbm, steps=10):

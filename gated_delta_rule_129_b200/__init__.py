@@ -22,7 +22,7 @@ import os
 import threading
 
 __all__ = ["chunk_fwd", "chunk_fwd_noalloc", "noalloc_status", "chunk_walk_flagged", "chunk_fwd_segmented",
-           "segmented_workspace_size", "state_map", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
+           "segmented_workspace_size", "state_map", "token_prologue", "token_epilogue", "token_path_fwd", "chunk_prep", "chunk_walk", "chunk_plan", "chunk_fused",
            "recurrent_step", "workspace_size",
            "workspace_layout", "status_string", "GDN2Error", "lib_path", "load_library"]
 
@@ -42,7 +42,8 @@ EXPORTED = ("gdn2_workspace_size", "gdn2_workspace_layout", "gdn2_chunk_fwd", "g
             "gdn2_chunk_prep", "gdn2_chunk_walk", "gdn2_chunk_plan", "gdn2_chunk_fused",
             "gdn2_recurrent_step", "gdn2_status_string", "gdn2_version", "gdn2_backward_workspace_size",
             "gdn2_chunk_bwd", "gdn2_noalloc_status", "gdn2_chunk_walk_flagged",
-            "gdn2_segmented_workspace_size", "gdn2_chunk_fwd_segmented", "gdn2_state_map")
+            "gdn2_segmented_workspace_size", "gdn2_chunk_fwd_segmented", "gdn2_state_map",
+            "gdn2_token_prologue", "gdn2_token_epilogue")
 
 
 class GDN2Error(RuntimeError):
@@ -107,6 +108,10 @@ def load_library():
         lib.gdn2_chunk_fwd_segmented.restype = i
         lib.gdn2_state_map.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn2_state_map.restype = i
+        lib.gdn2_token_prologue.argtypes = [dp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp]
+        lib.gdn2_token_prologue.restype = i
+        lib.gdn2_token_epilogue.argtypes = [dp, vp, vp, vp, vp, vp]
+        lib.gdn2_token_epilogue.restype = i
         lib.gdn2_chunk_prep.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.gdn2_chunk_prep.restype = i
         lib.gdn2_chunk_walk.argtypes = [dp, f, vp, vp, vp, vp, vp, vp]
@@ -419,6 +424,50 @@ def state_map(q, k, v, log_alpha, b, w, cu_seqlens=None, *, phi=None, psi=None, 
                                        _ptr(w), _ptr(cu_seqlens), _ptr(phi), _ptr(psi), _stream(stream))
     _check(st, "gdn2_state_map")
     return phi, psi
+
+
+def token_prologue(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cu_seqlens=None, *, q=None, k=None, v=None,
+                   stream=None):
+    """``gdn2_token_prologue``: ``(q, k, v)`` for the operator from the
+    projections' outputs (short causal convolution with weights ``conv_*``
+    ``[H * d, W]`` fp32, SiLU, and L2 normalisation of q and k)."""
+    torch = _torch()
+    B, T, H, dk, dv, ns = _shapes(q_raw, v_raw, cu_seqlens)
+    io = _io_of(q_raw.dtype)
+    _need_contig(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cu_seqlens)
+    W = int(conv_q.shape[-1])
+    q = torch.empty_like(q_raw) if q is None else q
+    k = torch.empty_like(k_raw) if k is None else k
+    v = torch.empty_like(v_raw) if v is None else v
+    d = make_desc(B, T, H, dk, dv, io, ns)
+    st = load_library().gdn2_token_prologue(ctypes.byref(d), _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q),
+                                            _ptr(conv_k), _ptr(conv_v), W, _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+                                            _stream(stream))
+    _check(st, "gdn2_token_prologue")
+    return q, k, v
+
+
+def token_epilogue(o, gate, norm_weight, *, out=None, stream=None):
+    """``gdn2_token_epilogue``: ``rmsnorm(o) * norm_weight * sigmoid(gate)``."""
+    torch = _torch()
+    B, T, H, dv = o.shape
+    _need_contig(o, gate, norm_weight)
+    out = torch.empty_like(o) if out is None else out
+    d = make_desc(B, T, H, 128, dv, _io_of(o.dtype))
+    st = load_library().gdn2_token_epilogue(ctypes.byref(d), _ptr(o), _ptr(gate), _ptr(norm_weight), _ptr(out),
+                                            _stream(stream))
+    _check(st, "gdn2_token_epilogue")
+    return out
+
+
+def token_path_fwd(q_raw, k_raw, v_raw, log_alpha, b, w, gate, conv_q, conv_k, conv_v, norm_weight, scale=None,
+                   h0=None, cu_seqlens=None, *, workspace=None, stream=None):
+    """The operator with its token path: :func:`token_prologue`, then
+    :func:`chunk_fwd`, then :func:`token_epilogue`.  Returns ``(out, hT)``
+    (``out`` before the caller's output projection)."""
+    q, k, v = token_prologue(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cu_seqlens, stream=stream)
+    o, hT = chunk_fwd(q, k, v, log_alpha, b, w, scale, h0, cu_seqlens, workspace=workspace, stream=stream)
+    return token_epilogue(o, gate, norm_weight, out=o, stream=stream), hT
 
 
 def backward_workspace_size(B, T, H, dk, dv, io=GDN2_IO_BF16, num_seqs=0) -> int:

@@ -21,6 +21,7 @@
 #include "prep_tc.cuh"
 #include "fused_tc.cuh"
 #include "segscan.cuh"
+#include "token_path.cuh"
 #include "tmap.cuh"
 #include "walk_simt.cuh"
 #include "walk_tc.cuh"
@@ -849,6 +850,81 @@ gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale, const fl
                                wait_budget_ns);
   return launch_walk_tc<64>(desc, L, scale, h0, cu_seqlens, out, hT, nullptr, stream, nullptr, true,
                             wait_budget_ns);
+}
+
+gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_raw, const void* k_raw, const void* v_raw,
+                                const float* conv_q, const float* conv_k, const float* conv_v, int conv_width,
+                                const int32_t* cu_seqlens, void* q, void* k, void* v, cudaStream_t stream) {
+  if (!desc) return GDN2_ERR_NULL;
+  const bool packed = cu_seqlens != nullptr;
+  gdn2_status st = check_dims(desc, packed);
+  if (st != GDN2_OK) return st;
+  if (conv_width < 1 || conv_width > gdn2::kMaxConvWidth) return GDN2_ERR_SHAPE;
+  const long long tokens = (long long)desc->B * desc->T;
+  if (tokens > 0 && (!q_raw || !k_raw || !v_raw || !conv_q || !conv_k || !conv_v || !q || !k || !v))
+    return GDN2_ERR_NULL;
+  if (!aligned16(q_raw) || !aligned16(k_raw) || !aligned16(v_raw) || !aligned16(q) || !aligned16(k) ||
+      !aligned16(v) || !aligned16(conv_q) || !aligned16(conv_k) || !aligned16(conv_v))
+    return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if (tokens == 0) return GDN2_OK;
+  gdn2::TokProArgs a;
+  a.q_raw = q_raw; a.k_raw = k_raw; a.v_raw = v_raw;
+  a.wq = conv_q; a.wk = conv_k; a.wv = conv_v;
+  a.W = conv_width;
+  a.cu = cu_seqlens;
+  a.N = packed ? desc->num_seqs : desc->B;
+  a.T = desc->T;
+  a.T_total = (int)tokens;
+  a.H = desc->H;
+  a.q = q; a.k = k; a.v = v;
+  const long long runs = (tokens + gdn2::kTokRun - 1) / gdn2::kTokRun;
+  const long long bx = (runs + gdn2::kTokThreads / 32 - 1) / (gdn2::kTokThreads / 32);
+  if (bx > INT32_MAX || desc->H > 65535) return GDN2_ERR_SHAPE;
+  const dim3 grid((unsigned)bx, (unsigned)desc->H, 3);
+  const bool f32 = desc->io == GDN2_IO_F32;
+#define GDN2_PRO(DK_, DV_)                                                                          \
+  if (desc->dk == DK_ && desc->dv == DV_) {                                                         \
+    if (f32) gdn2::token_prologue_kernel<float, DK_, DV_><<<grid, gdn2::kTokThreads, 0, stream>>>(a); \
+    else gdn2::token_prologue_kernel<bf16, DK_, DV_><<<grid, gdn2::kTokThreads, 0, stream>>>(a);      \
+    return launch_status();                                                                         \
+  }
+  GDN2_PRO(64, 64)
+  GDN2_PRO(64, 128)
+  GDN2_PRO(128, 64)
+  GDN2_PRO(128, 128)
+#undef GDN2_PRO
+  return GDN2_ERR_SHAPE;
+}
+
+gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void* gate, const float* norm_weight,
+                                void* out, cudaStream_t stream) {
+  if (!desc) return GDN2_ERR_NULL;
+  if (desc->io != GDN2_IO_F32 && desc->io != GDN2_IO_BF16) return GDN2_ERR_DTYPE;
+  if ((desc->dk != 64 && desc->dk != 128) || (desc->dv != 64 && desc->dv != 128)) return GDN2_ERR_SHAPE;
+  if (desc->H < 1 || desc->B < 1 || desc->T < 0) return GDN2_ERR_SHAPE;
+  const long long tokens = (long long)desc->B * desc->T;
+  if (tokens > INT32_MAX / 2) return GDN2_ERR_SHAPE;
+  if (tokens > 0 && (!o || !gate || !norm_weight || !out)) return GDN2_ERR_NULL;
+  if (!aligned16(o) || !aligned16(gate) || !aligned16(norm_weight) || !aligned16(out)) return GDN2_ERR_ALIGN;
+  if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
+  if (tokens == 0) return GDN2_OK;
+  gdn2::TokEpiArgs a;
+  a.o = o; a.g = gate; a.weight = norm_weight;
+  a.T_total = (int)tokens;
+  a.H = desc->H;
+  a.out = out;
+  const long long blocks = (tokens * desc->H + gdn2::kTokThreads / 32 - 1) / (gdn2::kTokThreads / 32);
+  if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+  const bool f32 = desc->io == GDN2_IO_F32;
+  if (desc->dv == 128) {
+    if (f32) gdn2::token_epilogue_kernel<float, 128><<<(unsigned)blocks, gdn2::kTokThreads, 0, stream>>>(a);
+    else gdn2::token_epilogue_kernel<bf16, 128><<<(unsigned)blocks, gdn2::kTokThreads, 0, stream>>>(a);
+  } else {
+    if (f32) gdn2::token_epilogue_kernel<float, 64><<<(unsigned)blocks, gdn2::kTokThreads, 0, stream>>>(a);
+    else gdn2::token_epilogue_kernel<bf16, 64><<<(unsigned)blocks, gdn2::kTokThreads, 0, stream>>>(a);
+  }
+  return launch_status();
 }
 
 gdn2_status gdn2_recurrent_step(const gdn2_desc* desc, const void* q, const void* k, const void* v,

@@ -257,6 +257,40 @@ GDN2_API gdn2_status gdn2_state_map(const gdn2_desc* desc, const void* q, const 
                                     const float* log_alpha, const float* b, const float* w,
                                     const int32_t* cu_seqlens, float* phi, float* psi, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Token path around the operator (page "Gated DeltaNet-2：将擦除与写入分开",
+ * section "词元路径与并行训练"): q and k pass through a short causal
+ * convolution, SiLU and L2 normalisation, v through the convolution and SiLU;
+ * the operator's output passes through RMS normalisation and an output gate of
+ * its own.  The linear projections before and after need trained weights and
+ * stay with the caller.  Readings where the pages are silent: depthwise
+ * convolution over the H*d channels of a projection, causal inside each
+ * sequence (tokens before its first count as zero), width conv_width (1..8);
+ * eps = 1e-6 in both norms; the gate is sigmoid(g).
+ * ------------------------------------------------------------------------ */
+
+/* q = l2norm(silu(conv(q_raw))), k = l2norm(silu(conv(k_raw))),
+ * v = silu(conv(v_raw)), per token and head.
+ *   q_raw, k_raw, q, k : [B, T, H, dk] io dtype;  v_raw, v : [B, T, H, dv]
+ *   conv_q, conv_k     : [H * dk, conv_width] fp32, tap i weighs token t - i
+ *   conv_v             : [H * dv, conv_width] fp32
+ *   cu_seqlens         : as for gdn2_chunk_fwd (sequence starts reset the
+ *                        convolution), or NULL for B dense sequences
+ * desc: B, T, H, dk, dv, num_seqs and io as for gdn2_chunk_fwd (the workspace
+ * is not used).  Outputs must not overlap the inputs.  Device pointers,
+ * 16-byte aligned.  Asynchronous on `stream`. */
+GDN2_API gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_raw, const void* k_raw,
+                                         const void* v_raw, const float* conv_q, const float* conv_k,
+                                         const float* conv_v, int conv_width, const int32_t* cu_seqlens, void* q,
+                                         void* k, void* v, cudaStream_t stream);
+
+/* out = rmsnorm(o) * norm_weight * sigmoid(gate), per token and head, the norm
+ * over the dv channels of a head.
+ *   o, gate, out : [B, T, H, dv] io dtype (out may be o);  norm_weight : [dv] fp32
+ * desc: B, T, H, dk, dv, io (the rest is not used).  Asynchronous on `stream`. */
+GDN2_API gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void* gate,
+                                         const float* norm_weight, void* out, cudaStream_t stream);
+
 /* gdn2_chunk_walk with the walk taking each chunk only once its ready flag in
  * the workspace (off_sync, the flags gdn2_chunk_fused's prep raises) reads 2,
  * and with every bounded device-side wait limited to wait_budget_ns (0 = the
