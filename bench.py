@@ -600,6 +600,42 @@ def ncu_case():
     print("ncu case ok", float(out.float().abs().mean()))
 
 
+def ncu_kernels():
+    """One launch of each kernel of the library on a small case, for per-kernel
+    ncu captures (nothing timed): the two stages of the chunked forward
+    (B=1, T=4096, H=16, dk=dv=128, strong decay: inputs and factors larger
+    than L2), the decode step on 256 states, the token path's prologue and
+    epilogue, the two-level chunk scan, and the backward on T=1024."""
+    import torch
+
+    import gated_delta_rule_129_b200 as gdn2
+    from workloads import decode_inputs, make_inputs
+    torch.cuda.set_device(0)
+    bf, f32 = torch.bfloat16, torch.float32
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to("cuda", dt)  # noqa: E731
+    x = make_inputs(1, 4096, 16, 128, 128, io="bf16", seed=2, decay="strong")
+    q, k, v = (t(a, bf) for a in (x.q, x.k, x.v))
+    la, b, w = (t(a, f32) for a in (x.log_alpha, x.b, x.w))
+    ws = torch.empty(gdn2.workspace_size(1, 4096, 16, 128, 128), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(v)
+    hT = torch.empty((1, 16, 128, 128), dtype=f32, device="cuda")
+    gdn2.chunk_prep(q, k, v, la, b, w, workspace=ws)
+    gdn2.chunk_walk(ws, (1, 4096, 16, 128, 128), bf, x.scale, out=out, hT=hT)
+    di = decode_inputs(B=256, H=16, dk=128, dv=128, io="bf16", seed=41)
+    state = t(di.state, f32)
+    gdn2.recurrent_step(t(di.q, bf), t(di.k, bf), t(di.v, bf), t(di.log_alpha, f32), t(di.b, f32), t(di.w, f32),
+                        di.scale, state)
+    wconv = torch.full((16 * 128, 4), 0.25, device="cuda")
+    q2, k2, v2 = gdn2.token_prologue(q, k, v, wconv, wconv, wconv)
+    gdn2.token_epilogue(out, v, torch.ones(128, device="cuda"), out=out)
+    gdn2.chunk_fwd_segmented(q, k, v, la, b, w, x.scale, segment_chunks=16)
+    xs = make_inputs(1, 1024, 16, 128, 128, io="bf16", seed=3, decay="strong")
+    gdn2.chunk_bwd(*(t(a, bf) for a in (xs.q, xs.k, xs.v)), *(t(a, f32) for a in (xs.log_alpha, xs.b, xs.w)),
+                   xs.scale, t(xs.v, bf))
+    torch.cuda.synchronize()
+    print("ncu kernels ok", float(out.float().abs().mean()), float(q2.float().abs().mean()))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -612,9 +648,14 @@ def main():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--ncu-case", action="store_true",
                     help="run the small fused-kernel case for ncu captures and exit")
+    ap.add_argument("--ncu-kernels", action="store_true",
+                    help="run one launch of each kernel on small cases for ncu captures and exit")
     args = ap.parse_args()
     if args.ncu_case:
         ncu_case()
+        return
+    if args.ncu_kernels:
+        ncu_kernels()
         return
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":

@@ -878,10 +878,10 @@ gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_raw, const 
   a.T_total = (int)tokens;
   a.H = desc->H;
   a.q = q; a.k = k; a.v = v;
-  const long long runs = (tokens + gdn2::kTokRun - 1) / gdn2::kTokRun;
-  const long long bx = (runs + gdn2::kTokThreads / 32 - 1) / (gdn2::kTokThreads / 32);
-  if (bx > INT32_MAX || desc->H > 65535) return GDN2_ERR_SHAPE;
-  const dim3 grid((unsigned)bx, (unsigned)desc->H, 3);
+  const int tile = desc->io == GDN2_IO_F32 ? gdn2::tok_tile<float>() : gdn2::tok_tile<bf16>();
+  const long long tiles = (tokens + tile - 1) / tile;
+  if (tiles > INT32_MAX || desc->H > 65535) return GDN2_ERR_SHAPE;
+  const dim3 grid((unsigned)tiles, (unsigned)desc->H, 3);
   const bool f32 = desc->io == GDN2_IO_F32;
 #define GDN2_PRO(DK_, DV_)                                                                          \
   if (desc->dk == DK_ && desc->dv == DV_) {                                                         \
@@ -914,7 +914,8 @@ gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void
   a.T_total = (int)tokens;
   a.H = desc->H;
   a.out = out;
-  const long long blocks = (tokens * desc->H + gdn2::kTokThreads / 32 - 1) / (gdn2::kTokThreads / 32);
+  const long long per_block = (gdn2::kTokThreads / 32) * gdn2::kEpiPairs;
+  const long long blocks = (tokens * desc->H + per_block - 1) / per_block;
   if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
   const bool f32 = desc->io == GDN2_IO_F32;
   if (desc->dv == 128) {

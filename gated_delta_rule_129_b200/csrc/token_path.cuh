@@ -14,9 +14,9 @@
 //
 // Both kernels are bound by HBM traffic; each lane owns a run of d/32
 // channels (8 or 4 bytes of a bf16 row), fp32 arithmetic, a head's sums of
-// squares by warp shuffles.  The prologue gives each warp one head of one
-// projection over 32 consecutive tokens and slides the convolution window
-// along them in registers; the epilogue gives each warp one (token, head).
+// squares by warp shuffles.  The prologue gives each block one head of one
+// projection over a 64-token tile staged in shared memory (with the W - 1
+// rows before it); the epilogue gives each warp one (token, head).
 #pragma once
 
 #include "common.cuh"
@@ -54,7 +54,10 @@ struct Row {
   }
 };
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+// __expf (the hardware exponential): its relative error, a few fp32 ulp, is
+// far below what the bf16 outputs keep and below the fp32 path's tolerance.
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
 
 // Sequence bookkeeping of the prologue: the sequence that holds token t, as
 // [start, next start).  Packed: the largest n with cu[n] <= t (empty
@@ -76,7 +79,10 @@ __device__ __forceinline__ void seq_bounds(const int32_t* cu, int N, int T, int 
   t1 = cu[lo + 1];
 }
 
-constexpr int kTokRun = 32;   // tokens per warp in the prologue
+// tokens per block in the prologue: 128 for bf16, 64 for fp32 rows (the
+// same shared-memory footprint)
+template <typename IO>
+constexpr int tok_tile() { return 256 / (int)sizeof(IO); }
 
 struct TokProArgs {
   const void *q_raw, *k_raw, *v_raw;
@@ -87,65 +93,63 @@ struct TokProArgs {
   void *q, *k, *v;
 };
 
-// One warp: one head of one projection over a run of kTokRun consecutive
-// tokens.  Each lane keeps its channels' taps and the last W - 1 input rows
-// in registers and slides along the run, so every input row is read from
-// memory once (plus W - 1 rows before the run); a sequence start inside the
-// run clears the window.
+// One block: one head of one projection over a tile of tok_tile<IO>() tokens.
+// The tile's rows, the W - 1 rows before it and the head's taps are first
+// copied to shared memory by all threads (16-byte loads, many in flight);
+// then each warp computes its tokens from there, a lane per d/32 channels.
+// A tap that reaches before the token's sequence start reads zero.
 template <typename IO, int D>
-__device__ __forceinline__ void conv_run(const IO* __restrict__ x, const float* __restrict__ wt, IO* __restrict__ y,
-                                         const TokProArgs& a, int h, int tb, bool l2, int lane) {
+__device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float* __restrict__ wt, IO* __restrict__ y,
+                                          const TokProArgs& a, int h, int tb, bool l2, uint8_t* smem) {
   constexpr int PER = D / 32;
-  constexpr int WM = kMaxConvWidth;
-  const int c0 = lane * PER;
+  constexpr int ROWB = D * (int)sizeof(IO);                  // bytes of one row
+  constexpr int TT = tok_tile<IO>();
   const int W = a.W;
-  float tap[WM][PER];
-#pragma unroll
-  for (int i = 0; i < WM; ++i)
-#pragma unroll
-    for (int e = 0; e < PER; ++e) tap[i][e] = i < W ? wt[((size_t)h * D + c0 + e) * W + i] : 0.f;
-  const int te = min(a.T_total, tb + kTokRun);
-  int n, t0, t1;
-  seq_bounds(a.cu, a.N, a.T, tb, n, t0, t1);
-  t0 = max(t0, 0);   // (a malformed cu_seqlens must not send a read before the row)
-  // win[i] = x_{t-i} for i = 1 .. WM-1 (zero before the sequence's start)
-  float win[WM][PER];
-#pragma unroll
-  for (int i = 1; i < WM; ++i) {
-    Row<IO, D> r;
-    if (i < W && tb - i >= t0) {
-      r.load(x + ((size_t)(tb - i) * a.H + h) * D + c0);
-    } else {
-#pragma unroll
-      for (int e = 0; e < PER; ++e) r.v[e] = 0.f;
-    }
-#pragma unroll
-    for (int e = 0; e < PER; ++e) win[i][e] = r.v[e];
+  const int r0 = tb - (W - 1);                               // first row held
+  const int nrows = min(a.T_total, tb + TT) - r0;
+  float* s_tap = reinterpret_cast<float*>(smem + (TT + kMaxConvWidth - 1) * ROWB);   // [D][W]
+  for (int i = threadIdx.x; i < D * W; i += kTokThreads) s_tap[i] = wt[(size_t)h * D * W + i];
+  // copy rows [r0, r0 + nrows) of head h (rows before 0 left out)
+  for (int i = threadIdx.x; i < nrows * (ROWB / 16); i += kTokThreads) {
+    const int r = i / (ROWB / 16), u = i % (ROWB / 16);
+    if (r0 + r >= 0)
+      reinterpret_cast<uint4*>(smem + r * ROWB)[u] =
+          *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(x + ((size_t)(r0 + r) * a.H + h) * D) + u * 16);
   }
-  for (int t = tb; t < te; ++t) {
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c0 = lane * PER;
+  float tap[kMaxConvWidth][PER];
+#pragma unroll
+  for (int i = 0; i < kMaxConvWidth; ++i)
+#pragma unroll
+    for (int e = 0; e < PER; ++e) tap[i][e] = i < W ? s_tap[(c0 + e) * W + i] : 0.f;
+  constexpr int PW = TT / (kTokThreads / 32);                // tokens per warp
+  const int tw = tb + warp * PW;
+  if (tw >= a.T_total) return;
+  int n, t0, t1;
+  seq_bounds(a.cu, a.N, a.T, tw, n, t0, t1);
+  t0 = max(t0, 0);
+#pragma unroll
+  for (int u = 0; u < PW; ++u) {
+    const int t = tw + u;
+    if (t >= a.T_total) break;
     if (t >= t1) {
-      // a new sequence starts here (skip empty ones): nothing before it counts
       seq_bounds(a.cu, a.N, a.T, t, n, t0, t1);
-#pragma unroll
-      for (int i = 1; i < WM; ++i)
-#pragma unroll
-        for (int e = 0; e < PER; ++e) win[i][e] = 0.f;
+      t0 = max(t0, 0);
     }
-    Row<IO, D> r;
-    r.load(x + ((size_t)t * a.H + h) * D + c0);
     float acc[PER];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = tap[0][e] * r.v[e];
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
 #pragma unroll
-    for (int i = 1; i < WM; ++i)
+    for (int i = 0; i < kMaxConvWidth; ++i) {
+      if (i < W && t - i >= t0) {
+        Row<IO, D> r;
+        r.load(reinterpret_cast<const IO*>(smem + (t - i - r0) * ROWB) + c0);
 #pragma unroll
-      for (int e = 0; e < PER; ++e) acc[e] = fmaf(tap[i][e], win[i][e], acc[e]);
-#pragma unroll
-    for (int i = WM - 1; i > 1; --i)
-#pragma unroll
-      for (int e = 0; e < PER; ++e) win[i][e] = win[i - 1][e];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) win[1][e] = r.v[e];
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(tap[i][e], r.v[e], acc[e]);
+      }
+    }
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
@@ -157,30 +161,31 @@ __device__ __forceinline__ void conv_run(const IO* __restrict__ x, const float* 
 #pragma unroll
       for (int e = 0; e < PER; ++e) acc[e] *= rn;
     }
+    Row<IO, D> o;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) r.v[e] = acc[e];
-    r.store(y + ((size_t)t * a.H + h) * D + c0);
+    for (int e = 0; e < PER; ++e) o.v[e] = acc[e];
+    o.store(y + ((size_t)t * a.H + h) * D + c0);
   }
 }
 
-// grid: (token runs / 8, H, 3 projections); block: 8 warps, one run each
+// rows of the tile and before it (as many bytes for bf16 and fp32), then the taps
+constexpr int kTokSmem = (tok_tile<float>() + kMaxConvWidth - 1) * 128 * 4 + 128 * kMaxConvWidth * 4;
+
+// grid: (token tiles, H, 3 projections)
 template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(kTokThreads)
 token_prologue_kernel(const TokProArgs a) {
-  const int lane = threadIdx.x & 31;
-  const long long run = (long long)blockIdx.x * (kTokThreads / 32) + (threadIdx.x >> 5);
-  const long long tb = run * kTokRun;
-  if (tb >= a.T_total) return;
-  const int h = blockIdx.y;
+  __shared__ __align__(16) uint8_t smem[kTokSmem];
+  const int tb = blockIdx.x * tok_tile<IO>(), h = blockIdx.y;
   switch (blockIdx.z) {
     case 0:
-      conv_run<IO, DK>(static_cast<const IO*>(a.q_raw), a.wq, static_cast<IO*>(a.q), a, h, (int)tb, true, lane);
+      conv_tile<IO, DK>(static_cast<const IO*>(a.q_raw), a.wq, static_cast<IO*>(a.q), a, h, tb, true, smem);
       break;
     case 1:
-      conv_run<IO, DK>(static_cast<const IO*>(a.k_raw), a.wk, static_cast<IO*>(a.k), a, h, (int)tb, true, lane);
+      conv_tile<IO, DK>(static_cast<const IO*>(a.k_raw), a.wk, static_cast<IO*>(a.k), a, h, tb, true, smem);
       break;
     default:
-      conv_run<IO, DV>(static_cast<const IO*>(a.v_raw), a.wv, static_cast<IO*>(a.v), a, h, (int)tb, false, lane);
+      conv_tile<IO, DV>(static_cast<const IO*>(a.v_raw), a.wv, static_cast<IO*>(a.v), a, h, tb, false, smem);
       break;
   }
 }
@@ -192,24 +197,38 @@ struct TokEpiArgs {
   void* out;
 };
 
+constexpr int kEpiPairs = 1;   // (token, head) pairs per warp in the epilogue
+
 template <typename IO, int DV>
 __global__ void __launch_bounds__(kTokThreads)
 token_epilogue_kernel(const TokEpiArgs a) {
   constexpr int PER = DV / 32;
   const int lane = threadIdx.x & 31;
-  const long long pair = (long long)blockIdx.x * (kTokThreads / 32) + (threadIdx.x >> 5);
-  if (pair >= (long long)a.T_total * a.H) return;
-  const size_t base = (size_t)pair * DV + lane * PER;
-  Row<IO, DV> o, g;
-  o.load(static_cast<const IO*>(a.o) + base);
-  g.load(static_cast<const IO*>(a.g) + base);
-  float ss = 0.f;
+  const long long p0 = ((long long)blockIdx.x * (kTokThreads / 32) + (threadIdx.x >> 5)) * kEpiPairs;
+  const long long np = (long long)a.T_total * a.H;
+  float wt[PER];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) ss = fmaf(o.v[e], o.v[e], ss);
-  const float r = rsqrtf(warp_sum(ss) * (1.f / DV) + kTokEps);
+  for (int e = 0; e < PER; ++e) wt[e] = a.weight[lane * PER + e];
+  Row<IO, DV> o[kEpiPairs], g[kEpiPairs];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) o.v[e] = o.v[e] * r * a.weight[lane * PER + e] / (1.f + expf(-g.v[e]));
-  o.store(static_cast<IO*>(a.out) + base);
+  for (int u = 0; u < kEpiPairs; ++u) {
+    if (p0 + u < np) {
+      const size_t base = (size_t)(p0 + u) * DV + lane * PER;
+      o[u].load(static_cast<const IO*>(a.o) + base);
+      g[u].load(static_cast<const IO*>(a.g) + base);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kEpiPairs; ++u) {
+    if (p0 + u >= np) break;
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) ss = fmaf(o[u].v[e], o[u].v[e], ss);
+    const float r = rsqrtf(warp_sum(ss) * (1.f / DV) + kTokEps);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[u].v[e] = o[u].v[e] * r * wt[e] * sigmoid_f(g[u].v[e]);
+    o[u].store(static_cast<IO*>(a.out) + (size_t)(p0 + u) * DV + lane * PER);
+  }
 }
 
 }  // namespace gdn2

@@ -56,6 +56,10 @@ CASES = [
     dict(B=1, T=None, H=3, dv=128, lengths=[130, 0, 64, 1, 500], h0=0.05),
     # 20 heads: the walk CTAs take prep tasks first (switch point above 0)
     dict(B=1, T=300, H=20, dv=128, lengths=None, h0=0.05),
+    # long sequences (79 and 71 chunks), and a packed row of long ones
+    dict(B=1, T=5000, H=3, dv=128, lengths=None, h0=0.05),
+    dict(B=1, T=4500, H=2, dv=64, lengths=None, h0=0.05),
+    dict(B=1, T=None, H=2, dv=128, lengths=[2100, 0, 70, 2500], h0=0.05),
 ]
 
 
@@ -110,6 +114,24 @@ def test_fused_stage_rejects_shapes_it_does_not_take(gdn2):
     with pytest.raises(gdn2.GDN2Error):
         gdn2.chunk_fused(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], x.scale, ws,
                          out=torch.empty_like(d["v"]))
+
+
+def test_fused_steep_chunk_in_a_long_sequence_redoes_the_walk(gdn2):
+    """A steep chunk early in an 80-chunk sequence: the fused walk stops
+    there, and the redo (exact chunks, walk again) still gives the sequential
+    result."""
+    import torch
+    x = make_inputs(1, 80 * 64, 2, 128, 128, io="bf16", seed=44, h0_std=0.05)
+    x.log_alpha[0, 5 * 64 + 2:5 * 64 + 30, :, :8] = -6.0     # chunk 5: ~170 nats in 28 tokens
+    d = to_device(x)
+    shape = (1, 80 * 64, 2, 128, 128)
+    o_s, h_s = _sequential(gdn2, x, d, shape)
+    o_f, h_f, ws, lay = _fused(gdn2, x, d, shape)
+    sync = ws[lay["off_sync"]:].view(torch.int32)
+    assert int(sync[1].item()) == 1
+    assert torch.equal(o_f, o_s) and torch.equal(h_f, h_s)
+    ro, rh = compare(x, o_f.float().cpu().numpy(), h_f.cpu().numpy())
+    assert ro <= TOL["bf16"] and rh <= TOL["bf16"], (ro, rh)
 
 
 def test_fused_steep_chunk_redoes_the_walk(gdn2):
