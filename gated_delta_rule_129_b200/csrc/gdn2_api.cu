@@ -883,11 +883,14 @@ gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_raw, const 
   if (tiles > INT32_MAX || desc->H > 65535) return GDN2_ERR_SHAPE;
   const dim3 grid((unsigned)tiles, (unsigned)desc->H, 3);
   const bool f32 = desc->io == GDN2_IO_F32;
-#define GDN2_PRO(DK_, DV_)                                                                          \
-  if (desc->dk == DK_ && desc->dv == DV_) {                                                         \
-    if (f32) gdn2::token_prologue_kernel<float, DK_, DV_><<<grid, gdn2::kTokThreads, 0, stream>>>(a); \
-    else gdn2::token_prologue_kernel<bf16, DK_, DV_><<<grid, gdn2::kTokThreads, 0, stream>>>(a);      \
-    return launch_status();                                                                         \
+  const bool narrow = conv_width <= 4;
+#define GDN2_PRO(DK_, DV_)                                                                                  \
+  if (desc->dk == DK_ && desc->dv == DV_) {                                                                 \
+    if (f32 && narrow) gdn2::token_prologue_kernel<float, DK_, DV_, 4><<<grid, gdn2::kTokThreads, 0, stream>>>(a); \
+    else if (f32) gdn2::token_prologue_kernel<float, DK_, DV_, 8><<<grid, gdn2::kTokThreads, 0, stream>>>(a);      \
+    else if (narrow) gdn2::token_prologue_kernel<bf16, DK_, DV_, 4><<<grid, gdn2::kTokThreads, 0, stream>>>(a);    \
+    else gdn2::token_prologue_kernel<bf16, DK_, DV_, 8><<<grid, gdn2::kTokThreads, 0, stream>>>(a);                \
+    return launch_status();                                                                                 \
   }
   GDN2_PRO(64, 64)
   GDN2_PRO(64, 128)

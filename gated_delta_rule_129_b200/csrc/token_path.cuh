@@ -98,7 +98,8 @@ struct TokProArgs {
 // copied to shared memory by all threads (16-byte loads, many in flight);
 // then each warp computes its tokens from there, a lane per d/32 channels.
 // A tap that reaches before the token's sequence start reads zero.
-template <typename IO, int D>
+// WM: the taps held in registers (4 for widths up to 4, else 8).
+template <typename IO, int D, int WM>
 __device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float* __restrict__ wt, IO* __restrict__ y,
                                           const TokProArgs& a, int h, int tb, bool l2, uint8_t* smem) {
   constexpr int PER = D / 32;
@@ -119,9 +120,9 @@ __device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float*
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c0 = lane * PER;
-  float tap[kMaxConvWidth][PER];
+  float tap[WM][PER];
 #pragma unroll
-  for (int i = 0; i < kMaxConvWidth; ++i)
+  for (int i = 0; i < WM; ++i)
 #pragma unroll
     for (int e = 0; e < PER; ++e) tap[i][e] = i < W ? s_tap[(c0 + e) * W + i] : 0.f;
   constexpr int PW = TT / (kTokThreads / 32);                // tokens per warp
@@ -130,7 +131,9 @@ __device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float*
   int n, t0, t1;
   seq_bounds(a.cu, a.N, a.T, tw, n, t0, t1);
   t0 = max(t0, 0);
-#pragma unroll
+  // (4 tokens at a time: enough independent work per warp, and a body small
+  // enough for the instruction cache)
+#pragma unroll 4
   for (int u = 0; u < PW; ++u) {
     const int t = tw + u;
     if (t >= a.T_total) break;
@@ -142,7 +145,7 @@ __device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float*
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[e] = 0.f;
 #pragma unroll
-    for (int i = 0; i < kMaxConvWidth; ++i) {
+    for (int i = 0; i < WM; ++i) {
       if (i < W && t - i >= t0) {
         Row<IO, D> r;
         r.load(reinterpret_cast<const IO*>(smem + (t - i - r0) * ROWB) + c0);
@@ -172,20 +175,20 @@ __device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float*
 constexpr int kTokSmem = (tok_tile<float>() + kMaxConvWidth - 1) * 128 * 4 + 128 * kMaxConvWidth * 4;
 
 // grid: (token tiles, H, 3 projections)
-template <typename IO, int DK, int DV>
+template <typename IO, int DK, int DV, int WM>
 __global__ void __launch_bounds__(kTokThreads)
 token_prologue_kernel(const TokProArgs a) {
   __shared__ __align__(16) uint8_t smem[kTokSmem];
   const int tb = blockIdx.x * tok_tile<IO>(), h = blockIdx.y;
   switch (blockIdx.z) {
     case 0:
-      conv_tile<IO, DK>(static_cast<const IO*>(a.q_raw), a.wq, static_cast<IO*>(a.q), a, h, tb, true, smem);
+      conv_tile<IO, DK, WM>(static_cast<const IO*>(a.q_raw), a.wq, static_cast<IO*>(a.q), a, h, tb, true, smem);
       break;
     case 1:
-      conv_tile<IO, DK>(static_cast<const IO*>(a.k_raw), a.wk, static_cast<IO*>(a.k), a, h, tb, true, smem);
+      conv_tile<IO, DK, WM>(static_cast<const IO*>(a.k_raw), a.wk, static_cast<IO*>(a.k), a, h, tb, true, smem);
       break;
     default:
-      conv_tile<IO, DV>(static_cast<const IO*>(a.v_raw), a.wv, static_cast<IO*>(a.v), a, h, tb, false, smem);
+      conv_tile<IO, DV, WM>(static_cast<const IO*>(a.v_raw), a.wv, static_cast<IO*>(a.v), a, h, tb, false, smem);
       break;
   }
 }
