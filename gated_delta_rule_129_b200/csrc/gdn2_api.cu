@@ -673,6 +673,26 @@ gdn2_status check_inputs(const void* q, const void* k, const void* v, const floa
 
 }  // namespace
 
+// one prologue launch with the width d and the tap count W as template
+// arguments (d in {64, 128}, 1 <= W <= 8, both checked by the caller)
+template <typename IO, int D>
+static void launch_prologue_d(int W, const gdn2::TokProArgs& a, dim3 grid, cudaStream_t stream) {
+  switch (W) {
+#define GDN2_PRO_W(W_) \
+  case W_: gdn2::token_prologue_kernel<IO, D, W_><<<grid, gdn2::kTokThreads, 0, stream>>>(a); break;
+    GDN2_PRO_W(1) GDN2_PRO_W(2) GDN2_PRO_W(3) GDN2_PRO_W(4)
+    GDN2_PRO_W(5) GDN2_PRO_W(6) GDN2_PRO_W(7) GDN2_PRO_W(8)
+#undef GDN2_PRO_W
+    default: break;
+  }
+}
+
+template <typename IO>
+static void launch_prologue(int d, int W, const gdn2::TokProArgs& a, dim3 grid, cudaStream_t stream) {
+  if (d == 64) launch_prologue_d<IO, 64>(W, a, grid, stream);
+  else launch_prologue_d<IO, 128>(W, a, grid, stream);
+}
+
 extern "C" {
 
 size_t gdn2_workspace_size(const gdn2_desc* desc) {
@@ -868,36 +888,32 @@ gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_raw, const 
     return GDN2_ERR_ALIGN;
   if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
   if (tokens == 0) return GDN2_OK;
-  gdn2::TokProArgs a;
-  a.q_raw = q_raw; a.k_raw = k_raw; a.v_raw = v_raw;
-  a.wq = conv_q; a.wk = conv_k; a.wv = conv_v;
-  a.W = conv_width;
+  gdn2::TokProArgs a{};
   a.cu = cu_seqlens;
   a.N = packed ? desc->num_seqs : desc->B;
   a.T = desc->T;
   a.T_total = (int)tokens;
   a.H = desc->H;
-  a.q = q; a.k = k; a.v = v;
   const int tile = desc->io == GDN2_IO_F32 ? gdn2::tok_tile<float>() : gdn2::tok_tile<bf16>();
   const long long tiles = (tokens + tile - 1) / tile;
   if (tiles > INT32_MAX || desc->H > 65535) return GDN2_ERR_SHAPE;
-  const dim3 grid((unsigned)tiles, (unsigned)desc->H, 3);
+  // q and k (and v when dv == dk) in one launch, v in a second one otherwise
+  a.x[0] = q_raw; a.wt[0] = conv_q; a.y[0] = q; a.l2[0] = 1;
+  a.x[1] = k_raw; a.wt[1] = conv_k; a.y[1] = k; a.l2[1] = 1;
+  gdn2::TokProArgs av = a;
+  av.x[0] = v_raw; av.wt[0] = conv_v; av.y[0] = v; av.l2[0] = 0;
+  const bool one = desc->dk == desc->dv;
+  if (one) { a.x[2] = v_raw; a.wt[2] = conv_v; a.y[2] = v; a.l2[2] = 0; }
+  const dim3 grid_qk((unsigned)tiles, (unsigned)desc->H, one ? 3 : 2), grid_v((unsigned)tiles, (unsigned)desc->H, 1);
   const bool f32 = desc->io == GDN2_IO_F32;
-  const bool narrow = conv_width <= 4;
-#define GDN2_PRO(DK_, DV_)                                                                                  \
-  if (desc->dk == DK_ && desc->dv == DV_) {                                                                 \
-    if (f32 && narrow) gdn2::token_prologue_kernel<float, DK_, DV_, 4><<<grid, gdn2::kTokThreads, 0, stream>>>(a); \
-    else if (f32) gdn2::token_prologue_kernel<float, DK_, DV_, 8><<<grid, gdn2::kTokThreads, 0, stream>>>(a);      \
-    else if (narrow) gdn2::token_prologue_kernel<bf16, DK_, DV_, 4><<<grid, gdn2::kTokThreads, 0, stream>>>(a);    \
-    else gdn2::token_prologue_kernel<bf16, DK_, DV_, 8><<<grid, gdn2::kTokThreads, 0, stream>>>(a);                \
-    return launch_status();                                                                                 \
+  if (f32) {
+    launch_prologue<float>(desc->dk, conv_width, a, grid_qk, stream);
+    if (!one) launch_prologue<float>(desc->dv, conv_width, av, grid_v, stream);
+  } else {
+    launch_prologue<bf16>(desc->dk, conv_width, a, grid_qk, stream);
+    if (!one) launch_prologue<bf16>(desc->dv, conv_width, av, grid_v, stream);
   }
-  GDN2_PRO(64, 64)
-  GDN2_PRO(64, 128)
-  GDN2_PRO(128, 64)
-  GDN2_PRO(128, 128)
-#undef GDN2_PRO
-  return GDN2_ERR_SHAPE;
+  return launch_status();
 }
 
 gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void* gate, const float* norm_weight,
@@ -914,11 +930,10 @@ gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void
   if (tokens == 0) return GDN2_OK;
   gdn2::TokEpiArgs a;
   a.o = o; a.g = gate; a.weight = norm_weight;
-  a.T_total = (int)tokens;
-  a.H = desc->H;
+  a.rows = tokens * desc->H;
   a.out = out;
-  const long long per_block = (gdn2::kTokThreads / 32) * gdn2::kEpiPairs;
-  const long long blocks = (tokens * desc->H + per_block - 1) / per_block;
+  const long long per_block = gdn2::kTokThreads / 16;          // a row per half-warp
+  const long long blocks = (a.rows + per_block - 1) / per_block;
   if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
   const bool f32 = desc->io == GDN2_IO_F32;
   if (desc->dv == 128) {

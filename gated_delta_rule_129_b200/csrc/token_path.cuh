@@ -12,37 +12,43 @@
 // sequence's start count as zero), of width W <= 8; both norms use eps = 1e-6;
 // the output gate is sigmoid(g), like the erase and write gates.
 //
-// Both kernels are bound by HBM traffic; each lane owns a run of d/32
-// channels (8 or 4 bytes of a bf16 row), fp32 arithmetic, a head's sums of
-// squares by warp shuffles.  The prologue gives each block one head of one
-// projection over a 64-token tile staged in shared memory (with the W - 1
-// rows before it); the epilogue gives each warp one (token, head).
+// Both kernels are bound by HBM traffic and written to issue few
+// instructions per token: fp32 arithmetic, a row of d channels spread over a
+// warp (prologue) or a half-warp (epilogue), a row's sum of squares by
+// shuffles.  The prologue gives each block one head of one projection over a
+// tile of tokens staged in shared memory by asynchronous copies (with the
+// W - 1 rows before it); each warp then walks a run of the tile's tokens with
+// the last W rows of its channels held in registers, so a token costs one
+// shared-memory read and W fused multiply-adds per channel.  The epilogue
+// gives each half-warp one (token, head) row, 16 bytes per lane for bf16.
 #pragma once
 
 #include "common.cuh"
 
 namespace gdn2 {
 
-constexpr int kTokThreads = 256;   // 8 warps, 8 (token, head) pairs per block
+constexpr int kTokThreads = 256;   // 8 warps
 constexpr int kMaxConvWidth = 8;
 constexpr float kTokEps = 1e-6f;
 
-// A lane's run of channels of one row, moved as one vector access (4, 8 or
-// 16 bytes: the run starts at a multiple of its own size).
+// PER consecutive elements of a row, loaded or stored as one or two vector
+// accesses (the run starts at a multiple of its own size, up to 16 bytes).
 template <int BYTES> struct VecT;
 template <> struct VecT<4> { using T = uint32_t; };
 template <> struct VecT<8> { using T = uint2; };
 template <> struct VecT<16> { using T = uint4; };
 
-template <typename IO, int D>
-struct Row {
-  static constexpr int PER = D / 32;   // channels per lane
-  using V = typename VecT<PER * (int)sizeof(IO)>::T;
-  union U { V vec; IO e[PER]; };
+template <typename IO, int PER>
+struct Run {
+  static constexpr int BYTES = PER * (int)sizeof(IO);
+  static constexpr int NV = BYTES > 16 ? BYTES / 16 : 1;   // vector accesses
+  using V = typename VecT<(BYTES > 16 ? 16 : BYTES)>::T;
+  union U { V vec[NV]; IO e[PER]; };
   float v[PER];
   __device__ __forceinline__ void load(const IO* p) {
     U u;
-    u.vec = *reinterpret_cast<const V*>(p);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) u.vec[j] = reinterpret_cast<const V*>(p)[j];
 #pragma unroll
     for (int i = 0; i < PER; ++i) v[i] = to_f32(u.e[i]);
   }
@@ -50,22 +56,30 @@ struct Row {
     U u;
 #pragma unroll
     for (int i = 0; i < PER; ++i) u.e[i] = from_f32<IO>(v[i]);
-    *reinterpret_cast<V*>(p) = u.vec;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) reinterpret_cast<V*>(p)[j] = u.vec[j];
   }
 };
 
-// __expf (the hardware exponential): its relative error, a few fp32 ulp, is
-// far below what the bf16 outputs keep and below the fp32 path's tolerance.
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+// Sigmoid with the hardware exponential and the fast divide: their relative
+// errors, a few fp32 ulp, are far below what the bf16 outputs keep and below
+// the fp32 path's tolerance.  Very negative x gives exp(-x) = inf and 0.
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 __device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
+
+// sum over the 16 lanes of each half-warp
+__device__ __forceinline__ float half_warp_sum(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
 
 // Sequence bookkeeping of the prologue: the sequence that holds token t, as
 // [start, next start).  Packed: the largest n with cu[n] <= t (empty
 // sequences skipped); dense: rows of T.
-__device__ __forceinline__ void seq_bounds(const int32_t* cu, int N, int T, int t, int& n, int& t0, int& t1) {
+__device__ __forceinline__ void seq_bounds(const int32_t* cu, int N, int T, int t, int& t0, int& t1) {
   if (!cu) {
-    n = t / T;
-    t0 = n * T;
+    t0 = (t / T) * T;
     t1 = t0 + T;
     return;
   }
@@ -74,7 +88,6 @@ __device__ __forceinline__ void seq_bounds(const int32_t* cu, int N, int T, int 
     const int mid = (lo + hi + 1) >> 1;
     if (cu[mid] <= t) lo = mid; else hi = mid - 1;
   }
-  n = lo;
   t0 = cu[lo];
   t1 = cu[lo + 1];
 }
@@ -84,154 +97,154 @@ __device__ __forceinline__ void seq_bounds(const int32_t* cu, int N, int T, int 
 template <typename IO>
 constexpr int tok_tile() { return 256 / (int)sizeof(IO); }
 
+// One launch covers up to three projections of the same width d (grid z):
+// q and k (L2-normalised) and v, or q and k alone, or v alone.
 struct TokProArgs {
-  const void *q_raw, *k_raw, *v_raw;
-  const float *wq, *wk, *wv;
-  int W;
+  const void* x[3];     // projections' outputs [T_total, H, d]
+  const float* wt[3];   // taps [H * d, W]
+  void* y[3];           // the operator's inputs [T_total, H, d]
+  int l2[3];            // 1: L2-normalise the row
   const int32_t* cu;
   int N, T, T_total, H;
-  void *q, *k, *v;
 };
 
-// One block: one head of one projection over a tile of tok_tile<IO>() tokens.
-// The tile's rows, the W - 1 rows before it and the head's taps are first
-// copied to shared memory by all threads (16-byte loads, many in flight);
-// then each warp computes its tokens from there, a lane per d/32 channels.
-// A tap that reaches before the token's sequence start reads zero.
-// WM: the taps held in registers (4 for widths up to 4, else 8).
-template <typename IO, int D, int WM>
-__device__ __forceinline__ void conv_tile(const IO* __restrict__ x, const float* __restrict__ wt, IO* __restrict__ y,
-                                          const TokProArgs& a, int h, int tb, bool l2, uint8_t* smem) {
-  constexpr int PER = D / 32;
+// rows of the tile and before it (as many bytes for bf16 and fp32)
+constexpr int kTokSmem = (tok_tile<float>() + kMaxConvWidth - 1) * 128 * 4;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+// grid: (token tiles, H, projections).  One block: one head of one projection
+// over tok_tile<IO>() tokens; D channels, exactly W taps (tap i weighs token
+// t - i; a tap that reaches before the token's sequence start reads zero).
+template <typename IO, int D, int W>
+__global__ void __launch_bounds__(kTokThreads)
+token_prologue_kernel(const TokProArgs a) {
+  constexpr int PER = D / 32;                                // channels per lane
   constexpr int ROWB = D * (int)sizeof(IO);                  // bytes of one row
   constexpr int TT = tok_tile<IO>();
-  const int W = a.W;
+  constexpr int PW = TT / (kTokThreads / 32);                // tokens per warp
+  __shared__ __align__(16) uint8_t smem[kTokSmem];
+  const int z = blockIdx.z, h = blockIdx.y, tb = blockIdx.x * TT;
+  // (selects, not an index: a dynamic index would copy the arguments to local memory)
+  const IO* __restrict__ x = static_cast<const IO*>(z == 0 ? a.x[0] : z == 1 ? a.x[1] : a.x[2]);
   const int r0 = tb - (W - 1);                               // first row held
   const int nrows = min(a.T_total, tb + TT) - r0;
-  float* s_tap = reinterpret_cast<float*>(smem + (TT + kMaxConvWidth - 1) * ROWB);   // [D][W]
-  for (int i = threadIdx.x; i < D * W; i += kTokThreads) s_tap[i] = wt[(size_t)h * D * W + i];
-  // copy rows [r0, r0 + nrows) of head h (rows before 0 left out)
+  // stage rows [r0, r0 + nrows) of head h (rows before 0 left out), all in flight at once
   for (int i = threadIdx.x; i < nrows * (ROWB / 16); i += kTokThreads) {
     const int r = i / (ROWB / 16), u = i % (ROWB / 16);
     if (r0 + r >= 0)
-      reinterpret_cast<uint4*>(smem + r * ROWB)[u] =
-          *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(x + ((size_t)(r0 + r) * a.H + h) * D) + u * 16);
+      cp_async16(smem + r * ROWB + u * 16,
+                 reinterpret_cast<const uint8_t*>(x + ((size_t)(r0 + r) * a.H + h) * D) + u * 16);
   }
-  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c0 = lane * PER;
-  float tap[WM][PER];
+  // the lane's taps: PER * W consecutive floats of the [H * d, W] table
+  float tap[W][PER];
+  {
+    const float* wp = (z == 0 ? a.wt[0] : z == 1 ? a.wt[1] : a.wt[2]) + ((size_t)h * D + c0) * W;
 #pragma unroll
-  for (int i = 0; i < WM; ++i)
+    for (int e = 0; e < PER; ++e)
 #pragma unroll
-    for (int e = 0; e < PER; ++e) tap[i][e] = i < W ? s_tap[(c0 + e) * W + i] : 0.f;
-  constexpr int PW = TT / (kTokThreads / 32);                // tokens per warp
-  const int tw = tb + warp * PW;
-  if (tw >= a.T_total) return;
-  int n, t0, t1;
-  seq_bounds(a.cu, a.N, a.T, tw, n, t0, t1);
-  t0 = max(t0, 0);
-  // (4 tokens at a time: enough independent work per warp, and a body small
-  // enough for the instruction cache)
+      for (int i = 0; i < W; ++i) tap[i][e] = wp[e * W + i];
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int ts = tb + warp * PW;                             // the warp's first token
+  if (ts >= a.T_total) return;
+  const bool l2 = (z == 0 ? a.l2[0] : z == 1 ? a.l2[1] : a.l2[2]) != 0;
+  IO* __restrict__ y = static_cast<IO*>(z == 0 ? a.y[0] : z == 1 ? a.y[1] : a.y[2]);
+  int t0, t1;
+  seq_bounds(a.cu, a.N, a.T, ts, t0, t1);
+  // win[i]: channels of row t - i for the current token t
+  float win[W][PER];
+#pragma unroll
+  for (int i = 1; i < W; ++i) {
+    if (ts - i >= t0) {
+      Run<IO, PER> r;
+      r.load(reinterpret_cast<const IO*>(smem + (ts - i - r0) * ROWB) + c0);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) win[i][e] = r.v[e];
+    } else {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) win[i][e] = 0.f;
+    }
+  }
 #pragma unroll 4
   for (int u = 0; u < PW; ++u) {
-    const int t = tw + u;
+    const int t = ts + u;
     if (t >= a.T_total) break;
-    if (t >= t1) {
-      seq_bounds(a.cu, a.N, a.T, t, n, t0, t1);
-      t0 = max(t0, 0);
+    if (t >= t1) {                                           // a sequence starts at t
+      seq_bounds(a.cu, a.N, a.T, t, t0, t1);
+#pragma unroll
+      for (int i = 1; i < W; ++i)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) win[i][e] = 0.f;
     }
-    float acc[PER];
+    {
+      Run<IO, PER> r;
+      r.load(reinterpret_cast<const IO*>(smem + (t - r0) * ROWB) + c0);
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int i = 0; i < WM; ++i) {
-      if (i < W && t - i >= t0) {
-        Row<IO, D> r;
-        r.load(reinterpret_cast<const IO*>(smem + (t - i - r0) * ROWB) + c0);
-#pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] = fmaf(tap[i][e], r.v[e], acc[e]);
-      }
+      for (int e = 0; e < PER; ++e) win[0][e] = r.v[e];
     }
+    Run<IO, PER> o;
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
-      acc[e] = silu_f(acc[e]);
-      ss = fmaf(acc[e], acc[e], ss);
+      float acc = tap[0][e] * win[0][e];
+#pragma unroll
+      for (int i = 1; i < W; ++i) acc = fmaf(tap[i][e], win[i][e], acc);
+      o.v[e] = silu_f(acc);
+      ss = fmaf(o.v[e], o.v[e], ss);
     }
     if (l2) {
       const float rn = rsqrtf(warp_sum(ss) + kTokEps);
 #pragma unroll
-      for (int e = 0; e < PER; ++e) acc[e] *= rn;
+      for (int e = 0; e < PER; ++e) o.v[e] *= rn;
     }
-    Row<IO, D> o;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) o.v[e] = acc[e];
     o.store(y + ((size_t)t * a.H + h) * D + c0);
-  }
-}
-
-// rows of the tile and before it (as many bytes for bf16 and fp32), then the taps
-constexpr int kTokSmem = (tok_tile<float>() + kMaxConvWidth - 1) * 128 * 4 + 128 * kMaxConvWidth * 4;
-
-// grid: (token tiles, H, 3 projections)
-template <typename IO, int DK, int DV, int WM>
-__global__ void __launch_bounds__(kTokThreads)
-token_prologue_kernel(const TokProArgs a) {
-  __shared__ __align__(16) uint8_t smem[kTokSmem];
-  const int tb = blockIdx.x * tok_tile<IO>(), h = blockIdx.y;
-  switch (blockIdx.z) {
-    case 0:
-      conv_tile<IO, DK, WM>(static_cast<const IO*>(a.q_raw), a.wq, static_cast<IO*>(a.q), a, h, tb, true, smem);
-      break;
-    case 1:
-      conv_tile<IO, DK, WM>(static_cast<const IO*>(a.k_raw), a.wk, static_cast<IO*>(a.k), a, h, tb, true, smem);
-      break;
-    default:
-      conv_tile<IO, DV, WM>(static_cast<const IO*>(a.v_raw), a.wv, static_cast<IO*>(a.v), a, h, tb, false, smem);
-      break;
+#pragma unroll
+    for (int i = W - 1; i > 0; --i)
+#pragma unroll
+      for (int e = 0; e < PER; ++e) win[i][e] = win[i - 1][e];
   }
 }
 
 struct TokEpiArgs {
   const void *o, *g;
   const float* weight;   // [dv]
-  int T_total, H;
+  long long rows;        // T_total * H
   void* out;
 };
 
-constexpr int kEpiPairs = 1;   // (token, head) pairs per warp in the epilogue
-
+// grid: ceil(rows / 16); one (token, head) row of DV channels per half-warp,
+// DV / 16 channels per lane.
 template <typename IO, int DV>
 __global__ void __launch_bounds__(kTokThreads)
 token_epilogue_kernel(const TokEpiArgs a) {
-  constexpr int PER = DV / 32;
-  const int lane = threadIdx.x & 31;
-  const long long p0 = ((long long)blockIdx.x * (kTokThreads / 32) + (threadIdx.x >> 5)) * kEpiPairs;
-  const long long np = (long long)a.T_total * a.H;
+  constexpr int PER = DV / 16;
+  const int l16 = threadIdx.x & 15;
+  const long long row = (long long)blockIdx.x * (kTokThreads / 16) + (threadIdx.x >> 4);
+  const bool live = row < a.rows;                            // shuffles below stay warp-wide
+  const size_t base = (size_t)(live ? row : 0) * DV + l16 * PER;
+  Run<IO, PER> o, g;
+  o.load(static_cast<const IO*>(a.o) + base);
+  g.load(static_cast<const IO*>(a.g) + base);
   float wt[PER];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) wt[e] = a.weight[lane * PER + e];
-  Row<IO, DV> o[kEpiPairs], g[kEpiPairs];
+  for (int e = 0; e < PER; ++e) wt[e] = a.weight[l16 * PER + e];
+  float ss = 0.f;
 #pragma unroll
-  for (int u = 0; u < kEpiPairs; ++u) {
-    if (p0 + u < np) {
-      const size_t base = (size_t)(p0 + u) * DV + lane * PER;
-      o[u].load(static_cast<const IO*>(a.o) + base);
-      g[u].load(static_cast<const IO*>(a.g) + base);
-    }
-  }
+  for (int e = 0; e < PER; ++e) ss = fmaf(o.v[e], o.v[e], ss);
+  const float r = rsqrtf(half_warp_sum(ss) * (1.f / DV) + kTokEps);
 #pragma unroll
-  for (int u = 0; u < kEpiPairs; ++u) {
-    if (p0 + u >= np) break;
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) ss = fmaf(o[u].v[e], o[u].v[e], ss);
-    const float r = rsqrtf(warp_sum(ss) * (1.f / DV) + kTokEps);
-#pragma unroll
-    for (int e = 0; e < PER; ++e) o[u].v[e] = o[u].v[e] * r * wt[e] * sigmoid_f(g[u].v[e]);
-    o[u].store(static_cast<IO*>(a.out) + (size_t)(p0 + u) * DV + lane * PER);
-  }
+  for (int e = 0; e < PER; ++e) o.v[e] = o.v[e] * r * wt[e] * sigmoid_f(g.v[e]);
+  if (live) o.store(static_cast<IO*>(a.out) + base);
 }
 
 }  // namespace gdn2

@@ -3,9 +3,11 @@ gdn2_token_epilogue), through the C ABI, against the fp64 oracle
 (oracle/token_path.py):
   * the prologue's q, k, v for dense and packed rows (sequence starts reset
     the convolution; empty and one-token sequences), dk / dv 64 and 128,
-    widths 1 and 4, fp32 I/O (rel-L2 <= 1e-5) and bf16 I/O (<= 1e-2: one
+    every width 1..8 (each its own kernel), tiles with sequence starts
+    inside a warp's run of tokens, fp32 I/O (rel-L2 <= 1e-5) and bf16 I/O (<= 1e-2: one
     bf16 rounding of the result);
-  * the epilogue likewise, and in place (out = o);
+  * the epilogue likewise (row counts that leave a block part-filled), and
+    in place (out = o);
   * the whole path (prologue, operator, epilogue) against the oracles chained,
     at the operator's bf16 bar.
 """
@@ -45,7 +47,10 @@ def _dev(a, dt):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
-@pytest.mark.parametrize("dk,dv,W,lengths", [(128, 128, 4, None), (64, 128, 1, None), (128, 64, 4, [9, 0, 1, 70])])
+@pytest.mark.parametrize("dk,dv,W,lengths", [(128, 128, 4, None), (64, 128, 1, None), (128, 64, 4, [9, 0, 1, 70]),
+                                             (128, 128, 3, [200, 17, 0, 90]), (64, 64, 8, [5, 1, 300, 0]),
+                                             (128, 128, 6, None), (64, 128, 2, [130, 7]), (128, 64, 5, None),
+                                             (128, 128, 7, [3, 140])])
 def test_prologue_matches_oracle(gdn2, io, dk, dv, W, lengths):
     import torch
     T = sum(lengths) if lengths else 50
@@ -66,11 +71,12 @@ def test_prologue_matches_oracle(gdn2, io, dk, dv, W, lengths):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("dv", [64, 128])
-def test_epilogue_matches_oracle(gdn2, io, dv):
+@pytest.mark.parametrize("shape", [(2, 40, 3), (1, 37, 3)])
+def test_epilogue_matches_oracle(gdn2, io, dv, shape):
     import torch
     rng = np.random.default_rng(82)
-    o = rng.standard_normal((2, 40, 3, dv)).astype(np.float32)
-    g = rng.standard_normal((2, 40, 3, dv)).astype(np.float32)
+    o = rng.standard_normal((*shape, dv)).astype(np.float32)
+    g = rng.standard_normal((*shape, dv)).astype(np.float32)
     if io == "bf16":
         o, g = round_bf16(o), round_bf16(g)
     wt = rng.uniform(0.5, 1.5, dv).astype(np.float32)
