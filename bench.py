@@ -422,8 +422,8 @@ def measure_decode(dev, stream, flush, reps=20):
 
 
 def measure_backward(dev, stream, hbm, reps=3):
-    """gdn2_chunk_bwd (the gradients of every input, a CUDA-core baseline) on
-    the 16K x 1 workload with a random bf16 dO.  Its algorithmic traffic per
+    """gdn2_chunk_bwd (the gradients of every input through the chunkwise WY
+    form, fp32 on the CUDA cores) on the 16K x 1 workload with a random bf16 dO.  Its algorithmic traffic per
     token-head: the inputs (768 + 1536 B), dO (256 B) and the six fp32
     gradients (4 x 512 + 2 x 512 B), plus dh0."""
     import torch
@@ -449,7 +449,8 @@ def measure_backward(dev, stream, hbm, reps=3):
     ms = tot / reps
     alg = TH * (768 + 1536 + 256 + 6 * 512) + B * H * DK * DV * 4
     gbs = alg / (ms / 1e3) / 1e9
-    return {"workload": "16Kx1 backward (gdn2_chunk_bwd, CUDA-core baseline), bf16 inputs, fp32 gradients",
+    return {"workload": "16Kx1 backward (gdn2_chunk_bwd: chunkwise WY form, fp32 on the CUDA cores), bf16 inputs, "
+                        "fp32 gradients",
             "ms": ms, "tokens_per_s": B * T / (ms / 1e3), "alg_bytes": alg,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
 

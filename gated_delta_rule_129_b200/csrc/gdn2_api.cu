@@ -13,7 +13,7 @@
 #include <cstring>
 #include <type_traits>
 
-#include "bwd_simt.cuh"
+#include "bwd_chunk.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "plan.cuh"
@@ -228,6 +228,8 @@ gdn2::PrepArgs<IO, FT> prep_args(const gdn2_desc* d, const Layout& L, const void
   a.Mp = at<FT>(d->workspace, L.l.off_Mp);
   a.Nc = at<FT>(d->workspace, L.l.off_Nc);
   a.colscale = L.l.factor_set == 1 ? at<float>(d->workspace, L.l.off_colscale) : nullptr;
+  a.Tm = nullptr;
+  a.Pm = nullptr;
   return a;
 }
 
@@ -522,59 +524,136 @@ struct DecodeOp {
 };
 
 // ------------------------------------------------------------- backward ----
-// Workspace of gdn2_chunk_bwd: the status word, then one fp32 state per
-// (checkpoint slot, head); a sequence's chunk m uses slot seq_begin / 64 + m + n,
-// so T_total / 64 + N + 1 slots cover every sequence without overlap.
-gdn2_status bwd_layout(const gdn2_desc* d, bool packed, size_t* total, size_t* off_ckpt) {
-  gdn2_status st = check_dims(d, packed);
+// Workspace of gdn2_chunk_bwd: the status word; the forward's fp32 WY factor
+// set (the layout gdn2_chunk_fwd uses for fp32 I/O, whatever the I/O type of
+// the call), with its chunk map; T and P of every (chunk, head); the state at
+// every chunk start (S0); the gradient reaching every chunk's end (dS1).
+struct BwdLayout {
+  Layout f;            // the factor set, relative to the workspace + kAlign
+  size_t off_T, off_P, off_S0, off_dS1, total;   // from the workspace start
+};
+
+gdn2_desc bwd_factor_desc(const gdn2_desc* d) {
+  gdn2_desc f = *d;
+  f.io = GDN2_IO_F32;
+  f.workspace = d->workspace ? static_cast<char*>(d->workspace) + kAlign : nullptr;
+  f.workspace_bytes = d->workspace_bytes > kAlign ? d->workspace_bytes - kAlign : 0;
+  return f;
+}
+
+gdn2_status bwd_layout(const gdn2_desc* d, bool packed, BwdLayout* B) {
+  const gdn2_desc f = bwd_factor_desc(d);
+  gdn2_status st = make_layout(&f, packed, &B->f);
   if (st != GDN2_OK) return st;
-  const long long N = packed ? d->num_seqs : d->B;
-  const long long slots = (long long)d->B * d->T / kChunk + N + 1;
-  *off_ckpt = kAlign;
-  *total = kAlign + align_up((size_t)slots * d->H * d->dk * d->dv * sizeof(float));
+  const size_t chunks_h = (size_t)B->f.l.max_chunks * d->H;
+  size_t off = kAlign + B->f.l.total_bytes;
+  B->off_T = off;   off = align_up(off + chunks_h * kChunk * kChunk * sizeof(float));
+  B->off_P = off;   off = align_up(off + chunks_h * kChunk * kChunk * sizeof(float));
+  B->off_S0 = off;  off = align_up(off + chunks_h * d->dk * d->dv * sizeof(float));
+  B->off_dS1 = off; off = align_up(off + chunks_h * d->dk * d->dv * sizeof(float));
+  B->total = off;
   return GDN2_OK;
 }
 
 template <int DK, int DV, typename IO, typename FT>
 struct BwdOp {
-  static gdn2_status run(const gdn2_desc* d, int N, const void* q, const void* k, const void* v, const float* la,
-                         const float* b, const float* w, float scale, const float* h0, const int32_t* cu,
-                         const void* dO, const float* dhT, float* dq, float* dk, float* dv, float* dla, float* db,
-                         float* dw, float* dh0, int* status, float* ckpt, cudaStream_t s) {
-    gdn2::BwdArgs<IO> a;
-    a.q = static_cast<const IO*>(q);
-    a.k = static_cast<const IO*>(k);
-    a.v = static_cast<const IO*>(v);
-    a.dO = static_cast<const IO*>(dO);
-    a.la = la;
-    a.b = b;
-    a.w = w;
-    a.h0 = h0;
-    a.dhT = dhT;
-    a.cu = cu;
-    a.N = N;
-    a.T = d->T;
-    a.T_total = d->B * d->T;
-    a.H = d->H;
-    a.scale = scale;
-    a.ckpt = ckpt;
-    a.dq = dq;
-    a.dk = dk;
-    a.dla = dla;
-    a.db = db;
-    a.dv = dv;
-    a.dw = dw;
-    a.dh0 = dh0;
-    a.status = status;
-    a.seqlens_err = (int)GDN2_ERR_SEQLENS;
-    const long long blocks = (long long)N * d->H * (DV / gdn2::kBwdCols);
-    if (blocks == 0) return GDN2_OK;
-    if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
-    constexpr size_t smem = (size_t)gdn2::bwd_smem_floats<DK, DV>() * sizeof(float);
-    auto kern = gdn2::bwd_simt_kernel<DK, DV, IO>;
+  static gdn2_status run(const gdn2_desc* d, const BwdLayout& B, const void* q, const void* k, const void* v,
+                         const float* la, const float* b, const float* w, float scale, const float* h0,
+                         const int32_t* cu, const void* dO, const float* dhT, float* dq, float* dk, float* dv,
+                         float* dla, float* db, float* dw, float* dh0, cudaStream_t s) {
+    const gdn2_desc f = bwd_factor_desc(d);
+    const Layout& L = B.f;
+    int32_t* status = at<int32_t>(d->workspace, 0);
+    // chunk map (and the check of cu_seqlens, into the status word)
+    gdn2::plan_kernel<<<1, gdn2::kPlanThreads, 0, s>>>(cu, L.N, d->T, d->B * d->T,
+                                                        at<int32_t>(f.workspace, L.l.off_chunk_offsets), status,
+                                                        (int)GDN2_ERR_SEQLENS, nullptr, nullptr, 0);
+    gdn2_status st = launch_status();
+    if (st != GDN2_OK) return st;
+    const gdn2::SeqMap map = seq_map(&f, L, cu);
+    // 1. factors, T and P in fp32
+    if (L.l.max_chunks > 0) {
+      auto pa = prep_args<DK, DV, IO, float>(&f, L, q, k, v, la, b, w, cu);
+      pa.Tm = at<float>(d->workspace, B.off_T);
+      pa.Pm = at<float>(d->workspace, B.off_P);
+      constexpr size_t smem = gdn2::prep_simt_smem_bytes<DK, DV>();
+      auto kern = gdn2::prep_simt_kernel<DK, DV, IO, float, false>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+      kern<<<dim3(L.l.max_chunks, d->H), gdn2::kPrepSimtThreads, smem, s>>>(pa);
+      if ((st = launch_status()) != GDN2_OK) return st;
+    }
+    if (L.N == 0) return GDN2_OK;
+    // 2. the state at every chunk start
+    {
+      gdn2::WalkArgs<IO, float> wa;
+      wa.W = at<const float>(f.workspace, L.l.off_W);
+      wa.Ut = at<const float>(f.workspace, L.l.off_Ut);
+      wa.Kbar = at<const float>(f.workspace, L.l.off_Kbar);
+      wa.Qeff = at<const float>(f.workspace, L.l.off_Qeff);
+      wa.Opart = at<const float>(f.workspace, L.l.off_Opart);
+      wa.gamma_last = at<const float>(f.workspace, L.l.off_gamma_last);
+      wa.map = map;
+      wa.H = d->H;
+      wa.scale = scale;
+      wa.h0 = h0;
+      wa.out = nullptr;
+      wa.hT = nullptr;
+      wa.chunk_states = at<float>(d->workspace, B.off_S0);
+      constexpr size_t smem = gdn2::walk_simt_smem_bytes<DK, DV>();
+      auto kern = gdn2::walk_simt_kernel<DK, DV, IO, float>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+      const long long blocks = (long long)L.N * d->H * (DV / gdn2::kWalkSimtDVS);
+      if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+      kern<<<(unsigned)blocks, gdn2::kWalkSimtThreads, smem, s>>>(wa);
+      if ((st = launch_status()) != GDN2_OK) return st;
+    }
+    // 3. the gradient reaching every chunk's end state, and dh0
+    {
+      gdn2::BwdStateArgs ra;
+      ra.W = at<const float>(f.workspace, L.l.off_W);
+      ra.Kbar = at<const float>(f.workspace, L.l.off_Kbar);
+      ra.Qeff = at<const float>(f.workspace, L.l.off_Qeff);
+      ra.gamma_last = at<const float>(f.workspace, L.l.off_gamma_last);
+      ra.dO = dO;
+      ra.map = map;
+      ra.H = d->H;
+      ra.scale = scale;
+      ra.dhT = dhT;
+      ra.dS1 = at<float>(d->workspace, B.off_dS1);
+      ra.dh0 = dh0;
+      ra.status = status;
+      constexpr size_t smem = gdn2::bwd_dstate_smem_bytes<DK>();
+      auto kern = gdn2::bwd_dstate_kernel<DK, DV, IO>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+      const long long blocks = (long long)L.N * d->H * (DV / gdn2::kBwdWalkCols);
+      if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
+      kern<<<(unsigned)blocks, gdn2::kBwdWalkThreads, smem, s>>>(ra);
+      if ((st = launch_status()) != GDN2_OK) return st;
+    }
+    // 4. every (chunk, head): the gradients of its tokens
+    if (L.l.max_chunks == 0) return GDN2_OK;
+    gdn2::BwdChunkArgs ca;
+    ca.q = q; ca.k = k; ca.v = v; ca.dO = dO;
+    ca.la = la; ca.b = b; ca.w = w;
+    ca.W = at<const float>(f.workspace, L.l.off_W);
+    ca.Ut = at<const float>(f.workspace, L.l.off_Ut);
+    ca.Kbar = at<const float>(f.workspace, L.l.off_Kbar);
+    ca.Tm = at<const float>(d->workspace, B.off_T);
+    ca.Pm = at<const float>(d->workspace, B.off_P);
+    ca.S0 = at<const float>(d->workspace, B.off_S0);
+    ca.dS1 = at<const float>(d->workspace, B.off_dS1);
+    ca.map = map;
+    ca.H = d->H;
+    ca.scale = scale;
+    ca.dq = dq; ca.dk = dk; ca.dla = dla; ca.db = db; ca.dv = dv; ca.dw = dw;
+    constexpr size_t smem = gdn2::BwdCfg<DK, DV>::SMEM;
+    auto kern = gdn2::bwd_chunk_kernel<DK, DV, IO>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return GDN2_ERR_CUDA;
-    kern<<<(unsigned)blocks, DK, smem, s>>>(a);
+    kern<<<dim3(L.l.max_chunks, d->H), gdn2::kBwdThreads, smem, s>>>(ca);
     return launch_status();
   }
 };
@@ -981,9 +1060,9 @@ int gdn2_version(void) { return 100; }
 
 size_t gdn2_backward_workspace_size(const gdn2_desc* desc) {
   if (!desc) return 0;
-  size_t total = 0, off = 0;
-  if (bwd_layout(desc, desc->num_seqs > 0, &total, &off) != GDN2_OK) return 0;
-  return total;
+  BwdLayout B;
+  if (bwd_layout(desc, desc->num_seqs > 0, &B) != GDN2_OK) return 0;
+  return B.total;
 }
 
 gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
@@ -992,14 +1071,13 @@ gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, 
                            float* dv, float* dlog_alpha, float* db, float* dw, float* dh0, cudaStream_t stream) {
   if (!desc) return GDN2_ERR_NULL;
   const bool packed = cu_seqlens != nullptr;
-  size_t total = 0, off_ckpt = 0;
-  gdn2_status st = bwd_layout(desc, packed, &total, &off_ckpt);
+  BwdLayout B;
+  gdn2_status st = bwd_layout(desc, packed, &B);
   if (st != GDN2_OK) return st;
   if (!desc->workspace) return GDN2_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(desc->workspace) & (kAlign - 1)) != 0) return GDN2_ERR_ALIGN;
-  if (desc->workspace_bytes < total) return GDN2_ERR_WORKSPACE;
+  if (desc->workspace_bytes < B.total) return GDN2_ERR_WORKSPACE;
   const long long tokens = (long long)desc->B * desc->T;
-  const int N = packed ? desc->num_seqs : desc->B;
   if ((st = check_inputs(q, k, v, log_alpha, b, w, tokens)) != GDN2_OK) return st;
   if (tokens > 0 && (!dO || !dq || !dk || !dv || !dlog_alpha || !db || !dw)) return GDN2_ERR_NULL;
   if (!dh0) return GDN2_ERR_NULL;
@@ -1008,21 +1086,20 @@ gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, 
     return GDN2_ERR_ALIGN;
   if (!device_ok()) return GDN2_ERR_UNSUPPORTED;
   int* status = at<int32_t>(desc->workspace, 0);
-  const size_t kbytes = (size_t)tokens * desc->H * desc->dk * sizeof(float);
-  const size_t vbytes = (size_t)tokens * desc->H * desc->dv * sizeof(float);
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), stream) != cudaSuccess) return GDN2_ERR_CUDA;
-  if (tokens > 0) {
-    // the key-side gradients are sums over every CTA of a head; the
-    // value-side ones are cleared too, so tokens outside every sequence of a
-    // malformed cu_seqlens read as zero
-    float* zero_k[4] = {dq, dk, dlog_alpha, db};
-    for (float* p : zero_k)
+  if (packed && tokens > 0) {
+    // every token of a well-formed packing belongs to one chunk, which writes
+    // all of its gradients; a malformed one leaves the chunk map empty, and
+    // the gradients must then read as zero
+    const size_t kbytes = (size_t)tokens * desc->H * desc->dk * sizeof(float);
+    const size_t vbytes = (size_t)tokens * desc->H * desc->dv * sizeof(float);
+    for (float* p : {dq, dk, dlog_alpha, db})
       if (cudaMemsetAsync(p, 0, kbytes, stream) != cudaSuccess) return GDN2_ERR_CUDA;
-    if (cudaMemsetAsync(dv, 0, vbytes, stream) != cudaSuccess || cudaMemsetAsync(dw, 0, vbytes, stream) != cudaSuccess)
-      return GDN2_ERR_CUDA;
+    for (float* p : {dv, dw})
+      if (cudaMemsetAsync(p, 0, vbytes, stream) != cudaSuccess) return GDN2_ERR_CUDA;
   }
-  return dispatch<BwdOp>(desc, N, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens, dO, dhT, dq, dk, dv, dlog_alpha,
-                         db, dw, dh0, status, at<float>(desc->workspace, off_ckpt), stream);
+  return dispatch<BwdOp>(desc, B, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens, dO, dhT, dq, dk, dv, dlog_alpha,
+                         db, dw, dh0, stream);
 }
 
 }  // extern "C"

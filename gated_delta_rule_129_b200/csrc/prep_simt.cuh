@@ -42,6 +42,8 @@ struct PrepArgs {
   float* colscale;   // affine set: column scale of Mp and Q_eff (1 here: stored unscaled)
   FT* Mp;  // affine factor set only: Kbar^T W   [., H, DK, DK]
   FT* Nc;  // affine factor set only: Kbar^T U~  [., H, DK, DV]
+  float* Tm;  // optional (the backward's recompute): T = (I + A)^-1  [., H, 64, 64]
+  float* Pm;  // optional: P, zero above the diagonal                 [., H, 64, 64]
 };
 
 constexpr int kPrepSimtThreads = 256;
@@ -181,6 +183,29 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     for (int j = 0; j <= i && j < len; ++j) acc = fmaf(sP[i * LA + j], sz[j * LV + cc], acc);
     a.Opart[tile_v + idx] = from_f32<FT>(acc);
     if constexpr (!AFFINE) a.Ut[tile_v + idx] = from_f32<FT>(sz[i * LV + cc]);
+  }
+  if (a.Tm) {
+    // T = (I + A)^-1 explicitly, for the backward: rows in order, each row's
+    // entries from the rows above it (T_ij = -A_ij - sum_{j<m<i} A_im T_mj),
+    // written over A once every thread has read the row (unit diagonal and
+    // zero upper part implied).  A is no longer needed for the factors.
+    __syncthreads();
+    for (int i = 1; i < len; ++i) {
+      float acc = 0.f;
+      if (tid < i) {
+        acc = -sA[i * LA + tid];
+        for (int m = tid + 1; m < i; ++m) acc = fmaf(-sA[i * LA + m], sA[m * LA + tid], acc);
+      }
+      __syncthreads();
+      if (tid < i) sA[i * LA + tid] = acc;
+      __syncthreads();
+    }
+    const size_t tile_t = ((size_t)c * H + h) * kChunk * kChunk;
+    for (int idx = tid; idx < kChunk * kChunk; idx += kPrepSimtThreads) {
+      const int i = idx / kChunk, j = idx % kChunk;
+      a.Tm[tile_t + idx] = j < i ? sA[i * LA + j] : (i == j ? 1.f : 0.f);
+      a.Pm[tile_t + idx] = j <= i ? sP[i * LA + j] : 0.f;
+    }
   }
   if constexpr (AFFINE) {
     // The chunk's affine state map: S' = diag(gamma) S - Mp S + Nc with

@@ -29,7 +29,7 @@ struct WalkArgs {
   int H;
   float scale;
   const float* h0;
-  IO* out;
+  IO* out;              // nullptr: states only (the backward's recompute)
   float* hT;
   float* chunk_states;  // optional [max_chunks, H, DK, DV]
 };
@@ -106,7 +106,7 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
         o = fmaf(sQe[i * LK + cc], s, o);
       }
       sU[idx] = u;
-      if (i < len) a.out[((size_t)(t0 + i) * H + h) * DV + j0 + j] = from_f32<IO>(a.scale * o);
+      if (a.out && i < len) a.out[((size_t)(t0 + i) * H + h) * DV + j0 + j] = from_f32<IO>(a.scale * o);
     }
     __syncthreads();
     for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads) {

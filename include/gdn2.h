@@ -304,27 +304,35 @@ GDN2_API gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale,
                                              unsigned long long wait_budget_ns, cudaStream_t stream);
 
 /* Bytes of workspace gdn2_chunk_bwd needs for `desc` (0 if desc is invalid):
- * a status word and one fp32 dk x dv state per head for every 64-token chunk
- * start (T_total / 64 + sequences + 1 of them). */
+ * a status word, the fp32 chunk factors of the forward (W, U~, Kbar, Q_eff,
+ * O_part, gamma_n, the chunk map), T and P of every (chunk, head), and two
+ * fp32 dk x dv states per (chunk, head): the forward state at the chunk's
+ * start and the gradient reaching its end. */
 GDN2_API size_t gdn2_backward_workspace_size(const gdn2_desc* desc);
 
 /* Gradients of gdn2_chunk_fwd's outputs: given dO (the gradient of out) and
- * dhT (of hT), the gradients of every input.  Reverse mode through the token
- * recurrence (page "Gated DeltaNet-2：将擦除与写入分开", section
- * "在两个维度上独立控制"; the pages train with the operator, section
- * "词元路径与并行训练"), fp32 on the CUDA cores: per (sequence, head) the
- * forward states at every 64-token chunk start are stored in the workspace,
- * and each chunk's token states are recomputed from there on the way back.
+ * dhT (of hT), the gradients of every input, through the 64-token chunk form
+ * (page "Gated DeltaNet-2：将擦除与写入分开", section "词元路径与并行训练":
+ * the operator is trained chunk by chunk, its gradients flowing through the
+ * gated keys and values; the update is the one of section "在两个维度上独立控制"),
+ * fp32 on the CUDA cores for both I/O types:
+ *   1. the chunk factors, T = (I + A)^-1 and P are recomputed in fp32;
+ *   2. the forward state at every chunk start is recomputed;
+ *   3. the chunks are walked in reverse: the gradient reaching a chunk's
+ *      start state is dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO
+ *      (dS1 of a sequence's last chunk is dhT; dh0 is dS0 of its first);
+ *   4. every (chunk, head) then gives its tokens' gradients from its start
+ *      state, the gradient at its end and dO, independently of the others.
  * desc, q, k, v, log_alpha, b, w, scale, h0, cu_seqlens: as for
  *   gdn2_chunk_fwd (the same call's inputs); desc->workspace holds at least
  *   gdn2_backward_workspace_size(desc) bytes, 256-byte aligned;
  * dO  : [B, T, H, dv] io dtype;  dhT : [N, H, dk, dv] fp32, NULL = zero;
  * dq, dk, dlog_alpha, db : [B, T, H, dk] fp32;  dv, dw : [B, T, H, dv] fp32;
  * dh0 : [N, H, dk, dv] fp32 (the gradient of h0, also when h0 is NULL).
- * Every gradient is written (the call clears them on `stream` first).
- * Device pointers, 16-byte aligned, owned by the caller.  A malformed
- * cu_seqlens sets GDN2_ERR_SEQLENS in the workspace's first int32 and leaves
- * the gradients of the affected sequences zero; nothing outside the arrays is
+ * Every gradient is written (for packed rows the call clears them on
+ * `stream` first).  Device pointers, 16-byte aligned, owned by the caller.
+ * A malformed cu_seqlens sets GDN2_ERR_SEQLENS in the workspace's first
+ * int32 and leaves every gradient zero; nothing outside the arrays is
  * touched.  Asynchronous on `stream`. */
 GDN2_API gdn2_status gdn2_chunk_bwd(const gdn2_desc* desc, const void* q, const void* k, const void* v,
                                     const float* log_alpha, const float* b, const float* w, float scale,
