@@ -66,31 +66,42 @@ struct BwdStateArgs {
   const int32_t* status;          // nonzero: malformed cu_seqlens (no chunks); dh0 = 0
 };
 
+// Shared memory, in bytes: two chunk buffers (W, Kbar, Q_eff rows padded by
+// 16 bytes, the dO slice, gamma_n), then dS [DK][CS] and X = Kbar dS [64][CS]
+// in fp32.
+template <int DK, typename IO>
+struct BwdDstateCfg {
+  static constexpr int CS = kBwdWalkCols, LK = DK + 4;
+  static constexpr int TILE = kChunk * LK * 4, DOB = kChunk * CS * (int)sizeof(IO);
+  static constexpr int OFF_W = 0, OFF_KB = TILE, OFF_QE = 2 * TILE, OFF_DO = 3 * TILE, OFF_GL = OFF_DO + DOB,
+                       BUF = OFF_GL + DK * 4;
+  static constexpr int OFF_S = 2 * BUF, OFF_X = OFF_S + DK * CS * 4, SMEM = OFF_X + kChunk * CS * 4;
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
 template <int DK>
 constexpr size_t bwd_dstate_smem_bytes() {
-  return sizeof(float) * (size_t)(3 * kChunk * (DK + 1) + DK * kBwdWalkCols + 2 * kChunk * kBwdWalkCols + DK);
+  return (size_t)BwdDstateCfg<DK, float>::SMEM;   // bounds the bf16 plan
 }
 
 // One CTA per (sequence, head, kBwdWalkCols value columns): the columns of
-// dS evolve independently, since every step multiplies it from the left.
+// dS evolve independently, since every step multiplies it from the left.  The
+// chunk's tiles are copied asynchronously into one of two buffers while the
+// chunk after it (in walk order) is computed.
 template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kBwdWalkThreads)
 bwd_dstate_kernel(const BwdStateArgs a) {
-  constexpr int CS = kBwdWalkCols, SL = DV / CS, LK = DK + 1;
+  using C = BwdDstateCfg<DK, IO>;
+  constexpr int CS = kBwdWalkCols, SL = DV / CS, LK = C::LK;
   const int H = a.H;
   const int sl = blockIdx.x % SL;
   const int h = (blockIdx.x / SL) % H;
   const int n = blockIdx.x / (SL * H);
   const int j0 = sl * CS, tid = threadIdx.x;
 
-  extern __shared__ float smem[];
-  float* sW = smem;                 // [64][LK]
-  float* sKb = sW + kChunk * LK;    // [64][LK]
-  float* sQe = sKb + kChunk * LK;   // [64][LK]
-  float* sdS = sQe + kChunk * LK;   // [DK][CS]
-  float* sdO = sdS + DK * CS;       // [64][CS], scale * dO
-  float* sX = sdO + kChunk * CS;    // [64][CS], Kbar dS1
-  float* sgl = sX + kChunk * CS;    // [DK]
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float* sdS = reinterpret_cast<float*>(dsm + C::OFF_S);   // [DK][CS]
+  float* sX = reinterpret_cast<float*>(dsm + C::OFF_X);    // [64][CS]
 
   const IO* dO = static_cast<const IO*>(a.dO);
   const size_t sbase = ((size_t)n * H + h) * DK * DV;
@@ -101,44 +112,85 @@ bwd_dstate_kernel(const BwdStateArgs a) {
   }
   const int c_begin = a.map.chunk_off[n], c_end = a.map.chunk_off[n + 1];
   const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
-  for (int c = c_end - 1; c >= c_begin; --c) {
+  auto issue = [&](int c, int slot) {
+    uint8_t* b = dsm + slot * C::BUF;
+    const size_t tk = ((size_t)c * H + h) * kChunk * DK;
+    const int t0 = s_begin + (c - c_begin) * kChunk, len = min(kChunk, s_end - t0);
+    stage_rows<DK * 4>(b + C::OFF_W, LK * 4, a.W + tk, DK * 4, kChunk, kChunk, tid, kBwdWalkThreads);
+    stage_rows<DK * 4>(b + C::OFF_KB, LK * 4, a.Kbar + tk, DK * 4, kChunk, kChunk, tid, kBwdWalkThreads);
+    stage_rows<DK * 4>(b + C::OFF_QE, LK * 4, a.Qeff + tk, DK * 4, kChunk, kChunk, tid, kBwdWalkThreads);
+    stage_rows<CS * (int)sizeof(IO)>(b + C::OFF_DO, CS * sizeof(IO), dO + ((size_t)t0 * H + h) * DV + j0,
+                                     (size_t)H * DV * sizeof(IO), kChunk, len, tid, kBwdWalkThreads);
+    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, kBwdWalkThreads);
+  };
+  if (c_begin < c_end) issue(c_end - 1, 0);
+  cp_async_commit();
+
+  constexpr int RS = DK / 32;                    // rows of dS per thread
+  const int ri = tid / 8, cj = 2 * (tid % 8);    // X: rows 2 ri, 2 ri + 1; columns cj, cj + 1
+  const int rs = RS * (tid / 8);                 // dS: rows rs .. rs + RS - 1; columns cj, cj + 1
+  for (int c = c_end - 1, it = 0; c >= c_begin; --c, ++it) {
+    if (c - 1 >= c_begin) issue(c - 1, (it + 1) & 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const uint8_t* b = dsm + (it & 1) * C::BUF;
+    const float* sW = reinterpret_cast<const float*>(b + C::OFF_W);
+    const float* sKb = reinterpret_cast<const float*>(b + C::OFF_KB);
+    const float* sQe = reinterpret_cast<const float*>(b + C::OFF_QE);
+    const IO* sdO = reinterpret_cast<const IO*>(b + C::OFF_DO);
+    const float* sgl = reinterpret_cast<const float*>(b + C::OFF_GL);
     const int t0 = s_begin + (c - c_begin) * kChunk;
     const int len = min(kChunk, s_end - t0);
-    __syncthreads();  // the previous chunk's readers are done
+    // the gradient reaching this chunk's end state
     const size_t cs = ((size_t)c * H + h) * DK * DV;
     for (int idx = tid; idx < DK * CS; idx += kBwdWalkThreads)
       a.dS1[cs + (size_t)(idx / CS) * DV + j0 + idx % CS] = sdS[idx];
-    const size_t tile_k = ((size_t)c * H + h) * kChunk * DK;
-    for (int idx = tid; idx < kChunk * DK; idx += kBwdWalkThreads) {
-      const int i = idx / DK, cc = idx % DK;
-      sW[i * LK + cc] = a.W[tile_k + idx];
-      sKb[i * LK + cc] = a.Kbar[tile_k + idx];
-      sQe[i * LK + cc] = a.Qeff[tile_k + idx];
-    }
-    for (int idx = tid; idx < kChunk * CS; idx += kBwdWalkThreads) {
-      const int i = idx / CS, j = idx % CS;
-      sdO[idx] = i < len ? a.scale * to_f32(dO[((size_t)(t0 + i) * H + h) * DV + j0 + j]) : 0.f;
-    }
-    if (tid < DK) sgl[tid] = a.gamma_last[((size_t)c * H + h) * DK + tid];
-    __syncthreads();
-    for (int idx = tid; idx < kChunk * CS; idx += kBwdWalkThreads) {
-      const int i = idx / CS, j = idx % CS;
-      float x = 0.f;
+    // X = Kbar dS1 on a 2 x 2 tile
+    {
+      float x[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll 8
-      for (int cc = 0; cc < DK; ++cc) x = fmaf(sKb[i * LK + cc], sdS[cc * CS + j], x);
-      sX[idx] = x;
+      for (int cc = 0; cc < DK; ++cc) {
+        const float2 d = *reinterpret_cast<const float2*>(sdS + cc * CS + cj);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float kb = sKb[(2 * ri + r) * LK + cc];
+          x[r][0] = fmaf(kb, d.x, x[r][0]);
+          x[r][1] = fmaf(kb, d.y, x[r][1]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) *reinterpret_cast<float2*>(sX + (2 * ri + r) * CS + cj) = make_float2(x[r][0], x[r][1]);
     }
     __syncthreads();
-    for (int idx = tid; idx < DK * CS; idx += kBwdWalkThreads) {
-      const int cc = idx / CS, j = idx % CS;
-      float s = sgl[cc] * sdS[idx];
-      for (int i = 0; i < len; ++i) {
-        s = fmaf(-sW[i * LK + cc], sX[i * CS + j], s);
-        s = fmaf(sQe[i * LK + cc], sdO[i * CS + j], s);
+    // dS0 = gamma_n dS1 - W^T X + Q_eff^T (scale dO) on an RS x 2 tile; every
+    // thread rewrites only the entries of dS it read
+    {
+      float s[RS][2];
+#pragma unroll
+      for (int r = 0; r < RS; ++r) {
+        const float g = sgl[rs + r];
+        s[r][0] = g * sdS[(rs + r) * CS + cj];
+        s[r][1] = g * sdS[(rs + r) * CS + cj + 1];
       }
-      sdS[idx] = s;
+#pragma unroll 4
+      for (int i = 0; i < len; ++i) {
+        const float2 xv = *reinterpret_cast<const float2*>(sX + i * CS + cj);
+        const float o0 = a.scale * to_f32(sdO[i * CS + cj]), o1 = a.scale * to_f32(sdO[i * CS + cj + 1]);
+#pragma unroll
+        for (int r = 0; r < RS; ++r) {
+          const float wv = sW[i * LK + rs + r], qv = sQe[i * LK + rs + r];
+          s[r][0] = fmaf(qv, o0, fmaf(-wv, xv.x, s[r][0]));
+          s[r][1] = fmaf(qv, o1, fmaf(-wv, xv.y, s[r][1]));
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RS; ++r)
+        *reinterpret_cast<float2*>(sdS + (rs + r) * CS + cj) = make_float2(s[r][0], s[r][1]);
     }
+    __syncthreads();   // this buffer is free for the chunk after next
   }
+  cp_async_wait<0>();
   __syncthreads();
   for (int idx = tid; idx < DK * CS; idx += kBwdWalkThreads) {
     const int cc = idx / CS, j = idx % CS;

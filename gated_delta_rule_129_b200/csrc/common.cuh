@@ -27,6 +27,37 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Asynchronous 16-byte global -> shared copies (cp.async, completion per
+// thread by commit groups; a barrier after the wait makes them visible).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() {
+  cp_async_commit();
+  cp_async_wait<0>();
+}
+
+// Rows [0, rows) of a row-major global array (row stride gstride bytes) into
+// shared memory (row stride sstride bytes), BYTES per row (a multiple of 16,
+// both addresses 16-byte aligned), by threads tid of nthr; rows >= valid are
+// written as zeros instead of read.
+template <int BYTES>
+__device__ __forceinline__ void stage_rows(void* dst, int sstride, const void* src, size_t gstride, int rows,
+                                           int valid, int tid, int nthr) {
+  static_assert(BYTES % 16 == 0, "16-byte pieces");
+  constexpr int PER = BYTES / 16;
+  for (int idx = tid; idx < rows * PER; idx += nthr) {
+    const int r = idx / PER, u = idx % PER;
+    char* d = static_cast<char*>(dst) + r * sstride + u * 16;
+    if (r < valid) cp_async16(d, static_cast<const char*>(src) + r * gstride + u * 16);
+    else *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -111,14 +111,6 @@ struct TokProArgs {
 // rows of the tile and before it (as many bytes for bf16 and fp32)
 constexpr int kTokSmem = (tok_tile<float>() + kMaxConvWidth - 1) * 128 * 4;
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
-}
-
 // grid: (token tiles, H, projections).  One block: one head of one projection
 // over tok_tile<IO>() tokens; D channels, exactly W taps (tap i weighs token
 // t - i; a tap that reaches before the token's sequence start reads zero).

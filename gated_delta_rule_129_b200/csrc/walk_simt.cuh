@@ -11,6 +11,11 @@
 //   O  = scale * (Q_eff S + O_part)          query reads the updated states
 //   S <- diag(gamma_last) S + Kbar^T U       state at the next chunk start
 // hT receives the final state; h0 (or zero) is the first start state.
+//
+// The chunk's factor tiles are copied to shared memory asynchronously into
+// one of two buffers while the previous chunk is computed; both products run
+// on register tiles (a thread holds 2 x 2 of U and O, dk / 32 x 2 of S; every
+// thread updates only the entries of S it read).
 #pragma once
 
 #include "common.cuh"
@@ -37,17 +42,31 @@ struct WalkArgs {
 constexpr int kWalkSimtThreads = 256;
 constexpr int kWalkSimtDVS = 16;
 
+// Shared memory, in bytes: two chunk buffers (W, Kbar, Q_eff rows padded by
+// 16 bytes; U~ and O_part slices; gamma_n), then S [DK][DVS] and U [64][DVS]
+// in fp32.
+template <int DK, typename FT>
+struct WalkSimtCfg {
+  static constexpr int LKF = DK + 16 / (int)sizeof(FT);           // elements per padded row
+  static constexpr int TILE = kChunk * LKF * (int)sizeof(FT);
+  static constexpr int VSL = kChunk * kWalkSimtDVS * (int)sizeof(FT);
+  static constexpr int OFF_W = 0, OFF_KB = TILE, OFF_QE = 2 * TILE, OFF_UT = 3 * TILE, OFF_OP = OFF_UT + VSL,
+                       OFF_GL = OFF_OP + VSL, BUF = OFF_GL + DK * 4;
+  static constexpr int OFF_S = 2 * BUF, OFF_U = OFF_S + DK * kWalkSimtDVS * 4;
+  static constexpr int SMEM = OFF_U + kChunk * kWalkSimtDVS * 4;
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
 template <int DK, int DV>
 constexpr size_t walk_simt_smem_bytes() {
-  return sizeof(float) * (size_t)(3 * kChunk * (DK + 1) + DK * kWalkSimtDVS + 3 * kChunk * kWalkSimtDVS + DK);
+  return (size_t)WalkSimtCfg<DK, float>::SMEM;   // the fp32 plan bounds the bf16 one
 }
 
 template <int DK, int DV, typename IO, typename FT>
 __global__ void __launch_bounds__(kWalkSimtThreads)
 walk_simt_kernel(const WalkArgs<IO, FT> a) {
-  constexpr int DVS = kWalkSimtDVS;
-  constexpr int SLICES = DV / DVS;
-  constexpr int LK = DK + 1;
+  using C = WalkSimtCfg<DK, FT>;
+  constexpr int DVS = kWalkSimtDVS, SLICES = DV / DVS, LKF = C::LKF;
   const int H = a.H;
   const int sl = blockIdx.x % SLICES;
   const int h = (blockIdx.x / SLICES) % H;
@@ -55,15 +74,9 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
   const int j0 = sl * DVS;
   const int tid = threadIdx.x;
 
-  extern __shared__ float smem[];
-  float* sW = smem;                 // [64][LK]
-  float* sKb = sW + kChunk * LK;    // [64][LK]
-  float* sQe = sKb + kChunk * LK;   // [64][LK]
-  float* sS = sQe + kChunk * LK;    // [DK][DVS] state slice
-  float* sUt = sS + DK * DVS;       // [64][DVS]
-  float* sOp = sUt + kChunk * DVS;  // [64][DVS]
-  float* sU = sOp + kChunk * DVS;   // [64][DVS]
-  float* sgl = sU + kChunk * DVS;   // [DK]
+  extern __shared__ __align__(16) uint8_t wsm[];
+  float* sS = reinterpret_cast<float*>(wsm + C::OFF_S);   // [DK][DVS]
+  float* sU = reinterpret_cast<float*>(wsm + C::OFF_U);   // [64][DVS]
 
   const size_t state_base = ((size_t)n * H + h) * DK * DV;
   for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads) {
@@ -72,50 +85,101 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
   }
   const int c_begin = a.map.chunk_off[n], c_end = a.map.chunk_off[n + 1];
   const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
+  auto issue = [&](int c) {   // chunk c's tiles into buffer c & 1
+    uint8_t* b = wsm + (c & 1) * C::BUF;
+    const size_t tk = ((size_t)c * H + h) * kChunk * DK, tv = ((size_t)c * H + h) * kChunk * DV;
+    constexpr int RB = DK * (int)sizeof(FT), SB = DVS * (int)sizeof(FT);
+    stage_rows<RB>(b + C::OFF_W, LKF * sizeof(FT), a.W + tk, RB, kChunk, kChunk, tid, kWalkSimtThreads);
+    stage_rows<RB>(b + C::OFF_KB, LKF * sizeof(FT), a.Kbar + tk, RB, kChunk, kChunk, tid, kWalkSimtThreads);
+    stage_rows<RB>(b + C::OFF_QE, LKF * sizeof(FT), a.Qeff + tk, RB, kChunk, kChunk, tid, kWalkSimtThreads);
+    stage_rows<SB>(b + C::OFF_UT, SB, a.Ut + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, kWalkSimtThreads);
+    stage_rows<SB>(b + C::OFF_OP, SB, a.Opart + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, kWalkSimtThreads);
+    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, kWalkSimtThreads);
+  };
+  if (c_begin < c_end) issue(c_begin);
+  cp_async_commit();
+
+  constexpr int RS = DK / 32;                     // rows of S per thread
+  const int ri = tid / 8, cj = 2 * (tid % 8);     // U, O: rows 2 ri, 2 ri + 1; columns cj, cj + 1
+  const int rs = RS * (tid / 8);                 // S: rows rs .. rs + RS - 1; columns cj, cj + 1
   for (int c = c_begin; c < c_end; ++c) {
+    if (c + 1 < c_end) issue(c + 1);
+    cp_async_commit();
+    cp_async_wait<1>();   // this chunk's copies have landed (the next chunk's may be in flight)
+    __syncthreads();
+    const uint8_t* b = wsm + (c & 1) * C::BUF;
+    const FT* sW = reinterpret_cast<const FT*>(b + C::OFF_W);
+    const FT* sKb = reinterpret_cast<const FT*>(b + C::OFF_KB);
+    const FT* sQe = reinterpret_cast<const FT*>(b + C::OFF_QE);
+    const FT* sUt = reinterpret_cast<const FT*>(b + C::OFF_UT);
+    const FT* sOp = reinterpret_cast<const FT*>(b + C::OFF_OP);
+    const float* sgl = reinterpret_cast<const float*>(b + C::OFF_GL);
     const int t0 = s_begin + (c - c_begin) * kChunk;
     const int len = min(kChunk, s_end - t0);
-    const size_t tile_k = ((size_t)c * H + h) * kChunk * DK;
-    const size_t tile_v = ((size_t)c * H + h) * kChunk * DV;
-    __syncthreads();  // previous chunk's readers of the tiles are done
-    for (int idx = tid; idx < kChunk * DK; idx += kWalkSimtThreads) {
-      const int i = idx / DK, cc = idx % DK;
-      sW[i * LK + cc] = to_f32(a.W[tile_k + idx]);
-      sKb[i * LK + cc] = to_f32(a.Kbar[tile_k + idx]);
-      sQe[i * LK + cc] = to_f32(a.Qeff[tile_k + idx]);
-    }
-    for (int idx = tid; idx < kChunk * DVS; idx += kWalkSimtThreads) {
-      const int i = idx / DVS, j = idx % DVS;
-      sUt[idx] = to_f32(a.Ut[tile_v + (size_t)i * DV + j0 + j]);
-      sOp[idx] = to_f32(a.Opart[tile_v + (size_t)i * DV + j0 + j]);
-    }
-    if (tid < DK) sgl[tid] = a.gamma_last[((size_t)c * H + h) * DK + tid];
     if (a.chunk_states) {
       const size_t cs = ((size_t)c * H + h) * DK * DV;
       for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads)
         a.chunk_states[cs + (size_t)(idx / DVS) * DV + j0 + idx % DVS] = sS[idx];
     }
-    __syncthreads();
-    for (int idx = tid; idx < kChunk * DVS; idx += kWalkSimtThreads) {
-      const int i = idx / DVS, j = idx % DVS;
-      float u = sUt[idx], o = sOp[idx];
+    // U = U~ - W S and O = Q_eff S + O_part on a 2 x 2 tile
+    {
+      float u[2][2], o[2][2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          u[r][q] = to_f32(sUt[(2 * ri + r) * DVS + cj + q]);
+          o[r][q] = to_f32(sOp[(2 * ri + r) * DVS + cj + q]);
+        }
 #pragma unroll 8
       for (int cc = 0; cc < DK; ++cc) {
-        const float s = sS[cc * DVS + j];
-        u = fmaf(-sW[i * LK + cc], s, u);
-        o = fmaf(sQe[i * LK + cc], s, o);
+        const float2 s = *reinterpret_cast<const float2*>(sS + cc * DVS + cj);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float wv = to_f32(sW[(2 * ri + r) * LKF + cc]), qv = to_f32(sQe[(2 * ri + r) * LKF + cc]);
+          u[r][0] = fmaf(-wv, s.x, u[r][0]); u[r][1] = fmaf(-wv, s.y, u[r][1]);
+          o[r][0] = fmaf(qv, s.x, o[r][0]); o[r][1] = fmaf(qv, s.y, o[r][1]);
+        }
       }
-      sU[idx] = u;
-      if (a.out && i < len) a.out[((size_t)(t0 + i) * H + h) * DV + j0 + j] = from_f32<IO>(a.scale * o);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = 2 * ri + r;
+        *reinterpret_cast<float2*>(sU + i * DVS + cj) = make_float2(u[r][0], u[r][1]);
+        if (a.out && i < len) {
+          const size_t off = ((size_t)(t0 + i) * H + h) * DV + j0 + cj;
+          a.out[off] = from_f32<IO>(a.scale * o[r][0]);
+          a.out[off + 1] = from_f32<IO>(a.scale * o[r][1]);
+        }
+      }
     }
     __syncthreads();
-    for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads) {
-      const int cc = idx / DVS, j = idx % DVS;
-      float s = sgl[cc] * sS[idx];
-      for (int i = 0; i < len; ++i) s = fmaf(sKb[i * LK + cc], sU[i * DVS + j], s);
-      sS[idx] = s;
+    // S <- diag(gamma_n) S + Kbar^T U on an RS x 2 tile (rows of Kbar and U
+    // past the chunk's last token are zero)
+    {
+      float s[RS][2];
+#pragma unroll
+      for (int r = 0; r < RS; ++r) {
+        const float g = sgl[rs + r];
+        s[r][0] = g * sS[(rs + r) * DVS + cj];
+        s[r][1] = g * sS[(rs + r) * DVS + cj + 1];
+      }
+#pragma unroll 4
+      for (int i = 0; i < len; ++i) {
+        const float2 uv = *reinterpret_cast<const float2*>(sU + i * DVS + cj);
+#pragma unroll
+        for (int r = 0; r < RS; ++r) {
+          const float kb = to_f32(sKb[i * LKF + rs + r]);
+          s[r][0] = fmaf(kb, uv.x, s[r][0]);
+          s[r][1] = fmaf(kb, uv.y, s[r][1]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RS; ++r)
+        *reinterpret_cast<float2*>(sS + (rs + r) * DVS + cj) = make_float2(s[r][0], s[r][1]);
     }
+    __syncthreads();   // this buffer is free for chunk c + 2
   }
+  cp_async_wait<0>();
   __syncthreads();
   if (a.hT) {
     for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads) {
