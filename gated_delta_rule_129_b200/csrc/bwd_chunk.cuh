@@ -200,7 +200,8 @@ bwd_dstate_kernel(const BwdStateArgs a) {
 
 // -------------------------------------------------- per-chunk gradients ----
 constexpr int kBwdThreads = 512;
-constexpr int kBwdVB = 16;   // value columns per pass of the value loop
+constexpr int kBwdVB = 32;            // value columns per pass of the value loop
+constexpr float kBwdFoldNats = 60.f;  // decay range (each side of the reference row) for the product form
 
 struct BwdChunkArgs {
   const void *q, *k, *v, *dO;     // io dtype, [T_total, H, d]
@@ -216,31 +217,31 @@ struct BwdChunkArgs {
 };
 
 // Shared-memory plan, in floats.  [64][DK] arrays have row stride LDK, 64 x 64
-// ones and the transposed [d][64] ones LT, value tiles LVB; strides are
-// multiples of 4 (float4 rows) and spread the rows over the banks.
-template <int DK, int DV>
+// ones and the transposed [d][64] ones LT, value tiles LVB: multiples of 4
+// (float4 rows) that also spread a column's rows over the banks.
+template <int DK, int DV, typename IO>
 struct BwdCfg {
   static constexpr int LDK = DK + 4, LT = kChunk + 4, VB = kBwdVB, LVB = VB + 4;
   static constexpr int MAT = kChunk * LDK > DK * LT ? kChunk * LDK : DK * LT;   // one key-sized slot
   static constexpr int SQ = kChunk * LT;                                         // one pair-sized slot
-  // the whole call: T and P
+  // T, and P (then dP), for the whole call
   static constexpr int OFF_T = 0, OFF_P = SQ, A0 = 2 * SQ;
-  // the value loop
+  // the value loop: W, Kbar, then the pass's tiles (dO and the raw v rows in io dtype)
   static constexpr int OFF_W = A0, OFF_KB = A0 + kChunk * LDK, OFF_V = A0 + 2 * kChunk * LDK;
-  static constexpr int OFF_S0 = OFF_V, OFF_S0T = OFF_S0 + DK * VB, OFF_D1 = OFF_S0T + VB * LDK,
-                       OFF_D1T = OFF_D1 + DK * VB, OFF_DO = OFF_D1T + VB * LDK, OFF_U = OFF_DO + kChunk * LVB,
-                       OFF_UT = OFF_U + kChunk * LVB, OFF_DU = OFF_UT + VB * LT, OFF_ZT = OFF_DU + kChunk * LVB,
-                       END_V = OFF_ZT + VB * LT;
-  // after it: g, k, then q / E~^T / q, dW / e, then dT / dA, X, dP
-  static constexpr int OFF_G = A0, OFF_K = A0 + MAT, SLOT2 = A0 + 2 * MAT, SLOT3 = A0 + 3 * MAT,
-                       OFF_DT = A0 + 4 * MAT, OFF_X = OFF_DT + SQ, OFF_DP = OFF_X + SQ, END_K = OFF_DP + SQ;
+  static constexpr int OFF_S0T = OFF_V, OFF_D1T = OFF_S0T + VB * LDK, OFF_U = OFF_D1T + VB * LDK,
+                       OFF_DU = OFF_U + kChunk * LVB, OFF_UT = OFF_DU + kChunk * LVB, OFF_ZT = OFF_UT + VB * LT,
+                       OFF_DO = OFF_ZT + VB * LT,                                  // [64][VB] io
+                       END_V = OFF_DO + (kChunk * VB * (int)sizeof(IO) + 3) / 4;
+  // after it, key-sized slots: g; k (then k beta); q / E~^T / T^T, X / q; dW / dT, X / dA; e alpha or e
+  static constexpr int S_G = A0, S_K = A0 + MAT, S_2 = A0 + 2 * MAT, S_3 = A0 + 3 * MAT, S_4 = A0 + 4 * MAT,
+                       END_K = A0 + 5 * MAT;
   static constexpr int OFF_RED = (END_V > END_K ? END_V : END_K);   // [DK] x 2: rowsum(dS1 S0), colsum(dKbar Kbar)
-  static constexpr int FLOATS = OFF_RED + 2 * DK;
+  static constexpr int FLOATS = OFF_RED + 2 * DK + 4;
   static constexpr size_t SMEM = sizeof(float) * (size_t)FLOATS;
-  // thread tiles: 64 x DK (4 columns, TMK rows), 64 x 64 (2 x 4), 64 x VB (1 x 2)
+  // thread tiles: 64 x DK (4 columns, TMK rows), 64 x 64 (2 x 4), 64 x VB (2 x 2)
   static constexpr int CGK = DK / 4, TMK = kChunk * CGK / kBwdThreads;
   static_assert(TMK * (kBwdThreads / CGK) == kChunk, "key tile");
-  static_assert(kChunk * VB == 2 * kBwdThreads && kChunk * kChunk == 8 * kBwdThreads, "value and pair tiles");
+  static_assert(kChunk * VB == 4 * kBwdThreads && kChunk * kChunk == 8 * kBwdThreads, "value and pair tiles");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -249,10 +250,15 @@ __device__ __forceinline__ float ld_io(const void* p, size_t i) {
   return to_f32(static_cast<const IO*>(p)[i]);
 }
 
+template <int N>
+__device__ __forceinline__ void unpack4(const float4 v, float (&o)[N], int at) {
+  o[at] = v.x; o[at + 1] = v.y; o[at + 2] = v.z; o[at + 3] = v.w;
+}
+
 template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_chunk_kernel(const BwdChunkArgs a) {
-  using C = BwdCfg<DK, DV>;
+  using C = BwdCfg<DK, DV, IO>;
   constexpr int LDK = C::LDK, LT = C::LT, VB = C::VB, LVB = C::LVB, TMK = C::TMK;
   const int c = blockIdx.x, h = blockIdx.y;
   if (c >= a.map.chunk_off[a.map.N]) return;
@@ -272,26 +278,17 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   float* sdgn = sgs + DK;              // colsum over i of dKbar * Kbar
 
   // ------------------------------------------------ persistent tiles ----
-  {
-    float* sW = sm + C::OFF_W;
-    float* sKb = sm + C::OFF_KB;
-    for (int idx = tid; idx < kChunk * kChunk; idx += kBwdThreads) {
-      const int i = idx / kChunk, j = idx % kChunk;
-      sT[i * LT + j] = a.Tm[tile_t + idx];
-      sP[i * LT + j] = a.Pm[tile_t + idx];
-    }
-    for (int idx = tid; idx < kChunk * DK / 4; idx += kBwdThreads) {
-      const int i = idx / (DK / 4), c4 = 4 * (idx % (DK / 4));
-      *reinterpret_cast<float4*>(sW + i * LDK + c4) = *reinterpret_cast<const float4*>(a.W + tile_k + i * DK + c4);
-      *reinterpret_cast<float4*>(sKb + i * LDK + c4) = *reinterpret_cast<const float4*>(a.Kbar + tile_k + i * DK + c4);
-    }
-    for (int i = tid; i < 2 * DK; i += kBwdThreads) sgs[i] = 0.f;
-  }
+  stage_rows<kChunk * 4>(sT, LT * 4, a.Tm + tile_t, kChunk * 4, kChunk, kChunk, tid, kBwdThreads);
+  stage_rows<kChunk * 4>(sP, LT * 4, a.Pm + tile_t, kChunk * 4, kChunk, kChunk, tid, kBwdThreads);
+  stage_rows<DK * 4>(sm + C::OFF_W, LDK * 4, a.W + tile_k, DK * 4, kChunk, kChunk, tid, kBwdThreads);
+  stage_rows<DK * 4>(sm + C::OFF_KB, LDK * 4, a.Kbar + tile_k, DK * 4, kChunk, kChunk, tid, kBwdThreads);
+  cp_async_commit();
+  for (int i = tid; i < 2 * DK; i += kBwdThreads) sgs[i] = 0.f;
 
   // thread tiles
   const int rk0 = TMK * (tid / C::CGK), ck0 = 4 * (tid % C::CGK);   // 64 x DK
   const int rp0 = 2 * (tid / 16), cp0 = 4 * (tid % 16);             // 64 x 64
-  const int rv = tid / 8, cv0 = 2 * (tid % 8);                      // 64 x VB
+  const int rv = 2 * (tid / 16), cv = tid % 16;                     // 64 x VB: rows rv, rv + 1; columns cv, cv + 16
   float accQ[TMK][4], accKb[TMK][4], accW[TMK][4], accP[2][4], accT[2][4];
 #pragma unroll
   for (int ii = 0; ii < TMK; ++ii)
@@ -303,137 +300,220 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     for (int jj = 0; jj < 4; ++jj) accP[ii][jj] = accT[ii][jj] = 0.f;
 
   // ---------------------------------------------------- value loop ----
+  // per pass of VB value columns: U = U~ - W S0 and dU = scale P^T dO + Kbar dS1,
+  // then dQ~, dKbar, dW (key tiles), dP, dT (pair tiles) gather the pass's
+  // terms, and dZ gives the pass's dv, dw.  (scale is applied to the sums of
+  // dO terms: here for dU, when dQ~ and dP are used.)
   {
     const float* sW = sm + C::OFF_W;
     const float* sKb = sm + C::OFF_KB;
-    float* sS0 = sm + C::OFF_S0;     // [DK][VB]
     float* sS0T = sm + C::OFF_S0T;   // [VB][LDK]
-    float* sD1 = sm + C::OFF_D1;     // [DK][VB]
     float* sD1T = sm + C::OFF_D1T;   // [VB][LDK]
-    float* sdO = sm + C::OFF_DO;     // [64][LVB], scale * dO
     float* sU = sm + C::OFF_U;       // [64][LVB], U~ then U
-    float* sUT = sm + C::OFF_UT;     // [VB][LT]
     float* sdU = sm + C::OFF_DU;     // [64][LVB]
+    float* sUT = sm + C::OFF_UT;     // [VB][LT]
     float* sZT = sm + C::OFF_ZT;     // [VB][LT]
+    IO* sdO = reinterpret_cast<IO*>(sm + C::OFF_DO);   // [64][VB]
     for (int v0 = 0; v0 < DV; v0 += VB) {
-      __syncthreads();  // the previous pass's readers are done (and the persistent tiles written)
-      for (int idx = tid; idx < DK * VB / 4; idx += kBwdThreads) {
-        const int cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
-        const float4 s = *reinterpret_cast<const float4*>(a.S0 + st + (size_t)cc * DV + v0 + v4);
-        const float4 d = *reinterpret_cast<const float4*>(a.dS1 + st + (size_t)cc * DV + v0 + v4);
-        *reinterpret_cast<float4*>(sS0 + cc * VB + v4) = s;
-        *reinterpret_cast<float4*>(sD1 + cc * VB + v4) = d;
-        sS0T[(v4 + 0) * LDK + cc] = s.x; sS0T[(v4 + 1) * LDK + cc] = s.y;
-        sS0T[(v4 + 2) * LDK + cc] = s.z; sS0T[(v4 + 3) * LDK + cc] = s.w;
-        sD1T[(v4 + 0) * LDK + cc] = d.x; sD1T[(v4 + 1) * LDK + cc] = d.y;
-        sD1T[(v4 + 2) * LDK + cc] = d.z; sD1T[(v4 + 3) * LDK + cc] = d.w;
+      __syncthreads();  // the previous pass's readers are done
+      stage_rows<VB * 4>(sU, LVB * 4, a.Ut + tile_v + v0, DV * 4, kChunk, kChunk, tid, kBwdThreads);
+      stage_rows<VB * (int)sizeof(IO)>(sdO, VB * sizeof(IO), static_cast<const IO*>(a.dO) + tok_v(0, v0),
+                                       (size_t)H * DV * sizeof(IO), kChunk, len, tid, kBwdThreads);
+      cp_async_commit();
+      // S0 and dS1 slices, transposed; Z^T (all loads of a thread issued first)
+      {
+        float4 s[DK * VB / 4 / kBwdThreads], d[DK * VB / 4 / kBwdThreads];
+        float zw[4], zv[4];
+#pragma unroll
+        for (int u = 0; u < DK * VB / 4 / kBwdThreads; ++u) {
+          const int idx = tid + u * kBwdThreads, cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
+          s[u] = *reinterpret_cast<const float4*>(a.S0 + st + (size_t)cc * DV + v0 + v4);
+          d[u] = *reinterpret_cast<const float4*>(a.dS1 + st + (size_t)cc * DV + v0 + v4);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = tid + u * kBwdThreads, i = idx / VB, j = idx % VB;
+          const bool live = i < len;
+          zw[u] = live ? a.w[tok_v(i, v0 + j)] : 0.f;
+          zv[u] = live ? ld_io<IO>(a.v, tok_v(i, v0 + j)) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < DK * VB / 4 / kBwdThreads; ++u) {
+          const int idx = tid + u * kBwdThreads, cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
+          sS0T[(v4 + 0) * LDK + cc] = s[u].x; sS0T[(v4 + 1) * LDK + cc] = s[u].y;
+          sS0T[(v4 + 2) * LDK + cc] = s[u].z; sS0T[(v4 + 3) * LDK + cc] = s[u].w;
+          sD1T[(v4 + 0) * LDK + cc] = d[u].x; sD1T[(v4 + 1) * LDK + cc] = d[u].y;
+          sD1T[(v4 + 2) * LDK + cc] = d[u].z; sD1T[(v4 + 3) * LDK + cc] = d[u].w;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = tid + u * kBwdThreads, i = idx / VB, j = idx % VB;
+          sZT[j * LT + i] = zw[u] * zv[u];
+        }
       }
-      for (int idx = tid; idx < kChunk * VB; idx += kBwdThreads) {
-        const int i = idx / VB, j = idx % VB;
-        const bool live = i < len;
-        sdO[i * LVB + j] = live ? a.scale * ld_io<IO>(a.dO, tok_v(i, v0 + j)) : 0.f;
-        sZT[j * LT + i] = live ? a.w[tok_v(i, v0 + j)] * ld_io<IO>(a.v, tok_v(i, v0 + j)) : 0.f;
-        sU[i * LVB + j] = a.Ut[tile_v + (size_t)i * DV + v0 + j];
-      }
+      cp_async_wait<0>();
       __syncthreads();
       if (tid < DK) {
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < VB; ++j) s = fmaf(sS0[tid * VB + j], sD1[tid * VB + j], s);
-        sgs[tid] += s;
+        float sacc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < VB; ++j) sacc = fmaf(sS0T[j * LDK + tid], sD1T[j * LDK + tid], sacc);
+        sgs[tid] += sacc;
       }
-      // U = U~ - W S0 and dU = P^T (scale dO) + Kbar dS1, two columns of one row
+      // U and dU on 2 x 2 tiles (rows rv, rv + 1; columns cv, cv + 16)
       {
-        float u0 = sU[rv * LVB + cv0], u1 = sU[rv * LVB + cv0 + 1], d0 = 0.f, d1 = 0.f;
-#pragma unroll 4
-        for (int cc = 0; cc < DK; ++cc) {
-          const float wv = sW[rv * LDK + cc], kb = sKb[rv * LDK + cc];
-          const float2 s = *reinterpret_cast<const float2*>(sS0 + cc * VB + cv0);
-          const float2 d = *reinterpret_cast<const float2*>(sD1 + cc * VB + cv0);
-          u0 = fmaf(-wv, s.x, u0); u1 = fmaf(-wv, s.y, u1);
-          d0 = fmaf(kb, d.x, d0); d1 = fmaf(kb, d.y, d1);
+        float u[2][2], kd[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pd[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          u[r][0] = sU[(rv + r) * LVB + cv];
+          u[r][1] = sU[(rv + r) * LVB + cv + 16];
         }
-        for (int j = rv; j < kChunk; ++j) {   // P_{j, rv} = 0 for j < rv
-          const float p = sP[j * LT + rv];
-          const float2 o = *reinterpret_cast<const float2*>(sdO + j * LVB + cv0);
-          d0 = fmaf(p, o.x, d0); d1 = fmaf(p, o.y, d1);
+#pragma unroll 2
+        for (int c4 = 0; c4 < DK; c4 += 4) {
+          float wr[2][4], kr[2][4], s0[2][4], d1[2][4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            unpack4(*reinterpret_cast<const float4*>(sW + (rv + r) * LDK + c4), wr[r], 0);
+            unpack4(*reinterpret_cast<const float4*>(sKb + (rv + r) * LDK + c4), kr[r], 0);
+            unpack4(*reinterpret_cast<const float4*>(sS0T + (cv + 16 * r) * LDK + c4), s0[r], 0);
+            unpack4(*reinterpret_cast<const float4*>(sD1T + (cv + 16 * r) * LDK + c4), d1[r], 0);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                u[r][q] = fmaf(-wr[r][e], s0[q][e], u[r][q]);
+                kd[r][q] = fmaf(kr[r][e], d1[q][e], kd[r][q]);
+              }
+        }
+        for (int j = rv; j < kChunk; ++j) {   // P_{j, i} = 0 for j < i
+          const float2 p = *reinterpret_cast<const float2*>(sP + j * LT + rv);
+          const float o0 = to_f32(sdO[j * VB + cv]), o1 = to_f32(sdO[j * VB + cv + 16]);
+          pd[0][0] = fmaf(p.x, o0, pd[0][0]); pd[0][1] = fmaf(p.x, o1, pd[0][1]);
+          pd[1][0] = fmaf(p.y, o0, pd[1][0]); pd[1][1] = fmaf(p.y, o1, pd[1][1]);
         }
         __syncthreads();   // every thread has read its U~ before any U is written
-        sU[rv * LVB + cv0] = u0; sU[rv * LVB + cv0 + 1] = u1;
-        sUT[cv0 * LT + rv] = u0; sUT[(cv0 + 1) * LT + rv] = u1;
-        sdU[rv * LVB + cv0] = d0; sdU[rv * LVB + cv0 + 1] = d1;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int i = rv + r, j = cv + 16 * q;
+            sU[i * LVB + j] = u[r][q];
+            sUT[j * LT + i] = u[r][q];
+            sdU[i * LVB + j] = fmaf(a.scale, pd[r][q], kd[r][q]);
+          }
       }
       __syncthreads();
-      // dQ~ += (scale dO) S0^T, dKbar += U dS1^T, dW += dU S0^T (negated below)
-#pragma unroll 4
-      for (int j = 0; j < VB; ++j) {
-        const float4 s = *reinterpret_cast<const float4*>(sS0T + j * LDK + ck0);
-        const float4 d = *reinterpret_cast<const float4*>(sD1T + j * LDK + ck0);
-        const float sv[4] = {s.x, s.y, s.z, s.w}, dv[4] = {d.x, d.y, d.z, d.w};
+      // dQ~ += dO S0^T, dKbar += U dS1^T, dW += dU S0^T (negated later), four columns at a time
+#pragma unroll 1
+      for (int j4 = 0; j4 < VB; j4 += 4) {
+        float sv[4][4], dv[4][4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          unpack4(*reinterpret_cast<const float4*>(sS0T + (j4 + jj) * LDK + ck0), sv[jj], 0);
+          unpack4(*reinterpret_cast<const float4*>(sD1T + (j4 + jj) * LDK + ck0), dv[jj], 0);
+        }
 #pragma unroll
         for (int ii = 0; ii < TMK; ++ii) {
-          const float o = sdO[(rk0 + ii) * LVB + j], u = sU[(rk0 + ii) * LVB + j], du = sdU[(rk0 + ii) * LVB + j];
+          const int i = rk0 + ii;
+          float o[4], uu[4], du[4];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            accQ[ii][jj] = fmaf(o, sv[jj], accQ[ii][jj]);
-            accKb[ii][jj] = fmaf(u, dv[jj], accKb[ii][jj]);
-            accW[ii][jj] = fmaf(du, sv[jj], accW[ii][jj]);
-          }
+          for (int jj = 0; jj < 4; ++jj) o[jj] = to_f32(sdO[i * VB + j4 + jj]);
+          unpack4(*reinterpret_cast<const float4*>(sU + i * LVB + j4), uu, 0);
+          unpack4(*reinterpret_cast<const float4*>(sdU + i * LVB + j4), du, 0);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              accQ[ii][e] = fmaf(o[jj], sv[jj][e], accQ[ii][e]);
+              accKb[ii][e] = fmaf(uu[jj], dv[jj][e], accKb[ii][e]);
+              accW[ii][e] = fmaf(du[jj], sv[jj][e], accW[ii][e]);
+            }
         }
       }
-      // dP += (scale dO) U^T, dT += dU Z^T
-#pragma unroll 4
-      for (int j = 0; j < VB; ++j) {
-        const float4 u = *reinterpret_cast<const float4*>(sUT + j * LT + cp0);
-        const float4 z = *reinterpret_cast<const float4*>(sZT + j * LT + cp0);
-        const float uv[4] = {u.x, u.y, u.z, u.w}, zv[4] = {z.x, z.y, z.z, z.w};
+      // dP += dO U^T, dT += dU Z^T
+#pragma unroll 1
+      for (int j4 = 0; j4 < VB; j4 += 4) {
+        float uv[4][4], zv[4][4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          unpack4(*reinterpret_cast<const float4*>(sUT + (j4 + jj) * LT + cp0), uv[jj], 0);
+          unpack4(*reinterpret_cast<const float4*>(sZT + (j4 + jj) * LT + cp0), zv[jj], 0);
+        }
 #pragma unroll
         for (int ii = 0; ii < 2; ++ii) {
-          const float o = sdO[(rp0 + ii) * LVB + j], du = sdU[(rp0 + ii) * LVB + j];
+          const int i = rp0 + ii;
+          float o[4], du[4];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            accP[ii][jj] = fmaf(o, uv[jj], accP[ii][jj]);
-            accT[ii][jj] = fmaf(du, zv[jj], accT[ii][jj]);
-          }
+          for (int jj = 0; jj < 4; ++jj) o[jj] = to_f32(sdO[i * VB + j4 + jj]);
+          unpack4(*reinterpret_cast<const float4*>(sdU + i * LVB + j4), du, 0);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              accP[ii][e] = fmaf(o[jj], uv[jj][e], accP[ii][e]);
+              accT[ii][e] = fmaf(du[jj], zv[jj][e], accT[ii][e]);
+            }
         }
       }
-      // dZ = T^T dU (rows >= rv of column rv), then dv = dZ w and dw = dZ v
+      // dZ = T^T dU on the 2 x 2 tile, then dv = dZ w and dw = dZ v
       {
-        float z0 = 0.f, z1 = 0.f;
-        for (int i = rv; i < kChunk; ++i) {
-          const float t = sT[i * LT + rv];
-          const float2 d = *reinterpret_cast<const float2*>(sdU + i * LVB + cv0);
-          z0 = fmaf(t, d.x, z0); z1 = fmaf(t, d.y, z1);
+        float z[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        for (int i = rv; i < kChunk; ++i) {   // T_{i, j} = 0 for i < j
+          const float2 t = *reinterpret_cast<const float2*>(sT + i * LT + rv);
+          const float d0 = sdU[i * LVB + cv], d1 = sdU[i * LVB + cv + 16];
+          z[0][0] = fmaf(t.x, d0, z[0][0]); z[0][1] = fmaf(t.x, d1, z[0][1]);
+          z[1][0] = fmaf(t.y, d0, z[1][0]); z[1][1] = fmaf(t.y, d1, z[1][1]);
         }
-        if (rv < len) {
-          const size_t o = tok_v(rv, v0 + cv0);
-          a.dv[o] = z0 * a.w[o];
-          a.dv[o + 1] = z1 * a.w[o + 1];
-          a.dw[o] = z0 * ld_io<IO>(a.v, o);
-          a.dw[o + 1] = z1 * ld_io<IO>(a.v, o + 1);
-        }
+        float wv[2][2], vv[2][2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const bool live = rv + r < len;
+            const size_t o = tok_v(live ? rv + r : 0, v0 + cv + 16 * q);
+            wv[r][q] = live ? a.w[o] : 0.f;
+            vv[r][q] = live ? ld_io<IO>(a.v, o) : 0.f;
+          }
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            if (rv + r < len) {
+              const size_t o = tok_v(rv + r, v0 + cv + 16 * q);
+              a.dv[o] = z[r][q] * wv[r][q];
+              a.dw[o] = z[r][q] * vv[r][q];
+            }
       }
     }
   }
   __syncthreads();  // the value loop's tiles are dead
 
   // ------------------------------------- g, k, q; dq, dk and dg partials ----
-  float* sg = sm + C::OFF_G;      // [64][LDK] cumulative log-decay
-  float* sk = sm + C::OFF_K;      // [64][LDK] k
-  float* sq = sm + C::SLOT2;      // [64][LDK] q
-  float* sdP = sm + C::OFF_DP;    // [64][LT]
-  for (int idx = tid; idx < kChunk * DK; idx += kBwdThreads) {
-    const int i = idx / DK, cc = idx % DK;
-    const bool live = i < len;
-    sg[i * LDK + cc] = live ? a.la[tok_k(i, cc)] : 0.f;
-    sk[i * LDK + cc] = live ? ld_io<IO>(a.k, tok_k(i, cc)) : 0.f;
-    sq[i * LDK + cc] = live ? ld_io<IO>(a.q, tok_k(i, cc)) : 0.f;
-  }
+  float* sg = sm + C::S_G;        // [64][LDK] cumulative log-decay
+  float* sk = sm + C::S_K;        // [64][LDK] k
+  float* sq = sm + C::S_2;        // [64][LDK] q
+  float* sdP = sm + C::OFF_P;     // [64][LT], over P
+  batched_copy<8, float4>(
+      kChunk * DK, tid, kBwdThreads,
+      [&](int idx) {
+        const int i = idx / DK, cc = idx % DK;
+        if (i >= len) return make_float4(0.f, 0.f, 0.f, 0.f);
+        const size_t o = tok_k(i, cc);
+        return make_float4(a.la[o], ld_io<IO>(a.k, o), ld_io<IO>(a.q, o), 0.f);
+      },
+      [&](int idx, float4 r) {
+        const int i = idx / DK, cc = idx % DK;
+        sg[i * LDK + cc] = r.x;
+        sk[i * LDK + cc] = r.y;
+        sq[i * LDK + cc] = r.z;
+      });
 #pragma unroll
   for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj)
-      sdP[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj <= rp0 + ii ? accP[ii][jj] : 0.f;
+      sdP[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj <= rp0 + ii ? a.scale * accP[ii][jj] : 0.f;
   __syncthreads();
   if (tid < DK) {   // in-chunk cumulative sum; padded rows keep g at its last value
     float acc = 0.f;
@@ -449,19 +529,22 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
     for (int ii = 0; ii < TMK; ++ii) {
       const int i = rk0 + ii;
+      float dqv[4], dkv[4];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int cc = ck0 + jj;
         const float g = sg[i * LDK + cc], gn = sg[(kChunk - 1) * LDK + cc];
         const float gam = expf(g), ks = expf(gn - g);
-        const float dQt = accQ[ii][jj], dKb = accKb[ii][jj];
+        const float dQt = a.scale * accQ[ii][jj], dKb = accKb[ii][jj];
         const float kb = sk[i * LDK + cc] * ks;   // Kbar
         dg[ii][jj] = dQt * sq[i * LDK + cc] * gam - dKb * kb;
         colsum[jj] = fmaf(dKb, kb, colsum[jj]);
-        if (i < len) {
-          a.dq[tok_k(i, cc)] = dQt * gam;
-          a.dk[tok_k(i, cc)] = dKb * ks;
-        }
+        dqv[jj] = dQt * gam;
+        dkv[jj] = dKb * ks;
+      }
+      if (i < len) {
+        *reinterpret_cast<float4*>(a.dq + tok_k(i, ck0)) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
+        *reinterpret_cast<float4*>(a.dk + tok_k(i, ck0)) = make_float4(dkv[0], dkv[1], dkv[2], dkv[3]);
       }
     }
 #pragma unroll
@@ -471,17 +554,22 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 
   // ------------------------------ dT += dW E~^T, dE~ = T^T dW, dE~ terms ----
   {
-    float* sEtT = sm + C::SLOT2;   // [DK][LT]
-    float* sdW = sm + C::SLOT3;    // [64][LDK]
-    for (int idx = tid; idx < kChunk * DK; idx += kBwdThreads) {
-      const int i = idx / DK, cc = idx % DK;
-      const float bv = i < len ? a.b[tok_k(i, cc)] : 0.f;
-      sEtT[cc * LT + i] = bv * sk[i * LDK + cc] * expf(sg[i * LDK + cc]);
-    }
+    float* sEtT = sm + C::S_2;     // [DK][LT]
+    float* sdW = sm + C::S_3;      // [64][LDK]
+    batched_copy<8, float>(
+        kChunk * DK, tid, kBwdThreads,
+        [&](int idx) {
+          const int i = idx / DK, cc = idx % DK;
+          return i < len ? a.b[tok_k(i, cc)] : 0.f;
+        },
+        [&](int idx, float bv) {
+          const int i = idx / DK, cc = idx % DK;
+          sEtT[cc * LT + i] = bv * sk[i * LDK + cc] * expf(sg[i * LDK + cc]);
+        });
 #pragma unroll
     for (int ii = 0; ii < TMK; ++ii)
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) sdW[(rk0 + ii) * LDK + ck0 + jj] = -accW[ii][jj];
+      *reinterpret_cast<float4*>(sdW + (rk0 + ii) * LDK + ck0) =
+          make_float4(-accW[ii][0], -accW[ii][1], -accW[ii][2], -accW[ii][3]);
     __syncthreads();
 #pragma unroll 4
     for (int cc = 0; cc < DK; ++cc) {
@@ -512,28 +600,31 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
     for (int ii = 0; ii < TMK; ++ii) {
       const int i = rk0 + ii;
+      float dev[4];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int cc = ck0 + jj;
         dg[ii][jj] = fmaf(dEt[ii][jj], sEtT[cc * LT + i], dg[ii][jj]);
-        if (i < len) {
-          a.db[tok_k(i, cc)] = dEt[ii][jj] * expf(sg[i * LDK + cc]);   // dE so far; made db below
-          a.dla[tok_k(i, cc)] = dg[ii][jj];                            // dg so far
-        }
+        dev[jj] = dEt[ii][jj] * expf(sg[i * LDK + cc]);
+      }
+      if (i < len) {   // dE so far (made db below) and dg so far
+        *reinterpret_cast<float4*>(a.db + tok_k(i, ck0)) = make_float4(dev[0], dev[1], dev[2], dev[3]);
+        *reinterpret_cast<float4*>(a.dla + tok_k(i, ck0)) = make_float4(dg[ii][0], dg[ii][1], dg[ii][2], dg[ii][3]);
       }
     }
   }
   __syncthreads();
 
   // ---------------------------------------------- dA = -T^T dT T^T ----
+  float* sdA = sm + C::S_3;        // [64][LT] (first half of the slot)
   {
-    float* sdT = sm + C::OFF_DT;   // [64][LT], then dA
-    float* sX = sm + C::OFF_X;     // [64][LT]
-    float* sTT = sm + C::SLOT3;    // [64][LT], T transposed
+    float* sdT = sdA;              // dT, then dA over it
+    float* sX = sm + C::S_3 + C::SQ;
+    float* sTT = sm + C::S_2;      // [64][LT], T transposed
 #pragma unroll
     for (int ii = 0; ii < 2; ++ii)
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) sdT[(rp0 + ii) * LT + cp0 + jj] = accT[ii][jj];
+      *reinterpret_cast<float4*>(sdT + (rp0 + ii) * LT + cp0) =
+          make_float4(accT[ii][0], accT[ii][1], accT[ii][2], accT[ii][3]);
     for (int idx = tid; idx < kChunk * kChunk; idx += kBwdThreads) {
       const int i = idx / kChunk, j = idx % kChunk;
       sTT[j * LT + i] = sT[i * LT + j];
@@ -553,8 +644,7 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     }
 #pragma unroll
     for (int ii = 0; ii < 2; ++ii)
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) sX[(rp0 + ii) * LT + cp0 + jj] = x[ii][jj];
+      *reinterpret_cast<float4*>(sX + (rp0 + ii) * LT + cp0) = make_float4(x[ii][0], x[ii][1], x[ii][2], x[ii][3]);
     __syncthreads();
     float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 4
@@ -572,21 +662,128 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
-        sdT[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj < rp0 + ii ? -y[ii][jj] : 0.f;   // dA, strictly lower
+        sdA[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj < rp0 + ii ? -y[ii][jj] : 0.f;   // strictly lower
+  }
+  // the chunk's decay range on each side of the reference row r (its middle
+  // token, or its last one when shorter): the product form below scales rows
+  // by exp(g_i - g_r) and exp(g_r - g_j), safe in fp32 while both ranges stay
+  // within kBwdFoldNats
+  const int rref = min(kChunk / 2, len - 1);
+  __shared__ int s_steep;
+  if (tid == 0) s_steep = 0;
+  __syncthreads();
+  if (tid < DK) {
+    const float g0 = sg[tid], gr = sg[rref * LDK + tid], gl = sg[(kChunk - 1) * LDK + tid];
+    if (g0 - gr > kBwdFoldNats || gr - gl > kBwdFoldNats) atomicOr(&s_steep, 1);
   }
   __syncthreads();
 
-  // ------------------------------- through the pairwise decays of A, P ----
-  {
-    const float* sdA = sm + C::OFF_DT;
-    float* sq2 = sm + C::SLOT2;    // q again
-    float* se = sm + C::SLOT3;     // e = b k
-    for (int idx = tid; idx < kChunk * DK; idx += kBwdThreads) {
-      const int i = idx / DK, cc = idx % DK;
-      const bool live = i < len;
-      sq2[i * LDK + cc] = live ? ld_io<IO>(a.q, tok_k(i, cc)) : 0.f;
-      se[i * LDK + cc] = live ? a.b[tok_k(i, cc)] * sk[i * LDK + cc] : 0.f;
+  if (!s_steep) {
+    // -------------------- through the pairwise decays, as products ----
+    // exp(g_ic - g_jc) = alpha_ic beta_jc with alpha = exp(g - g_r) and
+    // beta = exp(g_r - g):  dE^D = alpha (dA (k beta)), dQ^D = alpha (dP (k beta)),
+    // dK^D = beta (dA^T (e alpha) + dP^T (q alpha)).
+    float* skb = sk;                  // k beta, over k
+    float* sea = sm + C::S_2;         // e alpha
+    float* sqa = sm + C::S_4;         // q alpha
+    batched_copy<8, float2>(
+        kChunk * DK, tid, kBwdThreads,
+        [&](int idx) {
+          const int i = idx / DK, cc = idx % DK;
+          if (i >= len) return make_float2(0.f, 0.f);
+          const size_t o = tok_k(i, cc);
+          return make_float2(a.b[o], ld_io<IO>(a.q, o));
+        },
+        [&](int idx, float2 r) {
+          const int i = idx / DK, cc = idx % DK;
+          const float g = sg[i * LDK + cc], gr = sg[rref * LDK + cc], kv = sk[i * LDK + cc];
+          const float al = expf(g - gr), be = expf(gr - g);
+          sea[i * LDK + cc] = r.x * kv * al;
+          sqa[i * LDK + cc] = r.y * al;
+          skb[i * LDK + cc] = kv * be;
+        });
+    __syncthreads();
+    float ed[TMK][4], qd[TMK][4], kd[TMK][4];
+#pragma unroll
+    for (int ii = 0; ii < TMK; ++ii)
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) ed[ii][jj] = qd[ii][jj] = kd[ii][jj] = 0.f;
+    for (int m = 0; m < rk0 + TMK; ++m) {   // dA, dP vanish for m > i
+      float kbv[4];
+      unpack4(*reinterpret_cast<const float4*>(skb + m * LDK + ck0), kbv, 0);
+#pragma unroll
+      for (int ii = 0; ii < TMK; ++ii) {
+        const float av = sdA[(rk0 + ii) * LT + m], pv = sdP[(rk0 + ii) * LT + m];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          ed[ii][jj] = fmaf(av, kbv[jj], ed[ii][jj]);
+          qd[ii][jj] = fmaf(pv, kbv[jj], qd[ii][jj]);
+        }
+      }
     }
+    for (int i = rk0; i < kChunk; ++i) {   // dA_{i, j}, dP_{i, j} vanish for i < j
+      float ea[4], qa[4], av[TMK], pv[TMK];
+      unpack4(*reinterpret_cast<const float4*>(sea + i * LDK + ck0), ea, 0);
+      unpack4(*reinterpret_cast<const float4*>(sqa + i * LDK + ck0), qa, 0);
+#pragma unroll
+      for (int ii = 0; ii < TMK; ++ii) {
+        av[ii] = sdA[i * LT + rk0 + ii];
+        pv[ii] = sdP[i * LT + rk0 + ii];
+      }
+#pragma unroll
+      for (int ii = 0; ii < TMK; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) kd[ii][jj] = fmaf(av[ii], ea[jj], fmaf(pv[ii], qa[jj], kd[ii][jj]));
+    }
+    // combine with the partials this thread wrote (same rows and columns)
+#pragma unroll
+    for (int ii = 0; ii < TMK; ++ii) {
+      const int i = rk0 + ii;
+      if (i >= len) continue;
+      const size_t o = tok_k(i, ck0);
+      float4 pq = *reinterpret_cast<const float4*>(a.dq + o), pe = *reinterpret_cast<const float4*>(a.db + o);
+      float4 pk = *reinterpret_cast<const float4*>(a.dk + o), pg = *reinterpret_cast<const float4*>(a.dla + o);
+      const float4 bv = *reinterpret_cast<const float4*>(a.b + o);
+      float kv[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) kv[jj] = ld_io<IO>(a.k, o + jj);
+      float fq[4], fe[4], fk[4], fg[4], bq[4];
+      unpack4(pq, fq, 0); unpack4(pe, fe, 0); unpack4(pk, fk, 0); unpack4(pg, fg, 0); unpack4(bv, bq, 0);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int cc = ck0 + jj;
+        const float g = sg[i * LDK + cc], gr = sg[rref * LDK + cc];
+        const float al = expf(g - gr), be = expf(gr - g);
+        const float edv = al * ed[ii][jj], qdv = al * qd[ii][jj], kdv = be * kd[ii][jj];
+        const float dE = fe[jj] + edv;
+        fq[jj] += qdv;
+        fk[jj] += kdv + dE * bq[jj];
+        // e dE^D + q dQ^D - k dK^D, each from the scaled operands
+        fg[jj] += sea[i * LDK + cc] * ed[ii][jj] + sqa[i * LDK + cc] * qd[ii][jj] - skb[i * LDK + cc] * kd[ii][jj];
+        fe[jj] = dE * kv[jj];
+      }
+      *reinterpret_cast<float4*>(a.dq + o) = make_float4(fq[0], fq[1], fq[2], fq[3]);
+      *reinterpret_cast<float4*>(a.db + o) = make_float4(fe[0], fe[1], fe[2], fe[3]);
+      *reinterpret_cast<float4*>(a.dk + o) = make_float4(fk[0], fk[1], fk[2], fk[3]);
+      *reinterpret_cast<float4*>(a.dla + o) = make_float4(fg[0], fg[1], fg[2], fg[3]);
+    }
+  } else {
+    // -------------- through the pairwise decays, pair by pair (steep) ----
+    float* sq2 = sm + C::S_2;    // q again
+    float* se = sm + C::S_4;     // e = b k
+    batched_copy<8, float2>(
+        kChunk * DK, tid, kBwdThreads,
+        [&](int idx) {
+          const int i = idx / DK, cc = idx % DK;
+          if (i >= len) return make_float2(0.f, 0.f);
+          const size_t o = tok_k(i, cc);
+          return make_float2(ld_io<IO>(a.q, o), a.b[o]);
+        },
+        [&](int idx, float2 r) {
+          const int i = idx / DK, cc = idx % DK;
+          sq2[i * LDK + cc] = r.x;
+          se[i * LDK + cc] = r.y * sk[i * LDK + cc];
+        });
     __syncthreads();
     // thread (channel cc, part p): the row sums of its channel over the
     // columns j of its part (j mod 2*PARTS in {p, 2*PARTS-1-p}: every part

@@ -58,6 +58,26 @@ __device__ __forceinline__ void stage_rows(void* dst, int sstride, const void* s
   }
 }
 
+// Element-wise staging with many loads in flight: for idx = tid, tid + nthr,
+// ... < n, in batches of U per thread, every load(idx) of the batch is issued
+// before its store(idx, value).
+template <int U, typename T, typename L, typename S>
+__device__ __forceinline__ void batched_copy(int n, int tid, int nthr, L load, S store) {
+  for (int base = tid; base < n; base += U * nthr) {
+    T r[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int idx = base + u * nthr;
+      if (idx < n) r[u] = load(idx);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int idx = base + u * nthr;
+      if (idx < n) store(idx, r[u]);
+    }
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

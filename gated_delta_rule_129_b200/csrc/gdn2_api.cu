@@ -649,7 +649,7 @@ struct BwdOp {
     ca.H = d->H;
     ca.scale = scale;
     ca.dq = dq; ca.dk = dk; ca.dla = dla; ca.db = db; ca.dv = dv; ca.dw = dw;
-    constexpr size_t smem = gdn2::BwdCfg<DK, DV>::SMEM;
+    constexpr size_t smem = gdn2::BwdCfg<DK, DV, IO>::SMEM;
     auto kern = gdn2::bwd_chunk_kernel<DK, DV, IO>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return GDN2_ERR_CUDA;

@@ -73,30 +73,30 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   float* sP = sA + kChunk * LA;     // [64][LA]  P (lower, diagonal included)
   const int tid = threadIdx.x;
 
-  for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
-    const int i = idx / DK, cc = idx % DK;
-    float kv = 0.f, bv = 0.f, qv = 0.f, lv = 0.f;
-    if (i < len) {
-      const size_t off = ((size_t)(pos.t0 + i) * H + h) * DK + cc;
-      kv = to_f32(a.k[off]);
-      qv = to_f32(a.q[off]);
-      bv = a.b[off];
-      lv = a.la[off];
-    }
-    sk[i * LK + cc] = kv;
-    se[i * LK + cc] = bv * kv;
-    sq[i * LK + cc] = qv;
-    sg[i * LK + cc] = lv;
-  }
-  for (int idx = tid; idx < kChunk * DV; idx += kPrepSimtThreads) {
-    const int i = idx / DV, cc = idx % DV;
-    float z = 0.f;
-    if (i < len) {
-      const size_t off = ((size_t)(pos.t0 + i) * H + h) * DV + cc;
-      z = a.w[off] * to_f32(a.v[off]);
-    }
-    sz[i * LV + cc] = z;
-  }
+  batched_copy<8, float4>(
+      kChunk * DK, tid, kPrepSimtThreads,
+      [&](int idx) {
+        const int i = idx / DK, cc = idx % DK;
+        if (i >= len) return make_float4(0.f, 0.f, 0.f, 0.f);
+        const size_t off = ((size_t)(pos.t0 + i) * H + h) * DK + cc;
+        return make_float4(to_f32(a.k[off]), to_f32(a.q[off]), a.b[off], a.la[off]);
+      },
+      [&](int idx, float4 r) {
+        const int i = idx / DK, cc = idx % DK;
+        sk[i * LK + cc] = r.x;
+        se[i * LK + cc] = r.z * r.x;
+        sq[i * LK + cc] = r.y;
+        sg[i * LK + cc] = r.w;
+      });
+  batched_copy<8, float>(
+      kChunk * DV, tid, kPrepSimtThreads,
+      [&](int idx) {
+        const int i = idx / DV, cc = idx % DV;
+        if (i >= len) return 0.f;
+        const size_t off = ((size_t)(pos.t0 + i) * H + h) * DV + cc;
+        return a.w[off] * to_f32(a.v[off]);
+      },
+      [&](int idx, float z) { sz[(idx / DV) * LV + idx % DV] = z; });
   for (int idx = tid; idx < kChunk * LA; idx += kPrepSimtThreads) {
     sA[idx] = 0.f;
     sP[idx] = 0.f;
@@ -112,23 +112,47 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     }
   }
   __syncthreads();
-  // A and P: one warp per (i, j) pair, lanes over key channels.
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int i = warp; i < len; i += kPrepSimtThreads / 32) {
-    for (int j = 0; j <= i; ++j) {
-      float acc_a = 0.f, acc_p = 0.f;
+  // A and P on 2 x 2 blocks of (i, j) pairs of the lower triangle, a thread
+  // per block, the key channels summed in registers.  exp(g_i - g_j) is taken
+  // of min(g_i - g_j, 0), so the entries above the diagonal (masked below)
+  // cannot overflow; its hardware exponential's error, a few ulp, is far
+  // below the fp32 path's tolerance.
+  {
+    constexpr int NB = kChunk / 2;
+    for (int t = tid; t < NB * (NB + 1) / 2; t += kPrepSimtThreads) {
+      int bi = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+      while (bi * (bi + 1) / 2 > t) --bi;
+      while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
+      const int bj = t - bi * (bi + 1) / 2;
+      const int i0 = 2 * bi, j0 = 2 * bj;
+      if (i0 >= len) continue;   // rows past the last token stay zero
+      float aa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pp[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll 4
+      for (int cc = 0; cc < DK; ++cc) {
+        const float gi[2] = {sg[i0 * LK + cc], sg[(i0 + 1) * LK + cc]};
+        const float gj[2] = {sg[j0 * LK + cc], sg[(j0 + 1) * LK + cc]};
+        const float ev[2] = {se[i0 * LK + cc], se[(i0 + 1) * LK + cc]};
+        const float qv[2] = {sq[i0 * LK + cc], sq[(i0 + 1) * LK + cc]};
+        const float kv[2] = {sk[j0 * LK + cc], sk[(j0 + 1) * LK + cc]};
 #pragma unroll
-      for (int cc = lane; cc < DK; cc += 32) {
-        const float kd = sk[j * LK + cc] * expf(sg[i * LK + cc] - sg[j * LK + cc]);
-        acc_a = fmaf(se[i * LK + cc], kd, acc_a);
-        acc_p = fmaf(sq[i * LK + cc], kd, acc_p);
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const float kd = kv[q] * __expf(fminf(gi[r] - gj[q], 0.f));
+            aa[r][q] = fmaf(ev[r], kd, aa[r][q]);
+            pp[r][q] = fmaf(qv[r], kd, pp[r][q]);
+          }
       }
-      acc_a = warp_sum(acc_a);
-      acc_p = warp_sum(acc_p);
-      if (lane == 0) {
-        if (j < i) sA[i * LA + j] = acc_a;
-        sP[i * LA + j] = acc_p;
-      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int i = i0 + r, j = j0 + q;
+          if (i < len && j <= i) {
+            if (j < i) sA[i * LA + j] = aa[r][q];
+            sP[i * LA + j] = pp[r][q];
+          }
+        }
     }
   }
   __syncthreads();
@@ -154,18 +178,27 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
   if (AFFINE && a.colscale && tid < DK) a.colscale[((size_t)c * H + h) * DK + tid] = 1.f;
   __syncthreads();
+  // sum_{m0 <= m < i} A_im X_m,col with four partial sums (short dependency chains)
+  auto row_dot = [&](const float* X, int ld, int col, int i, int m0) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int m = m0;
+    for (; m + 3 < i; m += 4) {
+      s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
+      s1 = fmaf(sA[i * LA + m + 1], X[(m + 1) * ld + col], s1);
+      s2 = fmaf(sA[i * LA + m + 2], X[(m + 2) * ld + col], s2);
+      s3 = fmaf(sA[i * LA + m + 3], X[(m + 3) * ld + col], s3);
+    }
+    for (; m < i; ++m) s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
+    return (s0 + s1) + (s2 + s3);
+  };
   // Forward substitution, row by row: W_i = E~_i - sum_{j<i} A_ij W_j, and the
   // same for U~ with Z.  One thread per column of [W | U~].
   for (int i = 1; i < len; ++i) {
     if (tid < DK) {
-      float acc = se[i * LK + tid];
-      for (int j = 0; j < i; ++j) acc = fmaf(-sA[i * LA + j], se[j * LK + tid], acc);
-      se[i * LK + tid] = acc;
+      se[i * LK + tid] -= row_dot(se, LK, tid, i, 0);
     } else if (tid < DK + DV) {
       const int col = tid - DK;
-      float acc = sz[i * LV + col];
-      for (int j = 0; j < i; ++j) acc = fmaf(-sA[i * LA + j], sz[j * LV + col], acc);
-      sz[i * LV + col] = acc;
+      sz[i * LV + col] -= row_dot(sz, LV, col, i, 0);
     }
     __syncthreads();
   }
@@ -192,10 +225,7 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     __syncthreads();
     for (int i = 1; i < len; ++i) {
       float acc = 0.f;
-      if (tid < i) {
-        acc = -sA[i * LA + tid];
-        for (int m = tid + 1; m < i; ++m) acc = fmaf(-sA[i * LA + m], sA[m * LA + tid], acc);
-      }
+      if (tid < i) acc = -sA[i * LA + tid] - row_dot(sA, LA, tid, i, tid + 1);
       __syncthreads();
       if (tid < i) sA[i * LA + tid] = acc;
       __syncthreads();

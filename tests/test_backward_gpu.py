@@ -5,7 +5,9 @@ The kernel computes in fp32 from the same (bf16-representable) inputs the
 oracle sees and writes fp32 gradients, so the tolerance is the fp32 one in
 both I/O modes: rel-L2 <= 1e-4 over each gradient tensor (fp64 comparison),
 on shapes that span several chunks, a ragged tail, packed sequences with empty
-and one-token ones, dk / dv 64 and 128, with and without h0 and dhT.
+and one-token ones, dk / dv 64 and 128, with and without h0 and dhT, and
+chunks whose decay is too steep for the scaled-product form (the pair-by-pair
+path).
 """
 import numpy as np
 import pytest
@@ -30,11 +32,17 @@ CASES = [
     dict(io="bf16", dk=128, dv=128, B=1, T=200, H=2, lengths=None, decay="strong", h0=True, dhT=True),
     dict(io="f32", dk=128, dv=64, B=1, T=None, H=2, lengths=[70, 0, 1, 130], decay="mild", h0=True, dhT=True),
     dict(io="bf16", dk=64, dv=128, B=2, T=65, H=1, lengths=None, decay="mild", h0=False, dhT=False),
+    # a chunk whose decay spans ~96 nats on each side of its middle token: the
+    # pair-by-pair path instead of the scaled products
+    dict(io="bf16", dk=128, dv=128, B=1, T=192, H=2, lengths=None, decay="mild", h0=True, dhT=True, steep=True),
+    dict(io="f32", dk=64, dv=64, B=1, T=None, H=2, lengths=[100, 3, 90], decay="mild", h0=True, dhT=True,
+         steep=True),
 ]
 
 
 def _ids(c):
-    return f"{c['io']}-dk{c['dk']}-dv{c['dv']}-{'var' if c['lengths'] else 'B%d' % c['B']}"
+    return (f"{c['io']}-dk{c['dk']}-dv{c['dv']}-{'var' if c['lengths'] else 'B%d' % c['B']}"
+            + ("-steep" if c.get("steep") else ""))
 
 
 @pytest.mark.parametrize("case", CASES, ids=_ids)
@@ -46,6 +54,8 @@ def test_backward_matches_oracle(gdn2, case):
     T = sum(lengths) if lengths else case["T"]
     x = make_inputs(case["B"], T, case["H"], case["dk"], case["dv"], io=case["io"], seed=91 + case["dk"],
                     decay=case["decay"], h0_std=0.05 if case["h0"] else None, lengths=lengths)
+    if case.get("steep"):
+        x.log_alpha[:, 64:128] = -3.0
     rng = np.random.default_rng(92)
     dO = rng.standard_normal(x.v.shape).astype(np.float32)
     if case["io"] == "bf16":
