@@ -46,7 +46,7 @@ struct PrepArgs {
   float* Pm;  // optional: P, zero above the diagonal                 [., H, 64, 64]
 };
 
-constexpr int kPrepSimtThreads = 256;
+constexpr int kPrepSimtThreads = 512;
 
 template <int DK, int DV>
 constexpr size_t prep_simt_smem_bytes() {
@@ -58,7 +58,7 @@ constexpr size_t prep_simt_smem_bytes() {
 // One (chunk c, head h) per call; all kPrepSimtThreads threads take part.
 template <int DK, int DV, typename IO, typename FT, bool AFFINE>
 __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c, int h, float* smem) {
-  static_assert(DK + DV <= kPrepSimtThreads, "one thread per solve column");
+  static_assert(2 * (DK + DV) <= kPrepSimtThreads, "two threads per solve column");
   constexpr int LK = DK + 1, LV = DV + 1, LA = kChunk + 1;
   const int H = a.H;
   const ChunkPos pos = chunk_pos(a.map, c);
@@ -178,27 +178,30 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
   if (AFFINE && a.colscale && tid < DK) a.colscale[((size_t)c * H + h) * DK + tid] = 1.f;
   __syncthreads();
-  // sum_{m0 <= m < i} A_im X_m,col with four partial sums (short dependency chains)
-  auto row_dot = [&](const float* X, int ld, int col, int i, int m0) {
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    int m = m0;
-    for (; m + 3 < i; m += 4) {
+  // half of sum_{m0 <= m < i} A_im X_m,col: the terms m = m0 + half, m0 + half + 2,
+  // ... (two partial sums, short dependency chains); the other half comes
+  // from the neighbouring lane
+  const int scol = tid >> 1, half = tid & 1;
+  auto row_dot_half = [&](const float* X, int ld, int col, int i, int m0) {
+    float s0 = 0.f, s1 = 0.f;
+    int m = m0 + half;
+    for (; m + 2 < i; m += 4) {
       s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
-      s1 = fmaf(sA[i * LA + m + 1], X[(m + 1) * ld + col], s1);
-      s2 = fmaf(sA[i * LA + m + 2], X[(m + 2) * ld + col], s2);
-      s3 = fmaf(sA[i * LA + m + 3], X[(m + 3) * ld + col], s3);
+      s1 = fmaf(sA[i * LA + m + 2], X[(m + 2) * ld + col], s1);
     }
-    for (; m < i; ++m) s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
-    return (s0 + s1) + (s2 + s3);
+    for (; m < i; m += 2) s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
+    return s0 + s1;
   };
   // Forward substitution, row by row: W_i = E~_i - sum_{j<i} A_ij W_j, and the
-  // same for U~ with Z.  One thread per column of [W | U~].
+  // same for U~ with Z.  Two threads per column of [W | U~].
   for (int i = 1; i < len; ++i) {
-    if (tid < DK) {
-      se[i * LK + tid] -= row_dot(se, LK, tid, i, 0);
-    } else if (tid < DK + DV) {
-      const int col = tid - DK;
-      sz[i * LV + col] -= row_dot(sz, LV, col, i, 0);
+    float part = 0.f;
+    if (scol < DK) part = row_dot_half(se, LK, scol, i, 0);
+    else if (scol < DK + DV) part = row_dot_half(sz, LV, scol - DK, i, 0);
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    if (half == 0) {
+      if (scol < DK) se[i * LK + scol] -= part;
+      else if (scol < DK + DV) sz[i * LV + scol - DK] -= part;
     }
     __syncthreads();
   }
@@ -224,10 +227,11 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     // zero upper part implied).  A is no longer needed for the factors.
     __syncthreads();
     for (int i = 1; i < len; ++i) {
-      float acc = 0.f;
-      if (tid < i) acc = -sA[i * LA + tid] - row_dot(sA, LA, tid, i, tid + 1);
+      float part = scol < i ? row_dot_half(sA, LA, scol, i, scol + 1) : 0.f;
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      const float val = scol < i ? -sA[i * LA + scol] - part : 0.f;
       __syncthreads();
-      if (tid < i) sA[i * LA + tid] = acc;
+      if (scol < i && half == 0) sA[i * LA + scol] = val;
       __syncthreads();
     }
     const size_t tile_t = ((size_t)c * H + h) * kChunk * kChunk;
