@@ -50,7 +50,7 @@ constexpr int kPrepSimtThreads = 512;
 
 template <int DK, int DV>
 constexpr size_t prep_simt_smem_bytes() {
-  return sizeof(float) * (size_t)(4 * kChunk * (DK + 1) + kChunk * (DV + 1) + 2 * kChunk * (kChunk + 1));
+  return sizeof(float) * (size_t)(4 * kChunk * (DK + 1) + kChunk * (DV + 1) + 3 * kChunk * (kChunk + 1));
 }
 
 // AFFINE selects the factor set: false stores W, U~, Kbar (WY set); true
@@ -58,7 +58,7 @@ constexpr size_t prep_simt_smem_bytes() {
 // One (chunk c, head h) per call; all kPrepSimtThreads threads take part.
 template <int DK, int DV, typename IO, typename FT, bool AFFINE>
 __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c, int h, float* smem) {
-  static_assert(2 * (DK + DV) <= kPrepSimtThreads, "two threads per solve column");
+  static_assert(kPrepSimtThreads == 512 && (DK + DV) % 32 == 0, "16 warps; [W | U~] in 32-column groups");
   constexpr int LK = DK + 1, LV = DV + 1, LA = kChunk + 1;
   const int H = a.H;
   const ChunkPos pos = chunk_pos(a.map, c);
@@ -71,7 +71,9 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   float* sz = sq + kChunk * LK;     // [64][LV]  z, then U~
   float* sA = sz + kChunk * LV;     // [64][LA]  A (strictly lower)
   float* sP = sA + kChunk * LA;     // [64][LA]  P (lower, diagonal included)
+  float* sT = sP + kChunk * LA;     // [64][LA]  T = (I + A)^-1 (lower, unit diagonal)
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
 
   batched_copy<8, float4>(
       kChunk * DK, tid, kPrepSimtThreads,
@@ -100,6 +102,7 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   for (int idx = tid; idx < kChunk * LA; idx += kPrepSimtThreads) {
     sA[idx] = 0.f;
     sP[idx] = 0.f;
+    sT[idx] = 0.f;
   }
   __syncthreads();
   // In-chunk cumulative sum, one thread per key channel.  Padded rows carry
@@ -178,66 +181,138 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
   if (AFFINE && a.colscale && tid < DK) a.colscale[((size_t)c * H + h) * DK + tid] = 1.f;
   __syncthreads();
-  // half of sum_{m0 <= m < i} A_im X_m,col: the terms m = m0 + half, m0 + half + 2,
-  // ... (two partial sums, short dependency chains); the other half comes
-  // from the neighbouring lane
-  const int scol = tid >> 1, half = tid & 1;
-  auto row_dot_half = [&](const float* X, int ld, int col, int i, int m0) {
-    float s0 = 0.f, s1 = 0.f;
-    int m = m0 + half;
-    for (; m + 2 < i; m += 4) {
-      s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
-      s1 = fmaf(sA[i * LA + m + 2], X[(m + 2) * ld + col], s1);
+  // T = (I + A)^-1 by blocks: the four 16 x 16 diagonal blocks by forward
+  // substitution (warps 0-3, lane l < 16 owns column l), then the merges
+  // 16 -> 32 and 32 -> 64, each T21 = -T22 (A21 T11).  sT starts all zero.
+  if (warp < 4) {
+    const int I = 16 * warp, l = lane;
+    float t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < i; ++m) acc = fmaf(sA[(I + i) * LA + I + m], t[m], acc);   // t[m] = 0 for m < l
+      t[i] = i < l ? 0.f : (i == l ? 1.f : -acc);
     }
-    for (; m < i; m += 2) s0 = fmaf(sA[i * LA + m], X[m * ld + col], s0);
-    return s0 + s1;
-  };
-  // Forward substitution, row by row: W_i = E~_i - sum_{j<i} A_ij W_j, and the
-  // same for U~ with Z.  Two threads per column of [W | U~].
-  for (int i = 1; i < len; ++i) {
-    float part = 0.f;
-    if (scol < DK) part = row_dot_half(se, LK, scol, i, 0);
-    else if (scol < DK + DV) part = row_dot_half(sz, LV, scol - DK, i, 0);
-    part += __shfl_xor_sync(0xffffffffu, part, 1);
-    if (half == 0) {
-      if (scol < DK) se[i * LK + scol] -= part;
-      else if (scol < DK + DV) sz[i * LV + scol - DK] -= part;
+    if (l < 16)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sT[(I + i) * LA + I + l] = t[i];
+  }
+  __syncthreads();
+  {
+    // 16 -> 32: blocks (1, 0) and (3, 2); a thread per entry of X, then of T21
+    const int m = tid >> 8, r = (tid >> 4) & 15, cc = tid & 15;
+    const int ra = 32 * m + 16, ca = 32 * m;   // A21 / T21 at rows ra.., columns ca..; T11 at ca, T22 at ra
+    float x = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x = fmaf(sA[(ra + r) * LA + ca + k], sT[(ca + k) * LA + ca + cc], x);
+    float* X = sA + (ra + r) * LA + ca + cc;   // A21 is not read again: X goes over it
+    __syncthreads();
+    *X = x;
+    __syncthreads();
+    float y = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) y = fmaf(sT[(ra + r) * LA + ra + k], sA[(ra + k) * LA + ca + cc], y);
+    sT[(ra + r) * LA + ca + cc] = -y;
+  }
+  __syncthreads();
+  {
+    // 32 -> 64: rows 32.., columns 0..; two entries per thread
+    const int r = tid >> 4, c2 = 2 * (tid & 15);
+    float x0 = 0.f, x1 = 0.f;
+    for (int k = 0; k < 32; ++k) {
+      const float av = sA[(32 + r) * LA + k];
+      x0 = fmaf(av, sT[k * LA + c2], x0);
+      x1 = fmaf(av, sT[k * LA + c2 + 1], x1);
     }
     __syncthreads();
+    sA[(32 + r) * LA + c2] = x0;       // X over A21
+    sA[(32 + r) * LA + c2 + 1] = x1;
+    __syncthreads();
+    float y0 = 0.f, y1 = 0.f;
+    for (int k = 0; k < 32; ++k) {
+      const float tv = sT[(32 + r) * LA + 32 + k];
+      y0 = fmaf(tv, sA[(32 + k) * LA + c2], y0);
+      y1 = fmaf(tv, sA[(32 + k) * LA + c2 + 1], y1);
+    }
+    sT[(32 + r) * LA + c2] = -y0;
+    sT[(32 + r) * LA + c2 + 1] = -y1;
   }
-  // Q_eff = Q~ - P W and O_part = P U~ (P is lower triangular with diagonal).
-  for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
-    const int i = idx / DK, cc = idx % DK;
-    float acc = sq[i * LK + cc];
-    for (int j = 0; j <= i && j < len; ++j) acc = fmaf(-sP[i * LA + j], se[j * LK + cc], acc);
-    a.Qeff[tile_k + idx] = from_f32<FT>(acc);
-    if constexpr (!AFFINE) a.W[tile_k + idx] = from_f32<FT>(se[i * LK + cc]);
+  __syncthreads();
+  // [W | U~] = T [E~ | Z] and then Q_eff = Q~ - P W, O_part = P U~: warp w takes
+  // rows 4w .. 4w + 3, lane l the columns l + 32 e of [W | U~] (T and P are
+  // lower triangular, so the sums stop at the tile's last row)
+  constexpr int NE = (DK + DV) / 32;
+  auto colp = [&](float* base_k, float* base_v, int m, int e) -> float* {
+    const int col = lane + 32 * e;
+    return col < DK ? base_k + m * LK + col : base_v + m * LV + (col - DK);
+  };
+  {
+    float acc[4][NE];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < NE; ++e) acc[r][e] = 0.f;
+    for (int m = 0; m < 4 * warp + 4; ++m) {
+      float tv[4], xv[NE];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) tv[r] = sT[(4 * warp + r) * LA + m];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) xv[e] = *colp(se, sz, m, e);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(tv[r], xv[e], acc[r][e]);
+    }
+    __syncthreads();   // every thread has read E~ and Z
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < NE; ++e) *colp(se, sz, 4 * warp + r, e) = acc[r][e];
   }
-  for (int idx = tid; idx < kChunk * DV; idx += kPrepSimtThreads) {
-    const int i = idx / DV, cc = idx % DV;
-    float acc = 0.f;
-    for (int j = 0; j <= i && j < len; ++j) acc = fmaf(sP[i * LA + j], sz[j * LV + cc], acc);
-    a.Opart[tile_v + idx] = from_f32<FT>(acc);
-    if constexpr (!AFFINE) a.Ut[tile_v + idx] = from_f32<FT>(sz[i * LV + cc]);
+  __syncthreads();
+  {
+    float acc[4][NE];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < NE; ++e) acc[r][e] = lane + 32 * e < DK ? sq[(4 * warp + r) * LK + lane + 32 * e] : 0.f;
+    for (int m = 0; m < 4 * warp + 4; ++m) {
+      float pv[4], xv[NE];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) pv[r] = sP[(4 * warp + r) * LA + m];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) {
+        xv[e] = *colp(se, sz, m, e);
+        if (lane + 32 * e < DK) xv[e] = -xv[e];   // Q_eff takes -P W
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(pv[r], xv[e], acc[r][e]);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i = 4 * warp + r;
+#pragma unroll
+      for (int e = 0; e < NE; ++e) {
+        const int col = lane + 32 * e;
+        if (col < DK) {
+          a.Qeff[tile_k + i * DK + col] = from_f32<FT>(acc[r][e]);
+          if constexpr (!AFFINE) a.W[tile_k + i * DK + col] = from_f32<FT>(se[i * LK + col]);
+        } else {
+          a.Opart[tile_v + i * DV + col - DK] = from_f32<FT>(acc[r][e]);
+          if constexpr (!AFFINE) a.Ut[tile_v + i * DV + col - DK] = from_f32<FT>(sz[i * LV + col - DK]);
+        }
+      }
+    }
   }
   if (a.Tm) {
-    // T = (I + A)^-1 explicitly, for the backward: rows in order, each row's
-    // entries from the rows above it (T_ij = -A_ij - sum_{j<m<i} A_im T_mj),
-    // written over A once every thread has read the row (unit diagonal and
-    // zero upper part implied).  A is no longer needed for the factors.
-    __syncthreads();
-    for (int i = 1; i < len; ++i) {
-      float part = scol < i ? row_dot_half(sA, LA, scol, i, scol + 1) : 0.f;
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      const float val = scol < i ? -sA[i * LA + scol] - part : 0.f;
-      __syncthreads();
-      if (scol < i && half == 0) sA[i * LA + scol] = val;
-      __syncthreads();
-    }
+    // T and P for the backward (T with its unit diagonal, zero above it)
     const size_t tile_t = ((size_t)c * H + h) * kChunk * kChunk;
     for (int idx = tid; idx < kChunk * kChunk; idx += kPrepSimtThreads) {
       const int i = idx / kChunk, j = idx % kChunk;
-      a.Tm[tile_t + idx] = j < i ? sA[i * LA + j] : (i == j ? 1.f : 0.f);
+      a.Tm[tile_t + idx] = sT[i * LA + j];
       a.Pm[tile_t + idx] = j <= i ? sP[i * LA + j] : 0.f;
     }
   }
