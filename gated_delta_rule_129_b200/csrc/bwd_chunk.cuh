@@ -843,15 +843,31 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   }
   __syncthreads();
   // dlog_alpha: reverse cumulative sum of dg over the chunk; the last token
-  // also carries the gradient of gamma_n
-  if (tid < DK && len > 0) {
-    const float gn = sg[(kChunk - 1) * LDK + tid];
-    float run = expf(gn) * sgs[tid] + sdgn[tid];
-    for (int i = len - 1; i >= 0; --i) {
-      const size_t o = tok_k(i, tid);
-      run += a.dla[o];
-      a.dla[o] = run;
+  // also carries the gradient of gamma_n.  PARTS adjacent lanes per channel,
+  // each a run of 64 / PARTS rows: the run's values are loaded at once, summed
+  // from the end, and offset by the totals of the runs after it (shuffles).
+  {
+    constexpr int PARTS = kBwdThreads / DK, R = kChunk / PARTS;
+    const int cc = tid / PARTS, p = tid % PARTS, i0 = p * R;
+    float v[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) v[r] = i0 + r < len ? a.dla[tok_k(i0 + r, cc)] : 0.f;
+    float run = 0.f;
+#pragma unroll
+    for (int r = R - 1; r >= 0; --r) {
+      run += v[r];
+      v[r] = run;
     }
+    float after = p == 0 ? expf(sg[(kChunk - 1) * LDK + cc]) * sgs[cc] + sdgn[cc] : 0.f;   // added to every row
+    after = __shfl_sync(0xffffffffu, after, (tid & 31) - p);                             // the channel's first lane
+#pragma unroll
+    for (int d = 1; d < PARTS; ++d) {
+      const float tot = __shfl_sync(0xffffffffu, run, ((tid & 31) + d) & 31);
+      if (p + d < PARTS) after += tot;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (i0 + r < len) a.dla[tok_k(i0 + r, cc)] = v[r] + after;
   }
 }
 

@@ -75,7 +75,7 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  batched_copy<8, float4>(
+  batched_copy<16, float4>(
       kChunk * DK, tid, kPrepSimtThreads,
       [&](int idx) {
         const int i = idx / DK, cc = idx % DK;
@@ -90,7 +90,7 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
         sq[i * LK + cc] = r.y;
         sg[i * LK + cc] = r.w;
       });
-  batched_copy<8, float>(
+  batched_copy<16, float>(
       kChunk * DV, tid, kPrepSimtThreads,
       [&](int idx) {
         const int i = idx / DV, cc = idx % DV;
