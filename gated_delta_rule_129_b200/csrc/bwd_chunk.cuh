@@ -149,14 +149,19 @@ bwd_dstate_kernel(const BwdStateArgs a) {
     // X = Kbar dS1 on a 2 x 2 tile
     {
       float x[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll 8
-      for (int cc = 0; cc < DK; ++cc) {
-        const float2 d = *reinterpret_cast<const float2*>(sdS + cc * CS + cj);
+#pragma unroll 2
+      for (int c4 = 0; c4 < DK; c4 += 4) {   // four key rows of dS a step, Kbar read as vectors
+        float kb[2][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float kb = sKb[(2 * ri + r) * LK + cc];
-          x[r][0] = fmaf(kb, d.x, x[r][0]);
-          x[r][1] = fmaf(kb, d.y, x[r][1]);
+        for (int r = 0; r < 2; ++r) load_vec<4>(sKb + (2 * ri + r) * LK + c4, kb[r]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 d = *reinterpret_cast<const float2*>(sdS + (c4 + e) * CS + cj);
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            x[r][0] = fmaf(kb[r][e], d.x, x[r][0]);
+            x[r][1] = fmaf(kb[r][e], d.y, x[r][1]);
+          }
         }
       }
 #pragma unroll
@@ -177,11 +182,13 @@ bwd_dstate_kernel(const BwdStateArgs a) {
       for (int i = 0; i < len; ++i) {
         const float2 xv = *reinterpret_cast<const float2*>(sX + i * CS + cj);
         const float o0 = a.scale * to_f32(sdO[i * CS + cj]), o1 = a.scale * to_f32(sdO[i * CS + cj + 1]);
+        float wv[RS], qv[RS];
+        load_vec<RS>(sW + i * LK + rs, wv);
+        load_vec<RS>(sQe + i * LK + rs, qv);
 #pragma unroll
         for (int r = 0; r < RS; ++r) {
-          const float wv = sW[i * LK + rs + r], qv = sQe[i * LK + rs + r];
-          s[r][0] = fmaf(qv, o0, fmaf(-wv, xv.x, s[r][0]));
-          s[r][1] = fmaf(qv, o1, fmaf(-wv, xv.y, s[r][1]));
+          s[r][0] = fmaf(qv[r], o0, fmaf(-wv[r], xv.x, s[r][0]));
+          s[r][1] = fmaf(qv[r], o1, fmaf(-wv[r], xv.y, s[r][1]));
         }
       }
 #pragma unroll

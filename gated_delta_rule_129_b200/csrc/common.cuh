@@ -78,6 +78,31 @@ __device__ __forceinline__ void batched_copy(int n, int tid, int nthr, L load, S
   }
 }
 
+// N consecutive elements (N = 2 or 4, the address a multiple of their size)
+// of a shared-memory row of fp32 or bf16, as fp32.
+template <int N>
+__device__ __forceinline__ void load_vec(const float* p, float (&o)[N]) {
+  if constexpr (N == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  } else {
+    static_assert(N == 2, "2 or 4");
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    o[0] = v.x; o[1] = v.y;
+  }
+}
+template <int N>
+__device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float (&o)[N]) {
+  if constexpr (N == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    o[0] = bf16_lo_f(v.x); o[1] = bf16_hi_f(v.x); o[2] = bf16_lo_f(v.y); o[3] = bf16_hi_f(v.y);
+  } else {
+    static_assert(N == 2, "2 or 4");
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+    o[0] = bf16_lo_f(v); o[1] = bf16_hi_f(v);
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -131,14 +131,22 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
           u[r][q] = to_f32(sUt[(2 * ri + r) * DVS + cj + q]);
           o[r][q] = to_f32(sOp[(2 * ri + r) * DVS + cj + q]);
         }
-#pragma unroll 8
-      for (int cc = 0; cc < DK; ++cc) {
-        const float2 s = *reinterpret_cast<const float2*>(sS + cc * DVS + cj);
+#pragma unroll 2
+      for (int c4 = 0; c4 < DK; c4 += 4) {   // four key rows of S a step, W and Q_eff read as vectors
+        float wv[2][4], qv[2][4];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const float wv = to_f32(sW[(2 * ri + r) * LKF + cc]), qv = to_f32(sQe[(2 * ri + r) * LKF + cc]);
-          u[r][0] = fmaf(-wv, s.x, u[r][0]); u[r][1] = fmaf(-wv, s.y, u[r][1]);
-          o[r][0] = fmaf(qv, s.x, o[r][0]); o[r][1] = fmaf(qv, s.y, o[r][1]);
+          load_vec<4>(sW + (2 * ri + r) * LKF + c4, wv[r]);
+          load_vec<4>(sQe + (2 * ri + r) * LKF + c4, qv[r]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 s = *reinterpret_cast<const float2*>(sS + (c4 + e) * DVS + cj);
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            u[r][0] = fmaf(-wv[r][e], s.x, u[r][0]); u[r][1] = fmaf(-wv[r][e], s.y, u[r][1]);
+            o[r][0] = fmaf(qv[r][e], s.x, o[r][0]); o[r][1] = fmaf(qv[r][e], s.y, o[r][1]);
+          }
         }
       }
 #pragma unroll
@@ -166,11 +174,12 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
 #pragma unroll 4
       for (int i = 0; i < len; ++i) {
         const float2 uv = *reinterpret_cast<const float2*>(sU + i * DVS + cj);
+        float kb[RS];
+        load_vec<RS>(sKb + i * LKF + rs, kb);
 #pragma unroll
         for (int r = 0; r < RS; ++r) {
-          const float kb = to_f32(sKb[i * LKF + rs + r]);
-          s[r][0] = fmaf(kb, uv.x, s[r][0]);
-          s[r][1] = fmaf(kb, uv.y, s[r][1]);
+          s[r][0] = fmaf(kb[r], uv.x, s[r][0]);
+          s[r][1] = fmaf(kb[r], uv.y, s[r][1]);
         }
       }
 #pragma unroll
