@@ -14,11 +14,12 @@
 //   U = U~ - W S0,  O = scale (Q~ S0 + P U),  S1 = diag(gamma_n) S0 + Kbar^T U
 //
 // with Q~ = q gamma and Kbar = k exp(g_n - g).  The backward runs in four
-// launches (host: gdn2_chunk_bwd):
+// steps, three launches (host: gdn2_chunk_bwd):
 //   1. the CUDA-core prep recomputes every chunk's factors in fp32 (W, U~,
 //      Kbar, Q_eff = Q~ - P W, gamma_n) and also stores T and P;
 //   2. the CUDA-core walk recomputes the state at every chunk start (S0);
-//   3. bwd_dstate_kernel walks the chunks in reverse order: the gradient
+//   3. in other blocks of the same launch (bwd_walks_kernel: the two walks
+//      are independent), the chunks are walked in reverse order: the gradient
 //      reaching a chunk's start state is the transpose of the forward's
 //      affine chunk map applied to the one reaching its end, plus the
 //      outputs' share:  dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO
@@ -46,12 +47,13 @@
 #pragma once
 
 #include "common.cuh"
+#include "walk_simt.cuh"
 
 namespace gdn2 {
 
 // ------------------------------------------------ reverse state walk ----
-constexpr int kBwdWalkThreads = 256;
-constexpr int kBwdWalkCols = 16;   // value columns per CTA
+constexpr int kBwdWalkThreads = 512;
+constexpr int kBwdWalkCols = 32;   // value columns per CTA
 
 struct BwdStateArgs {
   const float *W, *Kbar, *Qeff;   // fp32 factors [chunks, H, 64, DK]
@@ -66,16 +68,16 @@ struct BwdStateArgs {
   const int32_t* status;          // nonzero: malformed cu_seqlens (no chunks); dh0 = 0
 };
 
-// Shared memory, in bytes: two chunk buffers (W, Kbar, Q_eff rows padded by
-// 16 bytes, the dO slice, gamma_n), then dS [DK][CS] and X = Kbar dS [64][CS]
-// in fp32.
+// Shared memory, in bytes: two buffers of (Kbar with rows padded by 16 bytes,
+// the dO slice, gamma_n), one W and one Q_eff tile, then dS [DK][CS] and
+// X = Kbar dS [64][CS] in fp32.
 template <int DK, typename IO>
 struct BwdDstateCfg {
   static constexpr int CS = kBwdWalkCols, LK = DK + 4;
   static constexpr int TILE = kChunk * LK * 4, DOB = kChunk * CS * (int)sizeof(IO);
-  static constexpr int OFF_W = 0, OFF_KB = TILE, OFF_QE = 2 * TILE, OFF_DO = 3 * TILE, OFF_GL = OFF_DO + DOB,
-                       BUF = OFF_GL + DK * 4;
-  static constexpr int OFF_S = 2 * BUF, OFF_X = OFF_S + DK * CS * 4, SMEM = OFF_X + kChunk * CS * 4;
+  static constexpr int OFF_KB = 0, OFF_DO = TILE, OFF_GL = OFF_DO + DOB, BUF = OFF_GL + DK * 4;
+  static constexpr int OFF_W = 2 * BUF, OFF_QE = OFF_W + TILE, OFF_S = OFF_QE + TILE, OFF_X = OFF_S + DK * CS * 4,
+                       SMEM = OFF_X + kChunk * CS * 4;
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -84,67 +86,73 @@ constexpr size_t bwd_dstate_smem_bytes() {
   return (size_t)BwdDstateCfg<DK, float>::SMEM;   // bounds the bf16 plan
 }
 
-// One CTA per (sequence, head, kBwdWalkCols value columns): the columns of
-// dS evolve independently, since every step multiplies it from the left.  The
-// chunk's tiles are copied asynchronously into one of two buffers while the
-// chunk after it (in walk order) is computed.
+// The reverse walk of block `blk` (sequence, head, kBwdWalkCols value
+// columns): the columns of dS evolve independently, since every step
+// multiplies it from the left.  Kbar, dO and gamma_n (used first) are copied
+// into one of two buffers a chunk ahead (in walk order), W and Q_eff (used
+// last) into single buffers as soon as the previous step has read them.
 template <int DK, int DV, typename IO>
-__global__ void __launch_bounds__(kBwdWalkThreads)
-bwd_dstate_kernel(const BwdStateArgs a) {
+__device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, uint8_t* dsm) {
   using C = BwdDstateCfg<DK, IO>;
-  constexpr int CS = kBwdWalkCols, SL = DV / CS, LK = C::LK;
+  constexpr int CS = kBwdWalkCols, SL = DV / CS, LK = C::LK, NT = kBwdWalkThreads;
   const int H = a.H;
-  const int sl = blockIdx.x % SL;
-  const int h = (blockIdx.x / SL) % H;
-  const int n = blockIdx.x / (SL * H);
+  const int sl = blk % SL;
+  const int h = (blk / SL) % H;
+  const int n = blk / (SL * H);
   const int j0 = sl * CS, tid = threadIdx.x;
 
-  extern __shared__ __align__(16) uint8_t dsm[];
   float* sdS = reinterpret_cast<float*>(dsm + C::OFF_S);   // [DK][CS]
   float* sX = reinterpret_cast<float*>(dsm + C::OFF_X);    // [64][CS]
+  const float* sW = reinterpret_cast<const float*>(dsm + C::OFF_W);
+  const float* sQe = reinterpret_cast<const float*>(dsm + C::OFF_QE);
 
   const IO* dO = static_cast<const IO*>(a.dO);
   const size_t sbase = ((size_t)n * H + h) * DK * DV;
   const bool bad = *a.status != 0;
-  for (int idx = tid; idx < DK * CS; idx += kBwdWalkThreads) {
+  for (int idx = tid; idx < DK * CS; idx += NT) {
     const int cc = idx / CS, j = idx % CS;
     sdS[idx] = (!bad && a.dhT) ? a.dhT[sbase + (size_t)cc * DV + j0 + j] : 0.f;
   }
   const int c_begin = a.map.chunk_off[n], c_end = a.map.chunk_off[n + 1];
   const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
-  auto issue = [&](int c, int slot) {
+  auto issue_b = [&](int c, int slot) {   // Kbar, the dO slice, gamma_n of chunk c
     uint8_t* b = dsm + slot * C::BUF;
     const size_t tk = ((size_t)c * H + h) * kChunk * DK;
     const int t0 = s_begin + (c - c_begin) * kChunk, len = min(kChunk, s_end - t0);
-    stage_rows<DK * 4>(b + C::OFF_W, LK * 4, a.W + tk, DK * 4, kChunk, kChunk, tid, kBwdWalkThreads);
-    stage_rows<DK * 4>(b + C::OFF_KB, LK * 4, a.Kbar + tk, DK * 4, kChunk, kChunk, tid, kBwdWalkThreads);
-    stage_rows<DK * 4>(b + C::OFF_QE, LK * 4, a.Qeff + tk, DK * 4, kChunk, kChunk, tid, kBwdWalkThreads);
+    stage_rows<DK * 4>(b + C::OFF_KB, LK * 4, a.Kbar + tk, DK * 4, kChunk, kChunk, tid, NT);
     stage_rows<CS * (int)sizeof(IO)>(b + C::OFF_DO, CS * sizeof(IO), dO + ((size_t)t0 * H + h) * DV + j0,
-                                     (size_t)H * DV * sizeof(IO), kChunk, len, tid, kBwdWalkThreads);
-    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, kBwdWalkThreads);
+                                     (size_t)H * DV * sizeof(IO), kChunk, len, tid, NT);
+    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, NT);
   };
-  if (c_begin < c_end) issue(c_end - 1, 0);
+  auto issue_w = [&](int c) {   // W and Q_eff of chunk c
+    const size_t tk = ((size_t)c * H + h) * kChunk * DK;
+    stage_rows<DK * 4>(dsm + C::OFF_W, LK * 4, a.W + tk, DK * 4, kChunk, kChunk, tid, NT);
+    stage_rows<DK * 4>(dsm + C::OFF_QE, LK * 4, a.Qeff + tk, DK * 4, kChunk, kChunk, tid, NT);
+  };
+  // commit groups, oldest first: B(last), W(last), then per chunk c (in walk
+  // order): B(c - 1) at its start and W(c - 1) at its end
+  if (c_begin < c_end) issue_b(c_end - 1, 0);
+  cp_async_commit();
+  if (c_begin < c_end) issue_w(c_end - 1);
   cp_async_commit();
 
-  constexpr int RS = DK / 32;                    // rows of dS per thread
-  const int ri = tid / 8, cj = 2 * (tid % 8);    // X: rows 2 ri, 2 ri + 1; columns cj, cj + 1
-  const int rs = RS * (tid / 8);                 // dS: rows rs .. rs + RS - 1; columns cj, cj + 1
+  constexpr int RS = DK / 32;                      // rows of dS per thread
+  const int ri = tid / 16, cj = 2 * (tid % 16);    // X: rows 2 ri, 2 ri + 1; columns cj, cj + 1
+  const int rs = RS * (tid / 16);                  // dS: rows rs .. rs + RS - 1; columns cj, cj + 1
   for (int c = c_end - 1, it = 0; c >= c_begin; --c, ++it) {
-    if (c - 1 >= c_begin) issue(c - 1, (it + 1) & 1);
+    if (c - 1 >= c_begin) issue_b(c - 1, (it + 1) & 1);
     cp_async_commit();
-    cp_async_wait<1>();
+    cp_async_wait<2>();   // B(c) has landed
     __syncthreads();
     const uint8_t* b = dsm + (it & 1) * C::BUF;
-    const float* sW = reinterpret_cast<const float*>(b + C::OFF_W);
     const float* sKb = reinterpret_cast<const float*>(b + C::OFF_KB);
-    const float* sQe = reinterpret_cast<const float*>(b + C::OFF_QE);
     const IO* sdO = reinterpret_cast<const IO*>(b + C::OFF_DO);
     const float* sgl = reinterpret_cast<const float*>(b + C::OFF_GL);
     const int t0 = s_begin + (c - c_begin) * kChunk;
     const int len = min(kChunk, s_end - t0);
     // the gradient reaching this chunk's end state
     const size_t cs = ((size_t)c * H + h) * DK * DV;
-    for (int idx = tid; idx < DK * CS; idx += kBwdWalkThreads)
+    for (int idx = tid; idx < DK * CS; idx += NT)
       a.dS1[cs + (size_t)(idx / CS) * DV + j0 + idx % CS] = sdS[idx];
     // X = Kbar dS1 on a 2 x 2 tile
     {
@@ -167,6 +175,7 @@ bwd_dstate_kernel(const BwdStateArgs a) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) *reinterpret_cast<float2*>(sX + (2 * ri + r) * CS + cj) = make_float2(x[r][0], x[r][1]);
     }
+    cp_async_wait<1>();   // W(c) has landed
     __syncthreads();
     // dS0 = gamma_n dS1 - W^T X + Q_eff^T (scale dO) on an RS x 2 tile; every
     // thread rewrites only the entries of dS it read
@@ -195,14 +204,28 @@ bwd_dstate_kernel(const BwdStateArgs a) {
       for (int r = 0; r < RS; ++r)
         *reinterpret_cast<float2*>(sdS + (rs + r) * CS + cj) = make_float2(s[r][0], s[r][1]);
     }
-    __syncthreads();   // this buffer is free for the chunk after next
+    __syncthreads();   // W, Q_eff and this chunk's buffer are free
+    if (c - 1 >= c_begin) issue_w(c - 1);
+    cp_async_commit();
   }
   cp_async_wait<0>();
   __syncthreads();
-  for (int idx = tid; idx < DK * CS; idx += kBwdWalkThreads) {
+  for (int idx = tid; idx < DK * CS; idx += NT) {
     const int cc = idx / CS, j = idx % CS;
     a.dh0[sbase + (size_t)cc * DV + j0 + j] = sdS[idx];
   }
+}
+
+// The two walks of the backward in one launch (they are independent): blocks
+// [0, n_fwd) walk the chunks forward and store every chunk's start state,
+// the others walk them in reverse for the state gradient.
+template <int DK, int DV, typename IO>
+__global__ void __launch_bounds__(kBwdWalkThreads)
+bwd_walks_kernel(const WalkArgs<IO, float> wa, const BwdStateArgs ra, int n_fwd) {
+  static_assert(kBwdWalkThreads == kWalkSimtThreads, "one block size for both walks");
+  extern __shared__ __align__(16) uint8_t bsm[];
+  if ((int)blockIdx.x < n_fwd) walk_simt_cta<DK, DV, IO, float>(wa, blockIdx.x, bsm);
+  else bwd_dstate_cta<DK, DV, IO>(ra, blockIdx.x - n_fwd, bsm);
 }
 
 // -------------------------------------------------- per-chunk gradients ----

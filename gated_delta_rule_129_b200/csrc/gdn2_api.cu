@@ -584,7 +584,8 @@ struct BwdOp {
       if ((st = launch_status()) != GDN2_OK) return st;
     }
     if (L.N == 0) return GDN2_OK;
-    // 2. the state at every chunk start
+    // 2. the state at every chunk start and 3. the gradient reaching every
+    // chunk's end state (and dh0), in one launch
     {
       gdn2::WalkArgs<IO, float> wa;
       wa.W = at<const float>(f.workspace, L.l.off_W);
@@ -600,22 +601,11 @@ struct BwdOp {
       wa.out = nullptr;
       wa.hT = nullptr;
       wa.chunk_states = at<float>(d->workspace, B.off_S0);
-      constexpr size_t smem = gdn2::walk_simt_smem_bytes<DK, DV>();
-      auto kern = gdn2::walk_simt_kernel<DK, DV, IO, float>;
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return GDN2_ERR_CUDA;
-      const long long blocks = (long long)L.N * d->H * (DV / gdn2::kWalkSimtDVS);
-      if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
-      kern<<<(unsigned)blocks, gdn2::kWalkSimtThreads, smem, s>>>(wa);
-      if ((st = launch_status()) != GDN2_OK) return st;
-    }
-    // 3. the gradient reaching every chunk's end state, and dh0
-    {
       gdn2::BwdStateArgs ra;
-      ra.W = at<const float>(f.workspace, L.l.off_W);
-      ra.Kbar = at<const float>(f.workspace, L.l.off_Kbar);
-      ra.Qeff = at<const float>(f.workspace, L.l.off_Qeff);
-      ra.gamma_last = at<const float>(f.workspace, L.l.off_gamma_last);
+      ra.W = wa.W;
+      ra.Kbar = wa.Kbar;
+      ra.Qeff = wa.Qeff;
+      ra.gamma_last = wa.gamma_last;
       ra.dO = dO;
       ra.map = map;
       ra.H = d->H;
@@ -624,13 +614,14 @@ struct BwdOp {
       ra.dS1 = at<float>(d->workspace, B.off_dS1);
       ra.dh0 = dh0;
       ra.status = status;
-      constexpr size_t smem = gdn2::bwd_dstate_smem_bytes<DK>();
-      auto kern = gdn2::bwd_dstate_kernel<DK, DV, IO>;
+      constexpr size_t smem = std::max(gdn2::walk_simt_smem_bytes<DK, DV>(), gdn2::bwd_dstate_smem_bytes<DK>());
+      auto kern = gdn2::bwd_walks_kernel<DK, DV, IO>;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GDN2_ERR_CUDA;
-      const long long blocks = (long long)L.N * d->H * (DV / gdn2::kBwdWalkCols);
-      if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
-      kern<<<(unsigned)blocks, gdn2::kBwdWalkThreads, smem, s>>>(ra);
+      const long long n_fwd = (long long)L.N * d->H * (DV / gdn2::kWalkSimtDVS);
+      const long long n_rev = (long long)L.N * d->H * (DV / gdn2::kBwdWalkCols);
+      if (n_fwd + n_rev > INT32_MAX) return GDN2_ERR_SHAPE;
+      kern<<<(unsigned)(n_fwd + n_rev), gdn2::kBwdWalkThreads, smem, s>>>(wa, ra, (int)n_fwd);
       if ((st = launch_status()) != GDN2_OK) return st;
     }
     // 4. every (chunk, head): the gradients of its tokens

@@ -12,10 +12,12 @@
 //   S <- diag(gamma_last) S + Kbar^T U       state at the next chunk start
 // hT receives the final state; h0 (or zero) is the first start state.
 //
-// The chunk's factor tiles are copied to shared memory asynchronously into
-// one of two buffers while the previous chunk is computed; both products run
-// on register tiles (a thread holds 2 x 2 of U and O, dk / 32 x 2 of S; every
-// thread updates only the entries of S it read).
+// The chunk's tiles are copied to shared memory asynchronously: W, Q_eff,
+// U~, O_part and gamma_n (used first) into one of two buffers a chunk ahead,
+// Kbar (used last) into a single buffer as soon as the previous chunk's
+// state update has read it.  Both products run on register tiles (a thread
+// holds 2 x 2 of U and O, dk / 32 x 2 of S, and updates only the entries of
+// S it read).
 #pragma once
 
 #include "common.cuh"
@@ -39,21 +41,22 @@ struct WalkArgs {
   float* chunk_states;  // optional [max_chunks, H, DK, DV]
 };
 
-constexpr int kWalkSimtThreads = 256;
-constexpr int kWalkSimtDVS = 16;
+constexpr int kWalkSimtThreads = 512;
+constexpr int kWalkSimtDVS = 32;
 
-// Shared memory, in bytes: two chunk buffers (W, Kbar, Q_eff rows padded by
-// 16 bytes; U~ and O_part slices; gamma_n), then S [DK][DVS] and U [64][DVS]
-// in fp32.
+// Shared memory, in bytes: two buffers of (W, Q_eff with rows padded by 16
+// bytes; the U~ and O_part slices; gamma_n), one Kbar tile, then S [DK][DVS]
+// and U [64][DVS] in fp32.
 template <int DK, typename FT>
 struct WalkSimtCfg {
+  static constexpr int DVS = kWalkSimtDVS;
   static constexpr int LKF = DK + 16 / (int)sizeof(FT);           // elements per padded row
   static constexpr int TILE = kChunk * LKF * (int)sizeof(FT);
-  static constexpr int VSL = kChunk * kWalkSimtDVS * (int)sizeof(FT);
-  static constexpr int OFF_W = 0, OFF_KB = TILE, OFF_QE = 2 * TILE, OFF_UT = 3 * TILE, OFF_OP = OFF_UT + VSL,
-                       OFF_GL = OFF_OP + VSL, BUF = OFF_GL + DK * 4;
-  static constexpr int OFF_S = 2 * BUF, OFF_U = OFF_S + DK * kWalkSimtDVS * 4;
-  static constexpr int SMEM = OFF_U + kChunk * kWalkSimtDVS * 4;
+  static constexpr int VSL = kChunk * DVS * (int)sizeof(FT);
+  static constexpr int OFF_W = 0, OFF_QE = TILE, OFF_UT = 2 * TILE, OFF_OP = OFF_UT + VSL, OFF_GL = OFF_OP + VSL,
+                       BUF = OFF_GL + DK * 4;
+  static constexpr int OFF_KB = 2 * BUF, OFF_S = OFF_KB + TILE, OFF_U = OFF_S + DK * DVS * 4;
+  static constexpr int SMEM = OFF_U + kChunk * DVS * 4;
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -62,54 +65,61 @@ constexpr size_t walk_simt_smem_bytes() {
   return (size_t)WalkSimtCfg<DK, float>::SMEM;   // the fp32 plan bounds the bf16 one
 }
 
+// The walk of block `blk` (sequence, head, value slice) with `wsm` its shared
+// memory; all kWalkSimtThreads threads of the CTA take part.
 template <int DK, int DV, typename IO, typename FT>
-__global__ void __launch_bounds__(kWalkSimtThreads)
-walk_simt_kernel(const WalkArgs<IO, FT> a) {
+__device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk, uint8_t* wsm) {
   using C = WalkSimtCfg<DK, FT>;
-  constexpr int DVS = kWalkSimtDVS, SLICES = DV / DVS, LKF = C::LKF;
+  constexpr int DVS = kWalkSimtDVS, SLICES = DV / DVS, LKF = C::LKF, NT = kWalkSimtThreads;
   const int H = a.H;
-  const int sl = blockIdx.x % SLICES;
-  const int h = (blockIdx.x / SLICES) % H;
-  const int n = blockIdx.x / (SLICES * H);
+  const int sl = blk % SLICES;
+  const int h = (blk / SLICES) % H;
+  const int n = blk / (SLICES * H);
   const int j0 = sl * DVS;
   const int tid = threadIdx.x;
 
-  extern __shared__ __align__(16) uint8_t wsm[];
   float* sS = reinterpret_cast<float*>(wsm + C::OFF_S);   // [DK][DVS]
   float* sU = reinterpret_cast<float*>(wsm + C::OFF_U);   // [64][DVS]
+  const FT* sKb = reinterpret_cast<const FT*>(wsm + C::OFF_KB);
 
   const size_t state_base = ((size_t)n * H + h) * DK * DV;
-  for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads) {
+  for (int idx = tid; idx < DK * DVS; idx += NT) {
     const int cc = idx / DVS, j = idx % DVS;
     sS[idx] = a.h0 ? a.h0[state_base + (size_t)cc * DV + j0 + j] : 0.f;
   }
   const int c_begin = a.map.chunk_off[n], c_end = a.map.chunk_off[n + 1];
   const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
-  auto issue = [&](int c) {   // chunk c's tiles into buffer c & 1
+  constexpr int RB = DK * (int)sizeof(FT), SB = DVS * (int)sizeof(FT);
+  auto issue_a = [&](int c) {   // W, Q_eff, U~, O_part, gamma_n of chunk c into buffer c & 1
     uint8_t* b = wsm + (c & 1) * C::BUF;
     const size_t tk = ((size_t)c * H + h) * kChunk * DK, tv = ((size_t)c * H + h) * kChunk * DV;
-    constexpr int RB = DK * (int)sizeof(FT), SB = DVS * (int)sizeof(FT);
-    stage_rows<RB>(b + C::OFF_W, LKF * sizeof(FT), a.W + tk, RB, kChunk, kChunk, tid, kWalkSimtThreads);
-    stage_rows<RB>(b + C::OFF_KB, LKF * sizeof(FT), a.Kbar + tk, RB, kChunk, kChunk, tid, kWalkSimtThreads);
-    stage_rows<RB>(b + C::OFF_QE, LKF * sizeof(FT), a.Qeff + tk, RB, kChunk, kChunk, tid, kWalkSimtThreads);
-    stage_rows<SB>(b + C::OFF_UT, SB, a.Ut + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, kWalkSimtThreads);
-    stage_rows<SB>(b + C::OFF_OP, SB, a.Opart + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, kWalkSimtThreads);
-    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, kWalkSimtThreads);
+    stage_rows<RB>(b + C::OFF_W, LKF * sizeof(FT), a.W + tk, RB, kChunk, kChunk, tid, NT);
+    stage_rows<RB>(b + C::OFF_QE, LKF * sizeof(FT), a.Qeff + tk, RB, kChunk, kChunk, tid, NT);
+    stage_rows<SB>(b + C::OFF_UT, SB, a.Ut + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, NT);
+    stage_rows<SB>(b + C::OFF_OP, SB, a.Opart + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, NT);
+    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, NT);
   };
-  if (c_begin < c_end) issue(c_begin);
+  auto issue_k = [&](int c) {   // Kbar of chunk c
+    stage_rows<RB>(wsm + C::OFF_KB, LKF * sizeof(FT), a.Kbar + ((size_t)c * H + h) * kChunk * DK, RB, kChunk, kChunk,
+                   tid, NT);
+  };
+  // commit groups, oldest first: A(c_begin), K(c_begin), then per chunk c:
+  // A(c + 1) at its start and K(c + 1) at its end (empty groups past the last)
+  if (c_begin < c_end) issue_a(c_begin);
+  cp_async_commit();
+  if (c_begin < c_end) issue_k(c_begin);
   cp_async_commit();
 
-  constexpr int RS = DK / 32;                     // rows of S per thread
-  const int ri = tid / 8, cj = 2 * (tid % 8);     // U, O: rows 2 ri, 2 ri + 1; columns cj, cj + 1
-  const int rs = RS * (tid / 8);                 // S: rows rs .. rs + RS - 1; columns cj, cj + 1
+  constexpr int RS = DK / 32;                      // rows of S per thread
+  const int ri = tid / 16, cj = 2 * (tid % 16);    // U, O: rows 2 ri, 2 ri + 1; columns cj, cj + 1
+  const int rs = RS * (tid / 16);                  // S: rows rs .. rs + RS - 1; columns cj, cj + 1
   for (int c = c_begin; c < c_end; ++c) {
-    if (c + 1 < c_end) issue(c + 1);
+    if (c + 1 < c_end) issue_a(c + 1);
     cp_async_commit();
-    cp_async_wait<1>();   // this chunk's copies have landed (the next chunk's may be in flight)
+    cp_async_wait<2>();   // A(c) has landed (K(c) and A(c + 1) may be in flight)
     __syncthreads();
     const uint8_t* b = wsm + (c & 1) * C::BUF;
     const FT* sW = reinterpret_cast<const FT*>(b + C::OFF_W);
-    const FT* sKb = reinterpret_cast<const FT*>(b + C::OFF_KB);
     const FT* sQe = reinterpret_cast<const FT*>(b + C::OFF_QE);
     const FT* sUt = reinterpret_cast<const FT*>(b + C::OFF_UT);
     const FT* sOp = reinterpret_cast<const FT*>(b + C::OFF_OP);
@@ -118,7 +128,7 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
     const int len = min(kChunk, s_end - t0);
     if (a.chunk_states) {
       const size_t cs = ((size_t)c * H + h) * DK * DV;
-      for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads)
+      for (int idx = tid; idx < DK * DVS; idx += NT)
         a.chunk_states[cs + (size_t)(idx / DVS) * DV + j0 + idx % DVS] = sS[idx];
     }
     // U = U~ - W S and O = Q_eff S + O_part on a 2 x 2 tile
@@ -160,6 +170,7 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
         }
       }
     }
+    cp_async_wait<1>();   // K(c) has landed
     __syncthreads();
     // S <- diag(gamma_n) S + Kbar^T U on an RS x 2 tile (rows of Kbar and U
     // past the chunk's last token are zero)
@@ -186,16 +197,25 @@ walk_simt_kernel(const WalkArgs<IO, FT> a) {
       for (int r = 0; r < RS; ++r)
         *reinterpret_cast<float2*>(sS + (rs + r) * DVS + cj) = make_float2(s[r][0], s[r][1]);
     }
-    __syncthreads();   // this buffer is free for chunk c + 2
+    __syncthreads();   // Kbar and this chunk's buffer are free
+    if (c + 1 < c_end) issue_k(c + 1);
+    cp_async_commit();
   }
   cp_async_wait<0>();
   __syncthreads();
   if (a.hT) {
-    for (int idx = tid; idx < DK * DVS; idx += kWalkSimtThreads) {
+    for (int idx = tid; idx < DK * DVS; idx += NT) {
       const int cc = idx / DVS, j = idx % DVS;
       a.hT[state_base + (size_t)cc * DV + j0 + j] = sS[idx];
     }
   }
+}
+
+template <int DK, int DV, typename IO, typename FT>
+__global__ void __launch_bounds__(kWalkSimtThreads)
+walk_simt_kernel(const WalkArgs<IO, FT> a) {
+  extern __shared__ __align__(16) uint8_t wsm[];
+  walk_simt_cta<DK, DV, IO, FT>(a, blockIdx.x, wsm);
 }
 
 }  // namespace gdn2
