@@ -64,6 +64,7 @@ struct BwdStateArgs {
   float scale;
   const float* dhT;               // [N, H, DK, DV] or nullptr (zero)
   float* dS1;                     // out: [chunks, H, DK, DV], gradient at each chunk's end state
+  float* X;                       // out: [chunks, H, 64, DV], Kbar dS1 of each chunk
   float* dh0;                     // out: [N, H, DK, DV]
   const int32_t* status;          // nonzero: malformed cu_seqlens (no chunks); dh0 = 0
 };
@@ -173,7 +174,11 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
         }
       }
 #pragma unroll
-      for (int r = 0; r < 2; ++r) *reinterpret_cast<float2*>(sX + (2 * ri + r) * CS + cj) = make_float2(x[r][0], x[r][1]);
+      for (int r = 0; r < 2; ++r) {
+        *reinterpret_cast<float2*>(sX + (2 * ri + r) * CS + cj) = make_float2(x[r][0], x[r][1]);
+        *reinterpret_cast<float2*>(a.X + (((size_t)c * H + h) * kChunk + 2 * ri + r) * DV + j0 + cj) =
+            make_float2(x[r][0], x[r][1]);
+      }
     }
     cp_async_wait<1>();   // W(c) has landed
     __syncthreads();
@@ -236,9 +241,9 @@ constexpr float kBwdFoldNats = 60.f;  // decay range (each side of the reference
 struct BwdChunkArgs {
   const void *q, *k, *v, *dO;     // io dtype, [T_total, H, d]
   const float *la, *b, *w;        // [T_total, H, d]
-  const float *W, *Ut, *Kbar;     // fp32 factors [chunks, H, 64, d]
   const float *Tm, *Pm;           // [chunks, H, 64, 64]
   const float *S0, *dS1;          // [chunks, H, DK, DV]
+  const float *U, *X;             // [chunks, H, 64, DV]: U = U~ - W S0 and Kbar dS1, from the two walks
   SeqMap map;
   int H;
   float scale;
@@ -256,8 +261,8 @@ struct BwdCfg {
   static constexpr int SQ = kChunk * LT;                                         // one pair-sized slot
   // T, and P (then dP), for the whole call
   static constexpr int OFF_T = 0, OFF_P = SQ, A0 = 2 * SQ;
-  // the value loop: W, Kbar, then the pass's tiles (dO and the raw v rows in io dtype)
-  static constexpr int OFF_W = A0, OFF_KB = A0 + kChunk * LDK, OFF_V = A0 + 2 * kChunk * LDK;
+  // the value loop: the pass's tiles (dO in io dtype)
+  static constexpr int OFF_V = A0;
   static constexpr int OFF_S0T = OFF_V, OFF_D1T = OFF_S0T + VB * LDK, OFF_U = OFF_D1T + VB * LDK,
                        OFF_DU = OFF_U + kChunk * LVB, OFF_UT = OFF_DU + kChunk * LVB, OFF_ZT = OFF_UT + VB * LT,
                        OFF_DO = OFF_ZT + VB * LT,                                  // [64][VB] io
@@ -296,7 +301,7 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   const ChunkPos pos = chunk_pos(a.map, c);
   const int len = pos.len, t0 = pos.t0;
   const size_t ch = (size_t)c * H + h;
-  const size_t tile_k = ch * kChunk * DK, tile_v = ch * kChunk * DV, tile_t = ch * kChunk * kChunk;
+  const size_t tile_v = ch * kChunk * DV, tile_t = ch * kChunk * kChunk;
   const size_t st = ch * DK * DV;
   auto tok_k = [&](int i, int cc) { return ((size_t)(t0 + i) * H + h) * DK + cc; };
   auto tok_v = [&](int i, int j) { return ((size_t)(t0 + i) * H + h) * DV + j; };
@@ -310,8 +315,6 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   // ------------------------------------------------ persistent tiles ----
   stage_rows<kChunk * 4>(sT, LT * 4, a.Tm + tile_t, kChunk * 4, kChunk, kChunk, tid, kBwdThreads);
   stage_rows<kChunk * 4>(sP, LT * 4, a.Pm + tile_t, kChunk * 4, kChunk, kChunk, tid, kBwdThreads);
-  stage_rows<DK * 4>(sm + C::OFF_W, LDK * 4, a.W + tile_k, DK * 4, kChunk, kChunk, tid, kBwdThreads);
-  stage_rows<DK * 4>(sm + C::OFF_KB, LDK * 4, a.Kbar + tile_k, DK * 4, kChunk, kChunk, tid, kBwdThreads);
   cp_async_commit();
   for (int i = tid; i < 2 * DK; i += kBwdThreads) sgs[i] = 0.f;
 
@@ -330,23 +333,23 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     for (int jj = 0; jj < 4; ++jj) accP[ii][jj] = accT[ii][jj] = 0.f;
 
   // ---------------------------------------------------- value loop ----
-  // per pass of VB value columns: U = U~ - W S0 and dU = scale P^T dO + Kbar dS1,
-  // then dQ~, dKbar, dW (key tiles), dP, dT (pair tiles) gather the pass's
-  // terms, and dZ gives the pass's dv, dw.  (scale is applied to the sums of
-  // dO terms: here for dU, when dQ~ and dP are used.)
+  // per pass of VB value columns: U (from the forward walk) and
+  // dU = scale P^T dO + Kbar dS1 (Kbar dS1 from the reverse walk), then dQ~,
+  // dKbar, dW (key tiles), dP, dT (pair tiles) gather the pass's terms, and
+  // dZ gives the pass's dv, dw.  (scale is applied to the sums of dO terms:
+  // here for dU, when dQ~ and dP are used.)
   {
-    const float* sW = sm + C::OFF_W;
-    const float* sKb = sm + C::OFF_KB;
     float* sS0T = sm + C::OFF_S0T;   // [VB][LDK]
     float* sD1T = sm + C::OFF_D1T;   // [VB][LDK]
-    float* sU = sm + C::OFF_U;       // [64][LVB], U~ then U
-    float* sdU = sm + C::OFF_DU;     // [64][LVB]
+    float* sU = sm + C::OFF_U;       // [64][LVB], U
+    float* sdU = sm + C::OFF_DU;     // [64][LVB], Kbar dS1 then dU
     float* sUT = sm + C::OFF_UT;     // [VB][LT]
     float* sZT = sm + C::OFF_ZT;     // [VB][LT]
     IO* sdO = reinterpret_cast<IO*>(sm + C::OFF_DO);   // [64][VB]
     for (int v0 = 0; v0 < DV; v0 += VB) {
       __syncthreads();  // the previous pass's readers are done
-      stage_rows<VB * 4>(sU, LVB * 4, a.Ut + tile_v + v0, DV * 4, kChunk, kChunk, tid, kBwdThreads);
+      stage_rows<VB * 4>(sU, LVB * 4, a.U + tile_v + v0, DV * 4, kChunk, kChunk, tid, kBwdThreads);
+      stage_rows<VB * 4>(sdU, LVB * 4, a.X + tile_v + v0, DV * 4, kChunk, kChunk, tid, kBwdThreads);
       stage_rows<VB * (int)sizeof(IO)>(sdO, VB * sizeof(IO), static_cast<const IO*>(a.dO) + tok_v(0, v0),
                                        (size_t)H * DV * sizeof(IO), kChunk, len, tid, kBwdThreads);
       cp_async_commit();
@@ -389,49 +392,23 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
         for (int j = 0; j < VB; ++j) sacc = fmaf(sS0T[j * LDK + tid], sD1T[j * LDK + tid], sacc);
         sgs[tid] += sacc;
       }
-      // U and dU on 2 x 2 tiles (rows rv, rv + 1; columns cv, cv + 16)
+      // dU = Kbar dS1 + scale P^T dO and U^T on 2 x 2 tiles (rows rv, rv + 1;
+      // columns cv, cv + 16: a thread rewrites only the entries it reads)
       {
-        float u[2][2], kd[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pd[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          u[r][0] = sU[(rv + r) * LVB + cv];
-          u[r][1] = sU[(rv + r) * LVB + cv + 16];
-        }
-#pragma unroll 2
-        for (int c4 = 0; c4 < DK; c4 += 4) {
-          float wr[2][4], kr[2][4], s0[2][4], d1[2][4];
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            unpack4(*reinterpret_cast<const float4*>(sW + (rv + r) * LDK + c4), wr[r], 0);
-            unpack4(*reinterpret_cast<const float4*>(sKb + (rv + r) * LDK + c4), kr[r], 0);
-            unpack4(*reinterpret_cast<const float4*>(sS0T + (cv + 16 * r) * LDK + c4), s0[r], 0);
-            unpack4(*reinterpret_cast<const float4*>(sD1T + (cv + 16 * r) * LDK + c4), d1[r], 0);
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                u[r][q] = fmaf(-wr[r][e], s0[q][e], u[r][q]);
-                kd[r][q] = fmaf(kr[r][e], d1[q][e], kd[r][q]);
-              }
-        }
+        float pd[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         for (int j = rv; j < kChunk; ++j) {   // P_{j, i} = 0 for j < i
           const float2 p = *reinterpret_cast<const float2*>(sP + j * LT + rv);
           const float o0 = to_f32(sdO[j * VB + cv]), o1 = to_f32(sdO[j * VB + cv + 16]);
           pd[0][0] = fmaf(p.x, o0, pd[0][0]); pd[0][1] = fmaf(p.x, o1, pd[0][1]);
           pd[1][0] = fmaf(p.y, o0, pd[1][0]); pd[1][1] = fmaf(p.y, o1, pd[1][1]);
         }
-        __syncthreads();   // every thread has read its U~ before any U is written
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             const int i = rv + r, j = cv + 16 * q;
-            sU[i * LVB + j] = u[r][q];
-            sUT[j * LT + i] = u[r][q];
-            sdU[i * LVB + j] = fmaf(a.scale, pd[r][q], kd[r][q]);
+            sUT[j * LT + i] = sU[i * LVB + j];
+            sdU[i * LVB + j] = fmaf(a.scale, pd[r][q], sdU[i * LVB + j]);
           }
       }
       __syncthreads();

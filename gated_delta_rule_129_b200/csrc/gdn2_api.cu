@@ -376,6 +376,7 @@ gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, cons
   a.out = static_cast<IO*>(out);
   a.hT = hT;
   a.chunk_states = chunk_states;
+  a.U_out = nullptr;
   if constexpr (DK == 128 && std::is_same<IO, bf16>::value) {
     if (L.l.factor_set == 1) return launch_walk_tc<DV>(d, L, scale, h0, cu, out, hT, chunk_states, s);
   }
@@ -527,10 +528,11 @@ struct DecodeOp {
 // Workspace of gdn2_chunk_bwd: the status word; the forward's fp32 WY factor
 // set (the layout gdn2_chunk_fwd uses for fp32 I/O, whatever the I/O type of
 // the call), with its chunk map; T and P of every (chunk, head); the state at
-// every chunk start (S0); the gradient reaching every chunk's end (dS1).
+// every chunk start (S0); the gradient reaching every chunk's end (dS1); and
+// from the two walks, U = U~ - W S0 and Kbar dS1 of every chunk.
 struct BwdLayout {
   Layout f;            // the factor set, relative to the workspace + kAlign
-  size_t off_T, off_P, off_S0, off_dS1, total;   // from the workspace start
+  size_t off_T, off_P, off_S0, off_dS1, off_U, off_X, total;   // from the workspace start
 };
 
 gdn2_desc bwd_factor_desc(const gdn2_desc* d) {
@@ -551,6 +553,8 @@ gdn2_status bwd_layout(const gdn2_desc* d, bool packed, BwdLayout* B) {
   B->off_P = off;   off = align_up(off + chunks_h * kChunk * kChunk * sizeof(float));
   B->off_S0 = off;  off = align_up(off + chunks_h * d->dk * d->dv * sizeof(float));
   B->off_dS1 = off; off = align_up(off + chunks_h * d->dk * d->dv * sizeof(float));
+  B->off_U = off;   off = align_up(off + chunks_h * kChunk * d->dv * sizeof(float));
+  B->off_X = off;   off = align_up(off + chunks_h * kChunk * d->dv * sizeof(float));
   B->total = off;
   return GDN2_OK;
 }
@@ -601,6 +605,7 @@ struct BwdOp {
       wa.out = nullptr;
       wa.hT = nullptr;
       wa.chunk_states = at<float>(d->workspace, B.off_S0);
+      wa.U_out = at<float>(d->workspace, B.off_U);
       gdn2::BwdStateArgs ra;
       ra.W = wa.W;
       ra.Kbar = wa.Kbar;
@@ -612,6 +617,7 @@ struct BwdOp {
       ra.scale = scale;
       ra.dhT = dhT;
       ra.dS1 = at<float>(d->workspace, B.off_dS1);
+      ra.X = at<float>(d->workspace, B.off_X);
       ra.dh0 = dh0;
       ra.status = status;
       constexpr size_t smem = std::max(gdn2::walk_simt_smem_bytes<DK, DV>(), gdn2::bwd_dstate_smem_bytes<DK>());
@@ -629,13 +635,12 @@ struct BwdOp {
     gdn2::BwdChunkArgs ca;
     ca.q = q; ca.k = k; ca.v = v; ca.dO = dO;
     ca.la = la; ca.b = b; ca.w = w;
-    ca.W = at<const float>(f.workspace, L.l.off_W);
-    ca.Ut = at<const float>(f.workspace, L.l.off_Ut);
-    ca.Kbar = at<const float>(f.workspace, L.l.off_Kbar);
     ca.Tm = at<const float>(d->workspace, B.off_T);
     ca.Pm = at<const float>(d->workspace, B.off_P);
     ca.S0 = at<const float>(d->workspace, B.off_S0);
     ca.dS1 = at<const float>(d->workspace, B.off_dS1);
+    ca.U = at<const float>(d->workspace, B.off_U);
+    ca.X = at<const float>(d->workspace, B.off_X);
     ca.map = map;
     ca.H = d->H;
     ca.scale = scale;

@@ -39,6 +39,7 @@ struct WalkArgs {
   IO* out;              // nullptr: states only (the backward's recompute)
   float* hT;
   float* chunk_states;  // optional [max_chunks, H, DK, DV]
+  float* U_out;         // optional [max_chunks, H, 64, DV]: every chunk's U (the backward)
 };
 
 constexpr int kWalkSimtThreads = 512;
@@ -163,6 +164,9 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
       for (int r = 0; r < 2; ++r) {
         const int i = 2 * ri + r;
         *reinterpret_cast<float2*>(sU + i * DVS + cj) = make_float2(u[r][0], u[r][1]);
+        if (a.U_out)
+          *reinterpret_cast<float2*>(a.U_out + (((size_t)c * H + h) * kChunk + i) * DV + j0 + cj) =
+              make_float2(u[r][0], u[r][1]);
         if (a.out && i < len) {
           const size_t off = ((size_t)(t0 + i) * H + h) * DV + j0 + cj;
           a.out[off] = from_f32<IO>(a.scale * o[r][0]);
