@@ -235,7 +235,7 @@ bwd_walks_kernel(const WalkArgs<IO, float> wa, const BwdStateArgs ra, int n_fwd)
 
 // -------------------------------------------------- per-chunk gradients ----
 constexpr int kBwdThreads = 512;
-constexpr int kBwdVB = 32;            // value columns per pass of the value loop
+constexpr int kBwdVB = 64;            // value columns per pass of the value loop
 constexpr float kBwdFoldNats = 60.f;  // decay range (each side of the reference row) for the product form
 
 struct BwdChunkArgs {
@@ -266,17 +266,19 @@ struct BwdCfg {
   static constexpr int OFF_S0T = OFF_V, OFF_D1T = OFF_S0T + VB * LDK, OFF_U = OFF_D1T + VB * LDK,
                        OFF_DU = OFF_U + kChunk * LVB, OFF_UT = OFF_DU + kChunk * LVB, OFF_ZT = OFF_UT + VB * LT,
                        OFF_DO = OFF_ZT + VB * LT,                                  // [64][VB] io
-                       END_V = OFF_DO + (kChunk * VB * (int)sizeof(IO) + 3) / 4;
+                       OFF_WS = OFF_DO + (kChunk * VB * (int)sizeof(IO) + 3) / 4,  // [64][VB] w (fp32)
+                       OFF_VS = OFF_WS + kChunk * VB,                              // [64][VB] v (io)
+                       END_V = OFF_VS + (kChunk * VB * (int)sizeof(IO) + 3) / 4;
   // after it, key-sized slots: g; k (then k beta); q / E~^T / T^T, X / q; dW / dT, X / dA; e alpha or e
   static constexpr int S_G = A0, S_K = A0 + MAT, S_2 = A0 + 2 * MAT, S_3 = A0 + 3 * MAT, S_4 = A0 + 4 * MAT,
                        END_K = A0 + 5 * MAT;
   static constexpr int OFF_RED = (END_V > END_K ? END_V : END_K);   // [DK] x 2: rowsum(dS1 S0), colsum(dKbar Kbar)
   static constexpr int FLOATS = OFF_RED + 2 * DK + 4;
   static constexpr size_t SMEM = sizeof(float) * (size_t)FLOATS;
-  // thread tiles: 64 x DK (4 columns, TMK rows), 64 x 64 (2 x 4), 64 x VB (2 x 2)
-  static constexpr int CGK = DK / 4, TMK = kChunk * CGK / kBwdThreads;
+  // thread tiles: 64 x DK (4 columns, TMK rows), 64 x 64 (2 x 4), 64 x VB (2 x QN)
+  static constexpr int CGK = DK / 4, TMK = kChunk * CGK / kBwdThreads, QN = VB / 16;
   static_assert(TMK * (kBwdThreads / CGK) == kChunk, "key tile");
-  static_assert(kChunk * VB == 4 * kBwdThreads && kChunk * kChunk == 8 * kBwdThreads, "value and pair tiles");
+  static_assert(kChunk * VB == 2 * QN * kBwdThreads && kChunk * kChunk == 8 * kBwdThreads, "value and pair tiles");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -294,7 +296,7 @@ template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_chunk_kernel(const BwdChunkArgs a) {
   using C = BwdCfg<DK, DV, IO>;
-  constexpr int LDK = C::LDK, LT = C::LT, VB = C::VB, LVB = C::LVB, TMK = C::TMK;
+  constexpr int LDK = C::LDK, LT = C::LT, VB = C::VB, LVB = C::LVB, TMK = C::TMK, QN = C::QN;
   const int c = blockIdx.x, h = blockIdx.y;
   if (c >= a.map.chunk_off[a.map.N]) return;
   const int H = a.H, tid = threadIdx.x;
@@ -321,7 +323,7 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   // thread tiles
   const int rk0 = TMK * (tid / C::CGK), ck0 = 4 * (tid % C::CGK);   // 64 x DK
   const int rp0 = 2 * (tid / 16), cp0 = 4 * (tid % 16);             // 64 x 64
-  const int rv = 2 * (tid / 16), cv = tid % 16;                     // 64 x VB: rows rv, rv + 1; columns cv, cv + 16
+  const int rv = 2 * (tid / 16), cv = tid % 16;                     // 64 x VB: rows rv, rv + 1; columns cv + 16 q
   float accQ[TMK][4], accKb[TMK][4], accW[TMK][4], accP[2][4], accT[2][4];
 #pragma unroll
   for (int ii = 0; ii < TMK; ++ii)
@@ -346,66 +348,69 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     float* sUT = sm + C::OFF_UT;     // [VB][LT]
     float* sZT = sm + C::OFF_ZT;     // [VB][LT]
     IO* sdO = reinterpret_cast<IO*>(sm + C::OFF_DO);   // [64][VB]
+    float* sws = sm + C::OFF_WS;                          // [64][VB] w
+    IO* svs = reinterpret_cast<IO*>(sm + C::OFF_VS);     // [64][VB] v
     for (int v0 = 0; v0 < DV; v0 += VB) {
       __syncthreads();  // the previous pass's readers are done
       stage_rows<VB * 4>(sU, LVB * 4, a.U + tile_v + v0, DV * 4, kChunk, kChunk, tid, kBwdThreads);
       stage_rows<VB * 4>(sdU, LVB * 4, a.X + tile_v + v0, DV * 4, kChunk, kChunk, tid, kBwdThreads);
       stage_rows<VB * (int)sizeof(IO)>(sdO, VB * sizeof(IO), static_cast<const IO*>(a.dO) + tok_v(0, v0),
                                        (size_t)H * DV * sizeof(IO), kChunk, len, tid, kBwdThreads);
+      stage_rows<VB * 4>(sws, VB * 4, a.w + tok_v(0, v0), (size_t)H * DV * 4, kChunk, len, tid, kBwdThreads);
+      stage_rows<VB * (int)sizeof(IO)>(svs, VB * sizeof(IO), static_cast<const IO*>(a.v) + tok_v(0, v0),
+                                       (size_t)H * DV * sizeof(IO), kChunk, len, tid, kBwdThreads);
       cp_async_commit();
-      // S0 and dS1 slices, transposed; Z^T (all loads of a thread issued first)
-      {
-        float4 s[DK * VB / 4 / kBwdThreads], d[DK * VB / 4 / kBwdThreads];
-        float zw[4], zv[4];
+      // S0 and dS1 slices, transposed (two float4 of each a thread in flight at a time)
+      constexpr int NS = DK * VB / 4 / kBwdThreads;
 #pragma unroll
-        for (int u = 0; u < DK * VB / 4 / kBwdThreads; ++u) {
-          const int idx = tid + u * kBwdThreads, cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
-          s[u] = *reinterpret_cast<const float4*>(a.S0 + st + (size_t)cc * DV + v0 + v4);
-          d[u] = *reinterpret_cast<const float4*>(a.dS1 + st + (size_t)cc * DV + v0 + v4);
+      for (int u0 = 0; u0 < NS; u0 += 2) {
+        float4 s4[2], d4[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int idx = tid + (u0 + u) * kBwdThreads, cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
+          s4[u] = *reinterpret_cast<const float4*>(a.S0 + st + (size_t)cc * DV + v0 + v4);
+          d4[u] = *reinterpret_cast<const float4*>(a.dS1 + st + (size_t)cc * DV + v0 + v4);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx = tid + u * kBwdThreads, i = idx / VB, j = idx % VB;
-          const bool live = i < len;
-          zw[u] = live ? a.w[tok_v(i, v0 + j)] : 0.f;
-          zv[u] = live ? ld_io<IO>(a.v, tok_v(i, v0 + j)) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < DK * VB / 4 / kBwdThreads; ++u) {
-          const int idx = tid + u * kBwdThreads, cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
-          sS0T[(v4 + 0) * LDK + cc] = s[u].x; sS0T[(v4 + 1) * LDK + cc] = s[u].y;
-          sS0T[(v4 + 2) * LDK + cc] = s[u].z; sS0T[(v4 + 3) * LDK + cc] = s[u].w;
-          sD1T[(v4 + 0) * LDK + cc] = d[u].x; sD1T[(v4 + 1) * LDK + cc] = d[u].y;
-          sD1T[(v4 + 2) * LDK + cc] = d[u].z; sD1T[(v4 + 3) * LDK + cc] = d[u].w;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx = tid + u * kBwdThreads, i = idx / VB, j = idx % VB;
-          sZT[j * LT + i] = zw[u] * zv[u];
+        for (int u = 0; u < 2; ++u) {
+          const int idx = tid + (u0 + u) * kBwdThreads, cc = idx / (VB / 4), v4 = 4 * (idx % (VB / 4));
+          sS0T[(v4 + 0) * LDK + cc] = s4[u].x; sS0T[(v4 + 1) * LDK + cc] = s4[u].y;
+          sS0T[(v4 + 2) * LDK + cc] = s4[u].z; sS0T[(v4 + 3) * LDK + cc] = s4[u].w;
+          sD1T[(v4 + 0) * LDK + cc] = d4[u].x; sD1T[(v4 + 1) * LDK + cc] = d4[u].y;
+          sD1T[(v4 + 2) * LDK + cc] = d4[u].z; sD1T[(v4 + 3) * LDK + cc] = d4[u].w;
         }
       }
       cp_async_wait<0>();
       __syncthreads();
+      for (int idx = tid; idx < kChunk * VB; idx += kBwdThreads) {   // Z^T (rows past the end are zero)
+        const int i = idx / VB, j = idx % VB;
+        sZT[j * LT + i] = sws[idx] * to_f32(svs[idx]);
+      }
       if (tid < DK) {
         float sacc = 0.f;
 #pragma unroll 8
         for (int j = 0; j < VB; ++j) sacc = fmaf(sS0T[j * LDK + tid], sD1T[j * LDK + tid], sacc);
         sgs[tid] += sacc;
       }
-      // dU = Kbar dS1 + scale P^T dO and U^T on 2 x 2 tiles (rows rv, rv + 1;
-      // columns cv, cv + 16: a thread rewrites only the entries it reads)
+      // dU = Kbar dS1 + scale P^T dO and U^T on 2 x QN tiles (rows rv, rv + 1;
+      // columns cv + 16 q: a thread rewrites only the entries it reads)
       {
-        float pd[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        float pd[2][QN];
+#pragma unroll
+        for (int q = 0; q < QN; ++q) pd[0][q] = pd[1][q] = 0.f;
         for (int j = rv; j < kChunk; ++j) {   // P_{j, i} = 0 for j < i
           const float2 p = *reinterpret_cast<const float2*>(sP + j * LT + rv);
-          const float o0 = to_f32(sdO[j * VB + cv]), o1 = to_f32(sdO[j * VB + cv + 16]);
-          pd[0][0] = fmaf(p.x, o0, pd[0][0]); pd[0][1] = fmaf(p.x, o1, pd[0][1]);
-          pd[1][0] = fmaf(p.y, o0, pd[1][0]); pd[1][1] = fmaf(p.y, o1, pd[1][1]);
+#pragma unroll
+          for (int q = 0; q < QN; ++q) {
+            const float o = to_f32(sdO[j * VB + cv + 16 * q]);
+            pd[0][q] = fmaf(p.x, o, pd[0][q]);
+            pd[1][q] = fmaf(p.y, o, pd[1][q]);
+          }
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          for (int q = 0; q < QN; ++q) {
             const int i = rv + r, j = cv + 16 * q;
             sUT[j * LT + i] = sU[i * LVB + j];
             sdU[i * LVB + j] = fmaf(a.scale, pd[r][q], sdU[i * LVB + j]);
@@ -464,33 +469,29 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
             }
         }
       }
-      // dZ = T^T dU on the 2 x 2 tile, then dv = dZ w and dw = dZ v
+      // dZ = T^T dU on the 2 x QN tile, then dv = dZ w and dw = dZ v
       {
-        float z[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        float z[2][QN];
+#pragma unroll
+        for (int q = 0; q < QN; ++q) z[0][q] = z[1][q] = 0.f;
         for (int i = rv; i < kChunk; ++i) {   // T_{i, j} = 0 for i < j
           const float2 t = *reinterpret_cast<const float2*>(sT + i * LT + rv);
-          const float d0 = sdU[i * LVB + cv], d1 = sdU[i * LVB + cv + 16];
-          z[0][0] = fmaf(t.x, d0, z[0][0]); z[0][1] = fmaf(t.x, d1, z[0][1]);
-          z[1][0] = fmaf(t.y, d0, z[1][0]); z[1][1] = fmaf(t.y, d1, z[1][1]);
-        }
-        float wv[2][2], vv[2][2];
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const bool live = rv + r < len;
-            const size_t o = tok_v(live ? rv + r : 0, v0 + cv + 16 * q);
-            wv[r][q] = live ? a.w[o] : 0.f;
-            vv[r][q] = live ? ld_io<IO>(a.v, o) : 0.f;
+          for (int q = 0; q < QN; ++q) {
+            const float d = sdU[i * LVB + cv + 16 * q];
+            z[0][q] = fmaf(t.x, d, z[0][q]);
+            z[1][q] = fmaf(t.y, d, z[1][q]);
           }
+        }
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int q = 0; q < 2; ++q)
+          for (int q = 0; q < QN; ++q)
             if (rv + r < len) {
-              const size_t o = tok_v(rv + r, v0 + cv + 16 * q);
-              a.dv[o] = z[r][q] * wv[r][q];
-              a.dw[o] = z[r][q] * vv[r][q];
+              const int j = cv + 16 * q;
+              const size_t o = tok_v(rv + r, v0 + j);
+              a.dv[o] = z[r][q] * sws[(rv + r) * VB + j];
+              a.dw[o] = z[r][q] * to_f32(svs[(rv + r) * VB + j]);
             }
       }
     }
