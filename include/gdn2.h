@@ -305,9 +305,10 @@ GDN2_API gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale,
 
 /* Bytes of workspace gdn2_chunk_bwd needs for `desc` (0 if desc is invalid):
  * a status word, the fp32 chunk factors of the forward (W, U~, Kbar, Q_eff,
- * O_part, gamma_n, the chunk map), T and P of every (chunk, head), and two
- * fp32 dk x dv states per (chunk, head): the forward state at the chunk's
- * start and the gradient reaching its end. */
+ * O_part, gamma_n, the chunk map), T and P of every (chunk, head), two fp32
+ * dk x dv states per (chunk, head) (the forward state at the chunk's start
+ * and the gradient reaching its end), and two fp32 64 x dv tiles per (chunk,
+ * head) (U = U~ - W S0 and Kbar times that gradient). */
 GDN2_API size_t gdn2_backward_workspace_size(const gdn2_desc* desc);
 
 /* Gradients of gdn2_chunk_fwd's outputs: given dO (the gradient of out) and
@@ -317,9 +318,10 @@ GDN2_API size_t gdn2_backward_workspace_size(const gdn2_desc* desc);
  * gated keys and values; the update is the one of section "在两个维度上独立控制"),
  * fp32 on the CUDA cores for both I/O types:
  *   1. the chunk factors, T = (I + A)^-1 and P are recomputed in fp32;
- *   2. the forward state at every chunk start is recomputed;
- *   3. the chunks are walked in reverse: the gradient reaching a chunk's
- *      start state is dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO
+ *   2. the forward state at every chunk start is recomputed, and
+ *   3. beside it (the two walks are independent) the chunks are walked in
+ *      reverse: the gradient reaching a chunk's start state is
+ *      dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO
  *      (dS1 of a sequence's last chunk is dhT; dh0 is dS0 of its first);
  *   4. every (chunk, head) then gives its tokens' gradients from its start
  *      state, the gradient at its end and dO, independently of the others.
