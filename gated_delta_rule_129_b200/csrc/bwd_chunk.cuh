@@ -503,20 +503,29 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   float* sk = sm + C::S_K;        // [64][LDK] k
   float* sq = sm + C::S_2;        // [64][LDK] q
   float* sdP = sm + C::OFF_P;     // [64][LT], over P
-  batched_copy<8, float4>(
-      kChunk * DK, tid, kBwdThreads,
-      [&](int idx) {
-        const int i = idx / DK, cc = idx % DK;
-        if (i >= len) return make_float4(0.f, 0.f, 0.f, 0.f);
-        const size_t o = tok_k(i, cc);
-        return make_float4(a.la[o], ld_io<IO>(a.k, o), ld_io<IO>(a.q, o), 0.f);
-      },
-      [&](int idx, float4 r) {
-        const int i = idx / DK, cc = idx % DK;
-        sg[i * LDK + cc] = r.x;
-        sk[i * LDK + cc] = r.y;
-        sq[i * LDK + cc] = r.z;
-      });
+  // the chunk's key-side rows: eight threads per token, DK / 8 channels each,
+  // read as 16-byte vectors eight channels at a time (rows past the end zero)
+  static_assert(kBwdThreads == 8 * kChunk, "eight threads per token row");
+  const int ri8 = tid >> 3, ck8 = (tid & 7) * (DK / 8);
+  auto row_pass = [&](auto&& body) {
+#pragma unroll
+    for (int c8 = ck8; c8 < ck8 + DK / 8; c8 += 8) body(ri8, c8, ri8 < len);
+  };
+  row_pass([&](int i, int c8, bool live) {
+    float lv[8], kv[8], qv[8];
+    if (live) {
+      const size_t o = tok_k(i, c8);
+      ldg_vec<8>(a.la + o, lv);
+      ldg_vec<8>(static_cast<const IO*>(a.k) + o, kv);
+      ldg_vec<8>(static_cast<const IO*>(a.q) + o, qv);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sg[i * LDK + c8 + e] = live ? lv[e] : 0.f;
+      sk[i * LDK + c8 + e] = live ? kv[e] : 0.f;
+      sq[i * LDK + c8 + e] = live ? qv[e] : 0.f;
+    }
+  });
 #pragma unroll
   for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
@@ -564,16 +573,13 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   {
     float* sEtT = sm + C::S_2;     // [DK][LT]
     float* sdW = sm + C::S_3;      // [64][LDK]
-    batched_copy<8, float>(
-        kChunk * DK, tid, kBwdThreads,
-        [&](int idx) {
-          const int i = idx / DK, cc = idx % DK;
-          return i < len ? a.b[tok_k(i, cc)] : 0.f;
-        },
-        [&](int idx, float bv) {
-          const int i = idx / DK, cc = idx % DK;
-          sEtT[cc * LT + i] = bv * sk[i * LDK + cc] * expf(sg[i * LDK + cc]);
-        });
+    row_pass([&](int i, int c8, bool live) {
+      float bv[8];
+      if (live) ldg_vec<8>(a.b + tok_k(i, c8), bv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        sEtT[(c8 + e) * LT + i] = live ? bv[e] * sk[i * LDK + c8 + e] * expf(sg[i * LDK + c8 + e]) : 0.f;
+    });
 #pragma unroll
     for (int ii = 0; ii < TMK; ++ii)
       *reinterpret_cast<float4*>(sdW + (rk0 + ii) * LDK + ck0) =
@@ -694,22 +700,22 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     float* skb = sk;                  // k beta, over k
     float* sea = sm + C::S_2;         // e alpha
     float* sqa = sm + C::S_4;         // q alpha
-    batched_copy<8, float2>(
-        kChunk * DK, tid, kBwdThreads,
-        [&](int idx) {
-          const int i = idx / DK, cc = idx % DK;
-          if (i >= len) return make_float2(0.f, 0.f);
-          const size_t o = tok_k(i, cc);
-          return make_float2(a.b[o], ld_io<IO>(a.q, o));
-        },
-        [&](int idx, float2 r) {
-          const int i = idx / DK, cc = idx % DK;
-          const float g = sg[i * LDK + cc], gr = sg[rref * LDK + cc], kv = sk[i * LDK + cc];
-          const float al = expf(g - gr), be = expf(gr - g);
-          sea[i * LDK + cc] = r.x * kv * al;
-          sqa[i * LDK + cc] = r.y * al;
-          skb[i * LDK + cc] = kv * be;
-        });
+    row_pass([&](int i, int c8, bool live) {
+      float bv[8], qv[8];
+      if (live) {
+        ldg_vec<8>(a.b + tok_k(i, c8), bv);
+        ldg_vec<8>(static_cast<const IO*>(a.q) + tok_k(i, c8), qv);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int cc = c8 + e;
+        const float g = sg[i * LDK + cc], gr = sg[rref * LDK + cc], kv = sk[i * LDK + cc];
+        const float al = expf(g - gr), be = expf(gr - g);
+        sea[i * LDK + cc] = live ? bv[e] * kv * al : 0.f;
+        sqa[i * LDK + cc] = live ? qv[e] * al : 0.f;
+        skb[i * LDK + cc] = kv * be;
+      }
+    });
     __syncthreads();
     float ed[TMK][4], qd[TMK][4], kd[TMK][4];
 #pragma unroll
@@ -779,19 +785,18 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
     // -------------- through the pairwise decays, pair by pair (steep) ----
     float* sq2 = sm + C::S_2;    // q again
     float* se = sm + C::S_4;     // e = b k
-    batched_copy<8, float2>(
-        kChunk * DK, tid, kBwdThreads,
-        [&](int idx) {
-          const int i = idx / DK, cc = idx % DK;
-          if (i >= len) return make_float2(0.f, 0.f);
-          const size_t o = tok_k(i, cc);
-          return make_float2(ld_io<IO>(a.q, o), a.b[o]);
-        },
-        [&](int idx, float2 r) {
-          const int i = idx / DK, cc = idx % DK;
-          sq2[i * LDK + cc] = r.x;
-          se[i * LDK + cc] = r.y * sk[i * LDK + cc];
-        });
+    row_pass([&](int i, int c8, bool live) {
+      float bv[8], qv[8];
+      if (live) {
+        ldg_vec<8>(a.b + tok_k(i, c8), bv);
+        ldg_vec<8>(static_cast<const IO*>(a.q) + tok_k(i, c8), qv);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sq2[i * LDK + c8 + e] = live ? qv[e] : 0.f;
+        se[i * LDK + c8 + e] = live ? bv[e] * sk[i * LDK + c8 + e] : 0.f;
+      }
+    });
     __syncthreads();
     // thread (channel cc, part p): the row sums of its channel over the
     // columns j of its part (j mod 2*PARTS in {p, 2*PARTS-1-p}: every part

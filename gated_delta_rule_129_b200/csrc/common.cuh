@@ -58,26 +58,6 @@ __device__ __forceinline__ void stage_rows(void* dst, int sstride, const void* s
   }
 }
 
-// Element-wise staging with many loads in flight: for idx = tid, tid + nthr,
-// ... < n, in batches of U per thread, every load(idx) of the batch is issued
-// before its store(idx, value).
-template <int U, typename T, typename L, typename S>
-__device__ __forceinline__ void batched_copy(int n, int tid, int nthr, L load, S store) {
-  for (int base = tid; base < n; base += U * nthr) {
-    T r[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int idx = base + u * nthr;
-      if (idx < n) r[u] = load(idx);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int idx = base + u * nthr;
-      if (idx < n) store(idx, r[u]);
-    }
-  }
-}
-
 // N consecutive elements (N = 2 or 4, the address a multiple of their size)
 // of a shared-memory row of fp32 or bf16, as fp32.
 template <int N>
@@ -100,6 +80,32 @@ __device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float (&o)[N]) 
     static_assert(N == 2, "2 or 4");
     const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
     o[0] = bf16_lo_f(v); o[1] = bf16_hi_f(v);
+  }
+}
+
+// N consecutive fp32 or bf16 elements of global memory (16-byte aligned, N a
+// multiple of 16 bytes' worth) as fp32, by 16-byte loads.
+template <int N>
+__device__ __forceinline__ void ldg_vec(const float* p, float (&o)[N]) {
+  static_assert(N % 4 == 0, "16-byte pieces");
+#pragma unroll
+  for (int j = 0; j < N / 4; ++j) {
+    const float4 v = *reinterpret_cast<const float4*>(p + 4 * j);
+    o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
+  }
+}
+template <int N>
+__device__ __forceinline__ void ldg_vec(const __nv_bfloat16* p, float (&o)[N]) {
+  static_assert(N % 8 == 0, "16-byte pieces");
+#pragma unroll
+  for (int j = 0; j < N / 8; ++j) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p + 8 * j);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      o[8 * j + 2 * e] = bf16_lo_f(w[e]);
+      o[8 * j + 2 * e + 1] = bf16_hi_f(w[e]);
+    }
   }
 }
 

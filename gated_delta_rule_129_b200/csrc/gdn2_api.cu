@@ -1007,7 +1007,7 @@ gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void
   a.o = o; a.g = gate; a.weight = norm_weight;
   a.rows = tokens * desc->H;
   a.out = out;
-  const long long per_block = gdn2::kTokThreads / 16;          // a row per half-warp
+  const long long per_block = gdn2::kTokThreads / 16 * gdn2::kEpiRows;   // kEpiRows rows per half-warp
   const long long blocks = (a.rows + per_block - 1) / per_block;
   if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
   const bool f32 = desc->io == GDN2_IO_F32;

@@ -75,30 +75,37 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  batched_copy<16, float4>(
-      kChunk * DK, tid, kPrepSimtThreads,
-      [&](int idx) {
-        const int i = idx / DK, cc = idx % DK;
-        if (i >= len) return make_float4(0.f, 0.f, 0.f, 0.f);
-        const size_t off = ((size_t)(pos.t0 + i) * H + h) * DK + cc;
-        return make_float4(to_f32(a.k[off]), to_f32(a.q[off]), a.b[off], a.la[off]);
-      },
-      [&](int idx, float4 r) {
-        const int i = idx / DK, cc = idx % DK;
-        sk[i * LK + cc] = r.x;
-        se[i * LK + cc] = r.z * r.x;
-        sq[i * LK + cc] = r.y;
-        sg[i * LK + cc] = r.w;
-      });
-  batched_copy<16, float>(
-      kChunk * DV, tid, kPrepSimtThreads,
-      [&](int idx) {
-        const int i = idx / DV, cc = idx % DV;
-        if (i >= len) return 0.f;
-        const size_t off = ((size_t)(pos.t0 + i) * H + h) * DV + cc;
-        return a.w[off] * to_f32(a.v[off]);
-      },
-      [&](int idx, float z) { sz[(idx / DV) * LV + idx % DV] = z; });
+  // the chunk's rows: eight threads per token, DK / 8 key and DV / 8 value
+  // channels each, read as 16-byte vectors (rows past the last token zero)
+  {
+    static_assert(kPrepSimtThreads == 8 * kChunk, "eight threads per token row");
+    constexpr int CK = DK / 8, CV = DV / 8;
+    const int i = tid >> 3, ck = (tid & 7) * CK, cv = (tid & 7) * CV;
+    float kv[CK], qv[CK], bv[CK], lv[CK], wv[CV], vv[CV];
+    if (i < len) {
+      const size_t ok = ((size_t)(pos.t0 + i) * H + h) * DK + ck, ov = ((size_t)(pos.t0 + i) * H + h) * DV + cv;
+      ldg_vec<CK>(a.k + ok, kv);
+      ldg_vec<CK>(a.q + ok, qv);
+      ldg_vec<CK>(a.b + ok, bv);
+      ldg_vec<CK>(a.la + ok, lv);
+      ldg_vec<CV>(a.w + ov, wv);
+      ldg_vec<CV>(a.v + ov, vv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < CK; ++e) kv[e] = qv[e] = bv[e] = lv[e] = 0.f;
+#pragma unroll
+      for (int e = 0; e < CV; ++e) wv[e] = vv[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < CK; ++e) {
+      sk[i * LK + ck + e] = kv[e];
+      se[i * LK + ck + e] = bv[e] * kv[e];
+      sq[i * LK + ck + e] = qv[e];
+      sg[i * LK + ck + e] = lv[e];
+    }
+#pragma unroll
+    for (int e = 0; e < CV; ++e) sz[i * LV + cv + e] = wv[e] * vv[e];
+  }
   for (int idx = tid; idx < kChunk * LA; idx += kPrepSimtThreads) {
     sA[idx] = 0.f;
     sP[idx] = 0.f;

@@ -214,29 +214,38 @@ struct TokEpiArgs {
   void* out;
 };
 
-// grid: ceil(rows / 16); one (token, head) row of DV channels per half-warp,
-// DV / 16 channels per lane.
+// grid: ceil(rows / (16 kEpiRows)); kEpiRows (token, head) rows of DV
+// channels per half-warp, DV / 16 channels per lane.
+constexpr int kEpiRows = 2;   // (token, head) rows per half-warp, loaded together
+
 template <typename IO, int DV>
 __global__ void __launch_bounds__(kTokThreads)
 token_epilogue_kernel(const TokEpiArgs a) {
-  constexpr int PER = DV / 16;
+  constexpr int PER = DV / 16, HW = kTokThreads / 16;
   const int l16 = threadIdx.x & 15;
-  const long long row = (long long)blockIdx.x * (kTokThreads / 16) + (threadIdx.x >> 4);
-  const bool live = row < a.rows;                            // shuffles below stay warp-wide
-  const size_t base = (size_t)(live ? row : 0) * DV + l16 * PER;
-  Run<IO, PER> o, g;
-  o.load(static_cast<const IO*>(a.o) + base);
-  g.load(static_cast<const IO*>(a.g) + base);
+  const long long row0 = (long long)blockIdx.x * (HW * kEpiRows) + (threadIdx.x >> 4);
+  Run<IO, PER> o[kEpiRows], g[kEpiRows];
+#pragma unroll
+  for (int u = 0; u < kEpiRows; ++u) {   // every load of the thread first
+    const long long row = row0 + u * HW;
+    const size_t base = (size_t)(row < a.rows ? row : 0) * DV + l16 * PER;   // shuffles below stay warp-wide
+    o[u].load(static_cast<const IO*>(a.o) + base);
+    g[u].load(static_cast<const IO*>(a.g) + base);
+  }
   float wt[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) wt[e] = a.weight[l16 * PER + e];
-  float ss = 0.f;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) ss = fmaf(o.v[e], o.v[e], ss);
-  const float r = rsqrtf(half_warp_sum(ss) * (1.f / DV) + kTokEps);
+  for (int u = 0; u < kEpiRows; ++u) {
+    const long long row = row0 + u * HW;
+    float ss = 0.f;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) o.v[e] = o.v[e] * r * wt[e] * sigmoid_f(g.v[e]);
-  if (live) o.store(static_cast<IO*>(a.out) + base);
+    for (int e = 0; e < PER; ++e) ss = fmaf(o[u].v[e], o[u].v[e], ss);
+    const float r = rsqrtf(half_warp_sum(ss) * (1.f / DV) + kTokEps);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[u].v[e] = o[u].v[e] * r * wt[e] * sigmoid_f(g[u].v[e]);
+    if (row < a.rows) o[u].store(static_cast<IO*>(a.out) + (size_t)row * DV + l16 * PER);
+  }
 }
 
 }  // namespace gdn2
