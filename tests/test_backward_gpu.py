@@ -5,9 +5,9 @@ The kernel computes in fp32 from the same (bf16-representable) inputs the
 oracle sees and writes fp32 gradients, so the tolerance is the fp32 one in
 both I/O modes: rel-L2 <= 1e-4 over each gradient tensor (fp64 comparison),
 on shapes that span several chunks, a ragged tail, packed sequences with empty
-and one-token ones, dk / dv 64 and 128, with and without h0 and dhT, and
+and one-token ones, dk / dv 64 and 128, with and without h0 and dhT,
 chunks whose decay is too steep for the scaled-product form (the pair-by-pair
-path).
+path), and two heads of the full 16K x 1 workload.
 """
 import numpy as np
 import pytest
@@ -88,3 +88,32 @@ def test_backward_malformed_seqlens_sets_status(gdn2):
     gdn2.chunk_bwd(t(x.q), t(x.k), t(x.v), t(x.log_alpha), t(x.b), t(x.w), x.scale, dO, cu_seqlens=cu, workspace=ws)
     torch.cuda.synchronize()
     assert gdn2.STATUS[int(ws[:4].view(torch.int32).item())] == "GDN2_ERR_SEQLENS"
+
+
+@pytest.mark.parametrize("heads", [(0, 11)])
+def test_backward_full_size_sampled_heads(gdn2, heads):
+    """The 16K x 1 workload (H = 16, bf16 inputs) in the launch configuration
+    bench.py times; heads are independent, so two of them are checked against
+    the chunkwise fp64 oracle run on that head alone."""
+    import torch
+
+    import oracle.chunk_backward as ocb
+    from workloads import config
+    x = config(2)
+    rng = np.random.default_rng(96)
+    dO = round_bf16(rng.standard_normal(x.v.shape).astype(np.float32))
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to("cuda", dt)  # noqa: E731
+    bf, f32 = torch.bfloat16, torch.float32
+    got = gdn2.chunk_bwd(t(x.q, bf), t(x.k, bf), t(x.v, bf), t(x.log_alpha, f32), t(x.b, f32), t(x.w, f32),
+                         x.scale, t(dO, bf))
+    torch.cuda.synchronize()
+    for h in heads:
+        one = lambda a: np.ascontiguousarray(a[:, :, h:h + 1])  # noqa: E731
+        ref = ocb.backward(one(x.q), one(x.k), one(x.v), one(x.log_alpha), one(x.b), one(x.w), x.scale, one(dO))
+        for name in NAMES:
+            g = got[name][:, :, h:h + 1].cpu().numpy()
+            assert np.all(np.isfinite(g)), (h, name)
+            r = rel_l2(g, ref[name])
+            assert r <= 1e-4, (h, name, r)
+        r = rel_l2(got["h0"][:, h:h + 1].cpu().numpy(), ref["h0"])
+        assert r <= 1e-4, (h, "h0", r)
