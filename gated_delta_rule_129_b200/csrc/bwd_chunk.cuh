@@ -269,7 +269,9 @@ struct BwdCfg {
                        OFF_WS = OFF_DO + (kChunk * VB * (int)sizeof(IO) + 3) / 4,  // [64][VB] w (fp32)
                        OFF_VS = OFF_WS + kChunk * VB,                              // [64][VB] v (io)
                        END_V = OFF_VS + (kChunk * VB * (int)sizeof(IO) + 3) / 4;
-  // after it, key-sized slots: g; k (then k beta); q / E~^T / T^T, X / q; dW / dT, X / dA; e alpha or e
+  // after it, key-sized slots: g; k (k beta in the product form); q, then E~^T,
+  // then T^T, then e alpha (product form) or q (pair by pair); dW, then dT /
+  // dA and X; q alpha (product form) or e (pair by pair)
   static constexpr int S_G = A0, S_K = A0 + MAT, S_2 = A0 + 2 * MAT, S_3 = A0 + 3 * MAT, S_4 = A0 + 4 * MAT,
                        END_K = A0 + 5 * MAT;
   static constexpr int OFF_RED = (END_V > END_K ? END_V : END_K);   // [DK] x 2: rowsum(dS1 S0), colsum(dKbar Kbar)
