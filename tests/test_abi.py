@@ -142,3 +142,50 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn2, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         gdn2.load_library()
+
+
+def test_backward_workspace_size(lib):
+    """The backward's workspace: the status word, the forward's fp32 factor
+    set (whatever the I/O type), T and P, two dk x dv states and two 64 x dv
+    tiles per (chunk, head), each region 256-byte aligned."""
+    B, T, H, dk, dv = 1, 16384, 16, 128, 128
+    chunks_h = (T // 64) * H
+    regions = 2 * chunks_h * 64 * 64 * 4 + 2 * chunks_h * dk * dv * 4 + 2 * chunks_h * 64 * dv * 4
+    wy = gdn2.workspace_size(B, T, H, dk, dv, gdn2.GDN2_IO_F32)
+    for io in (gdn2.GDN2_IO_BF16, gdn2.GDN2_IO_F32):
+        n = gdn2.backward_workspace_size(B, T, H, dk, dv, io)
+        assert wy + regions + 256 <= n <= wy + regions + 256 + 7 * 256
+    assert gdn2.backward_workspace_size(B, T, H, dk, dv, gdn2.GDN2_IO_BF16) == \
+        gdn2.backward_workspace_size(B, T, H, dk, dv, gdn2.GDN2_IO_F32)
+    assert gdn2.backward_workspace_size(1, 128, 2, 96, 64) == 0          # bad dk
+    # packed: T_total / 64 + N chunks bound the regions
+    n7 = gdn2.backward_workspace_size(1, 1000, 2, 64, 128, gdn2.GDN2_IO_F32, num_seqs=7)
+    ch7 = (1000 // 64 + 7) * 2
+    assert n7 >= gdn2.workspace_size(1, 1000, 2, 64, 128, gdn2.GDN2_IO_F32, num_seqs=7) + \
+        ch7 * (2 * 64 * 64 + 2 * 64 * 128 + 2 * 64 * 128) * 4
+
+
+def test_chunk_bwd_host_checks(lib):
+    """Failing argument checks of gdn2_chunk_bwd return before any CUDA call
+    (fake, never-dereferenced device addresses; no call passes every check)."""
+    size = gdn2.backward_workspace_size(1, 128, 2, 64, 64, 0)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    ins = [0x10000 + 0x100 * i for i in range(6)]
+    grads = [0x200000 + 0x1000 * i for i in range(7)]
+
+    def bwd(d, ins=ins, dO=0x80000, grads=grads, h0=None, dhT=None, cu=None):
+        return lib.gdn2_chunk_bwd(None if d is None else ctypes.byref(d), *(P(p) for p in ins), 0.125, P(h0),
+                                  P(cu), P(dO), P(dhT), *(P(g) for g in grads), None)
+    d = gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, 0x100000, size)
+    assert bwd(None) == NULL
+    assert bwd(gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, 0x100000, size - 1)) == WORKSPACE
+    assert bwd(gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, None, size)) == WORKSPACE
+    assert bwd(gdn2.make_desc(1, 128, 2, 64, 64, 0, 0, 0x100010, size)) == ALIGN
+    assert bwd(d, dO=None) == NULL
+    assert bwd(d, grads=grads[:6] + [None]) == NULL                    # dh0
+    assert bwd(d, grads=[grads[0] + 4] + grads[1:]) == ALIGN
+    assert bwd(d, dhT=0x90004) == ALIGN
+    bad = list(ins)
+    bad[2] = None
+    assert bwd(d, ins=bad) == NULL
+    assert bwd(gdn2.make_desc(1, 128, 2, 64, 80, 0, 0, 0x100000, size)) == SHAPE
