@@ -449,10 +449,40 @@ def measure_backward(dev, stream, hbm, reps=3):
     ms = tot / reps
     alg = TH * (768 + 1536 + 256 + 6 * 512) + B * H * DK * DV * 4
     gbs = alg / (ms / 1e3) / 1e9
+    flops = backward_flops()
+    tfs = flops / (ms / 1e3) / 1e12
     return {"workload": "16Kx1 backward (gdn2_chunk_bwd: chunkwise WY form, fp32 on the CUDA cores), bf16 inputs, "
                         "fp32 gradients",
-            "ms": ms, "tokens_per_s": B * T / (ms / 1e3), "alg_bytes": alg,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
+            "ms": ms, "tokens_per_s": B * T / (ms / 1e3), "alg_bytes": alg, "alg_flops": flops,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
+            "roofline_alu": {"bound": "alu", "achieved": tfs, "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s",
+                             "frac": tfs / FP32_FMA_TFLOPS,
+                             "peak_source": "nominal: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz"}}
+
+
+# fp32 CUDA-core peak of one B200 (nominal, from the unit counts and the
+# maximum SM clock): 148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_flops(C=64):
+    """Algorithmic FLOPs of the chunkwise backward at 16K x 1 (2 per
+    multiply-add; triangular products counted at half):
+      recompute: A, P (2 C^2/2 dk); T (C^3/6); W, Q_eff (2 C^2/2 dk);
+                 U~, O_part (2 C^2/2 dv)
+      the walks: U = U~ - W S0 and S1 (2 C dk dv); Kbar dS1 and the dS0
+                 update (3 C dk dv)
+      per chunk: P^T dO (C^2/2 dv); dQ~, dKbar, dW (3 C dk dv); dP (C^2 dv);
+                 dT (C^2 dv + C^2 dk); dZ (C^2/2 dv); dE~ (C^2/2 dk);
+                 dA (C^3); the three pairwise-decay sums (3 C^2/2 dk)"""
+    dk, dv = DK, DV
+    tri = C * C / 2
+    macs = (2 * tri * dk + C ** 3 / 6 + 2 * tri * dk + 2 * tri * dv
+            + 2 * C * dk * dv + 3 * C * dk * dv
+            + tri * dv + 3 * C * dk * dv + C * C * dv + C * C * (dv + dk) + tri * dv + tri * dk + C ** 3
+            + 3 * tri * dk)
+    chunks = B * T // C
+    return 2 * macs * chunks * H
 
 
 def measure_token_path(dev, stream, flush, hbm, reps=20):
