@@ -535,8 +535,10 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
     b = w = beta, 32 packed sequences) and on the gate ablations of the 16K x 1
     inputs (erase range [0, 2], channel-mean erase or write gate): tokens/s
     and the step roofline fraction, same timing rules as the headline number
-    (median of the timed steps); and the 16K x 1 workload through the two-level
-    chunk scan (gdn2_chunk_fwd_segmented)."""
+    (median of the timed steps); the 16K x 1 workload through the two-level
+    chunk scan (gdn2_chunk_fwd_segmented); and the 16K x 1 workload with fp32
+    q, k, v and O (the fp32 CUDA-core path, 3,584 algorithmic bytes per
+    token-head)."""
     import torch
 
     import gated_delta_rule_129_b200 as gdn2
@@ -548,32 +550,39 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
         ("16Kx1 channel-mean erase gate", dict(mean_gate="erase")),
         ("16Kx1 channel-mean write gate", dict(mean_gate="write")),
     ]
-    cases = [(lambda c=c, v_=v_: config(c, v_), False) for c, v_ in ((1, "a"), (3, "a"), (4, "a"))]
+    cases = [(lambda c=c, v_=v_: config(c, v_), False, "bf16") for c, v_ in ((1, "a"), (3, "a"), (4, "a"))]
     for name, kw in ablations:
         def mk(name=name, kw=kw):
             xi = make_inputs(1, 16384, 16, 128, 128, io="bf16", seed=2, decay="strong", **kw)
             xi.name = name
             return xi
-        cases.append((mk, False))
+        cases.append((mk, False, "bf16"))
 
     def mk_seg():
         xi = config(WORKLOAD_ID)
         xi.name = "16Kx1 through the two-level chunk scan (gdn2_chunk_fwd_segmented, 64-chunk segments)"
         return xi
-    cases.append((mk_seg, True))
-    for make, segmented in cases:
+    cases.append((mk_seg, True, "bf16"))
+
+    def mk_f32():
+        xi = make_inputs(1, 16384, 16, 128, 128, io="f32", seed=2, decay="strong")
+        xi.name = "16Kx1 fp32 q, k, v and O (the fp32 CUDA-core path)"
+        return xi
+    cases.append((mk_f32, False, "f32"))
+    for make, segmented, iot in cases:
         x = make()
         t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
         bf, f32 = torch.bfloat16, torch.float32
-        q, k, v = t(x.q, bf), t(x.k, bf), t(x.v, bf)
+        io_t = f32 if iot == "f32" else bf
+        io_c = gdn2.GDN2_IO_F32 if iot == "f32" else gdn2.GDN2_IO_BF16
+        q, k, v = t(x.q, io_t), t(x.k, io_t), t(x.v, io_t)
         la, b, w = t(x.log_alpha, f32), t(x.b, f32), t(x.w, f32)
         h0 = None if x.h0 is None else t(x.h0, f32)
         cu = None if x.cu_seqlens is None else t(x.cu_seqlens, torch.int32)
         Bc, Tc, Hc = x.q.shape[0], x.q.shape[1], x.q.shape[2]
         ns = 0 if cu is None else len(x.cu_seqlens) - 1
         nseq = ns if cu is not None else Bc
-        ws = torch.empty(gdn2.workspace_size(Bc, Tc, Hc, DK, DV, gdn2.GDN2_IO_BF16, ns), dtype=torch.uint8,
-                         device=dev)
+        ws = torch.empty(gdn2.workspace_size(Bc, Tc, Hc, DK, DV, io_c, ns), dtype=torch.uint8, device=dev)
         o = torch.empty_like(v)
         hT = torch.empty((nseq, Hc, DK, DV), dtype=f32, device=dev)
 
@@ -601,7 +610,8 @@ def measure_other_configs(dev, stream, flush, hbm, steps=10):
             times.append(e0.elapsed_time(e1))
         ms = statistics.median(times)
         tokens = Bc * Tc
-        alg = tokens * Hc * ALG_BYTES_PER_TH + nseq * Hc * DK * DV * 4 * (2 if h0 is not None else 1)
+        per_th = ALG_BYTES_PER_TH if iot == "bf16" else 3 * DK * 4 + 3 * DK * 4 + DV * 4
+        alg = tokens * Hc * per_th + nseq * Hc * DK * DV * 4 * (2 if h0 is not None else 1)
         out_cfg[x.name] = {"tokens_per_s": tokens / (ms / 1e3), "ms_per_step": ms,
                            "roofline_frac": (alg / (hbm * 1e9)) / (ms / 1e3)}
         del q, k, v, la, b, w, h0, cu, ws, o, hT

@@ -227,9 +227,9 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
 template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kBwdWalkThreads)
 bwd_walks_kernel(const WalkArgs<IO, float> wa, const BwdStateArgs ra, int n_fwd) {
-  static_assert(kBwdWalkThreads == kWalkSimtThreads, "one block size for both walks");
+  static_assert(kBwdWalkThreads == walk_simt_threads(kBwdWalkCols), "one block size for both walks");
   extern __shared__ __align__(16) uint8_t bsm[];
-  if ((int)blockIdx.x < n_fwd) walk_simt_cta<DK, DV, IO, float>(wa, blockIdx.x, bsm);
+  if ((int)blockIdx.x < n_fwd) walk_simt_cta<DK, DV, IO, float, kBwdWalkCols>(wa, blockIdx.x, bsm);
   else bwd_dstate_cta<DK, DV, IO>(ra, blockIdx.x - n_fwd, bsm);
 }
 

@@ -381,13 +381,13 @@ gdn2_status launch_walk_t(const gdn2_desc* d, const Layout& L, float scale, cons
     if (L.l.factor_set == 1) return launch_walk_tc<DV>(d, L, scale, h0, cu, out, hT, chunk_states, s);
   }
   if (L.N == 0) return GDN2_OK;
-  constexpr size_t smem = gdn2::walk_simt_smem_bytes<DK, DV>();
+  constexpr size_t smem = gdn2::walk_simt_smem_bytes<DK, gdn2::kWalkSimtDVS>();
   auto kern = gdn2::walk_simt_kernel<DK, DV, IO, FT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return GDN2_ERR_CUDA;
   const long long blocks = (long long)L.N * d->H * (DV / gdn2::kWalkSimtDVS);
   if (blocks > INT32_MAX) return GDN2_ERR_SHAPE;
-  kern<<<(unsigned)blocks, gdn2::kWalkSimtThreads, smem, s>>>(a);
+  kern<<<(unsigned)blocks, gdn2::walk_simt_threads(gdn2::kWalkSimtDVS), smem, s>>>(a);
   return launch_status();
 }
 
@@ -620,11 +620,12 @@ struct BwdOp {
       ra.X = at<float>(d->workspace, B.off_X);
       ra.dh0 = dh0;
       ra.status = status;
-      constexpr size_t smem = std::max(gdn2::walk_simt_smem_bytes<DK, DV>(), gdn2::bwd_dstate_smem_bytes<DK>());
+      constexpr size_t smem =
+          std::max(gdn2::walk_simt_smem_bytes<DK, gdn2::kBwdWalkCols>(), gdn2::bwd_dstate_smem_bytes<DK>());
       auto kern = gdn2::bwd_walks_kernel<DK, DV, IO>;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GDN2_ERR_CUDA;
-      const long long n_fwd = (long long)L.N * d->H * (DV / gdn2::kWalkSimtDVS);
+      const long long n_fwd = (long long)L.N * d->H * (DV / gdn2::kBwdWalkCols);
       const long long n_rev = (long long)L.N * d->H * (DV / gdn2::kBwdWalkCols);
       if (n_fwd + n_rev > INT32_MAX) return GDN2_ERR_SHAPE;
       kern<<<(unsigned)(n_fwd + n_rev), gdn2::kBwdWalkThreads, smem, s>>>(wa, ra, (int)n_fwd);

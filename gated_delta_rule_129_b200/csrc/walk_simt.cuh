@@ -42,15 +42,18 @@ struct WalkArgs {
   float* U_out;         // optional [max_chunks, H, 64, DV]: every chunk's U (the backward)
 };
 
-constexpr int kWalkSimtThreads = 512;
-constexpr int kWalkSimtDVS = 32;
+// Value columns per CTA: 16 (256 threads) for the forward, where the walk has
+// the GPU to itself; 32 (512 threads) beside the backward's reverse walk, so
+// that both walks fit on the SMs at once.  A CTA has 16 threads per column.
+constexpr int kWalkSimtDVS = 16;
+constexpr int walk_simt_threads(int dvs) { return 16 * dvs; }
 
 // Shared memory, in bytes: two buffers of (W, Q_eff with rows padded by 16
 // bytes; the U~ and O_part slices; gamma_n), one Kbar tile, then S [DK][DVS]
 // and U [64][DVS] in fp32.
-template <int DK, typename FT>
+template <int DK, typename FT, int DVS_>
 struct WalkSimtCfg {
-  static constexpr int DVS = kWalkSimtDVS;
+  static constexpr int DVS = DVS_;
   static constexpr int LKF = DK + 16 / (int)sizeof(FT);           // elements per padded row
   static constexpr int TILE = kChunk * LKF * (int)sizeof(FT);
   static constexpr int VSL = kChunk * DVS * (int)sizeof(FT);
@@ -61,17 +64,17 @@ struct WalkSimtCfg {
   static_assert(SMEM <= 232448, "shared memory");
 };
 
-template <int DK, int DV>
+template <int DK, int DVS>
 constexpr size_t walk_simt_smem_bytes() {
-  return (size_t)WalkSimtCfg<DK, float>::SMEM;   // the fp32 plan bounds the bf16 one
+  return (size_t)WalkSimtCfg<DK, float, DVS>::SMEM;   // the fp32 plan bounds the bf16 one
 }
 
-// The walk of block `blk` (sequence, head, value slice) with `wsm` its shared
-// memory; all kWalkSimtThreads threads of the CTA take part.
-template <int DK, int DV, typename IO, typename FT>
+// The walk of block `blk` (sequence, head, DVS value columns) with `wsm` its
+// shared memory; all 16 DVS threads of the CTA take part.
+template <int DK, int DV, typename IO, typename FT, int DVS>
 __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk, uint8_t* wsm) {
-  using C = WalkSimtCfg<DK, FT>;
-  constexpr int DVS = kWalkSimtDVS, SLICES = DV / DVS, LKF = C::LKF, NT = kWalkSimtThreads;
+  using C = WalkSimtCfg<DK, FT, DVS>;
+  constexpr int SLICES = DV / DVS, LKF = C::LKF, NT = walk_simt_threads(DVS), HC = DVS / 2;
   const int H = a.H;
   const int sl = blk % SLICES;
   const int h = (blk / SLICES) % H;
@@ -112,8 +115,8 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
   cp_async_commit();
 
   constexpr int RS = DK / 32;                      // rows of S per thread
-  const int ri = tid / 16, cj = 2 * (tid % 16);    // U, O: rows 2 ri, 2 ri + 1; columns cj, cj + 1
-  const int rs = RS * (tid / 16);                  // S: rows rs .. rs + RS - 1; columns cj, cj + 1
+  const int ri = tid / HC, cj = 2 * (tid % HC);    // U, O: rows 2 ri, 2 ri + 1; columns cj, cj + 1
+  const int rs = RS * (tid / HC);                  // S: rows rs .. rs + RS - 1; columns cj, cj + 1
   for (int c = c_begin; c < c_end; ++c) {
     if (c + 1 < c_end) issue_a(c + 1);
     cp_async_commit();
@@ -216,10 +219,10 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
 }
 
 template <int DK, int DV, typename IO, typename FT>
-__global__ void __launch_bounds__(kWalkSimtThreads)
+__global__ void __launch_bounds__(walk_simt_threads(kWalkSimtDVS))
 walk_simt_kernel(const WalkArgs<IO, FT> a) {
   extern __shared__ __align__(16) uint8_t wsm[];
-  walk_simt_cta<DK, DV, IO, FT>(a, blockIdx.x, wsm);
+  walk_simt_cta<DK, DV, IO, FT, kWalkSimtDVS>(a, blockIdx.x, wsm);
 }
 
 }  // namespace gdn2
