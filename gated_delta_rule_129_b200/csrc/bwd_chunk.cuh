@@ -13,18 +13,20 @@
 //   P_ij likewise with q (j <= i),  T = (I + A)^-1,  W = T E~,  U~ = T Z,
 //   U = U~ - W S0,  O = scale (Q~ S0 + P U),  S1 = diag(gamma_n) S0 + Kbar^T U
 //
-// with Q~ = q gamma and Kbar = k exp(g_n - g).  The backward runs in four
-// steps, three launches (host: gdn2_chunk_bwd):
+// with Q~ = q gamma and Kbar = k exp(g_n - g).  The backward runs in five
+// steps, four launches (host: gdn2_chunk_bwd):
 //   1. the CUDA-core prep recomputes every chunk's factors in fp32 (W, U~,
 //      Kbar, Q_eff = Q~ - P W, gamma_n) and also stores T and P;
-//   2. the CUDA-core walk recomputes the state at every chunk start (S0);
-//   3. in other blocks of the same launch (bwd_walks_kernel: the two walks
+//   2. bwd_g_kernel forms G = scale Q_eff^T dO of every chunk (the outputs'
+//      share of the state gradient, which does not depend on the state);
+//   3. the CUDA-core walk recomputes the state at every chunk start (S0);
+//   4. in other blocks of the same launch (bwd_walks_kernel: the two walks
 //      are independent), the chunks are walked in reverse order: the gradient
 //      reaching a chunk's start state is the transpose of the forward's
-//      affine chunk map applied to the one reaching its end, plus the
-//      outputs' share:  dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO
+//      affine chunk map applied to the one reaching its end, plus G:
+//      dS0 = gamma_n dS1 - W^T (Kbar dS1) + G
 //      (dS1 of a sequence's last chunk is dhT; dh0 is dS0 of its first);
-//   4. bwd_chunk_kernel then takes every (chunk, head) on its own, from S0,
+//   5. bwd_chunk_kernel then takes every (chunk, head) on its own, from S0,
 //      dS1 and dO:
 //        dQ~ = scale dO S0^T,  dP = scale dO U^T (j <= i),
 //        dU = scale P^T dO + Kbar dS1,  dKbar = U dS1^T,  dW = -dU S0^T,
@@ -56,12 +58,11 @@ constexpr int kBwdWalkThreads = 512;
 constexpr int kBwdWalkCols = 32;   // value columns per CTA
 
 struct BwdStateArgs {
-  const float *W, *Kbar, *Qeff;   // fp32 factors [chunks, H, 64, DK]
+  const float *W, *Kbar;          // fp32 factors [chunks, H, 64, DK]
   const float* gamma_last;        // [chunks, H, DK]
-  const void* dO;                 // [T_total, H, DV], io dtype
+  const float* G;                 // [chunks, H, DK, DV]: scale Q_eff^T dO of each chunk
   SeqMap map;
   int H;
-  float scale;
   const float* dhT;               // [N, H, DK, DV] or nullptr (zero)
   float* dS1;                     // out: [chunks, H, DK, DV], gradient at each chunk's end state
   float* X;                       // out: [chunks, H, 64, DV], Kbar dS1 of each chunk
@@ -70,31 +71,31 @@ struct BwdStateArgs {
 };
 
 // Shared memory, in bytes: two buffers of (Kbar with rows padded by 16 bytes,
-// the dO slice, gamma_n), one W and one Q_eff tile, then dS [DK][CS] and
+// the G slice [DK][CS], gamma_n), one W tile, then dS [DK][CS] and
 // X = Kbar dS [64][CS] in fp32.
-template <int DK, typename IO>
+template <int DK>
 struct BwdDstateCfg {
   static constexpr int CS = kBwdWalkCols, LK = DK + 4;
-  static constexpr int TILE = kChunk * LK * 4, DOB = kChunk * CS * (int)sizeof(IO);
-  static constexpr int OFF_KB = 0, OFF_DO = TILE, OFF_GL = OFF_DO + DOB, BUF = OFF_GL + DK * 4;
-  static constexpr int OFF_W = 2 * BUF, OFF_QE = OFF_W + TILE, OFF_S = OFF_QE + TILE, OFF_X = OFF_S + DK * CS * 4,
+  static constexpr int TILE = kChunk * LK * 4, GB = DK * CS * 4;
+  static constexpr int OFF_KB = 0, OFF_G = TILE, OFF_GL = OFF_G + GB, BUF = OFF_GL + DK * 4;
+  static constexpr int OFF_W = 2 * BUF, OFF_S = OFF_W + TILE, OFF_X = OFF_S + DK * CS * 4,
                        SMEM = OFF_X + kChunk * CS * 4;
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 template <int DK>
 constexpr size_t bwd_dstate_smem_bytes() {
-  return (size_t)BwdDstateCfg<DK, float>::SMEM;   // bounds the bf16 plan
+  return (size_t)BwdDstateCfg<DK>::SMEM;
 }
 
 // The reverse walk of block `blk` (sequence, head, kBwdWalkCols value
 // columns): the columns of dS evolve independently, since every step
-// multiplies it from the left.  Kbar, dO and gamma_n (used first) are copied
-// into one of two buffers a chunk ahead (in walk order), W and Q_eff (used
-// last) into single buffers as soon as the previous step has read them.
-template <int DK, int DV, typename IO>
+// multiplies it from the left.  Kbar, the G slice and gamma_n (used first)
+// are copied into one of two buffers a chunk ahead (in walk order), W (used
+// last) into a single buffer as soon as the previous step has read it.
+template <int DK, int DV>
 __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, uint8_t* dsm) {
-  using C = BwdDstateCfg<DK, IO>;
+  using C = BwdDstateCfg<DK>;
   constexpr int CS = kBwdWalkCols, SL = DV / CS, LK = C::LK, NT = kBwdWalkThreads;
   const int H = a.H;
   const int sl = blk % SL;
@@ -105,9 +106,7 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
   float* sdS = reinterpret_cast<float*>(dsm + C::OFF_S);   // [DK][CS]
   float* sX = reinterpret_cast<float*>(dsm + C::OFF_X);    // [64][CS]
   const float* sW = reinterpret_cast<const float*>(dsm + C::OFF_W);
-  const float* sQe = reinterpret_cast<const float*>(dsm + C::OFF_QE);
 
-  const IO* dO = static_cast<const IO*>(a.dO);
   const size_t sbase = ((size_t)n * H + h) * DK * DV;
   const bool bad = *a.status != 0;
   for (int idx = tid; idx < DK * CS; idx += NT) {
@@ -115,20 +114,16 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
     sdS[idx] = (!bad && a.dhT) ? a.dhT[sbase + (size_t)cc * DV + j0 + j] : 0.f;
   }
   const int c_begin = a.map.chunk_off[n], c_end = a.map.chunk_off[n + 1];
-  const int s_begin = a.map.seq_begin(n), s_end = a.map.seq_end(n);
-  auto issue_b = [&](int c, int slot) {   // Kbar, the dO slice, gamma_n of chunk c
+  auto issue_b = [&](int c, int slot) {   // Kbar, the G slice, gamma_n of chunk c
     uint8_t* b = dsm + slot * C::BUF;
-    const size_t tk = ((size_t)c * H + h) * kChunk * DK;
-    const int t0 = s_begin + (c - c_begin) * kChunk, len = min(kChunk, s_end - t0);
-    stage_rows<DK * 4>(b + C::OFF_KB, LK * 4, a.Kbar + tk, DK * 4, kChunk, kChunk, tid, NT);
-    stage_rows<CS * (int)sizeof(IO)>(b + C::OFF_DO, CS * sizeof(IO), dO + ((size_t)t0 * H + h) * DV + j0,
-                                     (size_t)H * DV * sizeof(IO), kChunk, len, tid, NT);
-    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, NT);
+    const size_t ch = (size_t)c * H + h;
+    stage_rows<DK * 4>(b + C::OFF_KB, LK * 4, a.Kbar + ch * kChunk * DK, DK * 4, kChunk, kChunk, tid, NT);
+    stage_rows<CS * 4>(b + C::OFF_G, CS * 4, a.G + ch * DK * DV + j0, DV * 4, DK, DK, tid, NT);
+    stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ch * DK, 0, 1, 1, tid, NT);
   };
-  auto issue_w = [&](int c) {   // W and Q_eff of chunk c
-    const size_t tk = ((size_t)c * H + h) * kChunk * DK;
-    stage_rows<DK * 4>(dsm + C::OFF_W, LK * 4, a.W + tk, DK * 4, kChunk, kChunk, tid, NT);
-    stage_rows<DK * 4>(dsm + C::OFF_QE, LK * 4, a.Qeff + tk, DK * 4, kChunk, kChunk, tid, NT);
+  auto issue_w = [&](int c) {   // W of chunk c
+    stage_rows<DK * 4>(dsm + C::OFF_W, LK * 4, a.W + ((size_t)c * H + h) * kChunk * DK, DK * 4, kChunk, kChunk,
+                       tid, NT);
   };
   // commit groups, oldest first: B(last), W(last), then per chunk c (in walk
   // order): B(c - 1) at its start and W(c - 1) at its end
@@ -147,10 +142,8 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
     __syncthreads();
     const uint8_t* b = dsm + (it & 1) * C::BUF;
     const float* sKb = reinterpret_cast<const float*>(b + C::OFF_KB);
-    const IO* sdO = reinterpret_cast<const IO*>(b + C::OFF_DO);
+    const float* sG = reinterpret_cast<const float*>(b + C::OFF_G);
     const float* sgl = reinterpret_cast<const float*>(b + C::OFF_GL);
-    const int t0 = s_begin + (c - c_begin) * kChunk;
-    const int len = min(kChunk, s_end - t0);
     // the gradient reaching this chunk's end state
     const size_t cs = ((size_t)c * H + h) * DK * DV;
     for (int idx = tid; idx < DK * CS; idx += NT)
@@ -182,34 +175,34 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
     }
     cp_async_wait<1>();   // W(c) has landed
     __syncthreads();
-    // dS0 = gamma_n dS1 - W^T X + Q_eff^T (scale dO) on an RS x 2 tile; every
-    // thread rewrites only the entries of dS it read
+    // dS0 = gamma_n dS1 - W^T X + G on an RS x 2 tile (rows of W and X past the
+    // chunk's last token are zero); every thread rewrites only the entries of
+    // dS it read
     {
       float s[RS][2];
 #pragma unroll
       for (int r = 0; r < RS; ++r) {
         const float g = sgl[rs + r];
-        s[r][0] = g * sdS[(rs + r) * CS + cj];
-        s[r][1] = g * sdS[(rs + r) * CS + cj + 1];
+        const float2 gv = *reinterpret_cast<const float2*>(sG + (rs + r) * CS + cj);
+        s[r][0] = fmaf(g, sdS[(rs + r) * CS + cj], gv.x);
+        s[r][1] = fmaf(g, sdS[(rs + r) * CS + cj + 1], gv.y);
       }
 #pragma unroll 4
-      for (int i = 0; i < len; ++i) {
+      for (int i = 0; i < kChunk; ++i) {
         const float2 xv = *reinterpret_cast<const float2*>(sX + i * CS + cj);
-        const float o0 = a.scale * to_f32(sdO[i * CS + cj]), o1 = a.scale * to_f32(sdO[i * CS + cj + 1]);
-        float wv[RS], qv[RS];
+        float wv[RS];
         load_vec<RS>(sW + i * LK + rs, wv);
-        load_vec<RS>(sQe + i * LK + rs, qv);
 #pragma unroll
         for (int r = 0; r < RS; ++r) {
-          s[r][0] = fmaf(qv[r], o0, fmaf(-wv[r], xv.x, s[r][0]));
-          s[r][1] = fmaf(qv[r], o1, fmaf(-wv[r], xv.y, s[r][1]));
+          s[r][0] = fmaf(-wv[r], xv.x, s[r][0]);
+          s[r][1] = fmaf(-wv[r], xv.y, s[r][1]);
         }
       }
 #pragma unroll
       for (int r = 0; r < RS; ++r)
         *reinterpret_cast<float2*>(sdS + (rs + r) * CS + cj) = make_float2(s[r][0], s[r][1]);
     }
-    __syncthreads();   // W, Q_eff and this chunk's buffer are free
+    __syncthreads();   // W and this chunk's buffer are free
     if (c - 1 >= c_begin) issue_w(c - 1);
     cp_async_commit();
   }
@@ -221,6 +214,70 @@ __device__ __forceinline__ void bwd_dstate_cta(const BwdStateArgs& a, int blk, u
   }
 }
 
+// G = scale Q_eff^T dO of every (chunk, head): the outputs' share of the
+// gradient reaching the chunk's start state, which does not depend on the
+// state, so it is formed for all chunks at once before the reverse walk.
+// grid (chunks, H); a thread holds 4 key rows x DK DV / 2048 value columns.
+constexpr int kBwdGThreads = 512;
+
+template <int DK, int DV, typename IO>
+__global__ void __launch_bounds__(kBwdGThreads)
+bwd_g_kernel(const float* __restrict__ Qeff, const void* dO_, SeqMap map, int H, float scale,
+             float* __restrict__ G) {
+  constexpr int RG = DK / 4, CG = kBwdGThreads / RG, CPT = DV / CG, LQ = DK + 4;
+  static_assert(CPT == 2 || CPT == 4 || CPT == 8, "2, 4 or 8 value columns a thread");
+  const int c = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  if (c >= map.chunk_off[map.N]) return;
+  const ChunkPos pos = chunk_pos(map, c);
+  const size_t ch = (size_t)c * H + h;
+  extern __shared__ __align__(16) float gsm[];
+  float* sQ = gsm;                                   // [64][LQ] Q_eff
+  IO* sO = reinterpret_cast<IO*>(gsm + kChunk * LQ); // [64][DV] dO (rows past the end zero)
+  const IO* dO = static_cast<const IO*>(dO_);
+  stage_rows<DK * 4>(sQ, LQ * 4, Qeff + ch * kChunk * DK, DK * 4, kChunk, kChunk, tid, kBwdGThreads);
+  stage_rows<DV * (int)sizeof(IO)>(sO, DV * sizeof(IO), dO + ((size_t)pos.t0 * H + h) * DV,
+                                   (size_t)H * DV * sizeof(IO), kChunk, pos.len, tid, kBwdGThreads);
+  cp_async_wait_all();
+  __syncthreads();
+  const int m0 = 4 * (tid / CG), j0 = CPT * (tid % CG);
+  float acc[4][CPT];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int e = 0; e < CPT; ++e) acc[r][e] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < kChunk; ++i) {
+    float qv[4], ov[CPT];
+    load_vec<4>(sQ + i * LQ + m0, qv);
+#pragma unroll
+    for (int e = 0; e < CPT; e += (CPT >= 4 ? 4 : 2)) {
+      if constexpr (CPT >= 4) {
+        float t4[4];
+        load_vec<4>(sO + i * DV + j0 + e, t4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) ov[e + u] = t4[u];
+      } else {
+        float t2[2];
+        load_vec<2>(sO + i * DV + j0 + e, t2);
+        ov[e] = t2[0]; ov[e + 1] = t2[1];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < CPT; ++e) acc[r][e] = fmaf(qv[r], ov[e], acc[r][e]);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int e = 0; e < CPT; ++e) G[(ch * DK + m0 + r) * DV + j0 + e] = scale * acc[r][e];
+}
+
+template <int DK, int DV, typename IO>
+constexpr size_t bwd_g_smem_bytes() {
+  return sizeof(float) * (size_t)kChunk * (DK + 4) + (size_t)kChunk * DV * sizeof(IO);
+}
+
 // The two walks of the backward in one launch (they are independent): blocks
 // [0, n_fwd) walk the chunks forward and store every chunk's start state,
 // the others walk them in reverse for the state gradient.
@@ -230,7 +287,7 @@ bwd_walks_kernel(const WalkArgs<IO, float> wa, const BwdStateArgs ra, int n_fwd)
   static_assert(kBwdWalkThreads == walk_simt_threads(kBwdWalkCols), "one block size for both walks");
   extern __shared__ __align__(16) uint8_t bsm[];
   if ((int)blockIdx.x < n_fwd) walk_simt_cta<DK, DV, IO, float, kBwdWalkCols>(wa, blockIdx.x, bsm);
-  else bwd_dstate_cta<DK, DV, IO>(ra, blockIdx.x - n_fwd, bsm);
+  else bwd_dstate_cta<DK, DV>(ra, blockIdx.x - n_fwd, bsm);
 }
 
 // -------------------------------------------------- per-chunk gradients ----

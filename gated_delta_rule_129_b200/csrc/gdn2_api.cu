@@ -528,11 +528,12 @@ struct DecodeOp {
 // Workspace of gdn2_chunk_bwd: the status word; the forward's fp32 WY factor
 // set (the layout gdn2_chunk_fwd uses for fp32 I/O, whatever the I/O type of
 // the call), with its chunk map; T and P of every (chunk, head); the state at
-// every chunk start (S0); the gradient reaching every chunk's end (dS1); and
-// from the two walks, U = U~ - W S0 and Kbar dS1 of every chunk.
+// every chunk start (S0); the gradient reaching every chunk's end (dS1); from
+// the two walks, U = U~ - W S0 and Kbar dS1 of every chunk; and the outputs'
+// share of the state gradient, G = scale Q_eff^T dO, of every chunk.
 struct BwdLayout {
   Layout f;            // the factor set, relative to the workspace + kAlign
-  size_t off_T, off_P, off_S0, off_dS1, off_U, off_X, total;   // from the workspace start
+  size_t off_T, off_P, off_S0, off_dS1, off_U, off_X, off_G, total;   // from the workspace start
 };
 
 gdn2_desc bwd_factor_desc(const gdn2_desc* d) {
@@ -555,6 +556,7 @@ gdn2_status bwd_layout(const gdn2_desc* d, bool packed, BwdLayout* B) {
   B->off_dS1 = off; off = align_up(off + chunks_h * d->dk * d->dv * sizeof(float));
   B->off_U = off;   off = align_up(off + chunks_h * kChunk * d->dv * sizeof(float));
   B->off_X = off;   off = align_up(off + chunks_h * kChunk * d->dv * sizeof(float));
+  B->off_G = off;   off = align_up(off + chunks_h * d->dk * d->dv * sizeof(float));
   B->total = off;
   return GDN2_OK;
 }
@@ -588,6 +590,16 @@ struct BwdOp {
       if ((st = launch_status()) != GDN2_OK) return st;
     }
     if (L.N == 0) return GDN2_OK;
+    // G = scale Q_eff^T dO of every chunk, for the reverse walk
+    if (L.l.max_chunks > 0) {
+      constexpr size_t smem = gdn2::bwd_g_smem_bytes<DK, DV, IO>();
+      auto kern = gdn2::bwd_g_kernel<DK, DV, IO>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+      kern<<<dim3(L.l.max_chunks, d->H), gdn2::kBwdGThreads, smem, s>>>(
+          at<const float>(f.workspace, L.l.off_Qeff), dO, map, d->H, scale, at<float>(d->workspace, B.off_G));
+      if ((st = launch_status()) != GDN2_OK) return st;
+    }
     // 2. the state at every chunk start and 3. the gradient reaching every
     // chunk's end state (and dh0), in one launch
     {
@@ -609,12 +621,10 @@ struct BwdOp {
       gdn2::BwdStateArgs ra;
       ra.W = wa.W;
       ra.Kbar = wa.Kbar;
-      ra.Qeff = wa.Qeff;
       ra.gamma_last = wa.gamma_last;
-      ra.dO = dO;
+      ra.G = at<const float>(d->workspace, B.off_G);
       ra.map = map;
       ra.H = d->H;
-      ra.scale = scale;
       ra.dhT = dhT;
       ra.dS1 = at<float>(d->workspace, B.off_dS1);
       ra.X = at<float>(d->workspace, B.off_X);

@@ -20,6 +20,8 @@
 // S it read).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace gdn2 {
@@ -98,9 +100,9 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
     uint8_t* b = wsm + (c & 1) * C::BUF;
     const size_t tk = ((size_t)c * H + h) * kChunk * DK, tv = ((size_t)c * H + h) * kChunk * DV;
     stage_rows<RB>(b + C::OFF_W, LKF * sizeof(FT), a.W + tk, RB, kChunk, kChunk, tid, NT);
-    stage_rows<RB>(b + C::OFF_QE, LKF * sizeof(FT), a.Qeff + tk, RB, kChunk, kChunk, tid, NT);
+    if (a.out) stage_rows<RB>(b + C::OFF_QE, LKF * sizeof(FT), a.Qeff + tk, RB, kChunk, kChunk, tid, NT);
     stage_rows<SB>(b + C::OFF_UT, SB, a.Ut + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, NT);
-    stage_rows<SB>(b + C::OFF_OP, SB, a.Opart + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, NT);
+    if (a.out) stage_rows<SB>(b + C::OFF_OP, SB, a.Opart + tv + j0, DV * sizeof(FT), kChunk, kChunk, tid, NT);
     stage_rows<DK * 4>(b + C::OFF_GL, 0, a.gamma_last + ((size_t)c * H + h) * DK, 0, 1, 1, tid, NT);
   };
   auto issue_k = [&](int c) {   // Kbar of chunk c
@@ -135,15 +137,17 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
       for (int idx = tid; idx < DK * DVS; idx += NT)
         a.chunk_states[cs + (size_t)(idx / DVS) * DV + j0 + idx % DVS] = sS[idx];
     }
-    // U = U~ - W S and O = Q_eff S + O_part on a 2 x 2 tile
-    {
+    // U = U~ - W S and O = Q_eff S + O_part on a 2 x 2 tile (O only when it
+    // is written: the backward's recompute needs the states and U alone)
+    auto phase1 = [&](auto with_o) {
+      constexpr bool WO = decltype(with_o)::value;
       float u[2][2], o[2][2];
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           u[r][q] = to_f32(sUt[(2 * ri + r) * DVS + cj + q]);
-          o[r][q] = to_f32(sOp[(2 * ri + r) * DVS + cj + q]);
+          o[r][q] = WO ? to_f32(sOp[(2 * ri + r) * DVS + cj + q]) : 0.f;
         }
 #pragma unroll 2
       for (int c4 = 0; c4 < DK; c4 += 4) {   // four key rows of S a step, W and Q_eff read as vectors
@@ -151,7 +155,7 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           load_vec<4>(sW + (2 * ri + r) * LKF + c4, wv[r]);
-          load_vec<4>(sQe + (2 * ri + r) * LKF + c4, qv[r]);
+          if constexpr (WO) load_vec<4>(sQe + (2 * ri + r) * LKF + c4, qv[r]);
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -159,7 +163,9 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             u[r][0] = fmaf(-wv[r][e], s.x, u[r][0]); u[r][1] = fmaf(-wv[r][e], s.y, u[r][1]);
-            o[r][0] = fmaf(qv[r][e], s.x, o[r][0]); o[r][1] = fmaf(qv[r][e], s.y, o[r][1]);
+            if constexpr (WO) {
+              o[r][0] = fmaf(qv[r][e], s.x, o[r][0]); o[r][1] = fmaf(qv[r][e], s.y, o[r][1]);
+            }
           }
         }
       }
@@ -170,13 +176,15 @@ __device__ __forceinline__ void walk_simt_cta(const WalkArgs<IO, FT>& a, int blk
         if (a.U_out)
           *reinterpret_cast<float2*>(a.U_out + (((size_t)c * H + h) * kChunk + i) * DV + j0 + cj) =
               make_float2(u[r][0], u[r][1]);
-        if (a.out && i < len) {
+        if (WO && i < len) {
           const size_t off = ((size_t)(t0 + i) * H + h) * DV + j0 + cj;
           a.out[off] = from_f32<IO>(a.scale * o[r][0]);
           a.out[off + 1] = from_f32<IO>(a.scale * o[r][1]);
         }
       }
-    }
+    };
+    if (a.out) phase1(std::true_type{});
+    else phase1(std::false_type{});
     cp_async_wait<1>();   // K(c) has landed
     __syncthreads();
     // S <- diag(gamma_n) S + Kbar^T U on an RS x 2 tile (rows of Kbar and U

@@ -305,10 +305,11 @@ GDN2_API gdn2_status gdn2_chunk_walk_flagged(const gdn2_desc* desc, float scale,
 
 /* Bytes of workspace gdn2_chunk_bwd needs for `desc` (0 if desc is invalid):
  * a status word, the fp32 chunk factors of the forward (W, U~, Kbar, Q_eff,
- * O_part, gamma_n, the chunk map), T and P of every (chunk, head), two fp32
- * dk x dv states per (chunk, head) (the forward state at the chunk's start
- * and the gradient reaching its end), and two fp32 64 x dv tiles per (chunk,
- * head) (U = U~ - W S0 and Kbar times that gradient). */
+ * O_part, gamma_n, the chunk map), T and P of every (chunk, head), three fp32
+ * dk x dv matrices per (chunk, head) (the forward state at the chunk's start,
+ * the gradient reaching its end, and the outputs' share scale Q_eff^T dO of
+ * the gradient reaching its start), and two fp32 64 x dv tiles per (chunk,
+ * head) (U = U~ - W S0 and Kbar times the gradient at its end). */
 GDN2_API size_t gdn2_backward_workspace_size(const gdn2_desc* desc);
 
 /* Gradients of gdn2_chunk_fwd's outputs: given dO (the gradient of out) and

@@ -146,15 +146,16 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_backward_workspace_size(lib):
     """The backward's workspace: the status word, the forward's fp32 factor
-    set (whatever the I/O type), T and P, two dk x dv states and two 64 x dv
-    tiles per (chunk, head), each region 256-byte aligned."""
+    set (whatever the I/O type), T and P, three dk x dv matrices (the state,
+    its gradient, G) and two 64 x dv tiles per (chunk, head), each region
+    256-byte aligned."""
     B, T, H, dk, dv = 1, 16384, 16, 128, 128
     chunks_h = (T // 64) * H
-    regions = 2 * chunks_h * 64 * 64 * 4 + 2 * chunks_h * dk * dv * 4 + 2 * chunks_h * 64 * dv * 4
+    regions = 2 * chunks_h * 64 * 64 * 4 + 3 * chunks_h * dk * dv * 4 + 2 * chunks_h * 64 * dv * 4
     wy = gdn2.workspace_size(B, T, H, dk, dv, gdn2.GDN2_IO_F32)
     for io in (gdn2.GDN2_IO_BF16, gdn2.GDN2_IO_F32):
         n = gdn2.backward_workspace_size(B, T, H, dk, dv, io)
-        assert wy + regions + 256 <= n <= wy + regions + 256 + 7 * 256
+        assert wy + regions + 256 <= n <= wy + regions + 256 + 8 * 256
     assert gdn2.backward_workspace_size(B, T, H, dk, dv, gdn2.GDN2_IO_BF16) == \
         gdn2.backward_workspace_size(B, T, H, dk, dv, gdn2.GDN2_IO_F32)
     assert gdn2.backward_workspace_size(1, 128, 2, 96, 64) == 0          # bad dk
@@ -162,7 +163,7 @@ def test_backward_workspace_size(lib):
     n7 = gdn2.backward_workspace_size(1, 1000, 2, 64, 128, gdn2.GDN2_IO_F32, num_seqs=7)
     ch7 = (1000 // 64 + 7) * 2
     assert n7 >= gdn2.workspace_size(1, 1000, 2, 64, 128, gdn2.GDN2_IO_F32, num_seqs=7) + \
-        ch7 * (2 * 64 * 64 + 2 * 64 * 128 + 2 * 64 * 128) * 4
+        ch7 * (2 * 64 * 64 + 3 * 64 * 128 + 2 * 64 * 128) * 4
 
 
 def test_chunk_bwd_host_checks(lib):
