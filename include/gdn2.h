@@ -322,7 +322,8 @@ GDN2_API size_t gdn2_backward_workspace_size(const gdn2_desc* desc);
  *   2. the forward state at every chunk start is recomputed, and
  *   3. beside it (the two walks are independent) the chunks are walked in
  *      reverse: the gradient reaching a chunk's start state is
- *      dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO
+ *      dS0 = gamma_n dS1 - W^T (Kbar dS1) + scale Q_eff^T dO, the last term
+ *      formed for every chunk before the walk
  *      (dS1 of a sequence's last chunk is dhT; dh0 is dS0 of its first);
  *   4. every (chunk, head) then gives its tokens' gradients from its start
  *      state, the gradient at its end and dO, independently of the others.
