@@ -47,6 +47,7 @@ struct PrepArgs {
 };
 
 constexpr int kPrepSimtThreads = 512;
+constexpr float kPrepFoldNats = 60.f;   // decay range (each side of the middle row) for the product form of A, P
 
 template <int DK, int DV>
 constexpr size_t prep_simt_smem_bytes() {
@@ -122,41 +123,59 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     }
   }
   __syncthreads();
-  // A and P on 2 x 2 blocks of (i, j) pairs of the lower triangle, a thread
-  // per block, the key channels summed in registers.  exp(g_i - g_j) is taken
-  // of min(g_i - g_j, 0), so the entries above the diagonal (masked below)
-  // cannot overflow; its hardware exponential's error, a few ulp, is far
-  // below the fp32 path's tolerance.
-  {
-    constexpr int NB = kChunk / 2;
-    for (int t = tid; t < NB * (NB + 1) / 2; t += kPrepSimtThreads) {
-      int bi = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
-      while (bi * (bi + 1) / 2 > t) --bi;
-      while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
-      const int bj = t - bi * (bi + 1) / 2;
-      const int i0 = 2 * bi, j0 = 2 * bj;
-      if (i0 >= len) continue;   // rows past the last token stay zero
-      float aa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pp[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  // A and P.  Where the chunk's decay stays within kPrepFoldNats on each side
+  // of its middle row r, exp(g_ic - g_jc) = exp(g_ic - g_rc) exp(g_rc - g_jc)
+  // (both factors in fp32 range), so with e, q scaled by the first and k by
+  // the second, A and P are plain products over the key channels.  Otherwise
+  // each pair takes its own exponential.
+  __shared__ int s_steep;
+  if (tid == 0) s_steep = 0;
+  __syncthreads();
+  const int rref = min(kChunk / 2, len - 1);
+  if (tid < DK) {
+    const float g0 = sg[tid], gr = sg[rref * LK + tid], gl = sg[(kChunk - 1) * LK + tid];
+    if (g0 - gr > kPrepFoldNats || gr - gl > kPrepFoldNats) atomicOr(&s_steep, 1);
+  }
+  __syncthreads();
+  const bool fold = s_steep == 0;
+  if (fold) {
+    for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
+      const int i = idx / DK, cc = idx % DK;
+      const float d = sg[i * LK + cc] - sg[rref * LK + cc];
+      const float al = expf(d), be = expf(-d);
+      se[i * LK + cc] *= al;
+      sq[i * LK + cc] *= al;
+      sk[i * LK + cc] *= be;
+    }
+    __syncthreads();
+    // a thread per 2 x 4 block of (i, j) pairs: rows 2 (t / 16) + {0, 1},
+    // columns 4 (t % 16) + {0 .. 3}; blocks wholly above the diagonal idle
+    const int i0 = 2 * (tid / 16), j0 = 4 * (tid % 16);
+    if (j0 <= i0 + 1 && i0 < len) {
+      float aa[2][4], pp[2][4];
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) aa[r][q] = pp[r][q] = 0.f;
 #pragma unroll 4
       for (int cc = 0; cc < DK; ++cc) {
-        const float gi[2] = {sg[i0 * LK + cc], sg[(i0 + 1) * LK + cc]};
-        const float gj[2] = {sg[j0 * LK + cc], sg[(j0 + 1) * LK + cc]};
         const float ev[2] = {se[i0 * LK + cc], se[(i0 + 1) * LK + cc]};
         const float qv[2] = {sq[i0 * LK + cc], sq[(i0 + 1) * LK + cc]};
-        const float kv[2] = {sk[j0 * LK + cc], sk[(j0 + 1) * LK + cc]};
+        float kv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) kv[q] = sk[(j0 + q) * LK + cc];
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const float kd = kv[q] * __expf(fminf(gi[r] - gj[q], 0.f));
-            aa[r][q] = fmaf(ev[r], kd, aa[r][q]);
-            pp[r][q] = fmaf(qv[r], kd, pp[r][q]);
+          for (int q = 0; q < 4; ++q) {
+            aa[r][q] = fmaf(ev[r], kv[q], aa[r][q]);
+            pp[r][q] = fmaf(qv[r], kv[q], pp[r][q]);
           }
       }
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 4; ++q) {
           const int i = i0 + r, j = j0 + q;
           if (i < len && j <= i) {
             if (j < i) sA[i * LA + j] = aa[r][q];
@@ -164,18 +183,64 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
           }
         }
     }
+  } else {
+    // A and P on 2 x 2 blocks of (i, j) pairs of the lower triangle, a thread
+    // per block, the key channels summed in registers.  exp(g_i - g_j) is taken
+    // of min(g_i - g_j, 0), so the entries above the diagonal (masked below)
+    // cannot overflow; its hardware exponential's error, a few ulp, is far
+    // below the fp32 path's tolerance.
+    {
+      constexpr int NB = kChunk / 2;
+      for (int t = tid; t < NB * (NB + 1) / 2; t += kPrepSimtThreads) {
+        int bi = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+        while (bi * (bi + 1) / 2 > t) --bi;
+        while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
+        const int bj = t - bi * (bi + 1) / 2;
+        const int i0 = 2 * bi, j0 = 2 * bj;
+        if (i0 >= len) continue;   // rows past the last token stay zero
+        float aa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, pp[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  #pragma unroll 4
+        for (int cc = 0; cc < DK; ++cc) {
+          const float gi[2] = {sg[i0 * LK + cc], sg[(i0 + 1) * LK + cc]};
+          const float gj[2] = {sg[j0 * LK + cc], sg[(j0 + 1) * LK + cc]};
+          const float ev[2] = {se[i0 * LK + cc], se[(i0 + 1) * LK + cc]};
+          const float qv[2] = {sq[i0 * LK + cc], sq[(i0 + 1) * LK + cc]};
+          const float kv[2] = {sk[j0 * LK + cc], sk[(j0 + 1) * LK + cc]};
+  #pragma unroll
+          for (int r = 0; r < 2; ++r)
+  #pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float kd = kv[q] * __expf(fminf(gi[r] - gj[q], 0.f));
+              aa[r][q] = fmaf(ev[r], kd, aa[r][q]);
+              pp[r][q] = fmaf(qv[r], kd, pp[r][q]);
+            }
+        }
+  #pragma unroll
+        for (int r = 0; r < 2; ++r)
+  #pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int i = i0 + r, j = j0 + q;
+            if (i < len && j <= i) {
+              if (j < i) sA[i * LA + j] = aa[r][q];
+              sP[i * LA + j] = pp[r][q];
+            }
+          }
+      }
+    }
   }
   __syncthreads();
   // Kbar (kept in sk, rows past the last token zero) and gamma_last; E~ and
   // Q~ are formed in place.
   const size_t tile_k = ((size_t)c * H + h) * kChunk * DK;
   const size_t tile_v = ((size_t)c * H + h) * kChunk * DV;
+  // (in the product form e, q and k are held scaled: e exp(g) = (e exp(g - g_r))
+  // exp(g_r), and Kbar = k exp(g_n - g) = (k exp(g_r - g)) exp(g_n - g_r))
   for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
     const int i = idx / DK, cc = idx % DK;
-    const float gi = sg[i * LK + cc];
-    const float kb = i < len ? sk[i * LK + cc] * expf(sg[(kChunk - 1) * LK + cc] - gi) : 0.f;
+    const float gi = sg[i * LK + cc], gn = sg[(kChunk - 1) * LK + cc], gr = sg[rref * LK + cc];
+    const float kb = i < len ? sk[i * LK + cc] * expf(fold ? gn - gr : gn - gi) : 0.f;
     if constexpr (!AFFINE) a.Kbar[tile_k + idx] = from_f32<FT>(kb);
-    const float gam = expf(gi);
+    const float gam = expf(fold ? gr : gi);
     se[i * LK + cc] *= gam;
     sq[i * LK + cc] *= gam;
   }
@@ -183,7 +248,8 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
   __syncthreads();
   for (int idx = tid; idx < kChunk * DK; idx += kPrepSimtThreads) {
     const int i = idx / DK, cc = idx % DK;
-    sk[i * LK + cc] = i < len ? sk[i * LK + cc] * expf(sg[(kChunk - 1) * LK + cc] - sg[i * LK + cc]) : 0.f;
+    const float gn = sg[(kChunk - 1) * LK + cc];
+    sk[i * LK + cc] = i < len ? sk[i * LK + cc] * expf(fold ? gn - sg[rref * LK + cc] : gn - sg[i * LK + cc]) : 0.f;
   }
   if (tid < DK) a.gamma_last[((size_t)c * H + h) * DK + tid] = expf(sg[(kChunk - 1) * LK + tid]);
   if (AFFINE && a.colscale && tid < DK) a.colscale[((size_t)c * H + h) * DK + tid] = 1.f;
