@@ -47,11 +47,11 @@ ALG_FLOPS = TH * (6 * DK * DV + 5 * 64 * 128 + 64 * 64 / 3)
 # O_part = 2 x 64 x 128 x 2 B: 1536 B per token-head; exp(g_n) fp32 8 B).
 FACTOR_BYTES_PER_TH = 1536 + 8
 # DRAM bytes (read + write) of one fused launch at 16K x 1, from one ncu
-# capture (dram__bytes_read.sum 605,008,384 + dram__bytes_write.sum
-# 429,505,280) of this build's fused kernel under this script's own command
+# capture (dram__bytes_read.sum 604,688,128 + dram__bytes_write.sum
+# 429,519,104) of this build's fused kernel under this script's own command
 # (profiles/ holds the command).  It is taken again (or set to None) whenever
 # the fused kernel changes.
-FUSED_TRAFFIC_BYTES = 605008384 + 429505280
+FUSED_TRAFFIC_BYTES = 604688128 + 429519104
 PREP_BYTES = TH * (2304 + FACTOR_BYTES_PER_TH)
 WALK_BYTES = TH * (FACTOR_BYTES_PER_TH + 256) + B * H * DK * DV * 4
 L2_FLUSH_BYTES = 256 << 20
