@@ -240,11 +240,11 @@ bwd_g_kernel(const float* __restrict__ Qeff, const void* dO_, SeqMap map, int H,
   cp_async_wait_all();
   __syncthreads();
   const int m0 = 4 * (tid / CG), j0 = CPT * (tid % CG);
-  float acc[4][CPT];
+  float2 acc[4][CPT / 2];   // columns j0 + 2 e2, j0 + 2 e2 + 1
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int e = 0; e < CPT; ++e) acc[r][e] = 0.f;
+    for (int e2 = 0; e2 < CPT / 2; ++e2) acc[r][e2] = make_float2(0.f, 0.f);
 #pragma unroll 4
   for (int i = 0; i < kChunk; ++i) {
     float qv[4], ov[CPT];
@@ -265,12 +265,15 @@ bwd_g_kernel(const float* __restrict__ Qeff, const void* dO_, SeqMap map, int H,
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int e = 0; e < CPT; ++e) acc[r][e] = fmaf(qv[r], ov[e], acc[r][e]);
+      for (int e2 = 0; e2 < CPT / 2; ++e2)
+        acc[r][e2] = fma2s(qv[r], make_float2(ov[2 * e2], ov[2 * e2 + 1]), acc[r][e2]);
   }
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int e = 0; e < CPT; ++e) G[(ch * DK + m0 + r) * DV + j0 + e] = scale * acc[r][e];
+    for (int e2 = 0; e2 < CPT / 2; ++e2)
+      *reinterpret_cast<float2*>(G + (ch * DK + m0 + r) * DV + j0 + 2 * e2) =
+          make_float2(scale * acc[r][e2].x, scale * acc[r][e2].y);
 }
 
 template <int DK, int DV, typename IO>
@@ -351,6 +354,16 @@ __device__ __forceinline__ void unpack4(const float4 v, float (&o)[N], int at) {
   o[at] = v.x; o[at + 1] = v.y; o[at + 2] = v.z; o[at + 3] = v.w;
 }
 
+// Four consecutive values held as two packed pairs: element j, and the pairs
+// of a float4.
+__device__ __forceinline__ float pick4(const float2 (&v)[2], int j) {
+  return (j & 2) ? ((j & 1) ? v[1].y : v[1].x) : ((j & 1) ? v[0].y : v[0].x);
+}
+__device__ __forceinline__ void pairs4(const float4 v, float2 (&o)[2]) {
+  o[0] = make_float2(v.x, v.y);
+  o[1] = make_float2(v.z, v.w);
+}
+
 template <int DK, int DV, typename IO>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_chunk_kernel(const BwdChunkArgs a) {
@@ -383,15 +396,16 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   const int rk0 = TMK * (tid / C::CGK), ck0 = 4 * (tid % C::CGK);   // 64 x DK
   const int rp0 = 2 * (tid / 16), cp0 = 4 * (tid % 16);             // 64 x 64
   const int rv = 2 * (tid / 16), cv = tid % 16;                     // 64 x VB: rows rv, rv + 1; columns cv + 16 q
-  float accQ[TMK][4], accKb[TMK][4], accW[TMK][4], accP[2][4], accT[2][4];
+  // accumulators of the four columns of a thread tile, as two packed pairs
+  float2 accQ[TMK][2], accKb[TMK][2], accW[TMK][2], accP[2][2], accT[2][2];
 #pragma unroll
   for (int ii = 0; ii < TMK; ++ii)
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) accQ[ii][jj] = accKb[ii][jj] = accW[ii][jj] = 0.f;
+    for (int hh = 0; hh < 2; ++hh) accQ[ii][hh] = accKb[ii][hh] = accW[ii][hh] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) accP[ii][jj] = accT[ii][jj] = 0.f;
+    for (int hh = 0; hh < 2; ++hh) accP[ii][hh] = accT[ii][hh] = make_float2(0.f, 0.f);
 
   // ---------------------------------------------------- value loop ----
   // per pass of VB value columns: U (from the forward walk) and
@@ -454,17 +468,13 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
       // dU = Kbar dS1 + scale P^T dO and U^T on 2 x QN tiles (rows rv, rv + 1;
       // columns cv + 16 q: a thread rewrites only the entries it reads)
       {
-        float pd[2][QN];
+        float2 pd[QN];   // rows rv, rv + 1 of column cv + 16 q
 #pragma unroll
-        for (int q = 0; q < QN; ++q) pd[0][q] = pd[1][q] = 0.f;
+        for (int q = 0; q < QN; ++q) pd[q] = make_float2(0.f, 0.f);
         for (int j = rv; j < kChunk; ++j) {   // P_{j, i} = 0 for j < i
           const float2 p = *reinterpret_cast<const float2*>(sP + j * LT + rv);
 #pragma unroll
-          for (int q = 0; q < QN; ++q) {
-            const float o = to_f32(sdO[j * VB + cv + 16 * q]);
-            pd[0][q] = fmaf(p.x, o, pd[0][q]);
-            pd[1][q] = fmaf(p.y, o, pd[1][q]);
-          }
+          for (int q = 0; q < QN; ++q) pd[q] = fma2s(to_f32(sdO[j * VB + cv + 16 * q]), p, pd[q]);
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r)
@@ -472,18 +482,18 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
           for (int q = 0; q < QN; ++q) {
             const int i = rv + r, j = cv + 16 * q;
             sUT[j * LT + i] = sU[i * LVB + j];
-            sdU[i * LVB + j] = fmaf(a.scale, pd[r][q], sdU[i * LVB + j]);
+            sdU[i * LVB + j] = fmaf(a.scale, r ? pd[q].y : pd[q].x, sdU[i * LVB + j]);
           }
       }
       __syncthreads();
       // dQ~ += dO S0^T, dKbar += U dS1^T, dW += dU S0^T (negated later), four columns at a time
 #pragma unroll 1
       for (int j4 = 0; j4 < VB; j4 += 4) {
-        float sv[4][4], dv[4][4];
+        float2 sv[4][2], dv[4][2];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          unpack4(*reinterpret_cast<const float4*>(sS0T + (j4 + jj) * LDK + ck0), sv[jj], 0);
-          unpack4(*reinterpret_cast<const float4*>(sD1T + (j4 + jj) * LDK + ck0), dv[jj], 0);
+          pairs4(*reinterpret_cast<const float4*>(sS0T + (j4 + jj) * LDK + ck0), sv[jj]);
+          pairs4(*reinterpret_cast<const float4*>(sD1T + (j4 + jj) * LDK + ck0), dv[jj]);
         }
 #pragma unroll
         for (int ii = 0; ii < TMK; ++ii) {
@@ -496,21 +506,21 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              accQ[ii][e] = fmaf(o[jj], sv[jj][e], accQ[ii][e]);
-              accKb[ii][e] = fmaf(uu[jj], dv[jj][e], accKb[ii][e]);
-              accW[ii][e] = fmaf(du[jj], sv[jj][e], accW[ii][e]);
+            for (int hh = 0; hh < 2; ++hh) {
+              accQ[ii][hh] = fma2s(o[jj], sv[jj][hh], accQ[ii][hh]);
+              accKb[ii][hh] = fma2s(uu[jj], dv[jj][hh], accKb[ii][hh]);
+              accW[ii][hh] = fma2s(du[jj], sv[jj][hh], accW[ii][hh]);
             }
         }
       }
       // dP += dO U^T, dT += dU Z^T
 #pragma unroll 1
       for (int j4 = 0; j4 < VB; j4 += 4) {
-        float uv[4][4], zv[4][4];
+        float2 uv[4][2], zv[4][2];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          unpack4(*reinterpret_cast<const float4*>(sUT + (j4 + jj) * LT + cp0), uv[jj], 0);
-          unpack4(*reinterpret_cast<const float4*>(sZT + (j4 + jj) * LT + cp0), zv[jj], 0);
+          pairs4(*reinterpret_cast<const float4*>(sUT + (j4 + jj) * LT + cp0), uv[jj]);
+          pairs4(*reinterpret_cast<const float4*>(sZT + (j4 + jj) * LT + cp0), zv[jj]);
         }
 #pragma unroll
         for (int ii = 0; ii < 2; ++ii) {
@@ -522,25 +532,21 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              accP[ii][e] = fmaf(o[jj], uv[jj][e], accP[ii][e]);
-              accT[ii][e] = fmaf(du[jj], zv[jj][e], accT[ii][e]);
+            for (int hh = 0; hh < 2; ++hh) {
+              accP[ii][hh] = fma2s(o[jj], uv[jj][hh], accP[ii][hh]);
+              accT[ii][hh] = fma2s(du[jj], zv[jj][hh], accT[ii][hh]);
             }
         }
       }
       // dZ = T^T dU on the 2 x QN tile, then dv = dZ w and dw = dZ v
       {
-        float z[2][QN];
+        float2 z[QN];   // rows rv, rv + 1 of column cv + 16 q
 #pragma unroll
-        for (int q = 0; q < QN; ++q) z[0][q] = z[1][q] = 0.f;
+        for (int q = 0; q < QN; ++q) z[q] = make_float2(0.f, 0.f);
         for (int i = rv; i < kChunk; ++i) {   // T_{i, j} = 0 for i < j
           const float2 t = *reinterpret_cast<const float2*>(sT + i * LT + rv);
 #pragma unroll
-          for (int q = 0; q < QN; ++q) {
-            const float d = sdU[i * LVB + cv + 16 * q];
-            z[0][q] = fmaf(t.x, d, z[0][q]);
-            z[1][q] = fmaf(t.y, d, z[1][q]);
-          }
+          for (int q = 0; q < QN; ++q) z[q] = fma2s(sdU[i * LVB + cv + 16 * q], t, z[q]);
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r)
@@ -549,8 +555,9 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
             if (rv + r < len) {
               const int j = cv + 16 * q;
               const size_t o = tok_v(rv + r, v0 + j);
-              a.dv[o] = z[r][q] * sws[(rv + r) * VB + j];
-              a.dw[o] = z[r][q] * to_f32(svs[(rv + r) * VB + j]);
+              const float zz = r ? z[q].y : z[q].x;
+              a.dv[o] = zz * sws[(rv + r) * VB + j];
+              a.dw[o] = zz * to_f32(svs[(rv + r) * VB + j]);
             }
       }
     }
@@ -589,7 +596,7 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
   for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj)
-      sdP[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj <= rp0 + ii ? a.scale * accP[ii][jj] : 0.f;
+      sdP[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj <= rp0 + ii ? a.scale * pick4(accP[ii], jj) : 0.f;
   __syncthreads();
   if (tid < DK) {   // in-chunk cumulative sum; padded rows keep g at its last value
     float acc = 0.f;
@@ -611,7 +618,7 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
         const int cc = ck0 + jj;
         const float g = sg[i * LDK + cc], gn = sg[(kChunk - 1) * LDK + cc];
         const float gam = expf(g), ks = expf(gn - g);
-        const float dQt = a.scale * accQ[ii][jj], dKb = accKb[ii][jj];
+        const float dQt = a.scale * pick4(accQ[ii], jj), dKb = pick4(accKb[ii], jj);
         const float kb = sk[i * LDK + cc] * ks;   // Kbar
         dg[ii][jj] = dQt * sq[i * LDK + cc] * gam - dKb * kb;
         colsum[jj] = fmaf(dKb, kb, colsum[jj]);
@@ -642,32 +649,30 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
     for (int ii = 0; ii < TMK; ++ii)
       *reinterpret_cast<float4*>(sdW + (rk0 + ii) * LDK + ck0) =
-          make_float4(-accW[ii][0], -accW[ii][1], -accW[ii][2], -accW[ii][3]);
+          make_float4(-accW[ii][0].x, -accW[ii][0].y, -accW[ii][1].x, -accW[ii][1].y);
     __syncthreads();
 #pragma unroll 4
     for (int cc = 0; cc < DK; ++cc) {
-      const float4 e = *reinterpret_cast<const float4*>(sEtT + cc * LT + cp0);
-      const float ev[4] = {e.x, e.y, e.z, e.w};
+      float2 ev[2];
+      pairs4(*reinterpret_cast<const float4*>(sEtT + cc * LT + cp0), ev);
 #pragma unroll
       for (int ii = 0; ii < 2; ++ii) {
         const float wv = sdW[(rp0 + ii) * LDK + cc];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) accT[ii][jj] = fmaf(wv, ev[jj], accT[ii][jj]);
+        for (int hh = 0; hh < 2; ++hh) accT[ii][hh] = fma2s(wv, ev[hh], accT[ii][hh]);
       }
     }
-    float dEt[TMK][4];
+    float2 dEt[TMK][2];
 #pragma unroll
-    for (int ii = 0; ii < TMK; ++ii)
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) dEt[ii][jj] = 0.f;
+    for (int ii = 0; ii < TMK; ++ii) dEt[ii][0] = dEt[ii][1] = make_float2(0.f, 0.f);
     for (int m = rk0; m < kChunk; ++m) {   // T_{m, i} = 0 for m < i
-      const float4 d = *reinterpret_cast<const float4*>(sdW + m * LDK + ck0);
-      const float dv[4] = {d.x, d.y, d.z, d.w};
+      float2 dv[2];
+      pairs4(*reinterpret_cast<const float4*>(sdW + m * LDK + ck0), dv);
 #pragma unroll
       for (int ii = 0; ii < TMK; ++ii) {
         const float t = sT[m * LT + rk0 + ii];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) dEt[ii][jj] = fmaf(t, dv[jj], dEt[ii][jj]);
+        for (int hh = 0; hh < 2; ++hh) dEt[ii][hh] = fma2s(t, dv[hh], dEt[ii][hh]);
       }
     }
 #pragma unroll
@@ -677,8 +682,8 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int cc = ck0 + jj;
-        dg[ii][jj] = fmaf(dEt[ii][jj], sEtT[cc * LT + i], dg[ii][jj]);
-        dev[jj] = dEt[ii][jj] * expf(sg[i * LDK + cc]);
+        dg[ii][jj] = fmaf(pick4(dEt[ii], jj), sEtT[cc * LT + i], dg[ii][jj]);
+        dev[jj] = pick4(dEt[ii], jj) * expf(sg[i * LDK + cc]);
       }
       if (i < len) {   // dE so far (made db below) and dg so far
         *reinterpret_cast<float4*>(a.db + tok_k(i, ck0)) = make_float4(dev[0], dev[1], dev[2], dev[3]);
@@ -697,45 +702,50 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
     for (int ii = 0; ii < 2; ++ii)
       *reinterpret_cast<float4*>(sdT + (rp0 + ii) * LT + cp0) =
-          make_float4(accT[ii][0], accT[ii][1], accT[ii][2], accT[ii][3]);
+          make_float4(accT[ii][0].x, accT[ii][0].y, accT[ii][1].x, accT[ii][1].y);
     for (int idx = tid; idx < kChunk * kChunk; idx += kBwdThreads) {
       const int i = idx / kChunk, j = idx % kChunk;
       sTT[j * LT + i] = sT[i * LT + j];
     }
     __syncthreads();
-    float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float2 x[2][2];
+#pragma unroll
+    for (int ii = 0; ii < 2; ++ii) x[ii][0] = x[ii][1] = make_float2(0.f, 0.f);
 #pragma unroll 4
     for (int m = 0; m < kChunk; ++m) {   // X = dT T^T
-      const float4 t = *reinterpret_cast<const float4*>(sTT + m * LT + cp0);
-      const float tv[4] = {t.x, t.y, t.z, t.w};
+      float2 tv[2];
+      pairs4(*reinterpret_cast<const float4*>(sTT + m * LT + cp0), tv);
 #pragma unroll
       for (int ii = 0; ii < 2; ++ii) {
         const float d = sdT[(rp0 + ii) * LT + m];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) x[ii][jj] = fmaf(d, tv[jj], x[ii][jj]);
+        for (int hh = 0; hh < 2; ++hh) x[ii][hh] = fma2s(d, tv[hh], x[ii][hh]);
       }
     }
 #pragma unroll
     for (int ii = 0; ii < 2; ++ii)
-      *reinterpret_cast<float4*>(sX + (rp0 + ii) * LT + cp0) = make_float4(x[ii][0], x[ii][1], x[ii][2], x[ii][3]);
+      *reinterpret_cast<float4*>(sX + (rp0 + ii) * LT + cp0) =
+          make_float4(x[ii][0].x, x[ii][0].y, x[ii][1].x, x[ii][1].y);
     __syncthreads();
-    float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float2 y[2][2];
+#pragma unroll
+    for (int ii = 0; ii < 2; ++ii) y[ii][0] = y[ii][1] = make_float2(0.f, 0.f);
 #pragma unroll 4
     for (int m = 0; m < kChunk; ++m) {   // T^T X
-      const float4 xv4 = *reinterpret_cast<const float4*>(sX + m * LT + cp0);
-      const float xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+      float2 xv[2];
+      pairs4(*reinterpret_cast<const float4*>(sX + m * LT + cp0), xv);
 #pragma unroll
       for (int ii = 0; ii < 2; ++ii) {
         const float t = sT[m * LT + rp0 + ii];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) y[ii][jj] = fmaf(t, xv[jj], y[ii][jj]);
+        for (int hh = 0; hh < 2; ++hh) y[ii][hh] = fma2s(t, xv[hh], y[ii][hh]);
       }
     }
 #pragma unroll
     for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
-        sdA[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj < rp0 + ii ? -y[ii][jj] : 0.f;   // strictly lower
+        sdA[(rp0 + ii) * LT + cp0 + jj] = cp0 + jj < rp0 + ii ? -pick4(y[ii], jj) : 0.f;   // strictly lower
   }
   // the chunk's decay range on each side of the reference row r (its middle
   // token, or its last one when shorter): the product form below scales rows
@@ -776,28 +786,29 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
       }
     });
     __syncthreads();
-    float ed[TMK][4], qd[TMK][4], kd[TMK][4];
+    float2 ed[TMK][2], qd[TMK][2], kd[TMK][2];
 #pragma unroll
     for (int ii = 0; ii < TMK; ++ii)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) ed[ii][jj] = qd[ii][jj] = kd[ii][jj] = 0.f;
+      for (int hh = 0; hh < 2; ++hh) ed[ii][hh] = qd[ii][hh] = kd[ii][hh] = make_float2(0.f, 0.f);
     for (int m = 0; m < rk0 + TMK; ++m) {   // dA, dP vanish for m > i
-      float kbv[4];
-      unpack4(*reinterpret_cast<const float4*>(skb + m * LDK + ck0), kbv, 0);
+      float2 kbv[2];
+      pairs4(*reinterpret_cast<const float4*>(skb + m * LDK + ck0), kbv);
 #pragma unroll
       for (int ii = 0; ii < TMK; ++ii) {
         const float av = sdA[(rk0 + ii) * LT + m], pv = sdP[(rk0 + ii) * LT + m];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          ed[ii][jj] = fmaf(av, kbv[jj], ed[ii][jj]);
-          qd[ii][jj] = fmaf(pv, kbv[jj], qd[ii][jj]);
+        for (int hh = 0; hh < 2; ++hh) {
+          ed[ii][hh] = fma2s(av, kbv[hh], ed[ii][hh]);
+          qd[ii][hh] = fma2s(pv, kbv[hh], qd[ii][hh]);
         }
       }
     }
     for (int i = rk0; i < kChunk; ++i) {   // dA_{i, j}, dP_{i, j} vanish for i < j
-      float ea[4], qa[4], av[TMK], pv[TMK];
-      unpack4(*reinterpret_cast<const float4*>(sea + i * LDK + ck0), ea, 0);
-      unpack4(*reinterpret_cast<const float4*>(sqa + i * LDK + ck0), qa, 0);
+      float2 ea[2], qa[2];
+      float av[TMK], pv[TMK];
+      pairs4(*reinterpret_cast<const float4*>(sea + i * LDK + ck0), ea);
+      pairs4(*reinterpret_cast<const float4*>(sqa + i * LDK + ck0), qa);
 #pragma unroll
       for (int ii = 0; ii < TMK; ++ii) {
         av[ii] = sdA[i * LT + rk0 + ii];
@@ -806,7 +817,7 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
 #pragma unroll
       for (int ii = 0; ii < TMK; ++ii)
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) kd[ii][jj] = fmaf(av[ii], ea[jj], fmaf(pv[ii], qa[jj], kd[ii][jj]));
+        for (int hh = 0; hh < 2; ++hh) kd[ii][hh] = fma2s(av[ii], ea[hh], fma2s(pv[ii], qa[hh], kd[ii][hh]));
     }
     // combine with the partials this thread wrote (same rows and columns)
 #pragma unroll
@@ -827,12 +838,13 @@ bwd_chunk_kernel(const BwdChunkArgs a) {
         const int cc = ck0 + jj;
         const float g = sg[i * LDK + cc], gr = sg[rref * LDK + cc];
         const float al = expf(g - gr), be = expf(gr - g);
-        const float edv = al * ed[ii][jj], qdv = al * qd[ii][jj], kdv = be * kd[ii][jj];
+        const float edj = pick4(ed[ii], jj), qdj = pick4(qd[ii], jj), kdj = pick4(kd[ii], jj);
+        const float edv = al * edj, qdv = al * qdj, kdv = be * kdj;
         const float dE = fe[jj] + edv;
         fq[jj] += qdv;
         fk[jj] += kdv + dE * bq[jj];
         // e dE^D + q dQ^D - k dK^D, each from the scaled operands
-        fg[jj] += sea[i * LDK + cc] * ed[ii][jj] + sqa[i * LDK + cc] * qd[ii][jj] - skb[i * LDK + cc] * kd[ii][jj];
+        fg[jj] += sea[i * LDK + cc] * edj + sqa[i * LDK + cc] * qdj - skb[i * LDK + cc] * kdj;
         fe[jj] = dE * kv[jj];
       }
       *reinterpret_cast<float4*>(a.dq + o) = make_float4(fq[0], fq[1], fq[2], fq[3]);

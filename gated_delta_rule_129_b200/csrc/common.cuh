@@ -23,6 +23,13 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
+// acc + (a, a) * b on a pair of fp32 values as one packed FMA (sm_100's
+// f32x2 FMA; each component is rounded exactly like fmaf, so a loop that
+// keeps each output's order of terms gives the same bits as with fmaf).
+__device__ __forceinline__ float2 fma2s(float a, float2 b, float2 acc) {
+  return __ffma2_rn(make_float2(a, a), b, acc);
+}
+
 // The two bf16 values packed in a 32-bit word, as fp32 (exact).
 __device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -152,24 +152,25 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     // columns 4 (t % 16) + {0 .. 3}; blocks wholly above the diagonal idle
     const int i0 = 2 * (tid / 16), j0 = 4 * (tid % 16);
     if (j0 <= i0 + 1 && i0 < len) {
-      float aa[2][4], pp[2][4];
+      float2 aa[2][2], pp[2][2];   // columns j0 + 2 h, j0 + 2 h + 1 of row i0 + r
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) aa[r][q] = pp[r][q] = 0.f;
+        for (int hh = 0; hh < 2; ++hh) aa[r][hh] = pp[r][hh] = make_float2(0.f, 0.f);
 #pragma unroll 4
       for (int cc = 0; cc < DK; ++cc) {
         const float ev[2] = {se[i0 * LK + cc], se[(i0 + 1) * LK + cc]};
         const float qv[2] = {sq[i0 * LK + cc], sq[(i0 + 1) * LK + cc]};
-        float kv[4];
+        float2 kv[2];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) kv[q] = sk[(j0 + q) * LK + cc];
+        for (int hh = 0; hh < 2; ++hh)
+          kv[hh] = make_float2(sk[(j0 + 2 * hh) * LK + cc], sk[(j0 + 2 * hh + 1) * LK + cc]);
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            aa[r][q] = fmaf(ev[r], kv[q], aa[r][q]);
-            pp[r][q] = fmaf(qv[r], kv[q], pp[r][q]);
+          for (int hh = 0; hh < 2; ++hh) {
+            aa[r][hh] = fma2s(ev[r], kv[hh], aa[r][hh]);
+            pp[r][hh] = fma2s(qv[r], kv[hh], pp[r][hh]);
           }
       }
 #pragma unroll
@@ -177,9 +178,11 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int i = i0 + r, j = j0 + q;
+          const float av = (q & 1) ? aa[r][q >> 1].y : aa[r][q >> 1].x;
+          const float pv = (q & 1) ? pp[r][q >> 1].y : pp[r][q >> 1].x;
           if (i < len && j <= i) {
-            if (j < i) sA[i * LA + j] = aa[r][q];
-            sP[i * LA + j] = pp[r][q];
+            if (j < i) sA[i * LA + j] = av;
+            sP[i * LA + j] = pv;
           }
         }
     }
@@ -320,36 +323,39 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
     const int col = lane + 32 * e;
     return col < DK ? base_k + m * LK + col : base_v + m * LV + (col - DK);
   };
+  static_assert(NE % 2 == 0, "column pairs");
   {
-    float acc[4][NE];
+    float2 acc[4][NE / 2];   // columns e = 2 e2, 2 e2 + 1 of row 4 w + r
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int e = 0; e < NE; ++e) acc[r][e] = 0.f;
+      for (int e2 = 0; e2 < NE / 2; ++e2) acc[r][e2] = make_float2(0.f, 0.f);
     for (int m = 0; m < 4 * warp + 4; ++m) {
-      float tv[4], xv[NE];
+      float tv[4];
+      float2 xv[NE / 2];
 #pragma unroll
       for (int r = 0; r < 4; ++r) tv[r] = sT[(4 * warp + r) * LA + m];
 #pragma unroll
-      for (int e = 0; e < NE; ++e) xv[e] = *colp(se, sz, m, e);
+      for (int e2 = 0; e2 < NE / 2; ++e2) xv[e2] = make_float2(*colp(se, sz, m, 2 * e2), *colp(se, sz, m, 2 * e2 + 1));
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(tv[r], xv[e], acc[r][e]);
+        for (int e2 = 0; e2 < NE / 2; ++e2) acc[r][e2] = fma2s(tv[r], xv[e2], acc[r][e2]);
     }
     __syncthreads();   // every thread has read E~ and Z
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int e = 0; e < NE; ++e) *colp(se, sz, 4 * warp + r, e) = acc[r][e];
+      for (int e = 0; e < NE; ++e) *colp(se, sz, 4 * warp + r, e) = (e & 1) ? acc[r][e >> 1].y : acc[r][e >> 1].x;
   }
   __syncthreads();
   {
-    float acc[4][NE];
+    float2 acc[4][NE / 2];   // columns e = 2 e2, 2 e2 + 1 of row 4 w + r
+    auto q0 = [&](int r, int e) { return lane + 32 * e < DK ? sq[(4 * warp + r) * LK + lane + 32 * e] : 0.f; };
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int e = 0; e < NE; ++e) acc[r][e] = lane + 32 * e < DK ? sq[(4 * warp + r) * LK + lane + 32 * e] : 0.f;
+      for (int e2 = 0; e2 < NE / 2; ++e2) acc[r][e2] = make_float2(q0(r, 2 * e2), q0(r, 2 * e2 + 1));
     for (int m = 0; m < 4 * warp + 4; ++m) {
       float pv[4], xv[NE];
 #pragma unroll
@@ -362,7 +368,7 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(pv[r], xv[e], acc[r][e]);
+        for (int e2 = 0; e2 < NE / 2; ++e2) acc[r][e2] = fma2s(pv[r], make_float2(xv[2 * e2], xv[2 * e2 + 1]), acc[r][e2]);
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -370,11 +376,12 @@ __device__ __forceinline__ void prep_simt_chunk(const PrepArgs<IO, FT>& a, int c
 #pragma unroll
       for (int e = 0; e < NE; ++e) {
         const int col = lane + 32 * e;
+        const float av = (e & 1) ? acc[r][e >> 1].y : acc[r][e >> 1].x;
         if (col < DK) {
-          a.Qeff[tile_k + i * DK + col] = from_f32<FT>(acc[r][e]);
+          a.Qeff[tile_k + i * DK + col] = from_f32<FT>(av);
           if constexpr (!AFFINE) a.W[tile_k + i * DK + col] = from_f32<FT>(se[i * LK + col]);
         } else {
-          a.Opart[tile_v + i * DV + col - DK] = from_f32<FT>(acc[r][e]);
+          a.Opart[tile_v + i * DV + col - DK] = from_f32<FT>(av);
           if constexpr (!AFFINE) a.Ut[tile_v + i * DV + col - DK] = from_f32<FT>(sz[i * LV + col - DK]);
         }
       }
