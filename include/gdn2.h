@@ -275,10 +275,17 @@ GDN2_API gdn2_status gdn2_state_map(const gdn2_desc* desc, const void* q, const 
  *   conv_q, conv_k     : [H * dk, conv_width] fp32, tap i weighs token t - i
  *   conv_v             : [H * dv, conv_width] fp32
  *   cu_seqlens         : as for gdn2_chunk_fwd (sequence starts reset the
- *                        convolution), or NULL for B dense sequences
+ *                        convolution), or NULL for B dense sequences.  It is
+ *                        not validated here (there is no status word): a
+ *                        malformed array gives unspecified outputs, but
+ *                        every access stays inside the buffers above and
+ *                        its num_seqs + 1 entries.
  * desc: B, T, H, dk, dv, num_seqs and io as for gdn2_chunk_fwd (the workspace
  * is not used).  Outputs must not overlap the inputs.  Device pointers,
- * 16-byte aligned.  Asynchronous on `stream`. */
+ * 16-byte aligned.  Asynchronous on `stream`.
+ * Errors (before any launch): GDN2_ERR_NULL, _DTYPE, _SHAPE (dims, num_seqs
+ * against cu_seqlens, conv_width outside 1..8), _ALIGN; _UNSUPPORTED without
+ * an sm_100 device. */
 GDN2_API gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_raw, const void* k_raw,
                                          const void* v_raw, const float* conv_q, const float* conv_k,
                                          const float* conv_v, int conv_width, const int32_t* cu_seqlens, void* q,
@@ -287,7 +294,9 @@ GDN2_API gdn2_status gdn2_token_prologue(const gdn2_desc* desc, const void* q_ra
 /* out = rmsnorm(o) * norm_weight * sigmoid(gate), per token and head, the norm
  * over the dv channels of a head.
  *   o, gate, out : [B, T, H, dv] io dtype (out may be o);  norm_weight : [dv] fp32
- * desc: B, T, H, dk, dv, io (the rest is not used).  Asynchronous on `stream`. */
+ * desc: B, T, H, dk, dv, io (the rest is not used).  Asynchronous on `stream`.
+ * Errors (before any launch): GDN2_ERR_NULL, _DTYPE, _SHAPE, _ALIGN (every
+ * pointer 16-byte aligned); _UNSUPPORTED without an sm_100 device. */
 GDN2_API gdn2_status gdn2_token_epilogue(const gdn2_desc* desc, const void* o, const void* gate,
                                          const float* norm_weight, void* out, cudaStream_t stream);
 

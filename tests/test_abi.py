@@ -190,3 +190,94 @@ def test_chunk_bwd_host_checks(lib):
     bad[2] = None
     assert bwd(d, ins=bad) == NULL
     assert bwd(gdn2.make_desc(1, 128, 2, 64, 80, 0, 0, 0x100000, size)) == SHAPE
+
+
+P_ = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+
+
+def test_token_path_host_checks(lib):
+    """Failing argument checks of gdn2_token_prologue / gdn2_token_epilogue
+    return before any CUDA call (fake, never-dereferenced device addresses;
+    no call passes every check)."""
+    raw = [0x10000, 0x20000, 0x30000]
+    taps = [0x40000, 0x41000, 0x42000]
+    outs = [0x50000, 0x60000, 0x70000]
+
+    def pro(d, raw=raw, taps=taps, width=4, cu=None, outs=outs):
+        return lib.gdn2_token_prologue(None if d is None else ctypes.byref(d), *(P_(p) for p in raw),
+                                       *(P_(p) for p in taps), width, P_(cu), *(P_(p) for p in outs), None)
+    d = gdn2.make_desc(1, 256, 2, 128, 128, gdn2.GDN2_IO_BF16)
+    assert pro(None) == NULL
+    assert pro(d, width=0) == SHAPE
+    assert pro(d, width=9) == SHAPE
+    assert pro(gdn2.make_desc(1, 256, 2, 96, 128, gdn2.GDN2_IO_BF16)) == SHAPE
+    assert pro(gdn2.make_desc(1, 256, 2, 128, 128, 7)) == DTYPE
+    assert pro(gdn2.make_desc(1, 256, 2, 128, 128, gdn2.GDN2_IO_BF16, num_seqs=3)) == SHAPE   # dense with num_seqs
+    assert pro(gdn2.make_desc(2, 256, 2, 128, 128, gdn2.GDN2_IO_BF16, num_seqs=2), cu=0x80000) == SHAPE  # packed, B 2
+    assert pro(d, raw=[raw[0], None, raw[2]]) == NULL
+    assert pro(d, taps=[taps[0], taps[1], None]) == NULL
+    assert pro(d, outs=[None, outs[1], outs[2]]) == NULL
+    assert pro(d, raw=[raw[0] + 8, raw[1], raw[2]]) == ALIGN
+    assert pro(d, taps=[taps[0], taps[1] + 4, taps[2]]) == ALIGN
+    assert pro(d, outs=[outs[0], outs[1], outs[2] + 2]) == ALIGN
+
+    def epi(d, o=0x10000, gate=0x20000, weight=0x30000, out=0x40000):
+        return lib.gdn2_token_epilogue(None if d is None else ctypes.byref(d), P_(o), P_(gate), P_(weight),
+                                       P_(out), None)
+    assert epi(None) == NULL
+    assert epi(gdn2.make_desc(1, 256, 2, 128, 128, 7)) == DTYPE
+    assert epi(gdn2.make_desc(1, 256, 2, 128, 80, gdn2.GDN2_IO_BF16)) == SHAPE
+    assert epi(gdn2.make_desc(1, 256, 0, 128, 128, gdn2.GDN2_IO_BF16)) == SHAPE
+    assert epi(gdn2.make_desc(1, 2 ** 30, 2, 128, 128, gdn2.GDN2_IO_BF16)) == SHAPE   # token count
+    assert epi(d, gate=None) == NULL
+    assert epi(d, weight=None) == NULL
+    assert epi(d, out=0x40004) == ALIGN
+
+
+def test_segmented_and_state_map_host_checks(lib):
+    """The two-level scan's workspace size and the host checks of
+    gdn2_chunk_fwd_segmented and gdn2_state_map (each call fails a check
+    before any CUDA call)."""
+    B, T, H, dk, dv = 1, 4096, 2, 128, 128
+    bf = gdn2.GDN2_IO_BF16
+    base = gdn2.workspace_size(B, T, H, dk, dv, bf)
+    size_seg = lambda d, L: int(lib.gdn2_segmented_workspace_size(None if d is None else ctypes.byref(d), L))  # noqa: E731
+    n8 = size_seg(gdn2.make_desc(B, T, H, dk, dv, bf), 8)
+    # beyond the usual layout: 8 segments of 8 chunks, each a [dk, dk] Phi and
+    # two [dk, dv] matrices (Psi and the start state) per head, fp32
+    assert n8 >= base + 8 * H * (dk * dk + 2 * dk * dv) * 4
+    assert size_seg(gdn2.make_desc(B, T, H, dk, dv, bf), 0) > base          # the library's choice
+    assert size_seg(None, 8) == 0
+    assert size_seg(gdn2.make_desc(B, T, H, dk, dv, bf), -1) == 0
+    assert size_seg(gdn2.make_desc(B, T, H, 64, dv, bf), 8) == 0          # not the affine factor set
+    assert size_seg(gdn2.make_desc(B, T, H, dk, dv, gdn2.GDN2_IO_F32), 8) == 0
+
+    ins = [0x10000 + 0x1000 * i for i in range(6)]
+
+    def seg(d, ins=ins, out=0x80000, h0=None, hT=None, L=8):
+        return lib.gdn2_chunk_fwd_segmented(None if d is None else ctypes.byref(d), *(P_(p) for p in ins),
+                                            0.125, P_(h0), None, P_(out), P_(hT), L, None)
+    d = gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000000, n8)
+    assert seg(None) == NULL
+    assert seg(gdn2.make_desc(B, T, H, dk, dv, gdn2.GDN2_IO_F32, 0, 0x1000000, n8)) == UNSUPPORTED
+    assert seg(gdn2.make_desc(B, T, H, dk, dv, bf, 0, None, n8)) == WORKSPACE
+    assert seg(gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000010, n8)) == ALIGN
+    assert seg(gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000000, n8 - 1)) == WORKSPACE
+    assert seg(d, L=-1) == SHAPE
+    assert seg(d, ins=ins[:5] + [None]) == NULL
+    assert seg(d, out=None) == NULL
+    assert seg(d, out=0x80008) == ALIGN
+    assert seg(d, h0=0x90004) == ALIGN
+
+    wsz = gdn2.workspace_size(B, T, H, dk, dv, bf)
+
+    def smap(d, ins=ins, phi=0xA0000, psi=0xB0000):
+        return lib.gdn2_state_map(None if d is None else ctypes.byref(d), *(P_(p) for p in ins), None,
+                                  P_(phi), P_(psi), None)
+    d = gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000000, wsz)
+    assert smap(None) == NULL
+    assert smap(gdn2.make_desc(B, T, H, dk, dv, gdn2.GDN2_IO_F32, 0, 0x1000000, 1 << 30)) == UNSUPPORTED
+    assert smap(gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000000, wsz - 1)) == WORKSPACE
+    assert smap(d, ins=[None] + ins[1:]) == NULL
+    assert smap(d, phi=None) == NULL
+    assert smap(d, psi=0xB0004) == ALIGN
