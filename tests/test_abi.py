@@ -281,3 +281,50 @@ def test_segmented_and_state_map_host_checks(lib):
     assert smap(d, ins=[None] + ins[1:]) == NULL
     assert smap(d, phi=None) == NULL
     assert smap(d, psi=0xB0004) == ALIGN
+
+
+def test_stage_entry_points_host_checks(lib):
+    """gdn2_chunk_prep, _walk, _plan, _fused and _walk_flagged reject a missing
+    or short workspace, missing or misaligned pointers, and (fused, flagged)
+    shapes outside the affine factor set, before any CUDA call (each call
+    fails a check)."""
+    B, T, H, dk, dv = 1, 256, 2, 128, 128
+    bf, f32 = gdn2.GDN2_IO_BF16, gdn2.GDN2_IO_F32
+    size = gdn2.workspace_size(B, T, H, dk, dv, bf)
+    ins = [0x10000 + 0x1000 * i for i in range(6)]
+    ok = gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000000, size)
+    short = gdn2.make_desc(B, T, H, dk, dv, bf, 0, 0x1000000, size - 1)
+    nows = gdn2.make_desc(B, T, H, dk, dv, bf, 0, None, size)
+    r = ctypes.byref
+
+    def prep(d, ins=ins):
+        return lib.gdn2_chunk_prep(r(d), *(P_(p) for p in ins), None, None)
+    assert prep(short) == WORKSPACE
+    assert prep(nows) == WORKSPACE
+    assert prep(ok, ins=ins[:2] + [None] + ins[3:]) == NULL
+    assert prep(ok, ins=ins[:4] + [ins[4] + 4, ins[5]]) == ALIGN
+
+    def walk(d, out=0x80000, h0=None, hT=None, states=None):
+        return lib.gdn2_chunk_walk(r(d), 0.125, P_(h0), None, P_(out), P_(hT), P_(states), None)
+    assert walk(short) == WORKSPACE
+    assert walk(ok, out=None) == NULL
+    assert walk(ok, hT=0x90008) == ALIGN
+    assert walk(ok, states=0x90004) == ALIGN
+
+    assert lib.gdn2_chunk_plan(r(short), None, None) == WORKSPACE
+    assert lib.gdn2_chunk_plan(r(gdn2.make_desc(B, T, H, dk, dv, bf, 2, 0x1000000, 1 << 30)), None, None) == SHAPE
+
+    def fused(d, ins=ins, out=0x80000):
+        return lib.gdn2_chunk_fused(r(d), *(P_(p) for p in ins), 0.125, None, None, P_(out), None, None)
+    assert fused(short) == WORKSPACE
+    assert fused(ok, out=None) == NULL
+    assert fused(ok, ins=[ins[0] + 2] + ins[1:]) == ALIGN
+    f32_size = gdn2.workspace_size(B, T, H, dk, dv, f32)
+    assert fused(gdn2.make_desc(B, T, H, dk, dv, f32, 0, 0x1000000, f32_size), out=0x80004) == ALIGN
+
+    def flagged(d, out=0x80000):
+        return lib.gdn2_chunk_walk_flagged(r(d), 0.125, None, None, P_(out), None, 1000000, None)
+    assert flagged(short) == WORKSPACE
+    assert flagged(ok, out=None) == NULL
+    assert flagged(ok, out=0x80004) == ALIGN
+    assert flagged(gdn2.make_desc(B, T, H, dk, dv, f32, 0, 0x1000000, f32_size)) == UNSUPPORTED   # WY factor set
