@@ -23,8 +23,9 @@ from workloads import make_inputs
 NAMES = ("q", "k", "v", "log_alpha", "b", "w")
 
 
-def _case(B, T, H, dk, dv, seed, decay="mild", lengths=None):
-    x = make_inputs(B, T, H, dk, dv, io="f32", seed=seed, decay=decay, h0_std=0.3, lengths=lengths)
+def _case(B, T, H, dk, dv, seed, decay="mild", lengths=None, erase_range=1.0):
+    x = make_inputs(B, T, H, dk, dv, io="f32", seed=seed, decay=decay, h0_std=0.3, lengths=lengths,
+                    erase_range=erase_range)
     arrs = {n: getattr(x, n).astype(np.float64) for n in NAMES}
     arrs["h0"] = x.h0.astype(np.float64)
     rng = np.random.default_rng(seed + 500)
@@ -71,6 +72,15 @@ def test_backward_matches_finite_differences_sampled_strong_decay():
     rng = np.random.default_rng(7)
     picks = {n: [tuple(int(rng.integers(s)) for s in a.shape) for _ in range(12)] for n, a in arrs.items()}
     _fd_check(x, arrs, dO, dhT, grads, picks)
+
+
+def test_backward_matches_finite_differences_widened_erase_range():
+    """The erase gate widened to (0, 2) (the gate ablation): the same
+    derivative, now through erase factors up to a reflection."""
+    x, arrs, dO, dhT = _case(1, 9, 2, 4, 3, seed=85, decay="strong", erase_range=2.0)
+    assert arrs["b"].max() > 1.0
+    grads = _grads(x, arrs, dO, dhT)
+    _fd_check(x, arrs, dO, dhT, grads, _all_elements(arrs))
 
 
 def test_backward_packed_equals_separate_sequences():
@@ -120,13 +130,16 @@ def _rel(a, b):
     return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
 
 
-@pytest.mark.parametrize("T,chunk,decay,lengths", [(23, 8, "mild", None), (150, 64, "strong", None),
-                                                    (None, 16, "strong", [40, 0, 1, 33])])
-def test_chunk_backward_equals_token_backward(T, chunk, decay, lengths):
+@pytest.mark.parametrize("T,chunk,decay,lengths,erase_range", [(23, 8, "mild", None, 1.0),
+                                                                (150, 64, "strong", None, 1.0),
+                                                                (None, 16, "strong", [40, 0, 1, 33], 1.0),
+                                                                (100, 16, "strong", None, 2.0)])
+def test_chunk_backward_equals_token_backward(T, chunk, decay, lengths, erase_range):
     from oracle.chunk_backward import backward as chunk_backward
     if lengths is not None:
         T = sum(lengths)
-    x, arrs, dO, dhT = _case(1 if lengths else 2, T, 2, 6, 5, seed=84, decay=decay, lengths=lengths)
+    x, arrs, dO, dhT = _case(1 if lengths else 2, T, 2, 6, 5, seed=84, decay=decay, lengths=lengths,
+                             erase_range=erase_range)
     ref = _grads(x, arrs, dO, dhT)
     got = chunk_backward(*(arrs[n] for n in NAMES), x.scale, dO, dhT=dhT, h0=arrs["h0"],
                          cu_seqlens=x.cu_seqlens, chunk=chunk)
